@@ -1,0 +1,38 @@
+"""CPU float64 oracle for the Hidden Decoding hot path.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product package imports this
+package; only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline``
+/ ``--impl reference`` legs of ``bench.py`` may use it.  It shares no code,
+constant or helper with the CUDA path.
+
+Sources (page "Hidden Decoding at Scale", WeLM blog):
+  * "Multi-Stream Expansion and Training Objective", eq. S_t = E_k(x_i) at
+    t = (i-1)n + k, and the statement that only the final stream E_n feeds the
+    LM head  ->  :func:`expand`, :func:`final_stream_gather`.
+  * "Stream-Factorized Attention", eqs. i(t) = ceil(t/n), s(t) = (t-1) mod n + 1
+    and Figure 2 masks (a) full cross-stream causal, (b) local cross-stream
+    causal sliding window, (c) intra-stream causal  ->  :func:`visible`,
+    :func:`attn`, :func:`attn_rows`.
+  * "Persistent KV and the KV-mirror Saving" (a KV cache kept for every
+    stream) and "Inference Throughput" (the n streams of a token are processed
+    together in one pass)  ->  :func:`decode`.
+
+Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
+against library routines (SDPA, index_select), closed forms, invariants and a
+pure-Python brute force written from the pages' 1-based formulas.  The pages
+print no worked numeric example, so no value of theirs pins a number.
+"""
+
+from .hd_oracle import (  # noqa: F401
+    token_index,
+    stream_index,
+    visible,
+    visible_matrix,
+    expand,
+    final_stream_gather,
+    attn,
+    attn_rows,
+    decode,
+    decode_rows,
+    pair_count,
+)

@@ -1,0 +1,245 @@
+"""Plain, slow, float64 definition of the Hidden Decoding hot path.
+
+TEST INFRASTRUCTURE ONLY (see the package docstring).  Every routine follows
+its definition literally: build the visible set from the index maps, take
+scores, softmax over the visible set, weight the values.  No blocking, no
+online softmax, no reordering beyond what a numpy matmul does internally.
+
+Indexing is 0-based throughout: token i in [0, L), stream s in [0, n), physical
+position p = i*n + s.  This is the pages' t = (i-1)n + k with i -> i+1 and
+k -> s+1 ("Hidden Decoding at Scale", "Multi-Stream Expansion and Training
+Objective").  The final stream is s = n-1.
+
+Readings where the pages are silent (each listed in the design notes):
+  * window W: intra-stream layers count W in tokens of the stream
+    (key (j,s) visible to query (i,s) iff i-W < j <= i); cross-stream layers
+    count W in physical positions (p-W < p' <= p).  W = 0 means no window.
+  * GQA: query head h reads KV head h // (Hq // Hkv).
+  * decode: ctx_len counts tokens per stream including the new one; the new
+    token's stream s sees the new token's streams s' <= s in cross mode
+    (causal in p), i.e. exactly the prefill row of that position.
+  * lse is the natural-log log-sum-exp of the scaled visible scores.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+INTRA = "intra"
+CROSS = "cross"
+
+
+def _mode(mode) -> str:
+    if mode in (INTRA, 0):
+        return INTRA
+    if mode in (CROSS, 1):
+        return CROSS
+    raise ValueError(f"unknown mode {mode!r}")
+
+
+def token_index(p, n):
+    """i(t) = ceil(t/n) of "Stream-Factorized Attention", 0-based: p // n."""
+    return np.asarray(p) // n
+
+
+def stream_index(p, n):
+    """s(t) = (t-1) mod n + 1 of "Stream-Factorized Attention", 0-based: p % n."""
+    return np.asarray(p) % n
+
+
+def visible(p, pk, n, mode, window=0):
+    """True where key position ``pk`` is visible to query position ``p``.
+
+    Figure 2 of "Stream-Factorized Attention":
+      (c) intra-stream: same stream and earlier-or-equal token
+          (optionally within ``window`` tokens of that stream);
+      (a) full cross-stream: standard causal over the interleaved order;
+      (b) local cross-stream: causal with a sliding window of ``window``
+          physical positions.
+    Broadcasts over array arguments.
+    """
+    mode = _mode(mode)
+    p = np.asarray(p)
+    pk = np.asarray(pk)
+    if mode == INTRA:
+        i, s = token_index(p, n), stream_index(p, n)
+        j, sk = token_index(pk, n), stream_index(pk, n)
+        ok = (sk == s) & (j <= i)
+        if window:
+            ok = ok & (i - j < window)
+    else:
+        ok = pk <= p
+        if window:
+            ok = ok & (p - pk < window)
+    return ok
+
+
+def visible_matrix(L, n, mode, window=0):
+    """[nL, nL] boolean mask, row = query position, column = key position."""
+    P = n * L
+    p = np.arange(P)[:, None]
+    pk = np.arange(P)[None, :]
+    return visible(p, pk, n, mode, window)
+
+
+def pair_count(L, n, mode, window=0):
+    """Number of visible (query, key) pairs per (batch, query head), counted by
+    enumerating the mask.  Useful FLOP = pairs * 4 * head_dim (QK^T and PV,
+    forward only, self pairs included)."""
+    total = 0
+    P = n * L
+    pk = np.arange(P)
+    for p in range(P):
+        total += int(np.count_nonzero(visible(p, pk, n, mode, window)))
+    return total
+
+
+def expand(tables, ids):
+    """S_t = E_k(x_i) ("Multi-Stream Expansion and Training Objective").
+
+    tables: [n, V, d]; ids: [B, L] integers in [0, V).
+    Returns out [B, n*L, d] with out[b, i*n + s] = tables[s, ids[b, i]].
+    Raises on an out-of-range id.
+    """
+    tables = np.asarray(tables)
+    ids = np.asarray(ids)
+    n, V, d = tables.shape
+    B, L = ids.shape
+    if ids.size and (ids.min() < 0 or ids.max() >= V):
+        raise ValueError("token id out of range")
+    out = np.empty((B, n * L, d), dtype=tables.dtype)
+    for b in range(B):
+        for i in range(L):
+            for s in range(n):
+                out[b, i * n + s] = tables[s, ids[b, i]]
+    return out
+
+
+def final_stream_gather(h, n):
+    """Rows of the final stream, the only ones fed to the shared LM head
+    ("Multi-Stream Expansion and Training Objective"; Figure 1).
+
+    h: [B, n*L, d] -> out [B, L, d], out[b, i] = h[b, i*n + n - 1].
+    """
+    h = np.asarray(h)
+    B, P, d = h.shape
+    if P % n:
+        raise ValueError("sequence length is not a multiple of n")
+    L = P // n
+    out = np.empty((B, L, d), dtype=h.dtype)
+    for b in range(B):
+        for i in range(L):
+            out[b, i] = h[b, i * n + n - 1]
+    return out
+
+
+def _softmax_weighted(scores, vals):
+    """Softmax over the last axis of ``scores`` (-inf = masked) applied to
+    ``vals``; returns (out, lse)."""
+    m = scores.max(axis=-1, keepdims=True)
+    w = np.exp(scores - m)
+    l = w.sum(axis=-1, keepdims=True)
+    out = (w / l) @ vals
+    lse = (m + np.log(l))[..., 0]
+    return out, lse
+
+
+def attn(q, k, v, n, mode, window=0, scale=None):
+    """Stream-Factorized Attention forward, float64.
+
+    q: [B, nL, Hq, D]; k, v: [B, nL, Hkv, D].  Returns (O [B, nL, Hq, D],
+    lse [B, Hq, nL]).  For each (b, h, p): scores over visible keys
+    scale * <q, k>, softmax, weighted sum of v.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, P, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if Hq % Hkv or P % n:
+        raise ValueError("bad shapes")
+    G = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    mask = visible_matrix(P // n, n, mode, window)
+    O = np.empty((B, P, Hq, D))
+    lse = np.empty((B, Hq, P))
+    for b in range(B):
+        for h in range(Hq):
+            kv = h // G
+            s = scale * (q[b, :, h, :] @ k[b, :, kv, :].T)
+            s = np.where(mask, s, -np.inf)
+            O[b, :, h, :], lse[b, h, :] = _softmax_weighted(s, v[b, :, kv, :])
+    return O, lse
+
+
+def attn_rows(q, k, v, n, mode, rows, window=0, scale=None):
+    """The same definition evaluated for selected output rows only.
+
+    rows: iterable of (b, h, p).  Returns (O [R, D], lse [R]).  Inputs may be
+    any array-likes indexable as q[b, p, h, :] (e.g. large float32 arrays);
+    each row's arithmetic is float64.
+    """
+    P = k.shape[1]
+    Hq = q.shape[2]
+    Hkv = k.shape[2]
+    G = Hq // Hkv
+    D = q.shape[3]
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    pk_all = np.arange(P)
+    outs, lses = [], []
+    for (b, h, p) in rows:
+        kv = h // G
+        keys = pk_all[visible(p, pk_all, n, mode, window)]
+        qv = np.asarray(q[b, p, h, :], dtype=np.float64)
+        kk = np.asarray(k[b, keys, kv, :], dtype=np.float64)
+        vv = np.asarray(v[b, keys, kv, :], dtype=np.float64)
+        o, l = _softmax_weighted(scale * (kk @ qv)[None, :], vv)
+        outs.append(o[0])
+        lses.append(l[0])
+    return np.array(outs), np.array(lses)
+
+
+def _decode_keys(T, n, s, mode, window):
+    """Visible cache entries (j, s') for the stream-s query of the new token
+    T-1, as physical positions of the expanded sequence."""
+    p = (T - 1) * n + s
+    pk = np.arange(T * n)
+    return pk[visible(p, pk, n, mode, window)]
+
+
+def decode_rows(q, k_cache, v_cache, ctx_len, n, mode, rows, window=0, scale=None):
+    """Decode for selected (b, s, h): the stream-s query of the newest token
+    of sequence b against the per-stream cache.
+
+    q: [B, n, Hq, D]; k_cache, v_cache: [B, n, Lmax, Hkv, D] (stream-major);
+    ctx_len: [B] tokens per stream, new token included.  Returns (O [R, D],
+    lse [R]).
+    """
+    Hq, D = q.shape[2], q.shape[3]
+    Hkv = k_cache.shape[3]
+    G = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    outs, lses = [], []
+    for (b, s, h) in rows:
+        T = int(ctx_len[b])
+        kv = h // G
+        pk = _decode_keys(T, n, s, mode, window)
+        j, sk = pk // n, pk % n
+        kk = np.asarray(k_cache[b, sk, j, kv, :], dtype=np.float64)
+        vv = np.asarray(v_cache[b, sk, j, kv, :], dtype=np.float64)
+        qv = np.asarray(q[b, s, h, :], dtype=np.float64)
+        o, l = _softmax_weighted(scale * (kk @ qv)[None, :], vv)
+        outs.append(o[0])
+        lses.append(l[0])
+    return np.array(outs), np.array(lses)
+
+
+def decode(q, k_cache, v_cache, ctx_len, n, mode, window=0, scale=None):
+    """All rows of :func:`decode_rows`: returns (O [B, n, Hq, D], lse [B, n, Hq])."""
+    B, _, Hq, D = q.shape
+    rows = [(b, s, h) for b in range(B) for s in range(n) for h in range(Hq)]
+    O, lse = decode_rows(q, k_cache, v_cache, ctx_len, n, mode, rows, window, scale)
+    return O.reshape(B, n, Hq, D), lse.reshape(B, n, Hq)
