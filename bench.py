@@ -1,0 +1,543 @@
+"""Benchmark of the Hidden Decoding hot path on B200; prints ONE JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload intra|cross|long|decode] [--no-extras]
+
+Default workload (intra): n=4 streams, L=4096 tokens (nL=16384), batch 2,
+32 query / 8 KV heads, head_dim 128, bf16.  One step is one pass of the
+prefill hot path over one batch: hd_expand_embed (4 tables of 152064 x 4096,
+Zipf(1.1) ids) -> hd_attn_fwd (intra-stream, causal) -> hd_final_stream_gather
+(final-stream rows of the expanded [B, nL, 4096] sequence).  The metric is
+useful attention TFLOP/s (visible pairs x 4 x head_dim per second of step
+time); the decode workload (batch 64, 32768 tokens per stream, both modes) is
+reported alongside in GB/s against HBM, and the cross-stream layer cost in
+TFLOP/s.
+
+Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
+on the launching stream, with an L2 flush (a 512 MiB write) between steps
+outside the events; a barrier and a device synchronise on both sides; the
+max over ranks.  With N > 1 every rank runs its own batch (data-parallel,
+weak scaling; no collective on the data path).
+
+--impl reference times the float64 CPU oracle on this machine's host cores
+(rank 0 only) on bounded samples of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOADS = {
+    "intra": dict(B=2, n=4, L=4096, Hq=32, Hkv=8, D=128, mode="intra", W=0, V=152064, dm=4096),
+    "cross": dict(B=2, n=4, L=4096, Hq=32, Hkv=8, D=128, mode="cross", W=0, V=152064, dm=4096),
+    "long": dict(B=1, n=4, L=32768, Hq=64, Hkv=8, D=128, mode="intra", W=4096, V=152064, dm=4096),
+    "decode": dict(B=64, n=4, T=32768, Hq=64, Hkv=8, D=128),
+}
+NAMES = {
+    "intra": "bf16 prefill, intra-stream, n=4 L=4096 B=2 32q/8kv D=128",
+    "cross": "bf16 prefill, cross-stream, n=4 L=4096 B=2 32q/8kv D=128",
+    "long": "long-context intra-stream W=4096, n=4 L=32768 B=1 64q/8kv D=128",
+    "decode": "decode B=64 n=4 ctx=32768 64q/8kv D=128, intra+cross",
+}
+FLUSH_BYTES = 512 << 20
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=None)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="intra", choices=list(WORKLOADS))
+    ap.add_argument("--no-extras", action="store_true", help="skip the side measurements")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"], bf16_sus=p.get("bf16_tflops_sustained"),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+
+
+def kernel_source_sha(names):
+    h = hashlib.sha256()
+    for nm in names:
+        with open(os.path.join(ROOT, "stream_sequence_attention_b200", "csrc", nm), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, sources, workload):
+    """DRAM bytes per launch from a committed ncu summary, or None when the
+    kernel source changed since the capture."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        t = json.load(f)
+    e = t.get(kernel, {}).get(workload)
+    if not e or e.get("source_sha") != kernel_source_sha(sources):
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ GPU workloads
+
+class Prefill:
+    """expand -> attention -> final-stream gather on device-resident inputs."""
+
+    def __init__(self, cfg, seed_base, torch, hd, synth):
+        self.cfg = c = cfg
+        self.torch, self.hd = torch, hd
+        P = c["n"] * c["L"]
+        self.P = P
+        ids = synth.ids_zipf(c["B"], c["L"], c["V"], 1.1, seed_base + 1)
+        self.ids_host = torch.from_numpy(ids).pin_memory()
+        self.ids = self.ids_host.cuda()
+        self.tables = synth.normal_device((c["n"], c["V"], c["dm"]), seed_base + 2, std=0.02)
+        self.q = synth.normal_device((c["B"], P, c["Hq"], c["D"]), seed_base + 3)
+        self.k = synth.normal_device((c["B"], P, c["Hkv"], c["D"]), seed_base + 4)
+        self.v = synth.normal_device((c["B"], P, c["Hkv"], c["D"]), seed_base + 5)
+        self.x = torch.empty((c["B"], P, c["dm"]), dtype=torch.bfloat16, device="cuda")
+        self.o = torch.empty_like(self.q)
+        self.g = torch.empty((c["B"], c["L"], c["dm"]), dtype=torch.bfloat16, device="cuda")
+        self.status = hd.new_status()
+
+    def step(self, ev=None):
+        c, hd = self.cfg, self.hd
+        hd.hd_expand_embed(self.tables, self.ids, self.x, dev_status=self.status)
+        if ev is not None:
+            ev[0].record()
+        hd.hd_attn_fwd(self.q, self.k, self.v, c["n"], c["mode"], c["W"], out=self.o, dev_status=self.status)
+        if ev is not None:
+            ev[1].record()
+        hd.hd_final_stream_gather(self.x, c["n"], out=self.g)
+
+    launches_per_step = 3
+
+    def e2e_buffers(self):
+        torch = self.torch
+        self.h_q = torch.empty_like(self.q, device="cpu").pin_memory()
+        self.h_k = torch.empty_like(self.k, device="cpu").pin_memory()
+        self.h_v = torch.empty_like(self.v, device="cpu").pin_memory()
+        self.h_q.copy_(self.q)
+        self.h_k.copy_(self.k)
+        self.h_v.copy_(self.v)
+        self.h_g = torch.empty_like(self.g, device="cpu").pin_memory()
+        self.h_o = torch.empty_like(self.o, device="cpu").pin_memory()
+        return (self.ids_host.numel() * 4 + 2 * (self.h_q.numel() + self.h_k.numel() + self.h_v.numel()),
+                2 * (self.h_g.numel() + self.h_o.numel()))
+
+    def e2e_step(self):
+        """Host inputs -> device, the step, results -> host (pinned buffers)."""
+        self.ids.copy_(self.ids_host, non_blocking=True)
+        self.q.copy_(self.h_q, non_blocking=True)
+        self.k.copy_(self.h_k, non_blocking=True)
+        self.v.copy_(self.h_v, non_blocking=True)
+        self.step()
+        self.h_o.copy_(self.o, non_blocking=True)
+        self.h_g.copy_(self.g, non_blocking=True)
+
+    def flops(self):
+        from stream_sequence_attention_b200 import accounting as acc
+        c = self.cfg
+        return acc.attn_flops(c["B"], c["L"], c["n"], c["Hq"], c["D"], c["mode"], c["W"])
+
+
+class Decode:
+    """hd_attn_decode, intra then cross, against a resident per-stream cache."""
+
+    def __init__(self, cfg, seed_base, torch, hd, synth):
+        self.cfg = c = cfg
+        self.torch, self.hd = torch, hd
+        self.q = synth.normal_device((c["B"], c["n"], c["Hq"], c["D"]), seed_base + 1)
+        self.kc = synth.normal_device((c["B"], c["n"], c["T"], c["Hkv"], c["D"]), seed_base + 2)
+        self.vc = synth.normal_device((c["B"], c["n"], c["T"], c["Hkv"], c["D"]), seed_base + 3)
+        self.ctx = torch.full((c["B"],), c["T"], dtype=torch.int32, device="cuda")
+        self.o = {m: torch.empty_like(self.q) for m in ("intra", "cross")}
+        wsb = max(hd.hd_attn_decode_workspace(c["B"], c["n"], c["T"], c["Hq"], c["Hkv"], c["D"], m)
+                  for m in ("intra", "cross"))
+        self.ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+        self.status = hd.new_status()
+
+    def run(self, mode):
+        self.hd.hd_attn_decode(self.q, self.kc, self.vc, self.ctx, mode, out=self.o[mode], workspace=self.ws,
+                               dev_status=self.status)
+
+    def step(self, ev=None):
+        if ev is not None:
+            ev[0].record()
+        self.run("intra")
+        if ev is not None:
+            ev[1].record()
+        self.run("cross")
+
+    launches_per_step = 4  # decode + combine, per mode
+
+    def bytes_per_mode(self):
+        from stream_sequence_attention_b200 import accounting as acc
+        c = self.cfg
+        return acc.decode_bytes(c["B"], c["n"], c["T"], c["Hq"], c["Hkv"], c["D"])
+
+    def e2e_buffers(self):
+        torch = self.torch
+        self.h_q = torch.empty_like(self.q, device="cpu").pin_memory()
+        self.h_q.copy_(self.q)
+        self.h_o = {m: torch.empty_like(self.q, device="cpu").pin_memory() for m in self.o}
+        return 2 * self.h_q.numel(), 2 * 2 * self.h_q.numel()
+
+    def e2e_step(self):
+        self.q.copy_(self.h_q, non_blocking=True)
+        self.step()
+        for m in self.o:
+            self.h_o[m].copy_(self.o[m], non_blocking=True)
+
+
+def timed(torch, work, K, flush, dist=None, use_e2e=False):
+    """Run K steps with per-step CUDA events (flush outside them).  Returns
+    (per-step ms list, dominant-kernel ms list)."""
+    st = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    en = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush()
+        st[i].record()
+        if use_e2e:
+            work.e2e_step()
+        else:
+            work.step(kev[i])
+        en[i].record()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    steps = [a.elapsed_time(b) for a, b in zip(st, en)]
+    kern = [] if use_e2e else [a.elapsed_time(b) for a, b in kev]
+    return steps, kern
+
+
+def max_over_ranks(torch, dist, x):
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_ours(args, rank, world, dist):
+    import torch
+
+    from stream_sequence_attention_b200 import build as hd_build
+    from stream_sequence_attention_b200 import hd, synth
+
+    hd_build.build()
+    hd.lib()
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+    peaks = load_peaks()
+    wl = args.workload
+    cfg = WORKLOADS[wl]
+    K = args.steps if args.steps is not None else (100 if wl != "decode" else 40)
+    W = args.warmup if args.warmup is not None else 5
+    W = max(W, 3)
+    seed_base = 1000 * (list(WORKLOADS).index(wl) + 1) + 97 * rank
+    work = Decode(cfg, seed_base, torch, hd, synth) if wl == "decode" else Prefill(cfg, seed_base, torch, hd, synth)
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush = lambda: flush_buf.fill_(1)  # noqa: E731
+
+    for _ in range(W):
+        flush()
+        work.step()
+    torch.cuda.synchronize()
+    if int(work.status.item()) != 0:
+        raise RuntimeError(f"device status {hd.status_string(int(work.status.item()))}")
+
+    clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", 0)))
+    clocks.start()
+    steps, kern = timed(torch, work, K, flush, dist)
+    clk = clocks.stop()
+    total_ms = sum(steps)
+    total_ms = max_over_ranks(torch, dist, total_ms)
+    ms_per_step = total_ms / K
+    kern_ms = statistics.mean(kern)
+
+    # e2e through the public API with host buffers
+    bi, bo = work.e2e_buffers()
+    for _ in range(2):
+        work.e2e_step()
+    e2e_steps, _ = timed(torch, work, args.e2e_steps, flush, dist, use_e2e=True)
+    e2e_ms = max_over_ranks(torch, dist, sum(e2e_steps)) / args.e2e_steps
+
+    out = {}
+    if wl == "decode":
+        nbytes = 2 * work.bytes_per_mode()
+        value = world * nbytes / (ms_per_step * 1e-3) / 1e9
+        metric, unit = "decode GB/s vs HBM (intra+cross, B=64 n=4 ctx=32768)", "GB/s"
+        achieved = work.bytes_per_mode() / (kern_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm"], 4), "kernel": "decode_kernel (intra) + combine",
+                "peak_source": peaks["source"] + " hbm_gbs",
+                "traffic": recorded_traffic("decode_kernel", ["decode.cu"], "decode_intra")}
+        e2e_value = world * nbytes / (e2e_ms * 1e-3) / 1e9
+        dtype = "bf16"
+    else:
+        fl = work.flops()
+        value = world * fl / (ms_per_step * 1e-3) / 1e12
+        metric = "useful attn TFLOP/s at n=4 (%s)" % cfg["mode"]
+        unit = "TFLOP/s"
+        achieved = fl / (kern_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16"], "unit": "TFLOP/s",
+                "frac": round(achieved / peaks["bf16"], 4), "kernel": "attn_tc_kernel<128>",
+                "peak_source": peaks["source"] + " bf16_tflops (burst)",
+                "traffic": recorded_traffic("attn_tc_kernel", ["attn_tc.cu", "hd_common.cuh"], wl)}
+        e2e_value = world * fl / (e2e_ms * 1e-3) / 1e12
+        dtype = "bf16"
+    out.update({
+        "metric": metric, "value": round(value, 2), "unit": unit, "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": dtype, "data": "synthetic (seeded; device-drawn N(0,1) q/k/v, N(0,0.02) tables, Zipf(1.1) ids)",
+        "config": {"workload": NAMES[wl], "global_batch": cfg["B"] * world,
+                   "seq_len": cfg.get("L", cfg.get("T")) * cfg["n"], "parallelism": f"dp{world}",
+                   "l2": "flushed between timed steps (512 MiB write, outside the step events)"},
+        "roofline": roof,
+        "e2e": {"value": round(e2e_value, 3), "unit": unit, "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
+                "ms_per_step": round(e2e_ms, 3)},
+        "gpu_launches": work.launches_per_step * K,
+        "clocks": clk,
+    })
+    return out, work, peaks
+
+
+def extras(torch, peaks, rank):
+    """Side measurements on one GPU: decode GB/s (both modes) and the
+    cross-stream prefill layer."""
+    from stream_sequence_attention_b200 import hd, synth
+
+    res = {}
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush = lambda: flush_buf.fill_(1)  # noqa: E731
+
+    def time_fn(fn, K=10, W=3):
+        for _ in range(W):
+            flush()
+            fn()
+        ts = []
+        for _ in range(K):
+            flush()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    dec = Decode(WORKLOADS["decode"], 7001 + rank, torch, hd, synth)
+    nb = dec.bytes_per_mode()
+    for mode in ("intra", "cross"):
+        ms = time_fn(lambda: dec.run(mode))
+        gbs = nb / (ms * 1e-3) / 1e9
+        res[f"decode_{mode}"] = {"ms": round(ms, 3), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm"], 4)}
+    del dec
+    torch.cuda.empty_cache()
+    cr = Prefill(WORKLOADS["cross"], 7101 + rank, torch, hd, synth)
+    c = WORKLOADS["cross"]
+    ms = time_fn(lambda: hd.hd_attn_fwd(cr.q, cr.k, cr.v, c["n"], "cross", out=cr.o))
+    tf = cr.flops() / (ms * 1e-3) / 1e12
+    res["cross_prefill"] = {"ms": round(ms, 3), "TFLOP/s": round(tf, 1), "frac_bf16": round(tf / peaks["bf16"], 4)}
+    del cr
+    torch.cuda.empty_cache()
+    return res
+
+
+# ------------------------------------------------------------ CPU oracle arm
+
+def oracle_sample_rate(wl, budget_s, seed=5):
+    """Run the float64 oracle on host cores on sampled output rows of the
+    workload for about ``budget_s`` seconds; returns (units/s, unit, sample
+    description, threads)."""
+    import numpy as np
+
+    import oracle
+    from stream_sequence_attention_b200 import synth
+
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        threads = 1
+    cfg = WORKLOADS[wl]
+    g = synth.rng(seed)
+    if wl == "decode":
+        n, T, D = cfg["n"], cfg["T"], cfg["D"]
+        G = cfg["Hq"] // cfg["Hkv"]
+        # one KV head of one sequence, host-drawn at full context length
+        q = synth.normal((1, n, G, D), seed + 1, dtype="bf16")
+        kc = synth.normal((1, n, T, 1, D), seed + 2, dtype="bf16")
+        vc = synth.normal((1, n, T, 1, D), seed + 3, dtype="bf16")
+        t0 = time.perf_counter()
+        rows = 0
+        while time.perf_counter() - t0 < budget_s:
+            for mode in ("intra", "cross"):
+                oracle.decode_rows(q, kc, vc, np.array([T]), n, mode, [(0, int(g.integers(n)), int(g.integers(G)))])
+                rows += 1
+        dt = time.perf_counter() - t0
+        # bytes each row's arithmetic reads from the cache: intra T, cross n*T entries of K and V
+        per_row_bytes = 0.5 * (2 * T * D * 2) + 0.5 * (2 * n * T * D * 2)
+        return rows * per_row_bytes / dt / 1e9, "GB/s", f"{rows} decode rows (one KV head, ctx {T}), {dt:.1f} s", threads
+    n, L, D, mode, W = cfg["n"], cfg["L"], cfg["D"], cfg["mode"], cfg["W"]
+    P = n * L
+    q = synth.normal((1, P, 1, D), seed + 1, dtype="bf16")
+    k = synth.normal((1, P, 1, D), seed + 2, dtype="bf16")
+    v = synth.normal((1, P, 1, D), seed + 3, dtype="bf16")
+    pk = np.arange(P)
+    t0 = time.perf_counter()
+    rows, pairs = 0, 0
+    while time.perf_counter() - t0 < budget_s:
+        p = int(g.integers(P))
+        oracle.attn_rows(q, k, v, n, mode, [(0, 0, p)], W, D ** -0.5)
+        pairs += int(np.count_nonzero(oracle.visible(p, pk, n, mode, W)))
+        rows += 1
+    dt = time.perf_counter() - t0
+    return (pairs * 4 * D / dt / 1e12, "TFLOP/s",
+            f"{rows} uniformly sampled output rows of one (batch, head), {dt:.1f} s", threads)
+
+
+def run_reference(args):
+    wl = args.workload
+    K = args.steps if args.steps is not None else 10
+    W = args.warmup if args.warmup is not None else 3
+    budget_total = 90.0
+    per_step = max(0.05, budget_total / max(1, K + W))
+    for _ in range(W):
+        oracle_sample_rate(wl, per_step, seed=11)
+    vals = []
+    t0 = time.perf_counter()
+    for i in range(K):
+        v, unit, sample, threads = oracle_sample_rate(wl, per_step, seed=100 + i)
+        vals.append(v)
+    wall = time.perf_counter() - t0
+    value = statistics.mean(vals)
+    metric = ("decode GB/s vs HBM (intra+cross, B=64 n=4 ctx=32768)" if wl == "decode"
+              else "useful attn TFLOP/s at n=4 (%s)" % WORKLOADS[wl]["mode"])
+    return {
+        "impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus, "steps": K,
+        "warmup": W, "ms_per_step": round(1000 * wall / K, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded host draws)",
+        "config": {"workload": NAMES[wl], "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
+                         "sample": f"per step: {sample}"},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        print(json.dumps(run_reference(args)), flush=True)
+        return
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as td
+
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        td.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = td
+    out, work, peaks = run_ours(args, rank, world, dist)
+    import torch
+
+    del work
+    torch.cuda.empty_cache()
+    if rank == 0:
+        if not args.no_extras and args.workload != "decode":
+            out["also"] = extras(torch, peaks, rank)
+        v, unit, sample, threads = oracle_sample_rate(args.workload, 15.0)
+        out["cpu_baseline"] = {"value": v, "unit": unit, "cores": threads, "kind": "oracle", "sample": sample}
+        print(json.dumps(out), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,145 @@
+/*
+ * hd.h — C ABI of the B200 (sm_100a) Hidden Decoding hot path.
+ *
+ * Method source: the WeLM blog page "Hidden Decoding at Scale" (sections
+ * "Multi-Stream Expansion and Training Objective", "Stream-Factorized
+ * Attention" with Figure 2, "Persistent KV and the KV-mirror Saving",
+ * "Inference Throughput").
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Indexing is 0-based: token i in [0, L), stream s in [0, n), physical
+ *    position p = i*n + s of the expanded sequence (the page's t = (i-1)n + k).
+ *    The final stream is s = n-1.
+ *  - All tensors are dense, row-major (last index fastest), on the current
+ *    CUDA device, owned by the caller.  Base pointers must be 16-byte aligned.
+ *  - The library allocates no device memory (the decode workspace is passed
+ *    in) and never synchronises: every call is enqueued on `stream` (a
+ *    cudaStream_t; NULL = legacy default stream) and returns at once.
+ *  - Host-side argument errors return a status synchronously and launch
+ *    nothing.  Problems found on the device (a token id out of range, a
+ *    pipeline wait that ran out of time) are written to `*dev_status` (a
+ *    device int32, nullable, first error wins, never reset by the library);
+ *    no kernel traps.
+ *  - Element types: HD_F32 = float32, HD_BF16 = bfloat16.
+ */
+#ifndef HD_H_
+#define HD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HD_OK = 0,
+  HD_ERR_INVALID_ARG = 1, /* null pointer, bad size, misalignment           */
+  HD_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. head_dim 96)    */
+  HD_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed            */
+  HD_ERR_TIMEOUT = 4,     /* device: a bounded pipeline wait gave up         */
+  HD_ERR_BAD_TOKEN = 5    /* device: token id outside [0, V)                 */
+} hd_status;
+
+typedef enum { HD_F32 = 0, HD_BF16 = 1 } hd_dtype;
+
+typedef enum {
+  HD_INTRA = 0, /* Figure 2(c): causal inside each stream                    */
+  HD_CROSS = 1  /* Figure 2(a)/(b): causal over the interleaved nL order     */
+} hd_mode;
+
+/*
+ * Multi-stream expansion ("Multi-Stream Expansion and Training Objective",
+ * eq. S_t = E_k(x_i)):   out[b, i*n + s, :] = tables[s, ids[b, i], :]
+ *
+ *   tables  [n, V, d]   element type `dt`
+ *   ids     [B, L]      int32, each in [0, V)
+ *   out     [B, n*L, d] element type `dt`
+ * d*sizeof(dt) must be a multiple of 16 bytes.  A row whose id is out of
+ * range is written as zeros and HD_ERR_BAD_TOKEN is recorded in *dev_status.
+ * The copy is bit-exact.
+ */
+hd_status hd_expand_embed(const void* tables, const int32_t* ids, void* out,
+                          int B, int L, int n, int64_t V, int d, hd_dtype dt,
+                          int32_t* dev_status, void* stream);
+
+/*
+ * Stream-Factorized Attention forward ("Stream-Factorized Attention",
+ * Figure 2).  For every batch b, query head h and position p = i*n + s:
+ *   O[b,p,h,:] = sum_{p' in vis(p)} softmax_{p'}(scale * <q[b,p,h], k[b,p',g]>) v[b,p',g]
+ * with g = h / (Hq/Hkv) (GQA, consecutive grouping) and
+ *   HD_INTRA: vis(p) = {(j, s) : j <= i, and i - j < window if window > 0}
+ *   HD_CROSS: vis(p) = {p' : p' <= p,   and p - p' < window if window > 0}
+ * (window counts tokens of the stream in intra mode, physical positions in
+ * cross mode; 0 = no window).
+ *
+ *   q   [B, n*L, Hq,  D]  element type `in_dt`
+ *   k,v [B, n*L, Hkv, D]  element type `in_dt`
+ *   o   [B, n*L, Hq,  D]  element type `out_dt`
+ *   lse [B, Hq, n*L]      float32 natural-log log-sum-exp, nullable
+ * D must be 64 or 128; Hq % Hkv == 0; L >= 1; n >= 1.
+ * in_dt = HD_BF16 runs the tcgen05/TMEM tensor-core kernel (fp32 accumulate);
+ * in_dt = HD_F32 runs the fp32 CUDA-core kernel.
+ */
+hd_status hd_attn_fwd(const void* q, const void* k, const void* v, void* o,
+                      float* lse, int B, int L, int n, int Hq, int Hkv, int D,
+                      hd_mode mode, int window, float scale, hd_dtype in_dt,
+                      hd_dtype out_dt, int32_t* dev_status, void* stream);
+
+/*
+ * Decode against the per-stream KV cache ("Persistent KV and the KV-mirror
+ * Saving": a separate cache per stream; "Inference Throughput": the n streams
+ * of a token are processed together in one pass).  For every b, the new
+ * token is T-1 with T = ctx_len[b] (tokens per stream, new token included;
+ * its K/V are already in the cache).  The stream-s query of that token sees
+ *   HD_INTRA: (j, s)  for j <= T-1            (and T-1-j < window)
+ *   HD_CROSS: (j, s') for j <  T-1, any s',   and (T-1, s') for s' <= s
+ *             (and p - p' < window, physical positions p = j*n + s)
+ * which is exactly the prefill row of position (T-1)*n + s.
+ *
+ *   q        [B, n, Hq, D]            element type `in_dt` (HD_BF16 only)
+ *   k_cache  [B, n, Lmax, Hkv, D]     stream-major, element type `in_dt`
+ *   v_cache  [B, n, Lmax, Hkv, D]
+ *   ctx_len  [B] int32 on the device, 1 <= T <= Lmax
+ *   o        [B, n, Hq, D]            element type `out_dt`
+ *   lse      [B, n, Hq] float32, nullable
+ *   workspace: device scratch of at least hd_attn_decode_workspace(...) bytes,
+ *              256-byte aligned, owned by the caller; its contents need no
+ *              initialisation and are dead after the call completes.
+ * Values of ctx_len outside [1, Lmax] record HD_ERR_INVALID_ARG in
+ * *dev_status and leave the rows of that sequence as zeros.
+ */
+hd_status hd_attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                         const int32_t* ctx_len, void* o, float* lse, int B,
+                         int n, int Lmax, int Hq, int Hkv, int D, hd_mode mode,
+                         int window, float scale, hd_dtype in_dt, hd_dtype out_dt,
+                         void* workspace, size_t ws_bytes, int32_t* dev_status,
+                         void* stream);
+
+/* Workspace bytes hd_attn_decode needs for these sizes on the current device
+ * (0 on invalid sizes). */
+size_t hd_attn_decode_workspace(int B, int n, int Lmax, int Hq, int Hkv, int D,
+                                hd_mode mode);
+
+/*
+ * Final-stream gather ("Multi-Stream Expansion and Training Objective": only
+ * the final stream E_n of each token feeds the shared LM head; Figure 1):
+ *   out[b, i, :] = h[b, i*n + n-1, :]
+ *   h   [B, n*L, d] element type `dt`;  out [B, L, d].
+ * d*sizeof(dt) must be a multiple of 16 bytes.  Bit-exact copy.
+ */
+hd_status hd_final_stream_gather(const void* h, void* out, int B, int L, int n,
+                                 int d, hd_dtype dt, void* stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* hd_status_string(hd_status st);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int hd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HD_H_ */

@@ -1,0 +1,468 @@
+// Stream-Factorized Attention forward, bf16 in / f32 accumulate, on the
+// 5th-generation tensor cores (tcgen05 + tensor memory) of sm_100a.
+//
+// ("Hidden Decoding at Scale", "Stream-Factorized Attention", Figure 2.)
+// Both modes run as "ns independent causal streams of Ls tokens": intra mode
+// is (ns = n, Ls = L), cross mode is (ns = 1, Ls = n*L).  The stream
+// structure lives entirely in the TMA tensor maps: q/k/v [B, ns*Ls, H, D] are
+// described as the 5-D tensor (D, H, ns, Ls, B), so a box of 128 tokens of
+// one stream is 128 rows at stride ns*H*D -- stride-n addressing in
+// hardware, no de-interleave pass, and keys of other streams are never
+// loaded.  A key at token j is visible to the query at token i iff j <= i
+// and (W == 0 or i - j < W); tiles entirely outside that band are never
+// visited and only the diagonal / band-edge tiles are masked.
+//
+// Work unit: 128 query tokens of one (batch, head, stream).  Units are
+// ordered longest-first (query block descending) with the G query heads of
+// one KV head adjacent, so concurrently running CTAs share K/V tiles in L2.
+// The kernel is persistent: one CTA per SM walks units with a static stride.
+//
+// CTA = 6 warps:
+//   warps 0-3  softmax / O-rescale / epilogue; thread r owns query row r
+//              (tensor-memory lane r)
+//   warp 4     TMA producer: Q (2 buffers), K and V (2 stages each)
+//   warp 5     MMA issuer: S = Q K^T (SS), O += P V (P from tensor memory)
+// Tensor memory (512 columns): S0 [0,128) S1 [128,256) P0 [256,320)
+// P1 [320,384) O [384, 384+D).  P is bf16 packed two per column.
+// The softmax keeps a running max m per row and only rescales O when a new
+// tile raises the max by more than 2^8 (the final 1/l normalisation makes
+// the result independent of which max was used).
+#include "hd_common.cuh"
+#include "hd_launch.h"
+
+namespace hd {
+
+namespace tc {
+constexpr int BM = 128;
+constexpr int BN = 128;
+constexpr int kThreads = 192;
+constexpr int KST = 2;
+constexpr int VST = 2;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0;
+constexpr uint32_t kColP = 256;
+constexpr uint32_t kColO = 384;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D>
+struct Layout {
+  static constexpr int KB = D / 64;       // 128-byte column blocks per row
+  static constexpr int BLK = BM * 128;    // bytes of one 128-row x 128-byte block
+  static constexpr int TILE = BLK * KB;   // bytes of a 128-row tile
+  static constexpr int Q_OFF = 0;
+  static constexpr int K_OFF = Q_OFF + 2 * TILE;
+  static constexpr int V_OFF = K_OFF + KST * TILE;
+  static constexpr int BAR_OFF = V_OFF + VST * TILE;
+  // barrier indices
+  static constexpr int B_QFULL = 0, B_QEMPTY = 2, B_KFULL = 4, B_KEMPTY = 4 + KST,
+                       B_VFULL = 4 + 2 * KST, B_VEMPTY = 4 + 2 * KST + VST,
+                       B_SFULL = 4 + 2 * KST + 2 * VST, B_PFULL = B_SFULL + 2,
+                       B_ODONE = B_PFULL + 2, B_OEMPTY = B_ODONE + 1, B_DRAIN = B_OEMPTY + 1,
+                       NBAR = B_DRAIN + 1;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int BYTES = MISC_OFF + 16;
+  static constexpr int ALLOC = BYTES + 1024;
+};
+}  // namespace tc
+
+struct TcParams {
+  void* o;
+  float* lse;
+  int32_t* status;
+  int B, Ls, ns, Hq, Hkv, W;
+  float scale_log2;
+  int out_bf16;
+  int nqb;
+  int total_units;
+};
+
+struct TcUnit {
+  int b, h, kvh, s, qblk, t_lo, t_hi;
+};
+
+__device__ __forceinline__ TcUnit tc_unit(int u, const TcParams& p) {
+  const int G = p.Hq / p.Hkv;
+  const int per = p.B * p.ns * p.Hq;
+  const int qi = u / per;
+  int rem = u - qi * per;
+  TcUnit x;
+  x.qblk = p.nqb - 1 - qi;
+  const int g = rem % G;
+  rem /= G;
+  x.kvh = rem % p.Hkv;
+  rem /= p.Hkv;
+  x.s = rem % p.ns;
+  x.b = rem / p.ns;
+  x.h = x.kvh * G + g;
+  const int q0 = x.qblk * tc::BM;
+  x.t_hi = x.qblk;  // BM == BN: the diagonal tile is the last one
+  x.t_lo = p.W > 0 ? max(0, q0 - p.W + 1) / tc::BN : 0;
+  return x;
+}
+
+template <int D>
+__global__ void __launch_bounds__(tc::kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const TcParams p) {
+  using Lay = tc::Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto bar = [&](int i) -> uint32_t { return sbase + Lay::BAR_OFF + 8 * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::MISC_OFF + 4);
+  volatile int* no_abort = reinterpret_cast<volatile int*>(smem + Lay::MISC_OFF + 8);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(Lay::B_QFULL + i), 1);
+      mbar_init(bar(Lay::B_QEMPTY + i), 1);
+      mbar_init(bar(Lay::B_SFULL + i), 1);
+      mbar_init(bar(Lay::B_PFULL + i), 128);
+    }
+    for (int i = 0; i < tc::KST; ++i) {
+      mbar_init(bar(Lay::B_KFULL + i), 1);
+      mbar_init(bar(Lay::B_KEMPTY + i), 1);
+    }
+    for (int i = 0; i < tc::VST; ++i) {
+      mbar_init(bar(Lay::B_VFULL + i), 1);
+      mbar_init(bar(Lay::B_VEMPTY + i), 1);
+    }
+    mbar_init(bar(Lay::B_ODONE), 1);
+    mbar_init(bar(Lay::B_OEMPTY), 128);
+    mbar_init(bar(Lay::B_DRAIN), 1);
+    *abort_flag = 0;
+    *no_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), tc::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto fail = [&]() {
+    *abort_flag = 1;
+    report(p.status, HD_ERR_TIMEOUT);
+  };
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int t = 0, ul = 0;
+      int q_issued[2] = {0, 0}, k_issued[tc::KST] = {}, v_issued[tc::VST] = {};
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++ul) {
+        const TcUnit x = tc_unit(u, p);
+        const int qb = ul & 1;
+        if (!mbar_wait(bar(Lay::B_QEMPTY + qb), ((ul >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+        mbar_arrive_expect_tx(bar(Lay::B_QFULL + qb), Lay::TILE);
+#pragma unroll
+        for (int kb = 0; kb < Lay::KB; ++kb)
+          tma_load_5d(sbase + Lay::Q_OFF + qb * Lay::TILE + kb * Lay::BLK, &tmQ,
+                      bar(Lay::B_QFULL + qb), kb * 64, x.h, x.s, x.qblk * tc::BM, x.b);
+        ++q_issued[qb];
+        for (int kt = x.t_lo; kt <= x.t_hi; ++kt, ++t) {
+          const int ks = t % tc::KST;
+          if (!mbar_wait(bar(Lay::B_KEMPTY + ks), ((t / tc::KST) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(bar(Lay::B_KFULL + ks), Lay::TILE);
+#pragma unroll
+          for (int kb = 0; kb < Lay::KB; ++kb)
+            tma_load_5d(sbase + Lay::K_OFF + ks * Lay::TILE + kb * Lay::BLK, &tmK,
+                        bar(Lay::B_KFULL + ks), kb * 64, x.kvh, x.s, kt * tc::BN, x.b);
+          ++k_issued[ks];
+          const int vs = t % tc::VST;
+          if (!mbar_wait(bar(Lay::B_VEMPTY + vs), ((t / tc::VST) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(bar(Lay::B_VFULL + vs), Lay::TILE);
+#pragma unroll
+          for (int kb = 0; kb < Lay::KB; ++kb)
+            tma_load_5d(sbase + Lay::V_OFF + vs * Lay::TILE + kb * Lay::BLK, &tmV,
+                        bar(Lay::B_VFULL + vs), kb * 64, x.kvh, x.s, kt * tc::BN, x.b);
+          ++v_issued[vs];
+        }
+      }
+      if (!ok) {
+        fail();
+        // Let every copy already issued land before the CTA can exit.
+        for (int i = 0; i < 2; ++i)
+          if (q_issued[i]) mbar_wait(bar(Lay::B_QFULL + i), (q_issued[i] - 1) & 1, no_abort);
+        for (int i = 0; i < tc::KST; ++i)
+          if (k_issued[i]) mbar_wait(bar(Lay::B_KFULL + i), (k_issued[i] - 1) & 1, no_abort);
+        for (int i = 0; i < tc::VST; ++i)
+          if (v_issued[i]) mbar_wait(bar(Lay::B_VFULL + i), (v_issued[i] - 1) & 1, no_abort);
+      }
+    }
+  } else if (warp == 5) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(tc::BM, tc::BN, false, false);
+      constexpr uint32_t idO = idesc_bf16_f32(tc::BM, D, false, true);
+      int t = 0, ul = 0;
+      bool ok = true;
+      auto issue_pv = [&](int tp, bool first, int ulc) -> bool {
+        if (!mbar_wait(bar(Lay::B_PFULL + (tp & 1)), (tp >> 1) & 1, abort_flag)) return false;
+        const int vs = tp % tc::VST;
+        if (!mbar_wait(bar(Lay::B_VFULL + vs), (tp / tc::VST) & 1, abort_flag)) return false;
+        if (first && ulc > 0)
+          if (!mbar_wait(bar(Lay::B_OEMPTY), (ulc - 1) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t pA = tmem + tc::kColP + (tp & 1) * 64;
+        const uint32_t vbase = sbase + Lay::V_OFF + vs * Lay::TILE;
+#pragma unroll
+        for (int kk = 0; kk < tc::BN / 16; ++kk) {
+          // V tile is MN-major (D contiguous): 16 keys = 16 rows of 128 B.
+          const uint64_t bdesc = smem_desc_sw128(vbase + kk * 2048, Lay::BLK, 1024);
+          mma_ts(tmem + tc::kColO, pA + kk * 8, bdesc, idO, (first && kk == 0) ? 0u : 1u);
+        }
+        tc_commit(bar(Lay::B_ODONE));
+        tc_commit(bar(Lay::B_VEMPTY + vs));
+        return true;
+      };
+      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++ul) {
+        const TcUnit x = tc_unit(u, p);
+        const int qb = ul & 1;
+        if (!mbar_wait(bar(Lay::B_QFULL + qb), (ul >> 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t qbase = sbase + Lay::Q_OFF + qb * Lay::TILE;
+        const int nt = x.t_hi - x.t_lo + 1;
+        for (int jj = 0; jj < nt; ++jj, ++t) {
+          const int ks = t % tc::KST;
+          if (!mbar_wait(bar(Lay::B_KFULL + ks), (t / tc::KST) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t kbase = sbase + Lay::K_OFF + ks * Lay::TILE;
+          const uint32_t dS = tmem + tc::kColS + (t & 1) * 128;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * Lay::BLK + (kk & 3) * 32;
+            mma_ss(dS, smem_desc_sw128(qbase + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
+                   idS, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(bar(Lay::B_SFULL + (t & 1)));
+          tc_commit(bar(Lay::B_KEMPTY + ks));
+          if (jj == nt - 1) tc_commit(bar(Lay::B_QEMPTY + qb));
+          if (jj > 0 && !issue_pv(t - 1, jj == 1, ul)) { ok = false; break; }
+        }
+        if (!ok) break;
+        if (!issue_pv(t - 1, nt == 1, ul)) { ok = false; break; }
+      }
+      if (!ok) fail();
+      // Drain: every MMA issued above has completed before TMEM is freed.
+      tc_commit(bar(Lay::B_DRAIN));
+      mbar_wait(bar(Lay::B_DRAIN), 0, no_abort);
+    }
+  } else {
+    // ------------------------------------------------- softmax + epilogue
+    const int r = threadIdx.x;  // 0..127, tensor-memory lane
+    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    const float sl2 = p.scale_log2;
+    const int P = p.Ls * p.ns;
+    int t = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
+      const TcUnit x = tc_unit(u, p);
+      const int q0 = x.qblk * tc::BM;
+      const int i = q0 + r;
+      float m = -INFINITY, l = 0.f;
+      const int nt = x.t_hi - x.t_lo + 1;
+      for (int jj = 0; jj < nt; ++jj, ++t) {
+        const int k0 = (x.t_lo + jj) * tc::BN;
+        const bool got = mbar_wait(bar(Lay::B_SFULL + (t & 1)), (t >> 1) & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t sv[128];
+        const uint32_t sS = tmem + lane_addr + tc::kColS + (t & 1) * 128;
+        tmem_ld32(sS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(sS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_ld32(sS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
+        tmem_ld32(sS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+        tmem_wait_ld();
+        const bool need_mask = (x.t_lo + jj >= x.qblk) || (p.W > 0 && k0 < q0 + tc::BM - p.W);
+        float mt = -INFINITY;
+        if (need_mask) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c) {
+            const int j = k0 + c;
+            float y = __uint_as_float(sv[c]) * sl2;
+            if (j > i || (p.W > 0 && i - j >= p.W)) y = -INFINITY;
+            sv[c] = __float_as_uint(y);
+            mt = fmaxf(mt, y);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 128; ++c) {
+            const float y = __uint_as_float(sv[c]) * sl2;
+            sv[c] = __float_as_uint(y);
+            mt = fmaxf(mt, y);
+          }
+        }
+        bool resc = false;
+        float alpha = 1.f;
+        if (jj == 0) {
+          m = mt;
+        } else if (mt > m + tc::kRescaleThreshold) {
+          alpha = ex2(m - mt);
+          l *= alpha;
+          m = mt;
+          resc = true;
+        }
+        const float mu = (m == -INFINITY) ? 0.f : m;
+        uint32_t pk[64];
+        float ls = 0.f;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float p0 = ex2(__uint_as_float(sv[2 * c]) - mu);
+          const float p1 = ex2(__uint_as_float(sv[2 * c + 1]) - mu);
+          ls += p0 + p1;
+          pk[c] = pack_bf16x2(p0, p1);
+        }
+        l += ls;
+        const uint32_t sP = tmem + lane_addr + tc::kColP + (t & 1) * 64;
+        tmem_st32(sP, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+        tmem_st32(sP + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+        if (__any_sync(0xffffffffu, resc)) {
+          // O must hold P_{t-1} V_{t-1} before it is rescaled.
+          if (!mbar_wait(bar(Lay::B_ODONE), (t - 1) & 1, abort_flag)) ok = false;
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            const uint32_t oA = tmem + lane_addr + tc::kColO + c * 32;
+            tmem_ld32(oA, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            tmem_st32(oA, ov);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(Lay::B_PFULL + (t & 1)));
+      }
+      if (!ok) break;
+      // Epilogue: O / l -> global.
+      if (!mbar_wait(bar(Lay::B_ODONE), (t - 1) & 1, abort_flag)) ok = false;
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const float inv = 1.f / l;
+      const bool row_ok = i < p.Ls;
+      const int64_t orow =
+          (static_cast<int64_t>(x.b) * P + static_cast<int64_t>(i) * p.ns + x.s) * p.Hq + x.h;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ov[32];
+        tmem_ld32(tmem + lane_addr + tc::kColO + c * 32, ov);
+        tmem_wait_ld();
+        if (row_ok) {
+          if (p.out_bf16) {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + orow * D + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(ov[8 * e + 0]) * inv, __uint_as_float(ov[8 * e + 1]) * inv);
+              w.y = pack_bf16x2(__uint_as_float(ov[8 * e + 2]) * inv, __uint_as_float(ov[8 * e + 3]) * inv);
+              w.z = pack_bf16x2(__uint_as_float(ov[8 * e + 4]) * inv, __uint_as_float(ov[8 * e + 5]) * inv);
+              w.w = pack_bf16x2(__uint_as_float(ov[8 * e + 6]) * inv, __uint_as_float(ov[8 * e + 7]) * inv);
+              dst[e] = w;
+            }
+          } else {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow * D + c * 32);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(__uint_as_float(ov[4 * e + 0]) * inv, __uint_as_float(ov[4 * e + 1]) * inv,
+                                   __uint_as_float(ov[4 * e + 2]) * inv, __uint_as_float(ov[4 * e + 3]) * inv);
+          }
+        }
+      }
+      if (row_ok && p.lse)
+        p.lse[(static_cast<int64_t>(x.b) * p.Hq + x.h) * P + static_cast<int64_t>(i) * p.ns + x.s] =
+            (m + log2f(l)) * 0.69314718055994531f;
+      tc_fence_before();
+      mbar_arrive(bar(Lay::B_OEMPTY));
+    }
+    if (!ok) fail();
+  }
+
+  __syncthreads();
+  if (warp == 5) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, tc::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------- host
+
+
+// (D, H, ns, Ls, B) view of a [B, ns*Ls, H, D] bf16 tensor; box = 64 x 1 x 1 x 128 x 1.
+static bool encode_stream_view(CUtensorMap* m, const void* ptr, int B, int Ls, int ns, int H, int D) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) return false;
+  const cuuint64_t dims[5] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)ns, (cuuint64_t)Ls, (cuuint64_t)B};
+  const cuuint64_t e = 2;
+  const cuuint64_t strides[4] = {(cuuint64_t)D * e, (cuuint64_t)H * D * e, (cuuint64_t)ns * H * D * e,
+                                 (cuuint64_t)Ls * ns * H * D * e};
+  const cuuint32_t box[5] = {64, 1, 1, (cuuint32_t)tc::BM, 1};
+  const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int attn_tc_smem_bytes(int D) { return D == 64 ? tc::Layout<64>::ALLOC : tc::Layout<128>::ALLOC; }
+
+cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                           int Ls, int ns, int Hq, int Hkv, int D, int W, float scale, bool out_bf16,
+                           int32_t* status, int sms, cudaStream_t st) {
+  CUtensorMap mq, mk, mv;
+  if (!encode_stream_view(&mq, q, B, Ls, ns, Hq, D) || !encode_stream_view(&mk, k, B, Ls, ns, Hkv, D) ||
+      !encode_stream_view(&mv, v, B, Ls, ns, Hkv, D))
+    return cudaErrorInvalidValue;
+  TcParams p;
+  p.o = o;
+  p.lse = lse;
+  p.status = status;
+  p.B = B;
+  p.Ls = Ls;
+  p.ns = ns;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.W = W;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.out_bf16 = out_bf16 ? 1 : 0;
+  p.nqb = (Ls + tc::BM - 1) / tc::BM;
+  const int64_t units = static_cast<int64_t>(p.nqb) * B * ns * Hq;
+  if (units <= 0) return cudaSuccess;
+  if (units > 0x7fffffff) return cudaErrorInvalidValue;
+  p.total_units = static_cast<int>(units);
+  const int grid = static_cast<int>(units < sms ? units : sms);
+  const int smem = attn_tc_smem_bytes(D);
+  cudaError_t err;
+  if (D == 64) {
+    err = cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    attn_tc_kernel<64><<<grid, tc::kThreads, smem, st>>>(mq, mk, mv, p);
+  } else {
+    err = cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    attn_tc_kernel<128><<<grid, tc::kThreads, smem, st>>>(mq, mk, mv, p);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace hd

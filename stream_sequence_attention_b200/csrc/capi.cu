@@ -1,0 +1,160 @@
+// C ABI of the library (include/hd.h): argument checks, the mode -> stream
+// view mapping, and dispatch to the kernels.  Nothing here allocates device
+// memory or synchronises.
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "hd_common.cuh"
+#include "hd_launch.h"
+
+namespace hd {
+
+// The driver's tensor-map encoder, fetched through the runtime so the
+// library does not link libcuda directly.
+EncodeTiledFn get_encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// SM count of the current device, cached per device.
+int sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;
+  if (dev < 64 && cache[dev] > 0) return cache[dev];
+  int v = 0;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev < 64) cache[dev] = v;
+  return v;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int esize(hd_dtype dt) { return dt == HD_BF16 ? 2 : 4; }
+
+static bool valid_dtype(hd_dtype dt) { return dt == HD_F32 || dt == HD_BF16; }
+
+static hd_status cuda_status(cudaError_t e) { return e == cudaSuccess ? HD_OK : HD_ERR_CUDA; }
+
+}  // namespace hd
+
+using namespace hd;
+
+extern "C" {
+
+hd_status hd_expand_embed(const void* tables, const int32_t* ids, void* out, int B, int L, int n, int64_t V,
+                          int d, hd_dtype dt, int32_t* dev_status, void* stream) {
+  if (B < 0 || L < 0 || n < 1 || V < 1 || d < 1 || !valid_dtype(dt)) return HD_ERR_INVALID_ARG;
+  const int64_t row_bytes = static_cast<int64_t>(d) * esize(dt);
+  if (row_bytes % 16 || row_bytes > (1 << 30)) return HD_ERR_INVALID_ARG;
+  const int64_t rows = static_cast<int64_t>(B) * L * n;
+  if (rows == 0) return HD_OK;
+  if (!tables || !ids || !out || !aligned16(tables) || !aligned16(out) || !aligned16(ids))
+    return HD_ERR_INVALID_ARG;
+  const int sms = sm_count();
+  if (sms <= 0) return HD_ERR_CUDA;
+  return cuda_status(launch_expand(tables, ids, out, rows, n, V, static_cast<int>(row_bytes), sms, dev_status,
+                                   static_cast<cudaStream_t>(stream)));
+}
+
+hd_status hd_final_stream_gather(const void* h, void* out, int B, int L, int n, int d, hd_dtype dt,
+                                 void* stream) {
+  if (B < 0 || L < 0 || n < 1 || d < 1 || !valid_dtype(dt)) return HD_ERR_INVALID_ARG;
+  const int64_t row_bytes = static_cast<int64_t>(d) * esize(dt);
+  if (row_bytes % 16 || row_bytes > (1 << 30)) return HD_ERR_INVALID_ARG;
+  const int64_t rows = static_cast<int64_t>(B) * L;
+  if (rows == 0) return HD_OK;
+  if (!h || !out || !aligned16(h) || !aligned16(out)) return HD_ERR_INVALID_ARG;
+  const int sms = sm_count();
+  if (sms <= 0) return HD_ERR_CUDA;
+  return cuda_status(
+      launch_gather(h, out, rows, n, static_cast<int>(row_bytes), sms, static_cast<cudaStream_t>(stream)));
+}
+
+hd_status hd_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int L, int n,
+                      int Hq, int Hkv, int D, hd_mode mode, int window, float scale, hd_dtype in_dt,
+                      hd_dtype out_dt, int32_t* dev_status, void* stream) {
+  if (B < 0 || L < 1 || n < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || window < 0) return HD_ERR_INVALID_ARG;
+  if (mode != HD_INTRA && mode != HD_CROSS) return HD_ERR_INVALID_ARG;
+  if (!valid_dtype(in_dt) || !valid_dtype(out_dt) || !std::isfinite(scale)) return HD_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return HD_ERR_UNSUPPORTED;
+  const int64_t P = static_cast<int64_t>(n) * L;
+  if (P > (1ll << 30) || static_cast<int64_t>(B) * P * Hq > (1ll << 40)) return HD_ERR_INVALID_ARG;
+  if (B == 0) return HD_OK;
+  if (!q || !k || !v || !o || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return HD_ERR_INVALID_ARG;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return HD_ERR_INVALID_ARG;
+  // Intra: n streams of L tokens.  Cross: one stream of n*L positions.
+  const int ns = mode == HD_INTRA ? n : 1;
+  const int Ls = mode == HD_INTRA ? L : static_cast<int>(P);
+  const bool out_bf16 = out_dt == HD_BF16;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (in_dt == HD_F32) {
+    if (Hq * ns > 65535 || B > 65535) return HD_ERR_UNSUPPORTED;
+    return cuda_status(launch_attn_f32(static_cast<const float*>(q), static_cast<const float*>(k),
+                                       static_cast<const float*>(v), o, lse, B, Ls, ns, Hq, Hkv, D, window,
+                                       scale, out_bf16, st));
+  }
+  const int sms = sm_count();
+  if (sms <= 0) return HD_ERR_CUDA;
+  return cuda_status(launch_attn_tc(q, k, v, o, lse, B, Ls, ns, Hq, Hkv, D, window, scale, out_bf16,
+                                    dev_status, sms, st));
+}
+
+size_t hd_attn_decode_workspace(int B, int n, int Lmax, int Hq, int Hkv, int D, hd_mode mode) {
+  if (B < 1 || n < 1 || Lmax < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || D != 128) return 0;
+  if (mode != HD_INTRA && mode != HD_CROSS) return 0;
+  const int sms = sm_count();
+  if (sms <= 0) return 0;
+  return decode_workspace_bytes(decode_plan(B, n, Lmax, Hq, Hkv, mode == HD_CROSS, sms));
+}
+
+hd_status hd_attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* ctx_len,
+                         void* o, float* lse, int B, int n, int Lmax, int Hq, int Hkv, int D, hd_mode mode,
+                         int window, float scale, hd_dtype in_dt, hd_dtype out_dt, void* workspace,
+                         size_t ws_bytes, int32_t* dev_status, void* stream) {
+  if (B < 0 || n < 1 || Lmax < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || window < 0) return HD_ERR_INVALID_ARG;
+  if (mode != HD_INTRA && mode != HD_CROSS) return HD_ERR_INVALID_ARG;
+  if (!valid_dtype(in_dt) || !valid_dtype(out_dt) || !std::isfinite(scale)) return HD_ERR_INVALID_ARG;
+  if (D != 128 || in_dt != HD_BF16) return HD_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(n) * Lmax > (1ll << 30)) return HD_ERR_INVALID_ARG;
+  if (B == 0) return HD_OK;
+  if (!q || !k_cache || !v_cache || !ctx_len || !o || !workspace) return HD_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) || (reinterpret_cast<uintptr_t>(ctx_len) & 3u))
+    return HD_ERR_INVALID_ARG;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return HD_ERR_INVALID_ARG;
+  const int sms = sm_count();
+  if (sms <= 0) return HD_ERR_CUDA;
+  const DecPlan pl = decode_plan(B, n, Lmax, Hq, Hkv, mode == HD_CROSS, sms);
+  if (pl.units > 65535) return HD_ERR_UNSUPPORTED;
+  if (ws_bytes < decode_workspace_bytes(pl)) return HD_ERR_INVALID_ARG;
+  return cuda_status(launch_decode(q, k_cache, v_cache, ctx_len, o, lse, B, n, Lmax, Hq, Hkv, window, scale,
+                                   mode == HD_CROSS, out_dt == HD_BF16, workspace, dev_status, sms,
+                                   static_cast<cudaStream_t>(stream)));
+}
+
+const char* hd_status_string(hd_status st) {
+  switch (st) {
+    case HD_OK: return "HD_OK";
+    case HD_ERR_INVALID_ARG: return "HD_ERR_INVALID_ARG";
+    case HD_ERR_UNSUPPORTED: return "HD_ERR_UNSUPPORTED";
+    case HD_ERR_CUDA: return "HD_ERR_CUDA";
+    case HD_ERR_TIMEOUT: return "HD_ERR_TIMEOUT";
+    case HD_ERR_BAD_TOKEN: return "HD_ERR_BAD_TOKEN";
+  }
+  return "HD_ERR_UNKNOWN";
+}
+
+int hd_version(void) { return 100; }
+
+}  // extern "C"

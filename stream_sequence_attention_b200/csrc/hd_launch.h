@@ -1,0 +1,42 @@
+// Host-side launchers shared between the C-ABI shim and the kernel files.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace hd {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// The driver's tensor-map encoder (fetched once through the runtime).
+EncodeTiledFn get_encode_tiled();
+
+cudaError_t launch_expand(const void* tables, const int32_t* ids, void* out, int64_t rows, int n,
+                          int64_t V, int row_bytes, int sms, int32_t* status, cudaStream_t st);
+cudaError_t launch_gather(const void* h, void* out, int64_t rows, int n, int row_bytes, int sms,
+                          cudaStream_t st);
+cudaError_t launch_attn_f32(const float* q, const float* k, const float* v, void* o, float* lse, int B,
+                            int Ls, int ns, int Hq, int Hkv, int D, int W, float scale, bool out_bf16,
+                            cudaStream_t st);
+cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Ls,
+                           int ns, int Hq, int Hkv, int D, int W, float scale, bool out_bf16,
+                           int32_t* status, int sms, cudaStream_t st);
+
+// Decode work decomposition: units (one KV head of one sequence, and for
+// intra mode one stream), row groups of at most 32 query rows, token splits.
+struct DecPlan {
+  int units, rg_count, nsplit, mt;
+  int64_t rows_total;
+};
+DecPlan decode_plan(int B, int n, int Lmax, int Hq, int Hkv, bool cross, int sms);
+size_t decode_workspace_bytes(const DecPlan& pl);
+cudaError_t launch_decode(const void* q, const void* kc, const void* vc, const int32_t* ctx, void* o,
+                          float* lse, int B, int n, int Lmax, int Hq, int Hkv, int W, float scale,
+                          bool cross, bool out_bf16, void* ws, int32_t* status, int sms, cudaStream_t st);
+
+}  // namespace hd

@@ -1,0 +1,230 @@
+"""Python binding of the C ABI in ``include/hd.h`` (ctypes, marshalling only).
+
+Each function takes torch tensors that already live on the current CUDA
+device, checks dtype / shape / contiguity, and passes raw pointers, sizes and
+the current CUDA stream to the library.  Every step of the computation runs in
+the library's kernels; there is no fallback: if ``libhd.so`` is missing or a
+call fails, an exception is raised.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhd.so")
+
+HD_OK, HD_ERR_INVALID_ARG, HD_ERR_UNSUPPORTED, HD_ERR_CUDA, HD_ERR_TIMEOUT, HD_ERR_BAD_TOKEN = range(6)
+HD_F32, HD_BF16 = 0, 1
+HD_INTRA, HD_CROSS = 0, 1
+
+_MODES = {"intra": HD_INTRA, "cross": HD_CROSS, HD_INTRA: HD_INTRA, HD_CROSS: HD_CROSS}
+
+EXPORTS = (
+    "hd_expand_embed",
+    "hd_attn_fwd",
+    "hd_attn_decode",
+    "hd_attn_decode_workspace",
+    "hd_final_stream_gather",
+    "hd_status_string",
+    "hd_version",
+)
+
+
+class HDError(RuntimeError):
+    def __init__(self, fn, code):
+        self.code = code
+        super().__init__(f"{fn} failed: {status_string(code)} ({code})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libhd.so (built in-tree by ``stream_sequence_attention_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m stream_sequence_attention_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+        L.hd_expand_embed.argtypes = [vp, vp, vp, i32, i32, i32, i64, i32, i32, vp, vp]
+        L.hd_expand_embed.restype = i32
+        L.hd_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, f32, i32, i32, vp, vp]
+        L.hd_attn_fwd.restype = i32
+        L.hd_attn_decode.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, f32, i32, i32,
+                                     vp, sz, vp, vp]
+        L.hd_attn_decode.restype = i32
+        L.hd_attn_decode_workspace.argtypes = [i32, i32, i32, i32, i32, i32, i32]
+        L.hd_attn_decode_workspace.restype = sz
+        L.hd_final_stream_gather.argtypes = [vp, vp, i32, i32, i32, i32, i32, vp]
+        L.hd_final_stream_gather.restype = i32
+        L.hd_status_string.argtypes = [i32]
+        L.hd_status_string.restype = ctypes.c_char_p
+        L.hd_version.argtypes = []
+        L.hd_version.restype = i32
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().hd_status_string(int(code)).decode()
+
+
+def version() -> int:
+    return lib().hd_version()
+
+
+def _check(fn, code):
+    if code != HD_OK:
+        raise HDError(fn, code)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return HD_BF16
+    if t.dtype == torch.float32:
+        return HD_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def new_status(device=None) -> torch.Tensor:
+    """A zeroed device status word for the ``dev_status`` arguments."""
+    return torch.zeros(1, dtype=torch.int32, device=device or "cuda")
+
+
+def hd_expand_embed(tables: torch.Tensor, ids: torch.Tensor, out: torch.Tensor | None = None,
+                    dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """tables [n, V, d], ids [B, L] int32 -> out [B, n*L, d]."""
+    _need(tables, "tables")
+    _need(ids, "ids")
+    n, V, d = tables.shape
+    B, L = ids.shape
+    if ids.dtype != torch.int32:
+        raise TypeError("ids must be int32")
+    if out is None:
+        out = torch.empty((B, n * L, d), dtype=tables.dtype, device=tables.device)
+    _need(out, "out")
+    if out.shape != (B, n * L, d) or out.dtype != tables.dtype:
+        raise ValueError("out has the wrong shape or dtype")
+    _check("hd_expand_embed", lib().hd_expand_embed(
+        _ptr(tables), _ptr(ids), _ptr(out), B, L, n, V, d, _dt(tables), _ptr(dev_status), _stream(stream)))
+    return out
+
+
+def hd_final_stream_gather(h: torch.Tensor, n: int, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """h [B, n*L, d] -> out [B, L, d] (rows of the final stream)."""
+    _need(h, "h")
+    B, P, d = h.shape
+    if P % n:
+        raise ValueError("sequence length is not a multiple of n")
+    L = P // n
+    if out is None:
+        out = torch.empty((B, L, d), dtype=h.dtype, device=h.device)
+    _need(out, "out")
+    if out.shape != (B, L, d) or out.dtype != h.dtype:
+        raise ValueError("out has the wrong shape or dtype")
+    _check("hd_final_stream_gather", lib().hd_final_stream_gather(
+        _ptr(h), _ptr(out), B, L, n, d, _dt(h), _stream(stream)))
+    return out
+
+
+def hd_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n: int, mode="intra", window: int = 0,
+                scale: float | None = None, out: torch.Tensor | None = None, out_dtype=None,
+                lse: torch.Tensor | bool | None = None, dev_status: torch.Tensor | None = None, stream=None):
+    """Stream-Factorized Attention forward.
+
+    q [B, n*L, Hq, D], k/v [B, n*L, Hkv, D] -> O [B, n*L, Hq, D] (and lse
+    [B, Hq, n*L] float32 when ``lse`` is True or a tensor).
+    """
+    for t, nm in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, nm)
+    B, P, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if k.shape != (B, P, Hkv, D) or v.shape != k.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q/k/v shapes or dtypes disagree")
+    if P % n:
+        raise ValueError("sequence length is not a multiple of n")
+    L = P // n
+    if scale is None:
+        scale = D ** -0.5
+    odt = out_dtype or q.dtype
+    if out is None:
+        out = torch.empty((B, P, Hq, D), dtype=odt, device=q.device)
+    _need(out, "out")
+    if out.shape != q.shape:
+        raise ValueError("out has the wrong shape")
+    want_lse = lse is True or isinstance(lse, torch.Tensor)
+    if lse is True:
+        lse = torch.empty((B, Hq, P), dtype=torch.float32, device=q.device)
+    elif lse is False:
+        lse = None
+    if isinstance(lse, torch.Tensor):
+        _need(lse, "lse")
+    _check("hd_attn_fwd", lib().hd_attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, L, n, Hq, Hkv, D, _MODES[mode], int(window),
+        float(scale), _dt(q), _dt(out), _ptr(dev_status), _stream(stream)))
+    return (out, lse) if want_lse else out
+
+
+def hd_attn_decode_workspace(B: int, n: int, Lmax: int, Hq: int, Hkv: int, D: int, mode="intra") -> int:
+    return int(lib().hd_attn_decode_workspace(B, n, Lmax, Hq, Hkv, D, _MODES[mode]))
+
+
+def hd_attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, ctx_len: torch.Tensor,
+                   mode="intra", window: int = 0, scale: float | None = None, out: torch.Tensor | None = None,
+                   out_dtype=None, lse: torch.Tensor | bool | None = None, workspace: torch.Tensor | None = None,
+                   dev_status: torch.Tensor | None = None, stream=None):
+    """q [B, n, Hq, D], caches [B, n, Lmax, Hkv, D], ctx_len [B] int32 ->
+    O [B, n, Hq, D] (and lse [B, n, Hq] when asked)."""
+    for t, nm in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"), (ctx_len, "ctx_len")):
+        _need(t, nm)
+    B, n, Hq, D = q.shape
+    _, _, Lmax, Hkv, _ = k_cache.shape
+    if k_cache.shape != (B, n, Lmax, Hkv, D) or v_cache.shape != k_cache.shape:
+        raise ValueError("cache shapes disagree with q")
+    if ctx_len.dtype != torch.int32 or ctx_len.shape != (B,):
+        raise ValueError("ctx_len must be int32 [B]")
+    if scale is None:
+        scale = D ** -0.5
+    odt = out_dtype or q.dtype
+    if out is None:
+        out = torch.empty((B, n, Hq, D), dtype=odt, device=q.device)
+    _need(out, "out")
+    want_lse = lse is True or isinstance(lse, torch.Tensor)
+    if lse is True:
+        lse = torch.empty((B, n, Hq), dtype=torch.float32, device=q.device)
+    elif lse is False:
+        lse = None
+    ws_bytes = hd_attn_decode_workspace(B, n, Lmax, Hq, Hkv, D, mode)
+    if ws_bytes == 0:
+        raise HDError("hd_attn_decode_workspace", HD_ERR_UNSUPPORTED)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    if workspace.numel() * workspace.element_size() < ws_bytes:
+        raise ValueError("workspace too small")
+    _check("hd_attn_decode", lib().hd_attn_decode(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(ctx_len), _ptr(out), _ptr(lse), B, n, Lmax, Hq, Hkv, D,
+        _MODES[mode], int(window), float(scale), _dt(q), _dt(out), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
+    return (out, lse) if want_lse else out

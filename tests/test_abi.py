@@ -1,0 +1,89 @@
+"""Host-side checks of the C ABI: the library loads without a GPU, exports
+every function ``include/hd.h`` declares, and rejects bad arguments before
+touching the device."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from stream_sequence_attention_b200 import build as hd_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hd.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    hd_build.build()
+    from stream_sequence_attention_b200 import hd
+    return hd.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(hd_[a-z0-9_]+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for want in ("hd_expand_embed", "hd_attn_fwd", "hd_attn_decode", "hd_attn_decode_workspace",
+                 "hd_final_stream_gather", "hd_status_string", "hd_version"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+        assert ctypes.cast(getattr(L, name), ctypes.c_void_p).value
+
+
+def test_binding_names_match_header():
+    from stream_sequence_attention_b200 import hd
+    assert sorted(hd.EXPORTS) == declared_functions()
+
+
+def test_status_strings_and_version(L):
+    from stream_sequence_attention_b200 import hd
+    assert hd.status_string(0) == "HD_OK"
+    assert hd.status_string(4) == "HD_ERR_TIMEOUT"
+    assert hd.status_string(5) == "HD_ERR_BAD_TOKEN"
+    assert hd.status_string(99) == "HD_ERR_UNKNOWN"
+    assert hd.version() >= 100
+
+
+def test_bad_arguments_rejected_on_host(L):
+    from stream_sequence_attention_b200 import hd
+    vp = ctypes.c_void_p
+    fake = vp(0x10000)  # never dereferenced: every call below fails validation first
+    # n = 0
+    assert L.hd_expand_embed(fake, fake, fake, 1, 4, 0, 10, 8, hd.HD_BF16, None, None) == hd.HD_ERR_INVALID_ARG
+    # row bytes not a multiple of 16 (d = 4 bf16)
+    assert L.hd_expand_embed(fake, fake, fake, 1, 4, 2, 10, 4, hd.HD_BF16, None, None) == hd.HD_ERR_INVALID_ARG
+    # Hq % Hkv != 0
+    assert L.hd_attn_fwd(fake, fake, fake, fake, None, 1, 8, 2, 3, 2, 64, 0, 0, 0.1, 1, 1, None, None) \
+        == hd.HD_ERR_INVALID_ARG
+    # unsupported head dim
+    assert L.hd_attn_fwd(fake, fake, fake, fake, None, 1, 8, 2, 2, 2, 96, 0, 0, 0.1, 1, 1, None, None) \
+        == hd.HD_ERR_UNSUPPORTED
+    # L = 0 and bad mode
+    assert L.hd_attn_fwd(fake, fake, fake, fake, None, 1, 0, 2, 2, 2, 64, 0, 0, 0.1, 1, 1, None, None) \
+        == hd.HD_ERR_INVALID_ARG
+    assert L.hd_attn_fwd(fake, fake, fake, fake, None, 1, 8, 2, 2, 2, 64, 7, 0, 0.1, 1, 1, None, None) \
+        == hd.HD_ERR_INVALID_ARG
+    # misaligned q
+    assert L.hd_attn_fwd(vp(0x10008), fake, fake, fake, None, 1, 8, 2, 2, 2, 64, 0, 0, 0.1, 1, 1, None, None) \
+        == hd.HD_ERR_INVALID_ARG
+    # decode: only bf16 / D = 128
+    assert L.hd_attn_decode(fake, fake, fake, fake, fake, None, 1, 2, 8, 2, 2, 64, 0, 0, 0.1, 1, 1,
+                            fake, 1 << 20, None, None) == hd.HD_ERR_UNSUPPORTED
+    assert L.hd_attn_decode(fake, fake, fake, fake, fake, None, 1, 2, 8, 2, 2, 128, 0, 0, 0.1, 0, 1,
+                            fake, 1 << 20, None, None) == hd.HD_ERR_UNSUPPORTED
+    # gather: negative sizes
+    assert L.hd_final_stream_gather(fake, fake, -1, 4, 2, 8, hd.HD_F32, None) == hd.HD_ERR_INVALID_ARG
+    # empty work is a no-op that succeeds without a device
+    assert L.hd_final_stream_gather(None, None, 0, 4, 2, 8, hd.HD_F32, None) == hd.HD_OK
+    assert L.hd_expand_embed(None, None, None, 0, 4, 2, 10, 8, hd.HD_F32, None, None) == hd.HD_OK
