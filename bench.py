@@ -63,6 +63,8 @@ def parse():
     ap.add_argument("--workload", default="intra", choices=list(WORKLOADS))
     ap.add_argument("--no-extras", action="store_true", help="skip the side measurements")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--profile", action="store_true",
+                    help="timed steps only (no e2e, side measurements or CPU oracle): for ncu captures")
     return ap.parse_args()
 
 
@@ -329,6 +331,8 @@ def run_ours(args, rank, world, dist):
     clocks.start()
     steps, kern = timed(torch, work, K, flush, dist)
     clk = clocks.stop()
+    if args.profile:
+        return {"profile": True, "ms_per_step": sum(steps) / K, "kernel_ms": statistics.mean(kern)}, work, peaks
     total_ms = sum(steps)
     total_ms = max_over_ranks(torch, dist, total_ms)
     ms_per_step = total_ms / K
@@ -528,6 +532,10 @@ def main():
 
     del work
     torch.cuda.empty_cache()
+    if args.profile:
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+        return
     if rank == 0:
         if not args.no_extras and args.workload != "decode":
             out["also"] = extras(torch, peaks, rank)

@@ -78,7 +78,7 @@ hd_status hd_expand_embed(const void* tables, const int32_t* ids, void* out,
  *   k,v [B, n*L, Hkv, D]  element type `in_dt`
  *   o   [B, n*L, Hq,  D]  element type `out_dt`
  *   lse [B, Hq, n*L]      float32 natural-log log-sum-exp, nullable
- * D must be 64 or 128; Hq % Hkv == 0; L >= 1; n >= 1.
+ * D must be 64 or 128; Hq % Hkv == 0; L >= 1; n >= 1; scale finite and > 0.
  * in_dt = HD_BF16 runs the tcgen05/TMEM tensor-core kernel (fp32 accumulate);
  * in_dt = HD_F32 runs the fp32 CUDA-core kernel.
  */

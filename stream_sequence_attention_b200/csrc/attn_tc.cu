@@ -12,21 +12,32 @@
 // and (W == 0 or i - j < W); tiles entirely outside that band are never
 // visited and only the diagonal / band-edge tiles are masked.
 //
-// Work unit: 128 query tokens of one (batch, head, stream).  Units are
-// ordered longest-first (query block descending) with the G query heads of
-// one KV head adjacent, so concurrently running CTAs share K/V tiles in L2.
-// The kernel is persistent: one CTA per SM walks units with a static stride.
+// Work unit: 128 query tokens of one (batch, stream) for TWO query heads of
+// the same KV head (GQA), which need exactly the same K/V tiles: every K/V
+// tile brought into shared memory feeds both heads.  Units are ordered
+// longest-first (query block descending); the kernel is persistent, one CTA
+// per SM walking units with a static stride.
 //
-// CTA = 6 warps:
-//   warps 0-3  softmax / O-rescale / epilogue; thread r owns query row r
-//              (tensor-memory lane r)
-//   warp 4     TMA producer: Q (2 buffers), K and V (2 stages each)
-//   warp 5     MMA issuer: S = Q K^T (SS), O += P V (P from tensor memory)
-// Tensor memory (512 columns): S0 [0,128) S1 [128,256) P0 [256,320)
-// P1 [320,384) O [384, 384+D).  P is bf16 packed two per column.
-// The softmax keeps a running max m per row and only rescales O when a new
-// tile raises the max by more than 2^8 (the final 1/l normalisation makes
-// the result independent of which max was used).
+// CTA = 10 warps:
+//   warps 0-3  softmax / O-rescale / epilogue of head slot 0 (thread r owns
+//              query row r = tensor-memory lane r)
+//   warps 4-7  the same for head slot 1
+//   warp 8     TMA producer: Q (both heads), K (3 stages), V (2 stages)
+//   warp 9     MMA issuer
+// Tensor memory (512 columns): S0 [0,128) S1 [128,256) O0 [256,384)
+// O1 [384,512).  P (bf16, two per column) overwrites the first 64 columns of
+// its S buffer.  The MMA warp issues, per tile, PV_0(t) S_0(t+1) PV_1(t)
+// S_1(t+1): S_h(t+1) lands in the columns PV_h(t) reads, which is safe
+// because tcgen05.mma operations issued by one thread execute in order.
+// While one softmax warpgroup works, the tensor core runs the other head's
+// PV and next S -- the two warpgroups ping-pong against the tensor core.
+//
+// Softmax: running max m per row in log2 units; O is rescaled only when a
+// tile raises the max by more than 2^8 (the final 1/l makes the result
+// independent of which max was used).  On tiles with no masked pair, one
+// exponential in four is evaluated on the FMA pipe (round to nearest
+// integer, cubic for 2^f on [-1/2, 1/2], exponent add; relative error
+// < 1e-4, below the bf16 rounding of P) to offload the MUFU unit.
 #include "hd_common.cuh"
 #include "hd_launch.h"
 
@@ -35,30 +46,27 @@ namespace hd {
 namespace tc {
 constexpr int BM = 128;
 constexpr int BN = 128;
-constexpr int kThreads = 192;
-constexpr int KST = 2;
+constexpr int kThreads = 320;
+constexpr int kWarpTMA = 8;
+constexpr int kWarpMMA = 9;
+constexpr int KST = 3;
 constexpr int VST = 2;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;
-constexpr uint32_t kColP = 256;
-constexpr uint32_t kColO = 384;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 template <int D>
 struct Layout {
-  static constexpr int KB = D / 64;       // 128-byte column blocks per row
-  static constexpr int BLK = BM * 128;    // bytes of one 128-row x 128-byte block
-  static constexpr int TILE = BLK * KB;   // bytes of a 128-row tile
-  static constexpr int Q_OFF = 0;
+  static constexpr int KB = D / 64;     // 128-byte column blocks per row
+  static constexpr int BLK = BM * 128;  // bytes of one 128-row x 128-byte block
+  static constexpr int TILE = BLK * KB; // bytes of a 128-row tile
+  static constexpr int Q_OFF = 0;       // head slots 0 and 1
   static constexpr int K_OFF = Q_OFF + 2 * TILE;
   static constexpr int V_OFF = K_OFF + KST * TILE;
   static constexpr int BAR_OFF = V_OFF + VST * TILE;
-  // barrier indices
-  static constexpr int B_QFULL = 0, B_QEMPTY = 2, B_KFULL = 4, B_KEMPTY = 4 + KST,
-                       B_VFULL = 4 + 2 * KST, B_VEMPTY = 4 + 2 * KST + VST,
-                       B_SFULL = 4 + 2 * KST + 2 * VST, B_PFULL = B_SFULL + 2,
-                       B_ODONE = B_PFULL + 2, B_OEMPTY = B_ODONE + 1, B_DRAIN = B_OEMPTY + 1,
-                       NBAR = B_DRAIN + 1;
+  static constexpr int B_QFULL = 0, B_QEMPTY = 1, B_KFULL = 2, B_KEMPTY = B_KFULL + KST,
+                       B_VFULL = B_KEMPTY + KST, B_VEMPTY = B_VFULL + VST, B_SFULL = B_VEMPTY + VST,
+                       B_PFULL = B_SFULL + 2, B_ODONE = B_PFULL + 2, B_OEMPTY = B_ODONE + 2,
+                       B_DRAIN = B_OEMPTY + 2, NBAR = B_DRAIN + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int ALLOC = BYTES + 1024;
@@ -72,32 +80,46 @@ struct TcParams {
   int B, Ls, ns, Hq, Hkv, W;
   float scale_log2;
   int out_bf16;
-  int nqb;
+  int nqb, npairs;
   int total_units;
 };
 
 struct TcUnit {
-  int b, h, kvh, s, qblk, t_lo, t_hi;
+  int b, s, kvh, qblk, h0, h1, t_lo, t_hi;  // h1 < 0: only one head in this unit
 };
 
 __device__ __forceinline__ TcUnit tc_unit(int u, const TcParams& p) {
   const int G = p.Hq / p.Hkv;
-  const int per = p.B * p.ns * p.Hq;
+  const int per = p.B * p.ns * p.Hkv * p.npairs;
   const int qi = u / per;
   int rem = u - qi * per;
   TcUnit x;
   x.qblk = p.nqb - 1 - qi;
-  const int g = rem % G;
-  rem /= G;
+  const int pair = rem % p.npairs;
+  rem /= p.npairs;
   x.kvh = rem % p.Hkv;
   rem /= p.Hkv;
   x.s = rem % p.ns;
   x.b = rem / p.ns;
-  x.h = x.kvh * G + g;
+  x.h0 = x.kvh * G + 2 * pair;
+  x.h1 = (2 * pair + 1 < G) ? x.h0 + 1 : -1;
   const int q0 = x.qblk * tc::BM;
   x.t_hi = x.qblk;  // BM == BN: the diagonal tile is the last one
   x.t_lo = p.W > 0 ? max(0, q0 - p.W + 1) / tc::BN : 0;
   return x;
+}
+
+// 2^x on the FMA pipe for finite x <= 2^22: x = n + f, n = rint(x),
+// f in [-1/2, 1/2]; cubic for 2^f (coefficients from fit_exp2_poly.py);
+// 2^n by adding n to the exponent field.  Inputs below -127 are clamped.
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -127.0f);
+  const float t = x + 12582912.0f;  // 1.5 * 2^23: rint(x) lands in the low mantissa bits
+  const float f = x - (t - 12582912.0f);
+  float p = fmaf(0.0551713444f, f, 0.242610335f);
+  p = fmaf(p, f, 0.693260968f);
+  p = fmaf(p, f, 0.999928117f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 template <int D>
@@ -118,12 +140,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(Lay::B_QFULL + i), 1);
-      mbar_init(bar(Lay::B_QEMPTY + i), 1);
-      mbar_init(bar(Lay::B_SFULL + i), 1);
-      mbar_init(bar(Lay::B_PFULL + i), 128);
-    }
+    mbar_init(bar(Lay::B_QFULL), 1);
+    mbar_init(bar(Lay::B_QEMPTY), 1);
     for (int i = 0; i < tc::KST; ++i) {
       mbar_init(bar(Lay::B_KFULL + i), 1);
       mbar_init(bar(Lay::B_KEMPTY + i), 1);
@@ -132,19 +150,23 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       mbar_init(bar(Lay::B_VFULL + i), 1);
       mbar_init(bar(Lay::B_VEMPTY + i), 1);
     }
-    mbar_init(bar(Lay::B_ODONE), 1);
-    mbar_init(bar(Lay::B_OEMPTY), 128);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(Lay::B_SFULL + i), 1);
+      mbar_init(bar(Lay::B_PFULL + i), 128);
+      mbar_init(bar(Lay::B_ODONE + i), 1);
+      mbar_init(bar(Lay::B_OEMPTY + i), 128);
+    }
     mbar_init(bar(Lay::B_DRAIN), 1);
     *abort_flag = 0;
     *no_abort = 0;
     fence_barrier_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == tc::kWarpTMA && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
   }
-  if (warp == 5) {
+  if (warp == tc::kWarpMMA) {
     tmem_alloc(smem_u32(tmem_slot), tc::kTmemCols);
     tmem_relinquish();
   }
@@ -158,104 +180,132 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     report(p.status, HD_ERR_TIMEOUT);
   };
 
-  if (warp == 4) {
+  if (warp == tc::kWarpTMA) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int t = 0, ul = 0;
-      int q_issued[2] = {0, 0}, k_issued[tc::KST] = {}, v_issued[tc::VST] = {};
+      int t = 0, ul = 0, q_issued = 0;
+      int k_issued[tc::KST] = {}, v_issued[tc::VST] = {};
       bool ok = true;
       for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++ul) {
         const TcUnit x = tc_unit(u, p);
-        const int qb = ul & 1;
-        if (!mbar_wait(bar(Lay::B_QEMPTY + qb), ((ul >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-        mbar_arrive_expect_tx(bar(Lay::B_QFULL + qb), Lay::TILE);
+        if (!mbar_wait(bar(Lay::B_QEMPTY), (ul & 1) ^ 1, abort_flag)) { ok = false; break; }
+        mbar_arrive_expect_tx(bar(Lay::B_QFULL), Lay::TILE * (x.h1 >= 0 ? 2 : 1));
 #pragma unroll
-        for (int kb = 0; kb < Lay::KB; ++kb)
-          tma_load_5d(sbase + Lay::Q_OFF + qb * Lay::TILE + kb * Lay::BLK, &tmQ,
-                      bar(Lay::B_QFULL + qb), kb * 64, x.h, x.s, x.qblk * tc::BM, x.b);
-        ++q_issued[qb];
+        for (int kb = 0; kb < Lay::KB; ++kb) {
+          tma_load_5d(sbase + Lay::Q_OFF + kb * Lay::BLK, &tmQ, bar(Lay::B_QFULL), kb * 64, x.h0, x.s,
+                      x.qblk * tc::BM, x.b);
+          if (x.h1 >= 0)
+            tma_load_5d(sbase + Lay::Q_OFF + Lay::TILE + kb * Lay::BLK, &tmQ, bar(Lay::B_QFULL), kb * 64,
+                        x.h1, x.s, x.qblk * tc::BM, x.b);
+        }
+        ++q_issued;
         for (int kt = x.t_lo; kt <= x.t_hi; ++kt, ++t) {
           const int ks = t % tc::KST;
           if (!mbar_wait(bar(Lay::B_KEMPTY + ks), ((t / tc::KST) & 1) ^ 1, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(bar(Lay::B_KFULL + ks), Lay::TILE);
 #pragma unroll
           for (int kb = 0; kb < Lay::KB; ++kb)
-            tma_load_5d(sbase + Lay::K_OFF + ks * Lay::TILE + kb * Lay::BLK, &tmK,
-                        bar(Lay::B_KFULL + ks), kb * 64, x.kvh, x.s, kt * tc::BN, x.b);
+            tma_load_5d(sbase + Lay::K_OFF + ks * Lay::TILE + kb * Lay::BLK, &tmK, bar(Lay::B_KFULL + ks),
+                        kb * 64, x.kvh, x.s, kt * tc::BN, x.b);
           ++k_issued[ks];
           const int vs = t % tc::VST;
           if (!mbar_wait(bar(Lay::B_VEMPTY + vs), ((t / tc::VST) & 1) ^ 1, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(bar(Lay::B_VFULL + vs), Lay::TILE);
 #pragma unroll
           for (int kb = 0; kb < Lay::KB; ++kb)
-            tma_load_5d(sbase + Lay::V_OFF + vs * Lay::TILE + kb * Lay::BLK, &tmV,
-                        bar(Lay::B_VFULL + vs), kb * 64, x.kvh, x.s, kt * tc::BN, x.b);
+            tma_load_5d(sbase + Lay::V_OFF + vs * Lay::TILE + kb * Lay::BLK, &tmV, bar(Lay::B_VFULL + vs),
+                        kb * 64, x.kvh, x.s, kt * tc::BN, x.b);
           ++v_issued[vs];
         }
       }
       if (!ok) {
         fail();
         // Let every copy already issued land before the CTA can exit.
-        for (int i = 0; i < 2; ++i)
-          if (q_issued[i]) mbar_wait(bar(Lay::B_QFULL + i), (q_issued[i] - 1) & 1, no_abort);
+        if (q_issued) mbar_wait(bar(Lay::B_QFULL), (q_issued - 1) & 1, no_abort);
         for (int i = 0; i < tc::KST; ++i)
           if (k_issued[i]) mbar_wait(bar(Lay::B_KFULL + i), (k_issued[i] - 1) & 1, no_abort);
         for (int i = 0; i < tc::VST; ++i)
           if (v_issued[i]) mbar_wait(bar(Lay::B_VFULL + i), (v_issued[i] - 1) & 1, no_abort);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == tc::kWarpMMA) {
     // ---------------------------------------------------------------- MMA
+    // Issue order per tile t (heads 0, 1):  PV_0(t) S_0(t+1) PV_1(t) S_1(t+1).
+    // S_h(t+1) overwrites the columns P_h(t) occupies; tcgen05.mma from one
+    // thread executes in issue order, so PV_h(t) has read P_h(t) by then.
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(tc::BM, tc::BN, false, false);
       constexpr uint32_t idO = idesc_bf16_f32(tc::BM, D, false, true);
-      int t = 0, ul = 0;
-      bool ok = true;
-      auto issue_pv = [&](int tp, bool first, int ulc) -> bool {
-        if (!mbar_wait(bar(Lay::B_PFULL + (tp & 1)), (tp >> 1) & 1, abort_flag)) return false;
-        const int vs = tp % tc::VST;
-        if (!mbar_wait(bar(Lay::B_VFULL + vs), (tp / tc::VST) & 1, abort_flag)) return false;
-        if (first && ulc > 0)
-          if (!mbar_wait(bar(Lay::B_OEMPTY), (ulc - 1) & 1, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t pA = tmem + tc::kColP + (tp & 1) * 64;
-        const uint32_t vbase = sbase + Lay::V_OFF + vs * Lay::TILE;
+      auto issue_S = [&](int h, int kst) {
+        const uint32_t qbase = sbase + Lay::Q_OFF + h * Lay::TILE;
+        const uint32_t kbase = sbase + Lay::K_OFF + kst * Lay::TILE;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * Lay::BLK + (kk & 3) * 32;
+          mma_ss(tmem + h * 128, smem_desc_sw128(qbase + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
+                 idS, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(Lay::B_SFULL + h));
+      };
+      auto issue_PV = [&](int h, int vst, bool acc) {
+        const uint32_t vbase = sbase + Lay::V_OFF + vst * Lay::TILE;
 #pragma unroll
         for (int kk = 0; kk < tc::BN / 16; ++kk) {
           // V tile is MN-major (D contiguous): 16 keys = 16 rows of 128 B.
           const uint64_t bdesc = smem_desc_sw128(vbase + kk * 2048, Lay::BLK, 1024);
-          mma_ts(tmem + tc::kColO, pA + kk * 8, bdesc, idO, (first && kk == 0) ? 0u : 1u);
+          mma_ts(tmem + 256 + h * 128, tmem + h * 128 + kk * 8, bdesc, idO, (acc || kk > 0) ? 1u : 0u);
         }
-        tc_commit(bar(Lay::B_ODONE));
-        tc_commit(bar(Lay::B_VEMPTY + vs));
-        return true;
       };
+      int t = 0, ul = 0;
+      int ts[2] = {0, 0};  // P_h V MMAs issued per head slot
+      int us[2] = {0, 0};  // units per head slot
+      bool ok = true;
       for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++ul) {
         const TcUnit x = tc_unit(u, p);
-        const int qb = ul & 1;
-        if (!mbar_wait(bar(Lay::B_QFULL + qb), (ul >> 1) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t qbase = sbase + Lay::Q_OFF + qb * Lay::TILE;
+        const int nslot = x.h1 >= 0 ? 2 : 1;
         const int nt = x.t_hi - x.t_lo + 1;
-        for (int jj = 0; jj < nt; ++jj, ++t) {
+        if (!mbar_wait(bar(Lay::B_QFULL), ul & 1, abort_flag)) { ok = false; break; }
+        {
           const int ks = t % tc::KST;
           if (!mbar_wait(bar(Lay::B_KFULL + ks), (t / tc::KST) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t kbase = sbase + Lay::K_OFF + ks * Lay::TILE;
-          const uint32_t dS = tmem + tc::kColS + (t & 1) * 128;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * Lay::BLK + (kk & 3) * 32;
-            mma_ss(dS, smem_desc_sw128(qbase + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
-                   idS, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(bar(Lay::B_SFULL + (t & 1)));
+          for (int h = 0; h < nslot; ++h) issue_S(h, ks);
           tc_commit(bar(Lay::B_KEMPTY + ks));
-          if (jj == nt - 1) tc_commit(bar(Lay::B_QEMPTY + qb));
-          if (jj > 0 && !issue_pv(t - 1, jj == 1, ul)) { ok = false; break; }
+          if (nt == 1) tc_commit(bar(Lay::B_QEMPTY));
         }
-        if (!ok) break;
-        if (!issue_pv(t - 1, nt == 1, ul)) { ok = false; break; }
+        for (int jj = 0; ok && jj < nt; ++jj, ++t) {
+          const int vs = t % tc::VST;
+          if (!mbar_wait(bar(Lay::B_VFULL + vs), (t / tc::VST) & 1, abort_flag)) { ok = false; break; }
+          const bool nxt = jj + 1 < nt;
+          const int ksn = (t + 1) % tc::KST;
+          for (int h = 0; h < nslot; ++h) {
+            if (!mbar_wait(bar(Lay::B_PFULL + h), ts[h] & 1, abort_flag)) { ok = false; break; }
+            if (jj == 0 && us[h] > 0 && !mbar_wait(bar(Lay::B_OEMPTY + h), (us[h] - 1) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_PV(h, vs, jj > 0);
+            ++ts[h];
+            if (nxt) {
+              if (h == 0 && !mbar_wait(bar(Lay::B_KFULL + ksn), ((t + 1) / tc::KST) & 1, abort_flag)) {
+                ok = false;
+                break;
+              }
+              issue_S(h, ksn);
+            } else {
+              tc_commit(bar(Lay::B_ODONE + h));
+            }
+          }
+          if (!ok) break;
+          tc_commit(bar(Lay::B_VEMPTY + vs));
+          if (nxt) {
+            tc_commit(bar(Lay::B_KEMPTY + ksn));
+            if (jj + 1 == nt - 1) tc_commit(bar(Lay::B_QEMPTY));
+          }
+        }
+        us[0]++;
+        if (nslot == 2) us[1]++;
       }
       if (!ok) fail();
       // Drain: every MMA issued above has completed before TMEM is freed.
@@ -264,49 +314,51 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     }
   } else {
     // ------------------------------------------------- softmax + epilogue
-    const int r = threadIdx.x;  // 0..127, tensor-memory lane
-    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    const int slot = warp >> 2;
+    const int r = threadIdx.x & 127;  // tensor-memory lane
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t sS = tmem + lane_addr + slot * 128;        // S_h, then P_h
+    const uint32_t sO = tmem + lane_addr + 256 + slot * 128;  // O_h
     const float sl2 = p.scale_log2;
     const int P = p.Ls * p.ns;
-    int t = 0;
+    int sc = 0, uc = 0;
     bool ok = true;
     for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
       const TcUnit x = tc_unit(u, p);
+      const int h = slot ? x.h1 : x.h0;
+      if (h < 0) continue;  // uniform across the warpgroup
       const int q0 = x.qblk * tc::BM;
       const int i = q0 + r;
       float m = -INFINITY, l = 0.f;
       const int nt = x.t_hi - x.t_lo + 1;
-      for (int jj = 0; jj < nt; ++jj, ++t) {
+      for (int jj = 0; jj < nt; ++jj, ++sc) {
         const int k0 = (x.t_lo + jj) * tc::BN;
-        const bool got = mbar_wait(bar(Lay::B_SFULL + (t & 1)), (t >> 1) & 1, abort_flag);
+        const bool got = mbar_wait(bar(Lay::B_SFULL + slot), sc & 1, abort_flag);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         tc_fence_after();
         uint32_t sv[128];
-        const uint32_t sS = tmem + lane_addr + tc::kColS + (t & 1) * 128;
         tmem_ld32(sS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
         tmem_ld32(sS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
         tmem_ld32(sS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
         tmem_ld32(sS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
         tmem_wait_ld();
         const bool need_mask = (x.t_lo + jj >= x.qblk) || (p.W > 0 && k0 < q0 + tc::BM - p.W);
-        float mt = -INFINITY;
         if (need_mask) {
 #pragma unroll
           for (int c = 0; c < 128; ++c) {
             const int j = k0 + c;
-            float y = __uint_as_float(sv[c]) * sl2;
-            if (j > i || (p.W > 0 && i - j >= p.W)) y = -INFINITY;
-            sv[c] = __float_as_uint(y);
-            mt = fmaxf(mt, y);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            const float y = __uint_as_float(sv[c]) * sl2;
-            sv[c] = __float_as_uint(y);
-            mt = fmaxf(mt, y);
+            if (j > i || (p.W > 0 && i - j >= p.W)) sv[c] = __float_as_uint(-INFINITY);
           }
         }
+        // Row max of the raw scores (scale > 0 commutes with max), 8 chains.
+        float mx[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx[e] = __uint_as_float(sv[e]);
+#pragma unroll
+        for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(sv[c]));
+        const float mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        const float mt = mraw * sl2;  // -inf stays -inf
         bool resc = false;
         float alpha = 1.f;
         if (jj == 0) {
@@ -317,55 +369,62 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
           m = mt;
           resc = true;
         }
-        const float mu = (m == -INFINITY) ? 0.f : m;
-        uint32_t pk[64];
-        float ls = 0.f;
+        const float nmu = (m == -INFINITY) ? 0.f : -m;
+        // P = 2^(s*scale - m) as bf16 pairs, written over the S columns 16 at
+        // a time (column 16j of P holds S columns 32j.. already consumed).
+        float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float p0 = ex2(__uint_as_float(sv[2 * c]) - mu);
-          const float p1 = ex2(__uint_as_float(sv[2 * c + 1]) - mu);
-          ls += p0 + p1;
-          pk[c] = pack_bf16x2(p0, p1);
+        for (int j = 0; j < 4; ++j) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c = 16 * j + e;
+            const float a0 = fmaf(__uint_as_float(sv[2 * c]), sl2, nmu);
+            const float a1 = fmaf(__uint_as_float(sv[2 * c + 1]), sl2, nmu);
+            float p0, p1;
+            if (!need_mask && (e & 3) == 3) {
+              p0 = exp2_fma(a0);
+              p1 = exp2_fma(a1);
+            } else {
+              p0 = ex2(a0);
+              p1 = ex2(a1);
+            }
+            ls[e & 7] += p0 + p1;
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(sS + 16 * j, pk);
         }
-        l += ls;
-        const uint32_t sP = tmem + lane_addr + tc::kColP + (t & 1) * 64;
-        tmem_st32(sP, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-        tmem_st32(sP + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+        l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
         if (__any_sync(0xffffffffu, resc)) {
-          // O must hold P_{t-1} V_{t-1} before it is rescaled.
-          if (!mbar_wait(bar(Lay::B_ODONE), (t - 1) & 1, abort_flag)) ok = false;
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          tc_fence_after();
+          // O_h is stable: the commit that signalled S_h of this tile also
+          // covers the P_h V MMA issued before it.
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t ov[32];
-            const uint32_t oA = tmem + lane_addr + tc::kColO + c * 32;
-            tmem_ld32(oA, ov);
+            tmem_ld32(sO + c * 32, ov);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-            tmem_st32(oA, ov);
+            tmem_st32(sO + c * 32, ov);
           }
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(Lay::B_PFULL + (t & 1)));
+        mbar_arrive(bar(Lay::B_PFULL + slot));
       }
       if (!ok) break;
-      // Epilogue: O / l -> global.
-      if (!mbar_wait(bar(Lay::B_ODONE), (t - 1) & 1, abort_flag)) ok = false;
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
+      // Epilogue: O / l -> global once the last P V MMA of this head is done.
+      const bool got = mbar_wait(bar(Lay::B_ODONE + slot), uc & 1, abort_flag);
+      ++uc;
+      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
       const float inv = 1.f / l;
       const bool row_ok = i < p.Ls;
-      const int64_t orow =
-          (static_cast<int64_t>(x.b) * P + static_cast<int64_t>(i) * p.ns + x.s) * p.Hq + x.h;
+      const int64_t orow = (static_cast<int64_t>(x.b) * P + static_cast<int64_t>(i) * p.ns + x.s) * p.Hq + h;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
-        tmem_ld32(tmem + lane_addr + tc::kColO + c * 32, ov);
+        tmem_ld32(sO + c * 32, ov);
         tmem_wait_ld();
         if (row_ok) {
           if (p.out_bf16) {
@@ -389,16 +448,16 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         }
       }
       if (row_ok && p.lse)
-        p.lse[(static_cast<int64_t>(x.b) * p.Hq + x.h) * P + static_cast<int64_t>(i) * p.ns + x.s] =
+        p.lse[(static_cast<int64_t>(x.b) * p.Hq + h) * P + static_cast<int64_t>(i) * p.ns + x.s] =
             (m + log2f(l)) * 0.69314718055994531f;
       tc_fence_before();
-      mbar_arrive(bar(Lay::B_OEMPTY));
+      mbar_arrive(bar(Lay::B_OEMPTY + slot));
     }
     if (!ok) fail();
   }
 
   __syncthreads();
-  if (warp == 5) {
+  if (warp == tc::kWarpMMA) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, tc::kTmemCols);
@@ -406,7 +465,6 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
 }
 
 // ------------------------------------------------------------------- host
-
 
 // (D, H, ns, Ls, B) view of a [B, ns*Ls, H, D] bf16 tensor; box = 64 x 1 x 1 x 128 x 1.
 static bool encode_stream_view(CUtensorMap* m, const void* ptr, int B, int Ls, int ns, int H, int D) {
@@ -426,9 +484,9 @@ static bool encode_stream_view(CUtensorMap* m, const void* ptr, int B, int Ls, i
 
 int attn_tc_smem_bytes(int D) { return D == 64 ? tc::Layout<64>::ALLOC : tc::Layout<128>::ALLOC; }
 
-cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                           int Ls, int ns, int Hq, int Hkv, int D, int W, float scale, bool out_bf16,
-                           int32_t* status, int sms, cudaStream_t st) {
+cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Ls,
+                           int ns, int Hq, int Hkv, int D, int W, float scale, bool out_bf16, int32_t* status,
+                           int sms, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
   if (!encode_stream_view(&mq, q, B, Ls, ns, Hq, D) || !encode_stream_view(&mk, k, B, Ls, ns, Hkv, D) ||
       !encode_stream_view(&mv, v, B, Ls, ns, Hkv, D))
@@ -446,7 +504,9 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o,
   p.scale_log2 = scale * 1.4426950408889634f;
   p.out_bf16 = out_bf16 ? 1 : 0;
   p.nqb = (Ls + tc::BM - 1) / tc::BM;
-  const int64_t units = static_cast<int64_t>(p.nqb) * B * ns * Hq;
+  const int G = Hq / Hkv;
+  p.npairs = (G + 1) / 2;
+  const int64_t units = static_cast<int64_t>(p.nqb) * B * ns * Hkv * p.npairs;
   if (units <= 0) return cudaSuccess;
   if (units > 0x7fffffff) return cudaErrorInvalidValue;
   p.total_units = static_cast<int>(units);

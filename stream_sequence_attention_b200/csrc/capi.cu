@@ -85,7 +85,8 @@ hd_status hd_attn_fwd(const void* q, const void* k, const void* v, void* o, floa
                       hd_dtype out_dt, int32_t* dev_status, void* stream) {
   if (B < 0 || L < 1 || n < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || window < 0) return HD_ERR_INVALID_ARG;
   if (mode != HD_INTRA && mode != HD_CROSS) return HD_ERR_INVALID_ARG;
-  if (!valid_dtype(in_dt) || !valid_dtype(out_dt) || !std::isfinite(scale)) return HD_ERR_INVALID_ARG;
+  if (!valid_dtype(in_dt) || !valid_dtype(out_dt) || !std::isfinite(scale) || !(scale > 0.f))
+    return HD_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return HD_ERR_UNSUPPORTED;
   const int64_t P = static_cast<int64_t>(n) * L;
   if (P > (1ll << 30) || static_cast<int64_t>(B) * P * Hq > (1ll << 40)) return HD_ERR_INVALID_ARG;
@@ -124,7 +125,8 @@ hd_status hd_attn_decode(const void* q, const void* k_cache, const void* v_cache
                          size_t ws_bytes, int32_t* dev_status, void* stream) {
   if (B < 0 || n < 1 || Lmax < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || window < 0) return HD_ERR_INVALID_ARG;
   if (mode != HD_INTRA && mode != HD_CROSS) return HD_ERR_INVALID_ARG;
-  if (!valid_dtype(in_dt) || !valid_dtype(out_dt) || !std::isfinite(scale)) return HD_ERR_INVALID_ARG;
+  if (!valid_dtype(in_dt) || !valid_dtype(out_dt) || !std::isfinite(scale) || !(scale > 0.f))
+    return HD_ERR_INVALID_ARG;
   if (D != 128 || in_dt != HD_BF16) return HD_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(n) * Lmax > (1ll << 30)) return HD_ERR_INVALID_ARG;
   if (B == 0) return HD_OK;
