@@ -34,10 +34,10 @@
 //
 // Softmax: running max m per row in log2 units; O is rescaled only when a
 // tile raises the max by more than 2^8 (the final 1/l makes the result
-// independent of which max was used).  On tiles with no masked pair, one
-// exponential in four is evaluated on the FMA pipe (round to nearest
-// integer, cubic for 2^f on [-1/2, 1/2], exponent add; relative error
-// < 1e-4, below the bf16 rounding of P) to offload the MUFU unit.
+// independent of which max was used).  The row max uses 3-input max.
+// Optionally (tc::kPolyEvery) part of the exponentials run on the FMA pipe
+// (round to nearest integer, cubic for 2^f on [-1/2, 1/2], exponent add;
+// relative error < 1e-4, below the bf16 rounding of P) to offload MUFU.
 #include "hd_common.cuh"
 #include "hd_launch.h"
 
@@ -53,6 +53,17 @@ constexpr int KST = 3;
 constexpr int VST = 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// On tiles without masking, one exp2 pair in kPolyEvery is evaluated on the
+// FMA pipe (0 = all on the MUFU unit).
+#ifndef HD_TC_POLY_EVERY
+#define HD_TC_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = HD_TC_POLY_EVERY;
+// The two softmax warpgroups take turns (ping-pong) when nonzero.
+#ifndef HD_TC_PINGPONG
+#define HD_TC_PINGPONG 0
+#endif
+constexpr bool kPingPong = HD_TC_PINGPONG != 0;
 
 template <int D>
 struct Layout {
@@ -66,7 +77,7 @@ struct Layout {
   static constexpr int B_QFULL = 0, B_QEMPTY = 1, B_KFULL = 2, B_KEMPTY = B_KFULL + KST,
                        B_VFULL = B_KEMPTY + KST, B_VEMPTY = B_VFULL + VST, B_SFULL = B_VEMPTY + VST,
                        B_PFULL = B_SFULL + 2, B_ODONE = B_PFULL + 2, B_OEMPTY = B_ODONE + 2,
-                       B_DRAIN = B_OEMPTY + 2, NBAR = B_DRAIN + 1;
+                       B_ORD = B_OEMPTY + 2, B_DRAIN = B_ORD + 2, NBAR = B_DRAIN + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int ALLOC = BYTES + 1024;
@@ -156,6 +167,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       mbar_init(bar(Lay::B_ODONE + i), 1);
       mbar_init(bar(Lay::B_OEMPTY + i), 128);
     }
+    mbar_init(bar(Lay::B_ORD + 0), 128);
+    mbar_init(bar(Lay::B_ORD + 1), 128);
     mbar_init(bar(Lay::B_DRAIN), 1);
     *abort_flag = 0;
     *no_abort = 0;
@@ -312,7 +325,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       tc_commit(bar(Lay::B_DRAIN));
       mbar_wait(bar(Lay::B_DRAIN), 0, no_abort);
     }
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------- softmax + epilogue
     const int slot = warp >> 2;
     const int r = threadIdx.x & 127;  // tensor-memory lane
@@ -321,19 +334,29 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     const uint32_t sO = tmem + lane_addr + 256 + slot * 128;  // O_h
     const float sl2 = p.scale_log2;
     const int P = p.Ls * p.ns;
-    int sc = 0, uc = 0;
+    int sc = 0, uc = 0, oc = 0;
     bool ok = true;
     for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
       const TcUnit x = tc_unit(u, p);
       const int h = slot ? x.h1 : x.h0;
       if (h < 0) continue;  // uniform across the warpgroup
+      const bool paired = x.h1 >= 0;
       const int q0 = x.qblk * tc::BM;
       const int i = q0 + r;
       float m = -INFINITY, l = 0.f;
       const int nt = x.t_hi - x.t_lo + 1;
       for (int jj = 0; jj < nt; ++jj, ++sc) {
         const int k0 = (x.t_lo + jj) * tc::BN;
-        const bool got = mbar_wait(bar(Lay::B_SFULL + slot), sc & 1, abort_flag);
+        bool got = mbar_wait(bar(Lay::B_SFULL + slot), sc & 1, abort_flag);
+        // Ping-pong: the two warpgroups take turns for the softmax arithmetic
+        // (slot 0 first), so each runs alone on the SM sub-partitions while
+        // the tensor core works on the other head.
+        if (tc::kPingPong && got && paired) {
+          if (slot == 1)
+            got = mbar_wait(bar(Lay::B_ORD + 1), oc & 1, abort_flag);
+          else if (oc > 0)
+            got = mbar_wait(bar(Lay::B_ORD + 0), (oc - 1) & 1, abort_flag);
+        }
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         tc_fence_after();
         uint32_t sv[128];
@@ -350,14 +373,13 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             if (j > i || (p.W > 0 && i - j >= p.W)) sv[c] = __float_as_uint(-INFINITY);
           }
         }
-        // Row max of the raw scores (scale > 0 commutes with max), 8 chains.
-        float mx[8];
+        // Row max of the raw scores (scale > 0 commutes with max): 3-input
+        // max, 4 independent chains.
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) mx[e] = __uint_as_float(sv[e]);
-#pragma unroll
-        for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(sv[c]));
-        const float mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        for (int c = 0; c < 128; c += 2)
+          mx[(c >> 1) & 3] = fmax3(mx[(c >> 1) & 3], __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]));
+        const float mraw = fmax3(fmax3(mx[0], mx[1], mx[2]), mx[3], mx[3]);
         const float mt = mraw * sl2;  // -inf stays -inf
         bool resc = false;
         float alpha = 1.f;
@@ -382,7 +404,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             const float a0 = fmaf(__uint_as_float(sv[2 * c]), sl2, nmu);
             const float a1 = fmaf(__uint_as_float(sv[2 * c + 1]), sl2, nmu);
             float p0, p1;
-            if (!need_mask && (e & 3) == 3) {
+            if (tc::kPolyEvery > 0 && !need_mask && (e % (tc::kPolyEvery > 0 ? tc::kPolyEvery : 1)) == tc::kPolyEvery - 1) {
               p0 = exp2_fma(a0);
               p1 = exp2_fma(a1);
             } else {
@@ -395,6 +417,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
           tmem_st16(sS + 16 * j, pk);
         }
         l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+        if (tc::kPingPong && paired) {
+          mbar_arrive(bar(Lay::B_ORD + (slot ^ 1)));
+          ++oc;
+        }
         if (__any_sync(0xffffffffu, resc)) {
           // O_h is stable: the commit that signalled S_h of this tile also
           // covers the P_h V MMA issued before it.
