@@ -122,6 +122,38 @@ hd_status hd_attn_decode(const void* q, const void* k_cache, const void* v_cache
 size_t hd_attn_decode_workspace(int B, int n, int Lmax, int Hq, int Hkv, int D,
                                 hd_mode mode);
 
+/* Size of the fixed device scratch used by hd_attn_decode_noalloc (64 MiB). */
+#define HD_DECODE_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/*
+ * hd_attn_decode without a workspace argument: the same computation, inputs,
+ * outputs and argument rules as hd_attn_decode, for callers that cannot
+ * allocate device memory or hand it to the library (an allocator-free
+ * serving loop, a host that owns no CUDA allocator, code running where a
+ * cudaMalloc is not permitted).  The pages have no counterpart of this call;
+ * it exists only for such callers.
+ *
+ * The split-KV partial results go to a fixed HD_DECODE_NOALLOC_SCRATCH_BYTES
+ * array in the library's own device memory (present on every GPU that loads
+ * the library, until the process exits).  Nothing is allocated: no cudaMalloc,
+ * cudaFree or allocating library routine is called.
+ *  - Sizes whose scratch need (hd_attn_decode_workspace for the same sizes)
+ *    exceeds HD_DECODE_NOALLOC_SCRATCH_BYTES return HD_ERR_UNSUPPORTED and
+ *    launch nothing; use hd_attn_decode with a workspace for those.
+ *  - The first call on a device looks up the scratch's device address for
+ *    that device; make that first call before any stream capture.
+ *  - All calls share the one scratch array.  Calls whose kernels can overlap
+ *    on the GPU (different streams with no ordering between them) race on it
+ *    and give wrong results; order them on one stream or with events.
+ *  - The scratch needs no clearing: every call writes each partial it reads.
+ */
+hd_status hd_attn_decode_noalloc(const void* q, const void* k_cache,
+                                 const void* v_cache, const int32_t* ctx_len,
+                                 void* o, float* lse, int B, int n, int Lmax,
+                                 int Hq, int Hkv, int D, hd_mode mode, int window,
+                                 float scale, hd_dtype in_dt, hd_dtype out_dt,
+                                 int32_t* dev_status, void* stream);
+
 /*
  * Final-stream gather ("Multi-Stream Expansion and Training Objective": only
  * the final stream E_n of each token feeds the shared LM head; Figure 1):

@@ -28,6 +28,7 @@ EXPORTS = (
     "hd_attn_fwd",
     "hd_attn_decode",
     "hd_attn_decode_workspace",
+    "hd_attn_decode_noalloc",
     "hd_final_stream_gather",
     "hd_status_string",
     "hd_version",
@@ -61,6 +62,9 @@ def lib() -> ctypes.CDLL:
         L.hd_attn_decode.restype = i32
         L.hd_attn_decode_workspace.argtypes = [i32, i32, i32, i32, i32, i32, i32]
         L.hd_attn_decode_workspace.restype = sz
+        L.hd_attn_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, f32,
+                                             i32, i32, vp, vp]
+        L.hd_attn_decode_noalloc.restype = i32
         L.hd_final_stream_gather.argtypes = [vp, vp, i32, i32, i32, i32, i32, vp]
         L.hd_final_stream_gather.restype = i32
         L.hd_status_string.argtypes = [i32]
@@ -227,4 +231,37 @@ def hd_attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(ctx_len), _ptr(out), _ptr(lse), B, n, Lmax, Hq, Hkv, D,
         _MODES[mode], int(window), float(scale), _dt(q), _dt(out), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
+    return (out, lse) if want_lse else out
+
+
+def hd_attn_decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, ctx_len: torch.Tensor,
+                           mode="intra", window: int = 0, scale: float | None = None,
+                           out: torch.Tensor | None = None, out_dtype=None, lse: torch.Tensor | bool | None = None,
+                           dev_status: torch.Tensor | None = None, stream=None):
+    """Same as :func:`hd_attn_decode` but the library uses its own fixed
+    device scratch instead of a workspace, for callers that cannot hand it
+    device memory (see ``hd_attn_decode_noalloc`` in ``include/hd.h``: sizes
+    needing more than 64 MiB of scratch are refused, and concurrent calls on
+    unordered streams race)."""
+    for t, nm in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"), (ctx_len, "ctx_len")):
+        _need(t, nm)
+    B, n, Hq, D = q.shape
+    _, _, Lmax, Hkv, _ = k_cache.shape
+    if k_cache.shape != (B, n, Lmax, Hkv, D) or v_cache.shape != k_cache.shape:
+        raise ValueError("cache shapes disagree with q")
+    if ctx_len.dtype != torch.int32 or ctx_len.shape != (B,):
+        raise ValueError("ctx_len must be int32 [B]")
+    if scale is None:
+        scale = D ** -0.5
+    if out is None:
+        out = torch.empty((B, n, Hq, D), dtype=out_dtype or q.dtype, device=q.device)
+    _need(out, "out")
+    want_lse = lse is True or isinstance(lse, torch.Tensor)
+    if lse is True:
+        lse = torch.empty((B, n, Hq), dtype=torch.float32, device=q.device)
+    elif lse is False:
+        lse = None
+    _check("hd_attn_decode_noalloc", lib().hd_attn_decode_noalloc(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(ctx_len), _ptr(out), _ptr(lse), B, n, Lmax, Hq, Hkv, D,
+        _MODES[mode], int(window), float(scale), _dt(q), _dt(out), _ptr(dev_status), _stream(stream)))
     return (out, lse) if want_lse else out
