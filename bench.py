@@ -63,6 +63,7 @@ def parse():
     ap.add_argument("--workload", default="intra", choices=list(WORKLOADS))
     ap.add_argument("--no-extras", action="store_true", help="skip the side measurements")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (small ncu captures)")
     ap.add_argument("--profile", action="store_true",
                     help="timed steps only (no e2e, side measurements or CPU oracle): for ncu captures")
     return ap.parse_args()
@@ -311,7 +312,9 @@ def run_ours(args, rank, world, dist):
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
     peaks = load_peaks()
     wl = args.workload
-    cfg = WORKLOADS[wl]
+    cfg = dict(WORKLOADS[wl])
+    if args.batch:
+        cfg["B"] = args.batch
     K = args.steps if args.steps is not None else (100 if wl != "decode" else 40)
     W = args.warmup if args.warmup is not None else 5
     W = max(W, 3)
