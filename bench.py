@@ -293,12 +293,18 @@ def timed(torch, work, K, flush, dist=None, use_e2e=False):
     return steps, kern
 
 
-def max_over_ranks(torch, dist, x):
+def max_over_ranks(torch, dist, x, device="cuda"):
+    """The slowest rank's time: every rank's share counts only when all are done."""
     if dist is None:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(workload, rank):
+    """Seed base of a rank's inputs: every rank draws its own batch."""
+    return 1000 * (list(WORKLOADS).index(workload) + 1) + 97 * rank
 
 
 def run_ours(args, rank, world, dist):
@@ -318,7 +324,7 @@ def run_ours(args, rank, world, dist):
     K = args.steps if args.steps is not None else (100 if wl != "decode" else 40)
     W = args.warmup if args.warmup is not None else 5
     W = max(W, 3)
-    seed_base = 1000 * (list(WORKLOADS).index(wl) + 1) + 97 * rank
+    seed_base = rank_seed(wl, rank)
     work = Decode(cfg, seed_base, torch, hd, synth) if wl == "decode" else Prefill(cfg, seed_base, torch, hd, synth)
     flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     flush = lambda: flush_buf.fill_(1)  # noqa: E731

@@ -38,6 +38,8 @@
 // Optionally (tc::kPolyEvery) part of the exponentials run on the FMA pipe
 // (round to nearest integer, cubic for 2^f on [-1/2, 1/2], exponent add;
 // relative error < 1e-4, below the bf16 rounding of P) to offload MUFU.
+#include <cstdlib>
+
 #include "hd_common.cuh"
 #include "hd_launch.h"
 
@@ -93,6 +95,10 @@ struct TcParams {
   int out_bf16;
   int nqb, npairs;
   int total_units;
+  // Test hook (environment HD_TEST_STALL_FIRST_S=1): the MMA warp of CTA 0
+  // never signals its first S tile, so the softmax wait runs out and the
+  // kernel must take its timeout path.  0 in normal use.
+  int stall_first_s;
 };
 
 struct TcUnit {
@@ -258,7 +264,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
           mma_ss(tmem + h * 128, smem_desc_sw128(qbase + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
                  idS, kk > 0 ? 1u : 0u);
         }
-        tc_commit(bar(Lay::B_SFULL + h));
+        if (!(p.stall_first_s && blockIdx.x == 0)) tc_commit(bar(Lay::B_SFULL + h));
       };
       auto issue_PV = [&](int h, int vst, bool acc) {
         const uint32_t vbase = sbase + Lay::V_OFF + vst * Lay::TILE;
@@ -536,6 +542,11 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o,
   if (units <= 0) return cudaSuccess;
   if (units > 0x7fffffff) return cudaErrorInvalidValue;
   p.total_units = static_cast<int>(units);
+  static const int stall = [] {
+    const char* e = getenv("HD_TEST_STALL_FIRST_S");
+    return (e && e[0] == '1') ? 1 : 0;
+  }();
+  p.stall_first_s = stall;
   const int grid = static_cast<int>(units < sms ? units : sms);
   const int smem = attn_tc_smem_bytes(D);
   cudaError_t err;

@@ -1,0 +1,46 @@
+"""The bounded-wait failure path of the tcgen05 attention kernel, on the GPU,
+without a fault: with HD_TEST_STALL_FIRST_S=1 the MMA warp of CTA 0 never
+signals its S tiles (a flag nothing sets), so the softmax wait runs out after
+its one-second limit.  The kernel must return with HD_ERR_TIMEOUT in the
+status word and leave the context usable for the next launches.  Runs in a
+child process because the hook is read once per process."""
+
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+pytestmark = pytest.mark.gpu
+
+CHILD = r"""
+import json, sys, torch
+sys.path.insert(0, ROOT)
+from stream_sequence_attention_b200 import build, hd, synth
+build.build(); hd.lib()
+q = synth.normal_device((1, 2 * 256, 4, 128), 1)
+k = synth.normal_device((1, 2 * 256, 2, 128), 2)
+v = synth.normal_device((1, 2 * 256, 2, 128), 3)
+st = hd.new_status()
+hd.hd_attn_fwd(q, k, v, 2, "intra", dev_status=st)
+torch.cuda.synchronize()
+status = int(st.item())
+# the context is still usable: other kernels run and give exact results
+h = synth.normal_device((1, 2 * 64, 16), 4)
+g = hd.hd_final_stream_gather(h, 2)
+torch.cuda.synchronize()
+usable = bool(torch.equal(g, h[:, 1::2]))
+print(json.dumps({"status": status, "usable": usable}))
+"""
+
+
+def test_attention_wait_times_out_cleanly():
+    env = dict(os.environ, HD_TEST_STALL_FIRST_S="1")
+    code = CHILD.replace("ROOT", repr(ROOT))
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=180)
+    assert r.returncode == 0, r.stderr[-2000:]
+    out = json.loads(r.stdout.strip().splitlines()[-1])
+    assert out["status"] == 4  # HD_ERR_TIMEOUT
+    assert out["usable"]
