@@ -43,12 +43,14 @@ WORKLOADS = {
     "cross": dict(B=2, n=4, L=4096, Hq=32, Hkv=8, D=128, mode="cross", W=0, V=152064, dm=4096),
     "long": dict(B=1, n=4, L=32768, Hq=64, Hkv=8, D=128, mode="intra", W=4096, V=152064, dm=4096),
     "decode": dict(B=64, n=4, T=32768, Hq=64, Hkv=8, D=128),
+    "mirror": dict(B=2, n=4, L=4096, Hq=32, Hkv=8, D=128, mode="cross", W=0, V=152064, dm=4096, final=True),
 }
 NAMES = {
     "intra": "bf16 prefill, intra-stream, n=4 L=4096 B=2 32q/8kv D=128",
     "cross": "bf16 prefill, cross-stream, n=4 L=4096 B=2 32q/8kv D=128",
     "long": "long-context intra-stream W=4096, n=4 L=32768 B=1 64q/8kv D=128",
     "decode": "decode B=64 n=4 ctx=32768 64q/8kv D=128, intra+cross",
+    "mirror": "bf16 KV-mirror layer: final-stream queries, cross-stream keys, n=4 L=4096 B=2 32q/8kv D=128",
 }
 FLUSH_BYTES = 512 << 20
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
@@ -170,7 +172,9 @@ class Prefill:
         self.ids_host = torch.from_numpy(ids).pin_memory()
         self.ids = self.ids_host.cuda()
         self.tables = synth.normal_device((c["n"], c["V"], c["dm"]), seed_base + 2, std=0.02)
-        self.q = synth.normal_device((c["B"], P, c["Hq"], c["D"]), seed_base + 3)
+        self.final = bool(c.get("final"))
+        qrows = c["L"] if self.final else P
+        self.q = synth.normal_device((c["B"], qrows, c["Hq"], c["D"]), seed_base + 3)
         self.k = synth.normal_device((c["B"], P, c["Hkv"], c["D"]), seed_base + 4)
         self.v = synth.normal_device((c["B"], P, c["Hkv"], c["D"]), seed_base + 5)
         self.x = torch.empty((c["B"], P, c["dm"]), dtype=torch.bfloat16, device="cuda")
@@ -183,7 +187,11 @@ class Prefill:
         hd.hd_expand_embed(self.tables, self.ids, self.x, dev_status=self.status)
         if ev is not None:
             ev[0].record()
-        hd.hd_attn_fwd(self.q, self.k, self.v, c["n"], c["mode"], c["W"], out=self.o, dev_status=self.status)
+        if self.final:
+            hd.hd_attn_fwd_final_stream(self.q, self.k, self.v, c["n"], c["mode"], c["W"], out=self.o,
+                                        dev_status=self.status)
+        else:
+            hd.hd_attn_fwd(self.q, self.k, self.v, c["n"], c["mode"], c["W"], out=self.o, dev_status=self.status)
         if ev is not None:
             ev[1].record()
         hd.hd_final_stream_gather(self.x, c["n"], out=self.g)
@@ -216,6 +224,8 @@ class Prefill:
     def flops(self):
         from stream_sequence_attention_b200 import accounting as acc
         c = self.cfg
+        if self.final:
+            return acc.attn_flops_final_stream(c["B"], c["L"], c["n"], c["Hq"], c["D"], c["mode"], c["W"])
         return acc.attn_flops(c["B"], c["L"], c["n"], c["Hq"], c["D"], c["mode"], c["W"])
 
 
@@ -369,7 +379,7 @@ def run_ours(args, rank, world, dist):
     else:
         fl = work.flops()
         value = world * fl / (ms_per_step * 1e-3) / 1e12
-        metric = "useful attn TFLOP/s at n=4 (%s)" % cfg["mode"]
+        metric = "useful attn TFLOP/s at n=4 (%s)" % (cfg["mode"] + (", final-stream queries" if cfg.get("final") else ""))
         unit = "TFLOP/s"
         achieved = fl / (kern_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16"], "unit": "TFLOP/s",
@@ -432,6 +442,14 @@ def extras(torch, peaks, rank):
     tf = cr.flops() / (ms * 1e-3) / 1e12
     res["cross_prefill"] = {"ms": round(ms, 3), "TFLOP/s": round(tf, 1), "frac_bf16": round(tf / peaks["bf16"], 4)}
     del cr
+    torch.cuda.empty_cache()
+    mi = Prefill(WORKLOADS["mirror"], 7201 + rank, torch, hd, synth)
+    c = WORKLOADS["mirror"]
+    ms = time_fn(lambda: hd.hd_attn_fwd_final_stream(mi.q, mi.k, mi.v, c["n"], "cross", out=mi.o))
+    tf = mi.flops() / (ms * 1e-3) / 1e12
+    res["mirror_final_stream_cross"] = {"ms": round(ms, 3), "TFLOP/s": round(tf, 1),
+                                        "frac_bf16": round(tf / peaks["bf16"], 4)}
+    del mi
     torch.cuda.empty_cache()
     return res
 

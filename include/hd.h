@@ -88,6 +88,27 @@ hd_status hd_attn_fwd(const void* q, const void* k, const void* v, void* o,
                       hd_dtype out_dt, int32_t* dev_status, void* stream);
 
 /*
+ * Final-stream queries only ("Persistent KV and the KV-mirror Saving": in the
+ * mirrored layers only the final stream is run, against keys and values that
+ * an earlier layer produced for every stream).  The rows of hd_attn_fwd at the
+ * final-stream positions p = i*n + n-1, computed without the other queries:
+ *   O[b,i,h,:] = sum_{p' in vis(i*n + n-1)} softmax(scale <qf[b,i,h], k[b,p',g]>) v[b,p',g]
+ * with vis as in hd_attn_fwd (intra: keys (j, n-1), j <= i; cross: all
+ * p' <= i*n + n-1; optional window in the same units).
+ *
+ *   q_final [B, L, Hq, D]     element type `in_dt` (the final-stream queries)
+ *   k, v    [B, n*L, Hkv, D]  element type `in_dt` (all streams)
+ *   o       [B, L, Hq, D]     element type `out_dt`
+ *   lse     [B, Hq, L]        float32, nullable
+ * Same argument rules and kernels as hd_attn_fwd.
+ */
+hd_status hd_attn_fwd_final_stream(const void* q_final, const void* k, const void* v,
+                                   void* o, float* lse, int B, int L, int n, int Hq,
+                                   int Hkv, int D, hd_mode mode, int window, float scale,
+                                   hd_dtype in_dt, hd_dtype out_dt, int32_t* dev_status,
+                                   void* stream);
+
+/*
  * Decode against the per-stream KV cache ("Persistent KV and the KV-mirror
  * Saving": a separate cache per stream; "Inference Throughput": the n streams
  * of a token are processed together in one pass).  For every b, the new

@@ -201,6 +201,37 @@ def attn_rows(q, k, v, n, mode, rows, window=0, scale=None):
     return np.array(outs), np.array(lses)
 
 
+def attn_final_stream(q_final, k, v, n, mode, window=0, scale=None):
+    """Attention of the final-stream queries only ("Persistent KV and the
+    KV-mirror Saving": in a mirrored layer only the final stream is run,
+    against the keys and values every stream contributed earlier).
+
+    q_final: [B, L, Hq, D] -- the query of token i sits at physical position
+    p = i*n + n-1; k, v: [B, nL, Hkv, D].  Returns (O [B, L, Hq, D],
+    lse [B, Hq, L]) by the same definition as :func:`attn`, one row at a time.
+    """
+    q_final = np.asarray(q_final, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, L, Hq, D = q_final.shape
+    Hkv = k.shape[2]
+    G = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    pk = np.arange(n * L)
+    O = np.empty((B, L, Hq, D))
+    lse = np.empty((B, Hq, L))
+    for i in range(L):
+        p = i * n + n - 1
+        keys = pk[visible(p, pk, n, mode, window)]
+        for b in range(B):
+            for h in range(Hq):
+                kv = h // G
+                o, l = _softmax_weighted(scale * (k[b, keys, kv, :] @ q_final[b, i, h, :])[None, :], v[b, keys, kv, :])
+                O[b, i, h], lse[b, h, i] = o[0], l[0]
+    return O, lse
+
+
 def _decode_keys(T, n, s, mode, window):
     """Visible cache entries (j, s') for the stream-s query of the new token
     T-1, as physical positions of the expanded sequence."""

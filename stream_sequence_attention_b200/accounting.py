@@ -56,3 +56,23 @@ def decode_flops(B: int, n: int, T: int, Hq: int, D: int, mode: str) -> int:
         # stream s sees n*(T-1) older entries plus s+1 entries of the new token
         pairs = n * n * (T - 1) + n * (n + 1) // 2
     return B * Hq * pairs * 4 * D
+
+
+def pairs_final_stream(L: int, n: int, mode: str, window: int = 0) -> int:
+    """Visible pairs per (batch, query head) when only the final-stream
+    queries run (KV-mirror layers): query i sits at position i*n + n-1.
+    intra: causal over the final stream's L tokens (window in tokens);
+    cross: all positions <= i*n + n-1 (window in positions)."""
+    if mode == "intra":
+        return pairs_per_head(L, 1, "intra", window)
+    if mode != "cross":
+        raise ValueError(mode)
+    total = 0
+    for i in range(L):
+        vis = (i + 1) * n
+        total += vis if window <= 0 else min(vis, window)
+    return total
+
+
+def attn_flops_final_stream(B: int, L: int, n: int, Hq: int, D: int, mode: str, window: int = 0) -> int:
+    return B * Hq * pairs_final_stream(L, n, mode, window) * 4 * D

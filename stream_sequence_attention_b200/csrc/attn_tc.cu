@@ -90,7 +90,8 @@ struct TcParams {
   void* o;
   float* lse;
   int32_t* status;
-  int B, Ls, ns, Hq, Hkv, W;
+  AttnGeom g;
+  int Hq, Hkv, W;
   float scale_log2;
   int out_bf16;
   int nqb, npairs;
@@ -107,7 +108,7 @@ struct TcUnit {
 
 __device__ __forceinline__ TcUnit tc_unit(int u, const TcParams& p) {
   const int G = p.Hq / p.Hkv;
-  const int per = p.B * p.ns * p.Hkv * p.npairs;
+  const int per = p.g.B * p.g.ns * p.Hkv * p.npairs;
   const int qi = u / per;
   int rem = u - qi * per;
   TcUnit x;
@@ -116,13 +117,16 @@ __device__ __forceinline__ TcUnit tc_unit(int u, const TcParams& p) {
   rem /= p.npairs;
   x.kvh = rem % p.Hkv;
   rem /= p.Hkv;
-  x.s = rem % p.ns;
-  x.b = rem / p.ns;
+  x.s = rem % p.g.ns;
+  x.b = rem / p.g.ns;
   x.h0 = x.kvh * G + 2 * pair;
   x.h1 = (2 * pair + 1 < G) ? x.h0 + 1 : -1;
+  // Key range of the block: up to the key index of its last query, from the
+  // window start of its first query.
   const int q0 = x.qblk * tc::BM;
-  x.t_hi = x.qblk;  // BM == BN: the diagonal tile is the last one
-  x.t_lo = p.W > 0 ? max(0, q0 - p.W + 1) / tc::BN : 0;
+  const int qlast = min(q0 + tc::BM - 1, p.g.Lq - 1);
+  x.t_hi = (qlast * p.g.qstride + p.g.qoff) / tc::BN;
+  x.t_lo = p.W > 0 ? max(0, q0 * p.g.qstride + p.g.qoff - p.W + 1) / tc::BN : 0;
   return x;
 }
 
@@ -218,6 +222,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                         x.h1, x.s, x.qblk * tc::BM, x.b);
         }
         ++q_issued;
+        const int skv = p.g.kv_stream >= 0 ? p.g.kv_stream : x.s;
         for (int kt = x.t_lo; kt <= x.t_hi; ++kt, ++t) {
           const int ks = t % tc::KST;
           if (!mbar_wait(bar(Lay::B_KEMPTY + ks), ((t / tc::KST) & 1) ^ 1, abort_flag)) { ok = false; break; }
@@ -225,7 +230,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
 #pragma unroll
           for (int kb = 0; kb < Lay::KB; ++kb)
             tma_load_5d(sbase + Lay::K_OFF + ks * Lay::TILE + kb * Lay::BLK, &tmK, bar(Lay::B_KFULL + ks),
-                        kb * 64, x.kvh, x.s, kt * tc::BN, x.b);
+                        kb * 64, x.kvh, skv, kt * tc::BN, x.b);
           ++k_issued[ks];
           const int vs = t % tc::VST;
           if (!mbar_wait(bar(Lay::B_VEMPTY + vs), ((t / tc::VST) & 1) ^ 1, abort_flag)) { ok = false; break; }
@@ -233,7 +238,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
 #pragma unroll
           for (int kb = 0; kb < Lay::KB; ++kb)
             tma_load_5d(sbase + Lay::V_OFF + vs * Lay::TILE + kb * Lay::BLK, &tmV, bar(Lay::B_VFULL + vs),
-                        kb * 64, x.kvh, x.s, kt * tc::BN, x.b);
+                        kb * 64, x.kvh, skv, kt * tc::BN, x.b);
           ++v_issued[vs];
         }
       }
@@ -339,7 +344,6 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     const uint32_t sS = tmem + lane_addr + slot * 128;        // S_h, then P_h
     const uint32_t sO = tmem + lane_addr + 256 + slot * 128;  // O_h
     const float sl2 = p.scale_log2;
-    const int P = p.Ls * p.ns;
     int sc = 0, uc = 0, oc = 0;
     bool ok = true;
     for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
@@ -349,6 +353,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       const bool paired = x.h1 >= 0;
       const int q0 = x.qblk * tc::BM;
       const int i = q0 + r;
+      const int pi = i * p.g.qstride + p.g.qoff;             // key index of this row's query
+      const int pfirst = q0 * p.g.qstride + p.g.qoff;         // ... of the block's first query
+      const int plast = (q0 + tc::BM - 1) * p.g.qstride + p.g.qoff;
       float m = -INFINITY, l = 0.f;
       const int nt = x.t_hi - x.t_lo + 1;
       for (int jj = 0; jj < nt; ++jj, ++sc) {
@@ -371,12 +378,12 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         tmem_ld32(sS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
         tmem_ld32(sS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
         tmem_wait_ld();
-        const bool need_mask = (x.t_lo + jj >= x.qblk) || (p.W > 0 && k0 < q0 + tc::BM - p.W);
+        const bool need_mask = (k0 + tc::BN - 1 > pfirst) || (p.W > 0 && k0 < plast - p.W + 1);
         if (need_mask) {
 #pragma unroll
           for (int c = 0; c < 128; ++c) {
             const int j = k0 + c;
-            if (j > i || (p.W > 0 && i - j >= p.W)) sv[c] = __float_as_uint(-INFINITY);
+            if (j > pi || (p.W > 0 && pi - j >= p.W)) sv[c] = __float_as_uint(-INFINITY);
           }
         }
         // Row max of the raw scores (scale > 0 commutes with max): 3-input
@@ -451,8 +458,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
       const float inv = 1.f / l;
-      const bool row_ok = i < p.Ls;
-      const int64_t orow = (static_cast<int64_t>(x.b) * P + static_cast<int64_t>(i) * p.ns + x.s) * p.Hq + h;
+      const bool row_ok = i < p.g.Lq;
+      const int64_t orow =
+          (static_cast<int64_t>(x.b) * p.g.o_rows + static_cast<int64_t>(i) * p.g.o_ns + x.s) * p.Hq + h;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
@@ -480,7 +488,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         }
       }
       if (row_ok && p.lse)
-        p.lse[(static_cast<int64_t>(x.b) * p.Hq + h) * P + static_cast<int64_t>(i) * p.ns + x.s] =
+        p.lse[(static_cast<int64_t>(x.b) * p.Hq + h) * p.g.o_rows + static_cast<int64_t>(i) * p.g.o_ns + x.s] =
             (m + log2f(l)) * 0.69314718055994531f;
       tc_fence_before();
       mbar_arrive(bar(Lay::B_OEMPTY + slot));
@@ -516,29 +524,28 @@ static bool encode_stream_view(CUtensorMap* m, const void* ptr, int B, int Ls, i
 
 int attn_tc_smem_bytes(int D) { return D == 64 ? tc::Layout<64>::ALLOC : tc::Layout<128>::ALLOC; }
 
-cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Ls,
-                           int ns, int Hq, int Hkv, int D, int W, float scale, bool out_bf16, int32_t* status,
-                           int sms, cudaStream_t st) {
+cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o, float* lse, const AttnGeom& g,
+                           int Hq, int Hkv, int D, int W, float scale, bool out_bf16, int32_t* status, int sms,
+                           cudaStream_t st) {
   CUtensorMap mq, mk, mv;
-  if (!encode_stream_view(&mq, q, B, Ls, ns, Hq, D) || !encode_stream_view(&mk, k, B, Ls, ns, Hkv, D) ||
-      !encode_stream_view(&mv, v, B, Ls, ns, Hkv, D))
+  if (!encode_stream_view(&mq, q, g.B, g.Lq, g.q_ns, Hq, D) ||
+      !encode_stream_view(&mk, k, g.B, g.Lk, g.kv_ns, Hkv, D) ||
+      !encode_stream_view(&mv, v, g.B, g.Lk, g.kv_ns, Hkv, D))
     return cudaErrorInvalidValue;
   TcParams p;
   p.o = o;
   p.lse = lse;
   p.status = status;
-  p.B = B;
-  p.Ls = Ls;
-  p.ns = ns;
+  p.g = g;
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.W = W;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.out_bf16 = out_bf16 ? 1 : 0;
-  p.nqb = (Ls + tc::BM - 1) / tc::BM;
+  p.nqb = (g.Lq + tc::BM - 1) / tc::BM;
   const int G = Hq / Hkv;
   p.npairs = (G + 1) / 2;
-  const int64_t units = static_cast<int64_t>(p.nqb) * B * ns * Hkv * p.npairs;
+  const int64_t units = static_cast<int64_t>(p.nqb) * g.B * g.ns * Hkv * p.npairs;
   if (units <= 0) return cudaSuccess;
   if (units > 0x7fffffff) return cudaErrorInvalidValue;
   p.total_units = static_cast<int>(units);

@@ -80,9 +80,10 @@ hd_status hd_final_stream_gather(const void* h, void* out, int B, int L, int n, 
       launch_gather(h, out, rows, n, static_cast<int>(row_bytes), sms, static_cast<cudaStream_t>(stream)));
 }
 
-hd_status hd_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int L, int n,
-                      int Hq, int Hkv, int D, hd_mode mode, int window, float scale, hd_dtype in_dt,
-                      hd_dtype out_dt, int32_t* dev_status, void* stream) {
+// Argument checks shared by both attention entry points.
+static hd_status check_attn_args(const void* q, const void* k, const void* v, void* o, float* lse, int B, int L,
+                                 int n, int Hq, int Hkv, int D, hd_mode mode, int window, float scale,
+                                 hd_dtype in_dt, hd_dtype out_dt) {
   if (B < 0 || L < 1 || n < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || window < 0) return HD_ERR_INVALID_ARG;
   if (mode != HD_INTRA && mode != HD_CROSS) return HD_ERR_INVALID_ARG;
   if (!valid_dtype(in_dt) || !valid_dtype(out_dt) || !std::isfinite(scale) || !(scale > 0.f))
@@ -94,21 +95,76 @@ hd_status hd_attn_fwd(const void* q, const void* k, const void* v, void* o, floa
   if (!q || !k || !v || !o || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
     return HD_ERR_INVALID_ARG;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return HD_ERR_INVALID_ARG;
-  // Intra: n streams of L tokens.  Cross: one stream of n*L positions.
-  const int ns = mode == HD_INTRA ? n : 1;
-  const int Ls = mode == HD_INTRA ? L : static_cast<int>(P);
+  return HD_OK;
+}
+
+static hd_status run_attn(const void* q, const void* k, const void* v, void* o, float* lse, const AttnGeom& g,
+                          int Hq, int Hkv, int D, int window, float scale, hd_dtype in_dt, hd_dtype out_dt,
+                          int32_t* dev_status, void* stream) {
   const bool out_bf16 = out_dt == HD_BF16;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (in_dt == HD_F32) {
-    if (Hq * ns > 65535 || B > 65535) return HD_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(Hq) * g.ns > 65535 || g.B > 65535) return HD_ERR_UNSUPPORTED;
     return cuda_status(launch_attn_f32(static_cast<const float*>(q), static_cast<const float*>(k),
-                                       static_cast<const float*>(v), o, lse, B, Ls, ns, Hq, Hkv, D, window,
-                                       scale, out_bf16, st));
+                                       static_cast<const float*>(v), o, lse, g, Hq, Hkv, D, window, scale, out_bf16,
+                                       st));
   }
   const int sms = sm_count();
   if (sms <= 0) return HD_ERR_CUDA;
-  return cuda_status(launch_attn_tc(q, k, v, o, lse, B, Ls, ns, Hq, Hkv, D, window, scale, out_bf16,
-                                    dev_status, sms, st));
+  return cuda_status(launch_attn_tc(q, k, v, o, lse, g, Hq, Hkv, D, window, scale, out_bf16, dev_status, sms, st));
+}
+
+hd_status hd_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int L, int n,
+                      int Hq, int Hkv, int D, hd_mode mode, int window, float scale, hd_dtype in_dt,
+                      hd_dtype out_dt, int32_t* dev_status, void* stream) {
+  hd_status stt = check_attn_args(q, k, v, o, lse, B, L, n, Hq, Hkv, D, mode, window, scale, in_dt, out_dt);
+  if (stt != HD_OK || B == 0) return stt;
+  // Intra: n streams of L tokens, read in place.  Cross: one stream of n*L positions.
+  const int P = n * L;
+  AttnGeom g;
+  g.B = B;
+  g.ns = mode == HD_INTRA ? n : 1;
+  g.Lq = mode == HD_INTRA ? L : P;
+  g.q_ns = g.ns;
+  g.kv_ns = g.ns;
+  g.Lk = g.Lq;
+  g.kv_stream = -1;
+  g.qstride = 1;
+  g.qoff = 0;
+  g.o_rows = P;
+  g.o_ns = g.ns;
+  return run_attn(q, k, v, o, lse, g, Hq, Hkv, D, window, scale, in_dt, out_dt, dev_status, stream);
+}
+
+hd_status hd_attn_fwd_final_stream(const void* q_final, const void* k, const void* v, void* o, float* lse, int B,
+                                   int L, int n, int Hq, int Hkv, int D, hd_mode mode, int window, float scale,
+                                   hd_dtype in_dt, hd_dtype out_dt, int32_t* dev_status, void* stream) {
+  hd_status stt = check_attn_args(q_final, k, v, o, lse, B, L, n, Hq, Hkv, D, mode, window, scale, in_dt, out_dt);
+  if (stt != HD_OK || B == 0) return stt;
+  // Queries: the L final-stream rows.  Intra: they read stream n-1 of the
+  // interleaved K/V in place.  Cross: query i sits at position i*n + n-1 of
+  // the single nL-position stream.
+  AttnGeom g;
+  g.B = B;
+  g.ns = 1;
+  g.Lq = L;
+  g.q_ns = 1;
+  g.o_rows = L;
+  g.o_ns = 1;
+  if (mode == HD_INTRA) {
+    g.kv_ns = n;
+    g.Lk = L;
+    g.kv_stream = n - 1;
+    g.qstride = 1;
+    g.qoff = 0;
+  } else {
+    g.kv_ns = 1;
+    g.Lk = n * L;
+    g.kv_stream = -1;
+    g.qstride = n;
+    g.qoff = n - 1;
+  }
+  return run_attn(q_final, k, v, o, lse, g, Hq, Hkv, D, window, scale, in_dt, out_dt, dev_status, stream);
 }
 
 size_t hd_attn_decode_workspace(int B, int n, int Lmax, int Hq, int Hkv, int D, hd_mode mode) {

@@ -20,12 +20,29 @@ cudaError_t launch_expand(const void* tables, const int32_t* ids, void* out, int
                           int64_t V, int row_bytes, int sms, int32_t* status, cudaStream_t st);
 cudaError_t launch_gather(const void* h, void* out, int64_t rows, int n, int row_bytes, int sms,
                           cudaStream_t st);
-cudaError_t launch_attn_f32(const float* q, const float* k, const float* v, void* o, float* lse, int B,
-                            int Ls, int ns, int Hq, int Hkv, int D, int W, float scale, bool out_bf16,
+// Geometry of one attention call, common to both attention kernels.  The
+// kernels walk query tokens i in [0, Lq) of ns query streams s.  Query token
+// i reads the key stream kv_stream (or s when kv_stream < 0), where it sits
+// at key index pos(i) = i*qstride + qoff; key j is visible iff j <= pos(i)
+// and, with a window W > 0, pos(i) - j < W.
+//   q   [B, q_ns*Lq, Hq, D]    query (i, s) is row i*q_ns + s
+//   k,v [B, kv_ns*Lk, Hkv, D]  key (j, t) is row j*kv_ns + t
+//   o   [B, o_rows, Hq, D]     query (i, s) writes row i*o_ns + s
+//   lse [B, Hq, o_rows]
+struct AttnGeom {
+  int B;
+  int ns, Lq, q_ns;
+  int kv_ns, Lk, kv_stream;
+  int qstride, qoff;
+  int o_rows, o_ns;
+};
+
+cudaError_t launch_attn_f32(const float* q, const float* k, const float* v, void* o, float* lse,
+                            const AttnGeom& g, int Hq, int Hkv, int D, int W, float scale, bool out_bf16,
                             cudaStream_t st);
-cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Ls,
-                           int ns, int Hq, int Hkv, int D, int W, float scale, bool out_bf16,
-                           int32_t* status, int sms, cudaStream_t st);
+cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o, float* lse, const AttnGeom& g,
+                           int Hq, int Hkv, int D, int W, float scale, bool out_bf16, int32_t* status, int sms,
+                           cudaStream_t st);
 
 // Decode work decomposition: units (one KV head of one sequence, and for
 // intra mode one stream), row groups of at most 32 query rows, token splits.

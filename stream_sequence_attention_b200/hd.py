@@ -26,6 +26,7 @@ _MODES = {"intra": HD_INTRA, "cross": HD_CROSS, HD_INTRA: HD_INTRA, HD_CROSS: HD
 EXPORTS = (
     "hd_expand_embed",
     "hd_attn_fwd",
+    "hd_attn_fwd_final_stream",
     "hd_attn_decode",
     "hd_attn_decode_workspace",
     "hd_attn_decode_noalloc",
@@ -57,6 +58,9 @@ def lib() -> ctypes.CDLL:
         L.hd_expand_embed.restype = i32
         L.hd_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, f32, i32, i32, vp, vp]
         L.hd_attn_fwd.restype = i32
+        L.hd_attn_fwd_final_stream.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, f32, i32,
+                                               i32, vp, vp]
+        L.hd_attn_fwd_final_stream.restype = i32
         L.hd_attn_decode.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, f32, i32, i32,
                                      vp, sz, vp, vp]
         L.hd_attn_decode.restype = i32
@@ -188,6 +192,40 @@ def hd_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n: int, mode=
     _check("hd_attn_fwd", lib().hd_attn_fwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, L, n, Hq, Hkv, D, _MODES[mode], int(window),
         float(scale), _dt(q), _dt(out), _ptr(dev_status), _stream(stream)))
+    return (out, lse) if want_lse else out
+
+
+def hd_attn_fwd_final_stream(q_final: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n: int, mode="intra",
+                             window: int = 0, scale: float | None = None, out: torch.Tensor | None = None,
+                             out_dtype=None, lse: torch.Tensor | bool | None = None,
+                             dev_status: torch.Tensor | None = None, stream=None):
+    """Attention of the final-stream queries only (KV-mirror layers).
+
+    q_final [B, L, Hq, D], k/v [B, n*L, Hkv, D] -> O [B, L, Hq, D] (and lse
+    [B, Hq, L] float32 when asked): the rows of :func:`hd_attn_fwd` at the
+    positions i*n + n-1.
+    """
+    for t, nm in ((q_final, "q_final"), (k, "k"), (v, "v")):
+        _need(t, nm)
+    B, L, Hq, D = q_final.shape
+    Hkv = k.shape[2]
+    if k.shape != (B, n * L, Hkv, D) or v.shape != k.shape or k.dtype != q_final.dtype or v.dtype != q_final.dtype:
+        raise ValueError("q_final/k/v shapes or dtypes disagree")
+    if scale is None:
+        scale = D ** -0.5
+    if out is None:
+        out = torch.empty((B, L, Hq, D), dtype=out_dtype or q_final.dtype, device=q_final.device)
+    _need(out, "out")
+    if out.shape != q_final.shape:
+        raise ValueError("out has the wrong shape")
+    want_lse = lse is True or isinstance(lse, torch.Tensor)
+    if lse is True:
+        lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q_final.device)
+    elif lse is False:
+        lse = None
+    _check("hd_attn_fwd_final_stream", lib().hd_attn_fwd_final_stream(
+        _ptr(q_final), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, L, n, Hq, Hkv, D, _MODES[mode], int(window),
+        float(scale), _dt(q_final), _dt(out), _ptr(dev_status), _stream(stream)))
     return (out, lse) if want_lse else out
 
 

@@ -32,3 +32,12 @@ def test_headline_workload_numbers():
     assert abs(acc.attn_flops(1, 32768, 4, 64, 128, "intra", 4096) / 1e12 - 16.493) < 1e-3
     # decode: batch 64, n=4, 32768 tokens, 64/8 heads
     assert abs(acc.decode_bytes(64, 4, 32768, 64, 8, 128) / 1e9 - 34.37) < 0.01
+
+
+@pytest.mark.parametrize("L,n", [(7, 1), (6, 2), (5, 4), (9, 3)])
+@pytest.mark.parametrize("mode", ["intra", "cross"])
+@pytest.mark.parametrize("W", [0, 1, 3, 50])
+def test_final_stream_pairs_match_enumeration(L, n, mode, W):
+    pk = np.arange(n * L)
+    want = sum(int(np.count_nonzero(oracle.visible(i * n + n - 1, pk, n, mode, W))) for i in range(L))
+    assert acc.pairs_final_stream(L, n, mode, W) == want

@@ -378,3 +378,41 @@ def test_planted_gqa_and_transpose_mistakes_are_caught(monkeypatch):
     # swapped K and V
     O_swap, _ = oracle.attn(q, v, k, 1, "cross", 0, 0.3)
     assert np.max(np.abs(O_swap - ref)) > 1e-3
+
+
+# ------------------------------------------- final-stream queries (KV mirror)
+
+@pytest.mark.parametrize("n,mode,W", [(1, "cross", 0), (2, "intra", 0), (3, "cross", 0), (4, "intra", 3),
+                                      (4, "cross", 7), (2, "cross", 1)])
+def test_final_stream_rows_equal_full_attention_rows(n, mode, W):
+    """Each output row depends only on its own query, so the final-stream
+    call equals the full call's rows p = i*n + n-1 whatever the other queries
+    are."""
+    B, L, Hq, Hkv, D = 2, 6, 4, 2, 8
+    P = n * L
+    q, k, v = _qkv(B, P, Hq, Hkv, D, 1400 + n + W)
+    qf = np.ascontiguousarray(q[:, n - 1::n])
+    O, lse = oracle.attn(q, k, v, n, mode, W, 0.35)
+    Of, lf = oracle.attn_final_stream(qf, k, v, n, mode, W, 0.35)
+    np.testing.assert_allclose(Of, O[:, n - 1::n], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lf, lse[:, :, n - 1::n], rtol=0, atol=1e-13)
+
+
+def test_final_stream_intra_is_causal_attention_on_last_stream():
+    B, n, L, Hq, Hkv, D = 1, 3, 9, 2, 1, 8
+    q, k, v = _qkv(B, n * L, Hq, Hkv, D, 1500)
+    qf = np.ascontiguousarray(q[:, n - 1::n])
+    Of, _ = oracle.attn_final_stream(qf, k, v, n, "intra", 0, 0.5)
+    ks = np.ascontiguousarray(k[:, n - 1::n])
+    vs = np.ascontiguousarray(v[:, n - 1::n])
+    ref = _sdpa(qf, ks, vs, 0.5, causal=True)
+    np.testing.assert_allclose(Of, ref, rtol=0, atol=1e-12)
+
+
+def test_final_stream_cross_pair_count_equals_intra():
+    # Final-stream queries over all streams: sum_i n*(i+1) = n L(L+1)/2 pairs,
+    # the intra-layer count -- the saving of running only the final stream.
+    for n, L in [(2, 5), (4, 7)]:
+        pk = np.arange(n * L)
+        pairs = sum(int(np.count_nonzero(oracle.visible(i * n + n - 1, pk, n, "cross"))) for i in range(L))
+        assert pairs == n * L * (L + 1) // 2
