@@ -15,11 +15,12 @@
 // (cross: all n*G query rows that share it -- the cache is read once and
 // reused by every stream's queries; intra: the G query rows of one stream),
 // its token range is split across CTAs, and each CTA streams 64-token K/V
-// tiles through a 3-stage TMA pipeline (one producer warp) into four compute
-// warps.  Each warp takes 16 keys of every tile and runs QK^T and PV on the
-// warp-level tensor-core MMA (m16n8k16 bf16 -> f32) with an online softmax;
-// the warps' partial (max, sum, O) are merged in shared memory and written
-// to the workspace, and a small combine kernel merges the splits.
+// tiles through a 3-stage TMA pipeline (one producer warp) into the compute
+// warps: four per 16 query rows, each taking 16 keys of every tile, running
+// QK^T and PV on the warp-level tensor-core MMA (m16n8k16 bf16 -> f32) with
+// an online softmax that only rescales O when the row max rises by more than
+// 2^8.  The four warps' partial (max, sum, O) are merged in shared memory and
+// written to the workspace, and a small combine kernel merges the splits.
 #include "hd_common.cuh"
 #include "hd_launch.h"
 
@@ -28,7 +29,6 @@ namespace hd {
 namespace dec {
 constexpr int kTok = 64;        // tokens per K/V tile
 constexpr int kStages = 3;
-constexpr int kThreads = 160;   // 4 compute warps + 1 TMA warp
 constexpr int kRowsMax = 32;    // query rows per unit
 constexpr int kBox = kTok * 128;        // one 64-token x 128-byte TMA box
 constexpr int kD = 128;
@@ -118,11 +118,24 @@ __device__ __forceinline__ void dec_row(const DecUnit& x, const DecParams& p, in
   }
 }
 
+// Compute warps per CTA: one 16-row m-tile per group of four warps; the four
+// warps of a group split every 64-key tile into 16-key quarters.
 template <int MT>
-__global__ void __launch_bounds__(dec::kThreads, 2) decode_kernel(const __grid_constant__ CUtensorMap tmK,
-                                                               const __grid_constant__ CUtensorMap tmV,
-                                                               const DecParams p) {
+struct DecShape {
+  static constexpr int kCompute = 4 * MT;
+  static constexpr int kThreads = 32 * (kCompute + 1);
+};
+
+#ifndef HD_DEC_MT2_CTAS
+#define HD_DEC_MT2_CTAS 2
+#endif
+template <int MT>
+__global__ void __launch_bounds__(DecShape<MT>::kThreads, MT == 2 ? HD_DEC_MT2_CTAS : 2)
+    decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const DecParams p) {
   using namespace dec;
+  constexpr int kCompute = DecShape<MT>::kCompute;
+  constexpr int kThr = DecShape<MT>::kThreads;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -157,7 +170,7 @@ __global__ void __launch_bounds__(dec::kThreads, 2) decode_kernel(const __grid_c
     if (bad_T && split == 0) report(p.status, HD_ERR_INVALID_ARG);
     for (int i = 0; i < kStages; ++i) {
       mbar_init(full0 + 8 * i, 1);
-      mbar_init(empty0 + 8 * i, 4);
+      mbar_init(empty0 + 8 * i, kCompute);
     }
     *abort_flag = 0;
     *no_abort = 0;
@@ -166,7 +179,7 @@ __global__ void __launch_bounds__(dec::kThreads, 2) decode_kernel(const __grid_c
   // Q rows -> padded shared tile (rows >= R are zero).
   {
     __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(smem + kQOff);
-    for (int e = threadIdx.x; e < MT * 16 * (kD / 8); e += kThreads) {
+    for (int e = threadIdx.x; e < MT * 16 * (kD / 8); e += kThr) {
       const int r = e / (kD / 8), c8 = e - r * (kD / 8);
       uint4 val = make_uint4(0, 0, 0, 0);
       if (r < x.R) {
@@ -179,7 +192,7 @@ __global__ void __launch_bounds__(dec::kThreads, 2) decode_kernel(const __grid_c
   }
   __syncthreads();
 
-  if (warp == 4) {
+  if (warp == kCompute) {
     if (lane == 0 && ntiles > 0) {
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
@@ -211,33 +224,30 @@ __global__ void __launch_bounds__(dec::kThreads, 2) decode_kernel(const __grid_c
   }
 
   // ------------------------------------------------------ compute warps
+  const int mt = warp >> 2;        // this warp's 16-row m-tile
+  const int kq = warp & 3;         // this warp's key quarter of every tile
+  const int kw = kq * 16;
   const int g = lane >> 2, tq = lane & 3;
   const uint32_t qs = sbase + kQOff;
-  float o[MT][kD / 8][4];
-  float mrow[MT][2], lrow[MT][2];
+  float o[kD / 8][4];
 #pragma unroll
-  for (int mt = 0; mt < MT; ++mt) {
+  for (int nt = 0; nt < kD / 8; ++nt)
 #pragma unroll
-    for (int nt = 0; nt < kD / 8; ++nt)
+    for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+  // Running max (log2 units) and sum of the two rows this thread holds.  The
+  // max is only raised when a tile exceeds it by more than 2^8, so O is
+  // rarely rescaled; any reference max gives the same final O / l.
+  float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
+  int srow[2];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) o[mt][nt][e] = 0.f;
-    mrow[mt][0] = mrow[mt][1] = -INFINITY;
-    lrow[mt][0] = lrow[mt][1] = 0.f;
+  for (int hh = 0; hh < 2; ++hh) {
+    const int r = mt * 16 + g + hh * 8;
+    int s, h;
+    dec_row(x, p, x.r0 + min(r, x.R - 1), s, h);
+    srow[hh] = s;
   }
-  // Per-row stream index (cross) for the rows this thread holds.
-  int srow[MT][2];
-#pragma unroll
-  for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int r = mt * 16 + g + hh * 8;
-      int s, h;
-      dec_row(x, p, x.r0 + min(r, x.R - 1), s, h);
-      srow[mt][hh] = s;
-    }
 
   bool ok = true;
-  const int kw = warp * 16;  // this warp's keys within a tile
   for (int t = 0; t < ntiles; ++t) {
     const int st = t % kStages;
     const bool got = mbar_wait(full0 + 8 * st, (t / kStages) & 1, abort_flag);
@@ -247,91 +257,84 @@ __global__ void __launch_bounds__(dec::kThreads, 2) decode_kernel(const __grid_c
     const uint32_t kbox = sbase + kStageOff + st * kStageBytes;
     const uint32_t vbox = kbox + kHalf * kBox;
 
-    // S = Q K^T for this warp's 16 keys.
-    float sc[MT][2][4];
+    // S = Q K^T for this warp's 16 rows x 16 keys.
+    float sc[2][4];
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
+    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sc[mt][nt][e] = 0.f;
+      for (int e = 0; e < 4; ++e) sc[nt][e] = 0.f;
 #pragma unroll
     for (int kk = 0; kk < kD / 16; ++kk) {
-      uint32_t b0, b1, b2, b3;
+      const int mi = lane >> 3, rr = lane & 7;
+      uint32_t b0, b1, b2, b3, a0, a1, a2, a3;
       {
-        const int mi = lane >> 3, rr = lane & 7;
         const int key = kw + rr + ((mi >> 1) << 3);
-        const int chunk = (kk & 3) * 2 + (mi & 1);
-        ldsm_x4(sw128(kbox + (kk >> 2) * kBox, key, chunk), b0, b1, b2, b3);
+        const int ch = (kk & 3) * 2 + (mi & 1);
+        ldsm_x4(sw128(kbox + (kk >> 2) * kBox, key, ch), b0, b1, b2, b3);
       }
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        uint32_t a0, a1, a2, a3;
-        const int mi = lane >> 3, rr = lane & 7;
+      {
         const int row = mt * 16 + rr + ((mi & 1) << 3);
         const int col = kk * 16 + ((mi >> 1) << 3);
         ldsm_x4(qs + (row * kQPitch + col) * 2, a0, a1, a2, a3);
-        mma_bf16_16816(sc[mt][0], a0, a1, a2, a3, b0, b1);
-        mma_bf16_16816(sc[mt][1], a0, a1, a2, a3, b2, b3);
       }
+      mma_bf16_16816(sc[0], a0, a1, a2, a3, b0, b1);
+      mma_bf16_16816(sc[1], a0, a1, a2, a3, b2, b3);
     }
 
-    // Scale, mask, online softmax.
+    // Scale, mask, online softmax with lazy rescaling.
     const bool edge = (j0 + kTok > T - 1) || (p.W > 0);
-    uint32_t pa[MT][4];
+    uint32_t pa[4];
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
+    for (int hh = 0; hh < 2; ++hh) {
+      float mx = -INFINITY;
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        float mx = -INFINITY;
+      for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            float y = sc[mt][nt][hh * 2 + e] * p.scale_log2;
-            if (edge) {
-              const int j = j0 + kw + nt * 8 + tq * 2 + e;
-              bool vis;
-              if (p.cross) {
-                const int64_t pq = static_cast<int64_t>(T - 1) * p.n + srow[mt][hh];
-                const int64_t pk = static_cast<int64_t>(j) * p.n + sp;
-                vis = pk <= pq && (p.W <= 0 || pq - pk < p.W);
-              } else {
-                vis = j <= T - 1 && (p.W <= 0 || T - 1 - j < p.W);
-              }
-              if (!vis) y = -INFINITY;
+        for (int e = 0; e < 2; ++e) {
+          float y = sc[nt][hh * 2 + e] * p.scale_log2;
+          if (edge) {
+            const int j = j0 + kw + nt * 8 + tq * 2 + e;
+            bool vis;
+            if (p.cross) {
+              const int64_t pq = static_cast<int64_t>(T - 1) * p.n + srow[hh];
+              const int64_t pk = static_cast<int64_t>(j) * p.n + sp;
+              vis = pk <= pq && (p.W <= 0 || pq - pk < p.W);
+            } else {
+              vis = j <= T - 1 && (p.W <= 0 || T - 1 - j < p.W);
             }
-            sc[mt][nt][hh * 2 + e] = y;
-            mx = fmaxf(mx, y);
+            if (!vis) y = -INFINITY;
           }
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        const float mold = mrow[mt][hh];
-        const float mnew = fmaxf(mold, mx);
-        const float alpha = (mold == -INFINITY) ? 0.f : ex2(mold - mnew);
-        const float mu = (mnew == -INFINITY) ? 0.f : mnew;
-        mrow[mt][hh] = mnew;
-        float ls = 0.f;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float pv = ex2(sc[mt][nt][hh * 2 + e] - mu);
-            sc[mt][nt][hh * 2 + e] = pv;
-            ls += pv;
-          }
-        lrow[mt][hh] = lrow[mt][hh] * alpha + ls;
+          sc[nt][hh * 2 + e] = y;
+          mx = fmaxf(mx, y);
+        }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      if (mx > mrow[hh] + 8.0f) {  // uniform across the quad holding the row
+        const float alpha = ex2(mrow[hh] - mx);  // mrow = -inf -> 0
+        lrow[hh] *= alpha;
 #pragma unroll
         for (int nt = 0; nt < kD / 8; ++nt) {
-          o[mt][nt][hh * 2 + 0] *= alpha;
-          o[mt][nt][hh * 2 + 1] *= alpha;
+          o[nt][hh * 2 + 0] *= alpha;
+          o[nt][hh * 2 + 1] *= alpha;
         }
+        mrow[hh] = mx;
       }
-      pa[mt][0] = pack_bf16x2(sc[mt][0][0], sc[mt][0][1]);
-      pa[mt][1] = pack_bf16x2(sc[mt][0][2], sc[mt][0][3]);
-      pa[mt][2] = pack_bf16x2(sc[mt][1][0], sc[mt][1][1]);
-      pa[mt][3] = pack_bf16x2(sc[mt][1][2], sc[mt][1][3]);
+      const float mu = (mrow[hh] == -INFINITY) ? 0.f : mrow[hh];
+      float ls = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float pv = ex2(sc[nt][hh * 2 + e] - mu);
+          sc[nt][hh * 2 + e] = pv;
+          ls += pv;
+        }
+      lrow[hh] += ls;
     }
+    pa[0] = pack_bf16x2(sc[0][0], sc[0][1]);
+    pa[1] = pack_bf16x2(sc[0][2], sc[0][3]);
+    pa[2] = pack_bf16x2(sc[1][0], sc[1][1]);
+    pa[3] = pack_bf16x2(sc[1][2], sc[1][3]);
 
     // O += P V.
 #pragma unroll
@@ -339,13 +342,10 @@ __global__ void __launch_bounds__(dec::kThreads, 2) decode_kernel(const __grid_c
       uint32_t b0, b1, b2, b3;
       const int mi = lane >> 3, rr = lane & 7;
       const int key = kw + rr + ((mi & 1) << 3);
-      const int chunk = ((2 * c) & 7) + (mi >> 1);
-      ldsm_x4_t(sw128(vbox + (c >> 2) * kBox, key, chunk), b0, b1, b2, b3);
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        mma_bf16_16816(o[mt][2 * c], pa[mt][0], pa[mt][1], pa[mt][2], pa[mt][3], b0, b1);
-        mma_bf16_16816(o[mt][2 * c + 1], pa[mt][0], pa[mt][1], pa[mt][2], pa[mt][3], b2, b3);
-      }
+      const int ch = ((2 * c) & 7) + (mi >> 1);
+      ldsm_x4_t(sw128(vbox + (c >> 2) * kBox, key, ch), b0, b1, b2, b3);
+      mma_bf16_16816(o[2 * c], pa[0], pa[1], pa[2], pa[3], b0, b1);
+      mma_bf16_16816(o[2 * c + 1], pa[0], pa[1], pa[2], pa[3], b2, b3);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty0 + 8 * st);
@@ -357,40 +357,37 @@ __global__ void __launch_bounds__(dec::kThreads, 2) decode_kernel(const __grid_c
 
   // Quad-reduce the row sums.
 #pragma unroll
-  for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      float l = lrow[mt][hh];
-      l += __shfl_xor_sync(0xffffffffu, l, 1);
-      l += __shfl_xor_sync(0xffffffffu, l, 2);
-      lrow[mt][hh] = l;
-    }
+  for (int hh = 0; hh < 2; ++hh) {
+    float l = lrow[hh];
+    l += __shfl_xor_sync(0xffffffffu, l, 1);
+    l += __shfl_xor_sync(0xffffffffu, l, 2);
+    lrow[hh] = l;
+  }
 
-  // Merge the four warps through shared memory (stage buffers are idle now).
-  asm volatile("bar.sync 1, 128;" ::: "memory");
-  float* so = reinterpret_cast<float*>(smem + kStageOff);                 // [4][32][D]
-  float* sm = so + 4 * kRowsMax * kD;                                     // [4][32]
-  float* sl = sm + 4 * kRowsMax;                                          // [4][32]
+  // Merge the four key quarters of each m-tile through shared memory (the
+  // stage buffers are idle now).
+  asm volatile("bar.sync 1, %0;" ::"n"(32 * kCompute) : "memory");
+  float* so = reinterpret_cast<float*>(smem + kStageOff);  // [4 quarters][32 rows][D]
+  float* sm = so + 4 * kRowsMax * kD;                      // [4][32]
+  float* sl = sm + 4 * kRowsMax;                           // [4][32]
 #pragma unroll
-  for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int r = mt * 16 + g + hh * 8;
-      if (tq == 0) {
-        sm[warp * kRowsMax + r] = mrow[mt][hh];
-        sl[warp * kRowsMax + r] = lrow[mt][hh];
-      }
-#pragma unroll
-      for (int nt = 0; nt < kD / 8; ++nt) {
-        float2 v2 = make_float2(o[mt][nt][hh * 2], o[mt][nt][hh * 2 + 1]);
-        *reinterpret_cast<float2*>(so + (warp * kRowsMax + r) * kD + nt * 8 + tq * 2) = v2;
-      }
+  for (int hh = 0; hh < 2; ++hh) {
+    const int r = mt * 16 + g + hh * 8;
+    if (tq == 0) {
+      sm[kq * kRowsMax + r] = mrow[hh];
+      sl[kq * kRowsMax + r] = lrow[hh];
     }
-  asm volatile("bar.sync 1, 128;" ::: "memory");
+#pragma unroll
+    for (int nt = 0; nt < kD / 8; ++nt) {
+      float2 v2 = make_float2(o[nt][hh * 2], o[nt][hh * 2 + 1]);
+      *reinterpret_cast<float2*>(so + (kq * kRowsMax + r) * kD + nt * 8 + tq * 2) = v2;
+    }
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(32 * kCompute) : "memory");
   {
-    const int tid = threadIdx.x;  // 0..127
-    const int r = tid >> 2;       // 0..31
-    const int d0 = (tid & 3) * (kD / 4);
+    const int tid = threadIdx.x;   // 0 .. 32*kCompute-1
+    const int r = tid >> 3;        // 16*MT rows, 8 threads per row
+    const int d0 = (tid & 7) * (kD / 8);
     if (r < x.R) {
       float M = -INFINITY;
 #pragma unroll
@@ -407,8 +404,8 @@ __global__ void __launch_bounds__(dec::kThreads, 2) decode_kernel(const __grid_c
       const int64_t row = (static_cast<int64_t>(x.b) * p.n + s) * p.Hq + h;
       float* dst = p.ws_o + (static_cast<int64_t>(split) * rows_total + row) * kD + d0;
       const float inv = L > 0.f ? 1.f / L : 0.f;
-#pragma unroll 4
-      for (int d = 0; d < kD / 4; d += 4) {
+#pragma unroll
+      for (int d = 0; d < kD / 8; d += 4) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
@@ -424,7 +421,7 @@ __global__ void __launch_bounds__(dec::kThreads, 2) decode_kernel(const __grid_c
         acc.w *= inv;
         *reinterpret_cast<float4*>(dst + d) = acc;
       }
-      if ((tid & 3) == 0)
+      if ((tid & 7) == 0)
         p.ws_lse[static_cast<int64_t>(split) * rows_total + row] = L > 0.f ? M + __log2f(L) : -INFINITY;
     }
   }
@@ -545,11 +542,11 @@ cudaError_t launch_decode(const void* q, const void* kc, const void* vc, const i
   if (pl.mt == 2) {
     err = cudaFuncSetAttribute(decode_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, dec::kAlloc);
     if (err != cudaSuccess) return err;
-    decode_kernel<2><<<grid, dec::kThreads, dec::kAlloc, st>>>(mk, mv, p);
+    decode_kernel<2><<<grid, DecShape<2>::kThreads, dec::kAlloc, st>>>(mk, mv, p);
   } else {
     err = cudaFuncSetAttribute(decode_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, dec::kAlloc);
     if (err != cudaSuccess) return err;
-    decode_kernel<1><<<grid, dec::kThreads, dec::kAlloc, st>>>(mk, mv, p);
+    decode_kernel<1><<<grid, DecShape<1>::kThreads, dec::kAlloc, st>>>(mk, mv, p);
   }
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
