@@ -13,6 +13,8 @@ Sources (page "Hidden Decoding at Scale", WeLM blog):
     and Figure 2 masks (a) full cross-stream causal, (b) local cross-stream
     causal sliding window, (c) intra-stream causal  ->  :func:`visible`,
     :func:`attn`, :func:`attn_rows`.
+  * "Computational Cost" (the layers are trained through): the gradient of
+    the attention forward  ->  :func:`attn_bwd`.
   * "Persistent KV and the KV-mirror Saving" (only the final stream runs
     through the mirrored layers)  ->  :func:`attn_final_stream`.
   * "Persistent KV and the KV-mirror Saving" (a KV cache kept for every
@@ -34,6 +36,7 @@ from .hd_oracle import (  # noqa: F401
     final_stream_gather,
     attn,
     attn_rows,
+    attn_bwd,
     attn_final_stream,
     decode,
     decode_rows,

@@ -173,6 +173,48 @@ def attn(q, k, v, n, mode, window=0, scale=None):
     return O, lse
 
 
+def attn_bwd(q, k, v, dO, n, mode, window=0, scale=None):
+    """Gradient of the Stream-Factorized Attention forward, float64.
+
+    The pages train through these layers ("Computational Cost", "Near-Linear
+    Training Cost") but print no backward; its plain definition is the
+    derivative of  sum(dO * O)  with O = attn(q, k, v) for the Figure 2 mask.
+    Per (b, h), with S = scale * q k^T over the visible set, P = softmax(S):
+        dV = P^T dO,  dP = dO V^T,  dS = P * (dP - rowsum(P * dP)),
+        dQ = scale * dS K,  dK = scale * dS^T Q,
+    and dK, dV of a KV head summed over the query heads that read it.
+    Returns (dQ [B, nL, Hq, D], dK [B, nL, Hkv, D], dV [B, nL, Hkv, D]).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    dO = np.asarray(dO, dtype=np.float64)
+    B, P, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if Hq % Hkv or P % n or dO.shape != q.shape:
+        raise ValueError("bad shapes")
+    G = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    mask = visible_matrix(P // n, n, mode, window)
+    dQ = np.zeros((B, P, Hq, D))
+    dK = np.zeros((B, P, Hkv, D))
+    dV = np.zeros((B, P, Hkv, D))
+    for b in range(B):
+        for h in range(Hq):
+            kv = h // G
+            s = np.where(mask, scale * (q[b, :, h, :] @ k[b, :, kv, :].T), -np.inf)
+            e = np.exp(s - s.max(axis=-1, keepdims=True))
+            p = e / e.sum(axis=-1, keepdims=True)
+            g = dO[b, :, h, :]
+            dp = g @ v[b, :, kv, :].T
+            ds = p * (dp - (p * dp).sum(axis=-1, keepdims=True))
+            dV[b, :, kv, :] += p.T @ g
+            dQ[b, :, h, :] = scale * (ds @ k[b, :, kv, :])
+            dK[b, :, kv, :] += scale * (ds.T @ q[b, :, h, :])
+    return dQ, dK, dV
+
+
 def attn_rows(q, k, v, n, mode, rows, window=0, scale=None):
     """The same definition evaluated for selected output rows only.
 
