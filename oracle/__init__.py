@@ -37,6 +37,8 @@ from .hd_oracle import (  # noqa: F401
     attn,
     attn_rows,
     attn_bwd,
+    attn_bwd_dq_rows,
+    attn_bwd_dkv_rows,
     attn_final_stream,
     decode,
     decode_rows,

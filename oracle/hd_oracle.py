@@ -215,6 +215,64 @@ def attn_bwd(q, k, v, dO, n, mode, window=0, scale=None):
     return dQ, dK, dV
 
 
+def _bwd_row(q, k, v, dO, n, mode, b, h, p, G, window, scale):
+    """Row p of head h: (visible keys, P over them, dS over them)."""
+    P = k.shape[1]
+    kv = h // G
+    keys = np.arange(P)[visible(p, np.arange(P), n, mode, window)]
+    kk = np.asarray(k[b, keys, kv, :], dtype=np.float64)
+    vv = np.asarray(v[b, keys, kv, :], dtype=np.float64)
+    qv = np.asarray(q[b, p, h, :], dtype=np.float64)
+    g = np.asarray(dO[b, p, h, :], dtype=np.float64)
+    s = scale * (kk @ qv)
+    e = np.exp(s - s.max())
+    pr = e / e.sum()
+    dp = vv @ g
+    ds = pr * (dp - pr @ dp)
+    return keys, kk, pr, ds
+
+
+def attn_bwd_dq_rows(q, k, v, dO, n, mode, rows, window=0, scale=None):
+    """dQ of :func:`attn_bwd` for selected (b, h, p), one row at a time:
+    dQ[p] = scale * sum over p's visible keys of dS[p, p'] k[p'].
+    Inputs may be any array-likes indexable as q[b, p, h, :].  Returns [R, D]."""
+    Hq, D = q.shape[2], q.shape[3]
+    G = Hq // k.shape[2]
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    out = []
+    for (b, h, p) in rows:
+        _, kk, _, ds = _bwd_row(q, k, v, dO, n, mode, b, h, p, G, window, scale)
+        out.append(scale * (ds @ kk))
+    return np.array(out)
+
+
+def attn_bwd_dkv_rows(q, k, v, dO, n, mode, rows, window=0, scale=None):
+    """dK and dV of :func:`attn_bwd` for selected (b, kv head g, key p'),
+    summing over the query heads of the group and every query position p
+    that sees p': each such row's softmax and dS are formed over the row's
+    own visible keys.  Returns (dK [R, D], dV [R, D])."""
+    P, Hq, D = q.shape[1], q.shape[2], q.shape[3]
+    G = Hq // k.shape[2]
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    dks, dvs = [], []
+    pos = np.arange(P)
+    for (b, kvh, pk) in rows:
+        queries = pos[visible(pos, pk, n, mode, window)]
+        dk = np.zeros(D)
+        dv = np.zeros(D)
+        for h in range(kvh * G, (kvh + 1) * G):
+            for p in queries:
+                keys, _, pr, ds = _bwd_row(q, k, v, dO, n, mode, b, h, p, G, window, scale)
+                c = int(np.searchsorted(keys, pk))
+                dv += pr[c] * np.asarray(dO[b, p, h, :], dtype=np.float64)
+                dk += scale * ds[c] * np.asarray(q[b, p, h, :], dtype=np.float64)
+        dks.append(dk)
+        dvs.append(dv)
+    return np.array(dks), np.array(dvs)
+
+
 def attn_rows(q, k, v, n, mode, rows, window=0, scale=None):
     """The same definition evaluated for selected output rows only.
 

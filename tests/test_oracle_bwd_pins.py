@@ -136,3 +136,18 @@ def test_planted_bwd_mistakes_are_caught(kind):
     with pytest.raises(AssertionError):
         for mode, W in CASES:
             _check_fd(ns["attn_bwd"], mode, W)
+
+
+@pytest.mark.parametrize("mode,W", CASES)
+def test_bwd_row_functions_match_full_backward(mode, W):
+    n, L, Hq, Hkv, D = 3, 7, 4, 2, 6
+    q, k, v, dO = _inputs(2, L, n, Hq, Hkv, D, 51)
+    dQ, dK, dV = oracle.attn_bwd(q, k, v, dO, n, mode, W)
+    P = n * L
+    qrows = [(b, h, p) for b in range(2) for h in range(Hq) for p in (0, 1, P // 2, P - 1)]
+    got = oracle.attn_bwd_dq_rows(q, k, v, dO, n, mode, qrows, W)
+    np.testing.assert_allclose(got, np.array([dQ[b, p, h] for b, h, p in qrows]), rtol=1e-12, atol=1e-12)
+    krows = [(b, g, p) for b in range(2) for g in range(Hkv) for p in (0, 2, P // 2, P - 2, P - 1)]
+    gk, gv = oracle.attn_bwd_dkv_rows(q, k, v, dO, n, mode, krows, W)
+    np.testing.assert_allclose(gk, np.array([dK[b, p, g] for b, g, p in krows]), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(gv, np.array([dV[b, p, g] for b, g, p in krows]), rtol=1e-12, atol=1e-12)
