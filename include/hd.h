@@ -109,6 +109,42 @@ hd_status hd_attn_fwd_final_stream(const void* q_final, const void* k, const voi
                                    void* stream);
 
 /*
+ * Backward of hd_attn_fwd ("Computational Cost", "Near-Linear Training Cost":
+ * the layers are trained through; the pages print no backward, so this is
+ * the gradient of the forward's definition).  Given the forward's inputs, its
+ * output o and lse, and dO = dLoss/dO, per (b, query head h) with
+ * P = softmax(scale q k^T) over vis(p) and delta_p = <dO[p], o[p]>:
+ *   dv[p'] = sum_{h in group} sum_p P[p,p'] dO[p]
+ *   dS[p,p'] = P[p,p'] (<dO[p], v[p']> - delta_p)
+ *   dq[p]  = scale sum_{p'} dS[p,p'] k[p']
+ *   dk[p'] = scale sum_{h in group} sum_p dS[p,p'] q[p]
+ * (group = the Hq/Hkv query heads that read KV head p''s head).
+ *
+ *   q, o, dO [B, n*L, Hq,  D]  element type `dt`
+ *   k, v     [B, n*L, Hkv, D]  element type `dt`
+ *   lse      [B, Hq, n*L]      float32, as written by hd_attn_fwd (required)
+ *   dq       [B, n*L, Hq,  D]  element type `dt`, overwritten
+ *   dk, dv   [B, n*L, Hkv, D]  element type `dt`, overwritten
+ *   workspace: device scratch of at least hd_attn_bwd_workspace(...) bytes,
+ *              256-byte aligned, owned by the caller, no initialisation
+ *              needed, dead after the call completes.
+ * Same shape, mode, window and scale rules as hd_attn_fwd.  dt = HD_BF16
+ * runs tcgen05/TMEM tensor-core kernels (fp32 accumulate, one bf16 rounding
+ * of P and dS); dt = HD_F32 runs fp32 CUDA-core kernels.  Output buffers must
+ * not overlap the inputs.
+ */
+hd_status hd_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                      const void* dO, const float* lse, void* dq, void* dk, void* dv,
+                      int B, int L, int n, int Hq, int Hkv, int D, hd_mode mode,
+                      int window, float scale, hd_dtype dt, void* workspace,
+                      size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/* Workspace bytes hd_attn_bwd needs for these sizes (0 on invalid sizes).
+ * It holds two floats per (b, query head, position), padded per stream to a
+ * multiple of 128 tokens. */
+size_t hd_attn_bwd_workspace(int B, int L, int n, int Hq, hd_mode mode);
+
+/*
  * Decode against the per-stream KV cache ("Persistent KV and the KV-mirror
  * Saving": a separate cache per stream; "Inference Throughput": the n streams
  * of a token are processed together in one pass).  For every b, the new

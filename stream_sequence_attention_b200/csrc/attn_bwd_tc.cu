@@ -1,0 +1,805 @@
+// Backward of Stream-Factorized Attention, bf16 in / f32 accumulate, on the
+// tcgen05 tensor cores and tensor memory of sm_100a.
+//
+// ("Hidden Decoding at Scale", "Stream-Factorized Attention", Figure 2; the
+// layers are trained through, "Computational Cost".)  Same stream views as
+// the forward: q/k/v/dO [B, ns*Ls, H, D] are read through 5-D TMA maps
+// (D, H, ns, Ls, B), so intra mode (ns = n) and cross mode (ns = 1, Ls = nL)
+// are the same kernels and keys of other streams are never loaded.  P is
+// recomputed from the forward's lse; per-row (lse*log2e, delta = <dO, O>)
+// come from the preparation kernel, stream-major and padded to 128 tokens
+// with (+inf, 0) so padded queries contribute nothing.
+//
+// Two kernels, each owning its output (no atomics):
+//
+// attn_bwd_dkv_kernel -- unit = 128 keys of one (batch, stream, KV head);
+//   walks every query tile of every query head of the GQA group that sees
+//   the key block.  Tensor memory: S^T [0,128) dP^T [128,256) dV [256,256+D)
+//   dK [256+D,256+2D).  Per query tile:  S^T = K Q^T,  dP^T = V dO^T,
+//   P^T = 2^(S^T scale log2e - lse2) (masked to 0),  dS^T = P^T (dP^T - delta),
+//   dV += P^T dO,  dK += dS^T Q, with P^T and dS^T written back as bf16 over
+//   their own f32 columns and fed to the tensor core from tensor memory.
+//   MMA issue order  dV(t) S(t+1) | dK(t) dP(t+1): while the softmax warps
+//   compute P(t+1) the tensor core runs dK(t) and dP(t+1); while they compute
+//   dS(t+1) it runs dV(t+1) and S(t+2).  Overwrites are safe because one
+//   thread's tcgen05.mma operations execute in issue order.
+//
+// attn_bwd_dq_kernel -- unit = 128 queries of one (batch, stream, query head);
+//   walks the visible key tiles.  Tensor memory: S double-buffered [0,256),
+//   dP [256,384), dQ [384,384+D).  Per key tile:  S = Q K^T,  dP = dO V^T,
+//   dS = P (dP - delta) written as bf16 over S,  dQ += dS K.  MMA order
+//   dQ(t) dP(t+1) S(t+2): the next S is ready when the softmax warps finish
+//   the current tile.
+//
+// CTA = 10 warps: 0-7 elementwise (warp w owns tensor-memory lanes
+// 32*(w&3).. and the column half w>>2 of each 128-column tile), 8 TMA
+// producer, 9 MMA issuer.  Persistent, longest units first.  Every wait is
+// bounded (1 s), after which the kernel records HD_ERR_TIMEOUT, lets its
+// copies land, drains its MMAs and frees tensor memory.
+#include "hd_common.cuh"
+#include "hd_launch.h"
+
+namespace hd {
+
+namespace bw {
+constexpr int BT = 128;  // tile rows (queries or keys)
+constexpr int kThreads = 320;
+constexpr int kWarpTMA = 8;
+constexpr int kWarpMMA = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kLdBytes = BT * 8;  // (lse2, delta) of one query tile
+
+template <int D>
+struct Tile {
+  static constexpr int KB = D / 64;     // 128-byte column blocks per row
+  static constexpr int BLK = BT * 128;  // one 128-row x 128-byte block
+  static constexpr int TILE = BLK * KB;
+};
+
+// dK/dV kernel: K, V resident per unit; Q (+ its lse/delta) and dO in 2 stages.
+template <int D>
+struct LayKV {
+  using T = Tile<D>;
+  static constexpr int QST = 2;
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = K_OFF + T::TILE;
+  static constexpr int Q_OFF = V_OFF + T::TILE;
+  static constexpr int O_OFF = Q_OFF + QST * T::TILE;
+  static constexpr int LD_OFF = O_OFF + QST * T::TILE;
+  static constexpr int BAR_OFF = LD_OFF + QST * kLdBytes;
+  static constexpr int B_KVFULL = 0, B_KVEMPTY = 1, B_QFULL = 2, B_QEMPTY = B_QFULL + QST,
+                       B_OFULL = B_QEMPTY + QST, B_OEMPTY = B_OFULL + QST, B_SFULL = B_OEMPTY + QST,
+                       B_DPFULL = B_SFULL + 1, B_PFULL = B_DPFULL + 1, B_DSFULL = B_PFULL + 1,
+                       B_ACCFULL = B_DSFULL + 1, B_ACCEMPTY = B_ACCFULL + 1, B_DRAIN = B_ACCEMPTY + 1,
+                       NBAR = B_DRAIN + 1;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int ALLOC = MISC_OFF + 16 + 1024;
+};
+
+// dQ kernel: Q, dO resident per unit; K in 3 stages, V in 2.
+template <int D>
+struct LayQ {
+  using T = Tile<D>;
+  static constexpr int KST = 3, VST = 2;
+  static constexpr int Q_OFF = 0;
+  static constexpr int O_OFF = Q_OFF + T::TILE;
+  static constexpr int K_OFF = O_OFF + T::TILE;
+  static constexpr int V_OFF = K_OFF + KST * T::TILE;
+  static constexpr int BAR_OFF = V_OFF + VST * T::TILE;
+  static constexpr int B_QFULL = 0, B_QEMPTY = 1, B_KFULL = 2, B_KEMPTY = B_KFULL + KST,
+                       B_VFULL = B_KEMPTY + KST, B_VEMPTY = B_VFULL + VST, B_SFULL = B_VEMPTY + VST,
+                       B_DPFULL = B_SFULL + 2, B_DSFULL = B_DPFULL + 1, B_ACCFULL = B_DSFULL + 1,
+                       B_ACCEMPTY = B_ACCFULL + 1, B_DRAIN = B_ACCEMPTY + 1, NBAR = B_DRAIN + 1;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int ALLOC = MISC_OFF + 16 + 1024;
+};
+}  // namespace bw
+
+struct BwParams {
+  const float2* ws;  // (lse2, delta), stream-major, padded
+  void* dq;
+  void* dk;
+  void* dv;
+  int32_t* status;
+  int B, ns, Lq, Lpad, Hq, Hkv, W;
+  int nblk;  // 128-token blocks per stream
+  float scale_log2, scale;
+  int total_units;
+};
+
+// dK/dV unit: key block ascending (causal: the first blocks see the most
+// query tiles), then (b, s, kvh).
+struct KvUnit {
+  int b, s, kvh, kblk, qt_lo, nqt;
+};
+__device__ __forceinline__ KvUnit kv_unit(int u, const BwParams& p) {
+  const int per = p.B * p.ns * p.Hkv;
+  KvUnit x;
+  x.kblk = u / per;
+  int rem = u - x.kblk * per;
+  x.kvh = rem % p.Hkv;
+  rem /= p.Hkv;
+  x.s = rem % p.ns;
+  x.b = rem / p.ns;
+  const int k0 = x.kblk * bw::BT;
+  x.qt_lo = x.kblk;  // queries >= first key of the block
+  const int qt_hi = p.W > 0 ? min(p.nblk - 1, (k0 + bw::BT - 1 + p.W - 1) / bw::BT) : p.nblk - 1;
+  x.nqt = qt_hi - x.qt_lo + 1;
+  return x;
+}
+
+// dQ unit: query block descending (causal: the last blocks see the most key
+// tiles), then (b, s, h).
+struct QUnit {
+  int b, s, h, qblk, kt_lo, nkt;
+};
+__device__ __forceinline__ QUnit q_unit(int u, const BwParams& p) {
+  const int per = p.B * p.ns * p.Hq;
+  QUnit x;
+  const int qi = u / per;
+  int rem = u - qi * per;
+  x.qblk = p.nblk - 1 - qi;
+  x.h = rem % p.Hq;
+  rem /= p.Hq;
+  x.s = rem % p.ns;
+  x.b = rem / p.ns;
+  const int q0 = x.qblk * bw::BT;
+  x.kt_lo = p.W > 0 ? max(0, q0 - p.W + 1) / bw::BT : 0;
+  x.nkt = x.qblk - x.kt_lo + 1;
+  return x;
+}
+
+// acc(tmem d) (+)= A(smem, K-major, 128 rows) * B(smem, K-major, 128 rows)^T
+// over the D-long reduction: the S-type products (S, dP, S^T, dP^T).
+template <int D>
+__device__ __forceinline__ void mma_rows_rows(uint32_t d, uint32_t a_smem, uint32_t b_smem) {
+  using T = bw::Tile<D>;
+  constexpr uint32_t id = idesc_bf16_f32(bw::BT, bw::BT, false, false);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * T::BLK + (kk & 3) * 32;
+    mma_ss(d, smem_desc_sw128(a_smem + off, 16, 1024), smem_desc_sw128(b_smem + off, 16, 1024), id,
+           kk > 0 ? 1u : 0u);
+  }
+}
+
+// acc(tmem d, 128 x D) (+)= A(tmem, 128 x 128 bf16, packed by column halves:
+// elements [64h, 64h+64) in columns [a + 64h, a + 64h + 32)) * B(smem tile
+// [128 rows][D], MN-major): the dV, dK and dQ products.
+template <int D>
+__device__ __forceinline__ void mma_tmem_rows(uint32_t d, uint32_t a_tmem, uint32_t b_smem, bool acc) {
+  using T = bw::Tile<D>;
+  constexpr uint32_t id = idesc_bf16_f32(bw::BT, D, false, true);
+#pragma unroll
+  for (int kk = 0; kk < bw::BT / 16; ++kk) {
+    const uint64_t bdesc = smem_desc_sw128(b_smem + kk * 2048, T::BLK, 1024);
+    mma_ts(d, a_tmem + 64 * (kk >> 2) + 8 * (kk & 3), bdesc, id, (acc || kk > 0) ? 1u : 0u);
+  }
+}
+
+// Store 64 f32 values of one row as bf16 (scaled) to 16-byte-aligned global memory.
+__device__ __forceinline__ void store_row64_bf16(__nv_bfloat16* dst, const uint32_t (&a)[32], const uint32_t (&b)[32],
+                                                 float mul) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    uint4 w;
+    w.x = pack_bf16x2(__uint_as_float(a[8 * e + 0]) * mul, __uint_as_float(a[8 * e + 1]) * mul);
+    w.y = pack_bf16x2(__uint_as_float(a[8 * e + 2]) * mul, __uint_as_float(a[8 * e + 3]) * mul);
+    w.z = pack_bf16x2(__uint_as_float(a[8 * e + 4]) * mul, __uint_as_float(a[8 * e + 5]) * mul);
+    w.w = pack_bf16x2(__uint_as_float(a[8 * e + 6]) * mul, __uint_as_float(a[8 * e + 7]) * mul);
+    d4[e] = w;
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    uint4 w;
+    w.x = pack_bf16x2(__uint_as_float(b[8 * e + 0]) * mul, __uint_as_float(b[8 * e + 1]) * mul);
+    w.y = pack_bf16x2(__uint_as_float(b[8 * e + 2]) * mul, __uint_as_float(b[8 * e + 3]) * mul);
+    w.z = pack_bf16x2(__uint_as_float(b[8 * e + 4]) * mul, __uint_as_float(b[8 * e + 5]) * mul);
+    w.w = pack_bf16x2(__uint_as_float(b[8 * e + 6]) * mul, __uint_as_float(b[8 * e + 7]) * mul);
+    d4[4 + e] = w;
+  }
+}
+
+// Write columns [c0, c0 + D/2) of a 128 x D f32 accumulator row (this
+// thread's lane) to dst as bf16 times mul.
+template <int D>
+__device__ __forceinline__ void acc_half_to_global(uint32_t taddr, __nv_bfloat16* dst, float mul, bool ok) {
+  if constexpr (D == 128) {
+    uint32_t a[32], b[32];
+    tmem_ld32(taddr, a);
+    tmem_ld32(taddr + 32, b);
+    tmem_wait_ld();
+    if (ok) store_row64_bf16(dst, a, b, mul);
+  } else {
+    uint32_t a[32];
+    tmem_ld32(taddr, a);
+    tmem_wait_ld();
+    if (ok) {
+      uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        uint4 w;
+        w.x = pack_bf16x2(__uint_as_float(a[8 * e + 0]) * mul, __uint_as_float(a[8 * e + 1]) * mul);
+        w.y = pack_bf16x2(__uint_as_float(a[8 * e + 2]) * mul, __uint_as_float(a[8 * e + 3]) * mul);
+        w.z = pack_bf16x2(__uint_as_float(a[8 * e + 4]) * mul, __uint_as_float(a[8 * e + 5]) * mul);
+        w.w = pack_bf16x2(__uint_as_float(a[8 * e + 6]) * mul, __uint_as_float(a[8 * e + 7]) * mul);
+        d4[e] = w;
+      }
+    }
+  }
+}
+
+// ======================================================= dK / dV kernel
+
+template <int D>
+__global__ void __launch_bounds__(bw::kThreads, 1)
+    attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                        const BwParams p) {
+  using Lay = bw::LayKV<D>;
+  using T = bw::Tile<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto bar = [&](int i) -> uint32_t { return sbase + Lay::BAR_OFF + 8 * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::MISC_OFF + 4);
+  volatile int* no_abort = reinterpret_cast<volatile int*>(smem + Lay::MISC_OFF + 8);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int G = p.Hq / p.Hkv;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(Lay::B_KVFULL), 1);
+    mbar_init(bar(Lay::B_KVEMPTY), 1);
+    for (int i = 0; i < Lay::QST; ++i) {
+      mbar_init(bar(Lay::B_QFULL + i), 1);
+      mbar_init(bar(Lay::B_QEMPTY + i), 1);
+      mbar_init(bar(Lay::B_OFULL + i), 1);
+      mbar_init(bar(Lay::B_OEMPTY + i), 1);
+    }
+    mbar_init(bar(Lay::B_SFULL), 1);
+    mbar_init(bar(Lay::B_DPFULL), 1);
+    mbar_init(bar(Lay::B_PFULL), 256);
+    mbar_init(bar(Lay::B_DSFULL), 256);
+    mbar_init(bar(Lay::B_ACCFULL), 1);
+    mbar_init(bar(Lay::B_ACCEMPTY), 256);
+    mbar_init(bar(Lay::B_DRAIN), 1);
+    *abort_flag = 0;
+    *no_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == bw::kWarpTMA && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmO);
+  }
+  if (warp == bw::kWarpMMA) {
+    tmem_alloc(smem_u32(tmem_slot), bw::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  auto fail = [&]() {
+    *abort_flag = 1;
+    report(p.status, HD_ERR_TIMEOUT);
+  };
+
+  if (warp == bw::kWarpTMA) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int t = 0, ul = 0, kv_issued = 0;
+      int q_issued[Lay::QST] = {}, o_issued[Lay::QST] = {};
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++ul) {
+        const KvUnit x = kv_unit(u, p);
+        if (!mbar_wait(bar(Lay::B_KVEMPTY), (ul & 1) ^ 1, abort_flag)) { ok = false; break; }
+        mbar_arrive_expect_tx(bar(Lay::B_KVFULL), 2 * T::TILE);
+#pragma unroll
+        for (int kb = 0; kb < T::KB; ++kb) {
+          tma_load_5d(sbase + Lay::K_OFF + kb * T::BLK, &tmK, bar(Lay::B_KVFULL), kb * 64, x.kvh, x.s,
+                      x.kblk * bw::BT, x.b);
+          tma_load_5d(sbase + Lay::V_OFF + kb * T::BLK, &tmV, bar(Lay::B_KVFULL), kb * 64, x.kvh, x.s,
+                      x.kblk * bw::BT, x.b);
+        }
+        ++kv_issued;
+        const int nt = G * x.nqt;
+        for (int j = 0; j < nt; ++j, ++t) {
+          const int h = x.kvh * G + j / x.nqt;
+          const int qt = x.qt_lo + j % x.nqt;
+          const int st = t % Lay::QST;
+          const uint32_t ph = ((t / Lay::QST) & 1) ^ 1;
+          if (!mbar_wait(bar(Lay::B_QEMPTY + st), ph, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(bar(Lay::B_QFULL + st), T::TILE + bw::kLdBytes);
+#pragma unroll
+          for (int kb = 0; kb < T::KB; ++kb)
+            tma_load_5d(sbase + Lay::Q_OFF + st * T::TILE + kb * T::BLK, &tmQ, bar(Lay::B_QFULL + st), kb * 64, h,
+                        x.s, qt * bw::BT, x.b);
+          bulk_load(sbase + Lay::LD_OFF + st * bw::kLdBytes,
+                    p.ws + ((static_cast<int64_t>(x.b) * p.Hq + h) * p.ns + x.s) * p.Lpad + qt * bw::BT,
+                    bw::kLdBytes, bar(Lay::B_QFULL + st));
+          ++q_issued[st];
+          if (!mbar_wait(bar(Lay::B_OEMPTY + st), ph, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(bar(Lay::B_OFULL + st), T::TILE);
+#pragma unroll
+          for (int kb = 0; kb < T::KB; ++kb)
+            tma_load_5d(sbase + Lay::O_OFF + st * T::TILE + kb * T::BLK, &tmO, bar(Lay::B_OFULL + st), kb * 64, h,
+                        x.s, qt * bw::BT, x.b);
+          ++o_issued[st];
+        }
+      }
+      if (!ok) {
+        fail();
+        if (kv_issued) mbar_wait(bar(Lay::B_KVFULL), (kv_issued - 1) & 1, no_abort);
+        for (int i = 0; i < Lay::QST; ++i) {
+          if (q_issued[i]) mbar_wait(bar(Lay::B_QFULL + i), (q_issued[i] - 1) & 1, no_abort);
+          if (o_issued[i]) mbar_wait(bar(Lay::B_OFULL + i), (o_issued[i] - 1) & 1, no_abort);
+        }
+      }
+    }
+  } else if (warp == bw::kWarpMMA) {
+    // ---------------------------------------------------------------- MMA
+    // Per tile t:  [P(t) ready] dV(t) S(t+1)  [dS(t) ready] dK(t) dP(t+1).
+    if (lane == 0) {
+      const uint32_t tS = tmem, tDP = tmem + 128, tDV = tmem + 256, tDK = tmem + 256 + D;
+      int t = 0, ul = 0;
+      bool ok = true;
+      auto issue_S = [&](int tt) {
+        const int st = tt % Lay::QST;
+        mma_rows_rows<D>(tS, sbase + Lay::K_OFF, sbase + Lay::Q_OFF + st * T::TILE);
+        tc_commit(bar(Lay::B_SFULL));
+      };
+      auto issue_dP = [&](int tt) {
+        const int st = tt % Lay::QST;
+        mma_rows_rows<D>(tDP, sbase + Lay::V_OFF, sbase + Lay::O_OFF + st * T::TILE);
+        tc_commit(bar(Lay::B_DPFULL));
+      };
+      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++ul) {
+        const KvUnit x = kv_unit(u, p);
+        const int nt = G * x.nqt;
+        if (!mbar_wait(bar(Lay::B_KVFULL), ul & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(bar(Lay::B_QFULL + t % Lay::QST), (t / Lay::QST) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        issue_S(t);
+        if (!mbar_wait(bar(Lay::B_OFULL + t % Lay::QST), (t / Lay::QST) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        issue_dP(t);
+        for (int j = 0; j < nt; ++j, ++t) {
+          const int st = t % Lay::QST;
+          const int stn = (t + 1) % Lay::QST;
+          const uint32_t phn = ((t + 1) / Lay::QST) & 1;
+          if (!mbar_wait(bar(Lay::B_PFULL), t & 1, abort_flag)) { ok = false; break; }
+          if (j == 0 && ul > 0 && !mbar_wait(bar(Lay::B_ACCEMPTY), (ul - 1) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          mma_tmem_rows<D>(tDV, tS, sbase + Lay::O_OFF + st * T::TILE, j > 0);
+          tc_commit(bar(Lay::B_OEMPTY + st));
+          if (j + 1 < nt) {
+            if (!mbar_wait(bar(Lay::B_QFULL + stn), phn, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            issue_S(t + 1);
+          }
+          if (!mbar_wait(bar(Lay::B_DSFULL), t & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          mma_tmem_rows<D>(tDK, tDP, sbase + Lay::Q_OFF + st * T::TILE, j > 0);
+          tc_commit(bar(Lay::B_QEMPTY + st));
+          if (j + 1 < nt) {
+            if (!mbar_wait(bar(Lay::B_OFULL + stn), phn, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            issue_dP(t + 1);
+          }
+        }
+        if (!ok) break;
+        tc_commit(bar(Lay::B_ACCFULL));
+        tc_commit(bar(Lay::B_KVEMPTY));
+      }
+      if (!ok) fail();
+      tc_commit(bar(Lay::B_DRAIN));
+      mbar_wait(bar(Lay::B_DRAIN), 0, no_abort);
+    }
+  } else {
+    // ------------------------------------------- elementwise + epilogue
+    const int ch = warp >> 2;  // column half
+    const int r = (warp & 3) * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_addr + 64 * ch;
+    const uint32_t tDP = tmem + lane_addr + 128 + 64 * ch;
+    const float sl2 = p.scale_log2;
+    int t = 0, ul = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++ul) {
+      const KvUnit x = kv_unit(u, p);
+      const int nt = G * x.nqt;
+      const int k0 = x.kblk * bw::BT;
+      const int jkey = k0 + r;  // this thread's key token
+      for (int j = 0; j < nt; ++j, ++t) {
+        const int st = t % Lay::QST;
+        const int q0 = (x.qt_lo + j % x.nqt) * bw::BT + 64 * ch;  // first query of this half
+        bool got = mbar_wait(bar(Lay::B_SFULL), t & 1, abort_flag);
+        got = got && mbar_wait(bar(Lay::B_QFULL + st), (t / Lay::QST) & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t sv[64];
+        tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        const float2* ld = reinterpret_cast<const float2*>(smem + Lay::LD_OFF + st * bw::kLdBytes) + 64 * ch;
+        tmem_wait_ld();
+        const bool need_mask = (q0 < k0 + bw::BT - 1) || (p.W > 0 && q0 + 63 - k0 >= p.W);
+        float pv[64];
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float a = fmaf(__uint_as_float(sv[c]), sl2, -ld[c].x);
+          pv[c] = ex2(a);
+        }
+        if (need_mask) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const int i = q0 + c;
+            if (i < jkey || (p.W > 0 && i - jkey >= p.W)) pv[c] = 0.f;
+          }
+        }
+        {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
+          tmem_st16(tS, pk);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(pv[32 + 2 * e], pv[32 + 2 * e + 1]);
+          tmem_st16(tS + 16, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(Lay::B_PFULL));
+        got = mbar_wait(bar(Lay::B_DPFULL), t & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        tc_fence_after();
+        tmem_ld32(tDP, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(tDP + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_wait_ld();
+        {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c = 2 * e;
+            pk[e] = pack_bf16x2(pv[c] * (__uint_as_float(sv[c]) - ld[c].y),
+                                pv[c + 1] * (__uint_as_float(sv[c + 1]) - ld[c + 1].y));
+          }
+          tmem_st16(tDP, pk);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c = 32 + 2 * e;
+            pk[e] = pack_bf16x2(pv[c] * (__uint_as_float(sv[c]) - ld[c].y),
+                                pv[c + 1] * (__uint_as_float(sv[c + 1]) - ld[c + 1].y));
+          }
+          tmem_st16(tDP + 16, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(Lay::B_DSFULL));
+      }
+      if (!ok) break;
+      // Epilogue: dV and scale*dK rows of this unit's keys.
+      const bool got = mbar_wait(bar(Lay::B_ACCFULL), ul & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      tc_fence_after();
+      const bool row_ok = jkey < p.Lq;
+      const int64_t orow =
+          ((static_cast<int64_t>(x.b) * p.ns * p.Lq + static_cast<int64_t>(row_ok ? jkey : 0) * p.ns + x.s) * p.Hkv +
+           x.kvh) * D + ch * (D / 2);
+      acc_half_to_global<D>(tmem + lane_addr + 256 + ch * (D / 2), static_cast<__nv_bfloat16*>(p.dv) + orow, 1.f,
+                            row_ok);
+      acc_half_to_global<D>(tmem + lane_addr + 256 + D + ch * (D / 2), static_cast<__nv_bfloat16*>(p.dk) + orow,
+                            p.scale, row_ok);
+      tc_fence_before();
+      mbar_arrive(bar(Lay::B_ACCEMPTY));
+    }
+    if (!ok) fail();
+  }
+
+  __syncthreads();
+  if (warp == bw::kWarpMMA) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, bw::kTmemCols);
+  }
+}
+
+// ============================================================ dQ kernel
+
+template <int D>
+__global__ void __launch_bounds__(bw::kThreads, 1)
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                       const BwParams p) {
+  using Lay = bw::LayQ<D>;
+  using T = bw::Tile<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto bar = [&](int i) -> uint32_t { return sbase + Lay::BAR_OFF + 8 * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::MISC_OFF + 4);
+  volatile int* no_abort = reinterpret_cast<volatile int*>(smem + Lay::MISC_OFF + 8);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int G = p.Hq / p.Hkv;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(Lay::B_QFULL), 1);
+    mbar_init(bar(Lay::B_QEMPTY), 1);
+    for (int i = 0; i < Lay::KST; ++i) {
+      mbar_init(bar(Lay::B_KFULL + i), 1);
+      mbar_init(bar(Lay::B_KEMPTY + i), 1);
+    }
+    for (int i = 0; i < Lay::VST; ++i) {
+      mbar_init(bar(Lay::B_VFULL + i), 1);
+      mbar_init(bar(Lay::B_VEMPTY + i), 1);
+    }
+    mbar_init(bar(Lay::B_SFULL + 0), 1);
+    mbar_init(bar(Lay::B_SFULL + 1), 1);
+    mbar_init(bar(Lay::B_DPFULL), 1);
+    mbar_init(bar(Lay::B_DSFULL), 256);
+    mbar_init(bar(Lay::B_ACCFULL), 1);
+    mbar_init(bar(Lay::B_ACCEMPTY), 256);
+    mbar_init(bar(Lay::B_DRAIN), 1);
+    *abort_flag = 0;
+    *no_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == bw::kWarpTMA && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmO);
+  }
+  if (warp == bw::kWarpMMA) {
+    tmem_alloc(smem_u32(tmem_slot), bw::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  auto fail = [&]() {
+    *abort_flag = 1;
+    report(p.status, HD_ERR_TIMEOUT);
+  };
+
+  if (warp == bw::kWarpTMA) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int t = 0, ul = 0, q_issued = 0;
+      int k_issued[Lay::KST] = {}, v_issued[Lay::VST] = {};
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++ul) {
+        const QUnit x = q_unit(u, p);
+        const int kvh = x.h / G;
+        if (!mbar_wait(bar(Lay::B_QEMPTY), (ul & 1) ^ 1, abort_flag)) { ok = false; break; }
+        mbar_arrive_expect_tx(bar(Lay::B_QFULL), 2 * T::TILE);
+#pragma unroll
+        for (int kb = 0; kb < T::KB; ++kb) {
+          tma_load_5d(sbase + Lay::Q_OFF + kb * T::BLK, &tmQ, bar(Lay::B_QFULL), kb * 64, x.h, x.s, x.qblk * bw::BT,
+                      x.b);
+          tma_load_5d(sbase + Lay::O_OFF + kb * T::BLK, &tmO, bar(Lay::B_QFULL), kb * 64, x.h, x.s, x.qblk * bw::BT,
+                      x.b);
+        }
+        ++q_issued;
+        for (int j = 0; j < x.nkt; ++j, ++t) {
+          const int kt = x.kt_lo + j;
+          const int ks = t % Lay::KST;
+          if (!mbar_wait(bar(Lay::B_KEMPTY + ks), ((t / Lay::KST) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(bar(Lay::B_KFULL + ks), T::TILE);
+#pragma unroll
+          for (int kb = 0; kb < T::KB; ++kb)
+            tma_load_5d(sbase + Lay::K_OFF + ks * T::TILE + kb * T::BLK, &tmK, bar(Lay::B_KFULL + ks), kb * 64, kvh,
+                        x.s, kt * bw::BT, x.b);
+          ++k_issued[ks];
+          const int vs = t % Lay::VST;
+          if (!mbar_wait(bar(Lay::B_VEMPTY + vs), ((t / Lay::VST) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(bar(Lay::B_VFULL + vs), T::TILE);
+#pragma unroll
+          for (int kb = 0; kb < T::KB; ++kb)
+            tma_load_5d(sbase + Lay::V_OFF + vs * T::TILE + kb * T::BLK, &tmV, bar(Lay::B_VFULL + vs), kb * 64, kvh,
+                        x.s, kt * bw::BT, x.b);
+          ++v_issued[vs];
+        }
+      }
+      if (!ok) {
+        fail();
+        if (q_issued) mbar_wait(bar(Lay::B_QFULL), (q_issued - 1) & 1, no_abort);
+        for (int i = 0; i < Lay::KST; ++i)
+          if (k_issued[i]) mbar_wait(bar(Lay::B_KFULL + i), (k_issued[i] - 1) & 1, no_abort);
+        for (int i = 0; i < Lay::VST; ++i)
+          if (v_issued[i]) mbar_wait(bar(Lay::B_VFULL + i), (v_issued[i] - 1) & 1, no_abort);
+      }
+    }
+  } else if (warp == bw::kWarpMMA) {
+    // ---------------------------------------------------------------- MMA
+    // Unit start: S(t0) dP(t0) S(t0+1); per tile t: [dS(t) ready] dQ(t)
+    // dP(t+1) S(t+2).  S(t) lives in buffer t&1.
+    if (lane == 0) {
+      const uint32_t tDP = tmem + 256, tDQ = tmem + 384;
+      int t = 0, ul = 0;
+      bool ok = true;
+      auto issue_S = [&](int tt) -> bool {
+        const int ks = tt % Lay::KST;
+        if (!mbar_wait(bar(Lay::B_KFULL + ks), (tt / Lay::KST) & 1, abort_flag)) return false;
+        tc_fence_after();
+        mma_rows_rows<D>(tmem + (tt & 1) * 128, sbase + Lay::Q_OFF, sbase + Lay::K_OFF + ks * T::TILE);
+        tc_commit(bar(Lay::B_SFULL + (tt & 1)));
+        return true;
+      };
+      auto issue_dP = [&](int tt) -> bool {
+        const int vs = tt % Lay::VST;
+        if (!mbar_wait(bar(Lay::B_VFULL + vs), (tt / Lay::VST) & 1, abort_flag)) return false;
+        tc_fence_after();
+        mma_rows_rows<D>(tDP, sbase + Lay::O_OFF, sbase + Lay::V_OFF + vs * T::TILE);
+        tc_commit(bar(Lay::B_DPFULL));
+        tc_commit(bar(Lay::B_VEMPTY + vs));
+        return true;
+      };
+      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++ul) {
+        const QUnit x = q_unit(u, p);
+        const int nt = x.nkt;
+        if (!mbar_wait(bar(Lay::B_QFULL), ul & 1, abort_flag)) { ok = false; break; }
+        const int t0 = t;
+        if (!issue_S(t0) || !issue_dP(t0) || (nt > 1 && !issue_S(t0 + 1))) { ok = false; break; }
+        for (int j = 0; j < nt; ++j, ++t) {
+          if (!mbar_wait(bar(Lay::B_DSFULL), t & 1, abort_flag)) { ok = false; break; }
+          if (j == 0 && ul > 0 && !mbar_wait(bar(Lay::B_ACCEMPTY), (ul - 1) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          mma_tmem_rows<D>(tDQ, tmem + (t & 1) * 128, sbase + Lay::K_OFF + (t % Lay::KST) * T::TILE, j > 0);
+          tc_commit(bar(Lay::B_KEMPTY + t % Lay::KST));
+          if (j + 1 < nt && !issue_dP(t + 1)) { ok = false; break; }
+          if (j + 2 < nt && !issue_S(t + 2)) { ok = false; break; }
+        }
+        if (!ok) break;
+        tc_commit(bar(Lay::B_ACCFULL));
+        tc_commit(bar(Lay::B_QEMPTY));
+      }
+      if (!ok) fail();
+      tc_commit(bar(Lay::B_DRAIN));
+      mbar_wait(bar(Lay::B_DRAIN), 0, no_abort);
+    }
+  } else {
+    // ------------------------------------------- elementwise + epilogue
+    const int ch = warp >> 2;  // column half (keys [64ch, 64ch+64) of a tile)
+    const int r = (warp & 3) * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tDP = tmem + lane_addr + 256 + 64 * ch;
+    const float sl2 = p.scale_log2;
+    int t = 0, ul = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++ul) {
+      const QUnit x = q_unit(u, p);
+      const int iq = x.qblk * bw::BT + r;  // this thread's query token
+      const float2 ld = p.ws[((static_cast<int64_t>(x.b) * p.Hq + x.h) * p.ns + x.s) * p.Lpad + iq];
+      for (int j = 0; j < x.nkt; ++j, ++t) {
+        const int k0 = (x.kt_lo + j) * bw::BT + 64 * ch;  // first key of this half
+        const uint32_t tS = tmem + lane_addr + (t & 1) * 128 + 64 * ch;
+        bool got = mbar_wait(bar(Lay::B_SFULL + (t & 1)), (t >> 1) & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t sv[64];
+        tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_wait_ld();
+        const int qfirst = x.qblk * bw::BT;
+        const bool need_mask = (k0 + 63 > qfirst) || (p.W > 0 && k0 < qfirst + bw::BT - 1 - p.W + 1);
+        float pv[64];
+#pragma unroll
+        for (int c = 0; c < 64; ++c) pv[c] = ex2(fmaf(__uint_as_float(sv[c]), sl2, -ld.x));
+        if (need_mask) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const int jk = k0 + c;
+            if (jk > iq || (p.W > 0 && iq - jk >= p.W)) pv[c] = 0.f;
+          }
+        }
+        got = mbar_wait(bar(Lay::B_DPFULL), t & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        tc_fence_after();
+        tmem_ld32(tDP, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(tDP + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_wait_ld();
+        {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c = 2 * e;
+            pk[e] = pack_bf16x2(pv[c] * (__uint_as_float(sv[c]) - ld.y), pv[c + 1] * (__uint_as_float(sv[c + 1]) - ld.y));
+          }
+          tmem_st16(tS, pk);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c = 32 + 2 * e;
+            pk[e] = pack_bf16x2(pv[c] * (__uint_as_float(sv[c]) - ld.y), pv[c + 1] * (__uint_as_float(sv[c + 1]) - ld.y));
+          }
+          tmem_st16(tS + 16, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(Lay::B_DSFULL));
+      }
+      if (!ok) break;
+      const bool got = mbar_wait(bar(Lay::B_ACCFULL), ul & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      tc_fence_after();
+      const bool row_ok = iq < p.Lq;
+      const int64_t orow =
+          ((static_cast<int64_t>(x.b) * p.ns * p.Lq + static_cast<int64_t>(row_ok ? iq : 0) * p.ns + x.s) * p.Hq +
+           x.h) * D + ch * (D / 2);
+      acc_half_to_global<D>(tmem + lane_addr + 384 + ch * (D / 2), static_cast<__nv_bfloat16*>(p.dq) + orow, p.scale,
+                            row_ok);
+      tc_fence_before();
+      mbar_arrive(bar(Lay::B_ACCEMPTY));
+    }
+    if (!ok) fail();
+  }
+
+  __syncthreads();
+  if (warp == bw::kWarpMMA) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, bw::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------- host
+
+template <int D>
+static cudaError_t launch_bwd_tc_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                                   const CUtensorMap& mo, BwParams p, int kv_units, int q_units, int sms,
+                                   cudaStream_t st) {
+  cudaError_t err;
+  const int skv = bw::LayKV<D>::ALLOC, sq = bw::LayQ<D>::ALLOC;
+  err = cudaFuncSetAttribute(attn_bwd_dkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, skv);
+  if (err != cudaSuccess) return err;
+  err = cudaFuncSetAttribute(attn_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, sq);
+  if (err != cudaSuccess) return err;
+  p.total_units = kv_units;
+  attn_bwd_dkv_kernel<D><<<kv_units < sms ? kv_units : sms, bw::kThreads, skv, st>>>(mq, mk, mv, mo, p);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  p.total_units = q_units;
+  attn_bwd_dq_kernel<D><<<q_units < sms ? q_units : sms, bw::kThreads, sq, st>>>(mq, mk, mv, mo, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, const void* dO, const float2* ws,
+                               void* dq, void* dk, void* dv, const AttnGeom& g, int Hq, int Hkv, int D, int W,
+                               float scale, int32_t* status, int sms, cudaStream_t st) {
+  CUtensorMap mq, mk, mv, mo;
+  if (!encode_stream_view(&mq, q, g.B, g.Lq, g.ns, Hq, D) || !encode_stream_view(&mk, k, g.B, g.Lq, g.ns, Hkv, D) ||
+      !encode_stream_view(&mv, v, g.B, g.Lq, g.ns, Hkv, D) || !encode_stream_view(&mo, dO, g.B, g.Lq, g.ns, Hq, D))
+    return cudaErrorInvalidValue;
+  BwParams p;
+  p.ws = ws;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.status = status;
+  p.B = g.B;
+  p.ns = g.ns;
+  p.Lq = g.Lq;
+  p.Lpad = bwd_lpad(g.Lq);
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.W = W;
+  p.nblk = p.Lpad / bw::BT;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.scale = scale;
+  const int64_t kv_units = static_cast<int64_t>(p.nblk) * g.B * g.ns * Hkv;
+  const int64_t q_units = static_cast<int64_t>(p.nblk) * g.B * g.ns * Hq;
+  if (q_units <= 0) return cudaSuccess;
+  if (q_units > 0x7fffffff) return cudaErrorInvalidValue;
+  if (D == 64) return launch_bwd_tc_d<64>(mq, mk, mv, mo, p, (int)kv_units, (int)q_units, sms, st);
+  return launch_bwd_tc_d<128>(mq, mk, mv, mo, p, (int)kv_units, (int)q_units, sms, st);
+}
+
+}  // namespace hd

@@ -507,7 +507,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
 // ------------------------------------------------------------------- host
 
 // (D, H, ns, Ls, B) view of a [B, ns*Ls, H, D] bf16 tensor; box = 64 x 1 x 1 x 128 x 1.
-static bool encode_stream_view(CUtensorMap* m, const void* ptr, int B, int Ls, int ns, int H, int D) {
+bool encode_stream_view(CUtensorMap* m, const void* ptr, int B, int Ls, int ns, int H, int D) {
   EncodeTiledFn enc = get_encode_tiled();
   if (!enc) return false;
   const cuuint64_t dims[5] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)ns, (cuuint64_t)Ls, (cuuint64_t)B};

@@ -98,6 +98,24 @@ static hd_status check_attn_args(const void* q, const void* k, const void* v, vo
   return HD_OK;
 }
 
+// Regular (all-query) geometry of hd_attn_fwd for the given mode.
+static AttnGeom regular_geom(int B, int L, int n, hd_mode mode) {
+  const int P = n * L;
+  AttnGeom g;
+  g.B = B;
+  g.ns = mode == HD_INTRA ? n : 1;
+  g.Lq = mode == HD_INTRA ? L : P;
+  g.q_ns = g.ns;
+  g.kv_ns = g.ns;
+  g.Lk = g.Lq;
+  g.kv_stream = -1;
+  g.qstride = 1;
+  g.qoff = 0;
+  g.o_rows = P;
+  g.o_ns = g.ns;
+  return g;
+}
+
 static hd_status run_attn(const void* q, const void* k, const void* v, void* o, float* lse, const AttnGeom& g,
                           int Hq, int Hkv, int D, int window, float scale, hd_dtype in_dt, hd_dtype out_dt,
                           int32_t* dev_status, void* stream) {
@@ -120,19 +138,7 @@ hd_status hd_attn_fwd(const void* q, const void* k, const void* v, void* o, floa
   hd_status stt = check_attn_args(q, k, v, o, lse, B, L, n, Hq, Hkv, D, mode, window, scale, in_dt, out_dt);
   if (stt != HD_OK || B == 0) return stt;
   // Intra: n streams of L tokens, read in place.  Cross: one stream of n*L positions.
-  const int P = n * L;
-  AttnGeom g;
-  g.B = B;
-  g.ns = mode == HD_INTRA ? n : 1;
-  g.Lq = mode == HD_INTRA ? L : P;
-  g.q_ns = g.ns;
-  g.kv_ns = g.ns;
-  g.Lk = g.Lq;
-  g.kv_stream = -1;
-  g.qstride = 1;
-  g.qoff = 0;
-  g.o_rows = P;
-  g.o_ns = g.ns;
+  const AttnGeom g = regular_geom(B, L, n, mode);
   return run_attn(q, k, v, o, lse, g, Hq, Hkv, D, window, scale, in_dt, out_dt, dev_status, stream);
 }
 
@@ -165,6 +171,42 @@ hd_status hd_attn_fwd_final_stream(const void* q_final, const void* k, const voi
     g.qoff = n - 1;
   }
   return run_attn(q_final, k, v, o, lse, g, Hq, Hkv, D, window, scale, in_dt, out_dt, dev_status, stream);
+}
+
+size_t hd_attn_bwd_workspace(int B, int L, int n, int Hq, hd_mode mode) {
+  if (B < 1 || L < 1 || n < 1 || Hq < 1 || (mode != HD_INTRA && mode != HD_CROSS)) return 0;
+  if (static_cast<int64_t>(n) * L > (1ll << 30)) return 0;
+  const AttnGeom g = regular_geom(B, L, n, mode);
+  return static_cast<size_t>(B) * Hq * g.ns * bwd_lpad(g.Lq) * sizeof(float2);
+}
+
+hd_status hd_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                      void* dq, void* dk, void* dv, int B, int L, int n, int Hq, int Hkv, int D, hd_mode mode,
+                      int window, float scale, hd_dtype dt, void* workspace, size_t ws_bytes, int32_t* dev_status,
+                      void* stream) {
+  hd_status stt = check_attn_args(q, k, v, dq, nullptr, B, L, n, Hq, Hkv, D, mode, window, scale, dt, dt);
+  if (stt != HD_OK || B == 0) return stt;
+  if (!o || !dO || !lse || !dk || !dv || !workspace || !aligned16(o) || !aligned16(dO) || !aligned16(dk) ||
+      !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return HD_ERR_INVALID_ARG;
+  if (ws_bytes < hd_attn_bwd_workspace(B, L, n, Hq, mode)) return HD_ERR_INVALID_ARG;
+  const AttnGeom g = regular_geom(B, L, n, mode);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float2* ws = static_cast<float2*>(workspace);
+  const bool bf16 = dt == HD_BF16;
+  cudaError_t e = launch_bwd_prep(o, dO, lse, ws, g, Hq, D, bf16, st);
+  if (e != cudaSuccess) return HD_ERR_CUDA;
+  if (!bf16) {
+    if (static_cast<int64_t>(Hq) * g.ns > 65535 || g.B > 65535) return HD_ERR_UNSUPPORTED;
+    return cuda_status(launch_attn_bwd_f32(static_cast<const float*>(q), static_cast<const float*>(k),
+                                           static_cast<const float*>(v), static_cast<const float*>(dO), ws,
+                                           static_cast<float*>(dq), static_cast<float*>(dk), static_cast<float*>(dv),
+                                           g, Hq, Hkv, D, window, scale, st));
+  }
+  const int sms = sm_count();
+  if (sms <= 0) return HD_ERR_CUDA;
+  return cuda_status(
+      launch_attn_bwd_tc(q, k, v, dO, ws, dq, dk, dv, g, Hq, Hkv, D, window, scale, dev_status, sms, st));
 }
 
 size_t hd_attn_decode_workspace(int B, int n, int Lmax, int Hq, int Hkv, int D, hd_mode mode) {

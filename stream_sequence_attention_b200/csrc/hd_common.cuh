@@ -118,6 +118,15 @@ __device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* m,
       : "memory");
 }
 
+// Untiled bulk copy global -> shared (this CTA): both addresses 16-byte
+// aligned, bytes a multiple of 16; completion counted on `bar`.  No multicast.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
 // ----------------------------------------------------------------- tcgen05
 
 // Tensor-memory allocation (whole warp).  Writes the base address to *slot.

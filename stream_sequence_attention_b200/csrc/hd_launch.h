@@ -37,12 +37,33 @@ struct AttnGeom {
   int o_rows, o_ns;
 };
 
+// TMA view (D, H, ns, Ls, B) of a [B, ns*Ls, H, D] bf16 tensor with a
+// 64 x 1 x 1 x 128 x 1 box and 128-byte swizzle: one box is 128 tokens of one
+// stream and head, 64 features wide.
+bool encode_stream_view(CUtensorMap* m, const void* ptr, int B, int Ls, int ns, int H, int D);
+
 cudaError_t launch_attn_f32(const float* q, const float* k, const float* v, void* o, float* lse,
                             const AttnGeom& g, int Hq, int Hkv, int D, int W, float scale, bool out_bf16,
                             cudaStream_t st);
 cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o, float* lse, const AttnGeom& g,
                            int Hq, int Hkv, int D, int W, float scale, bool out_bf16, int32_t* status, int sms,
                            cudaStream_t st);
+
+// Backward.  Regular geometry only (qstride 1, qoff 0, kv_stream -1, the
+// key streams equal the query streams).  The workspace holds, per
+// (b, query head, stream s, token i), the pair (lse * log2 e, delta =
+// <dO, o>) as float2 at ((b*Hq + h)*ns + s)*Lpad + i, with Lpad = Lq rounded
+// up to 128 and the padding rows set to (+inf, 0) so they contribute nothing.
+constexpr int kBwdPad = 128;
+__host__ __device__ inline int bwd_lpad(int Lq) { return (Lq + kBwdPad - 1) / kBwdPad * kBwdPad; }
+cudaError_t launch_bwd_prep(const void* o, const void* dO, const float* lse, float2* ws, const AttnGeom& g, int Hq,
+                            int D, bool bf16, cudaStream_t st);
+cudaError_t launch_attn_bwd_f32(const float* q, const float* k, const float* v, const float* dO, const float2* ws,
+                                float* dq, float* dk, float* dv, const AttnGeom& g, int Hq, int Hkv, int D, int W,
+                                float scale, cudaStream_t st);
+cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, const void* dO, const float2* ws,
+                               void* dq, void* dk, void* dv, const AttnGeom& g, int Hq, int Hkv, int D, int W,
+                               float scale, int32_t* status, int sms, cudaStream_t st);
 
 // Decode work decomposition: units (one KV head of one sequence, and for
 // intra mode one stream), row groups of at most 32 query rows, token splits.

@@ -27,6 +27,8 @@ EXPORTS = (
     "hd_expand_embed",
     "hd_attn_fwd",
     "hd_attn_fwd_final_stream",
+    "hd_attn_bwd",
+    "hd_attn_bwd_workspace",
     "hd_attn_decode",
     "hd_attn_decode_workspace",
     "hd_attn_decode_noalloc",
@@ -61,6 +63,11 @@ def lib() -> ctypes.CDLL:
         L.hd_attn_fwd_final_stream.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, f32, i32,
                                                i32, vp, vp]
         L.hd_attn_fwd_final_stream.restype = i32
+        L.hd_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, f32,
+                                  i32, vp, sz, vp, vp]
+        L.hd_attn_bwd.restype = i32
+        L.hd_attn_bwd_workspace.argtypes = [i32, i32, i32, i32, i32]
+        L.hd_attn_bwd_workspace.restype = sz
         L.hd_attn_decode.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, f32, i32, i32,
                                      vp, sz, vp, vp]
         L.hd_attn_decode.restype = i32
@@ -227,6 +234,53 @@ def hd_attn_fwd_final_stream(q_final: torch.Tensor, k: torch.Tensor, v: torch.Te
         _ptr(q_final), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, L, n, Hq, Hkv, D, _MODES[mode], int(window),
         float(scale), _dt(q_final), _dt(out), _ptr(dev_status), _stream(stream)))
     return (out, lse) if want_lse else out
+
+
+def hd_attn_bwd_workspace(B: int, L: int, n: int, Hq: int, mode="intra") -> int:
+    return int(lib().hd_attn_bwd_workspace(B, L, n, Hq, _MODES[mode]))
+
+
+def hd_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, dO: torch.Tensor,
+                lse: torch.Tensor, n: int, mode="intra", window: int = 0, scale: float | None = None,
+                dq: torch.Tensor | None = None, dk: torch.Tensor | None = None, dv: torch.Tensor | None = None,
+                workspace: torch.Tensor | None = None, dev_status: torch.Tensor | None = None, stream=None):
+    """Backward of :func:`hd_attn_fwd`: returns (dq, dk, dv).
+
+    q/o/dO [B, n*L, Hq, D], k/v [B, n*L, Hkv, D] (one dtype), lse [B, Hq, n*L]
+    float32 from the forward.  ``workspace`` (uint8, at least
+    :func:`hd_attn_bwd_workspace` bytes) is allocated when not given.
+    """
+    for t, nm in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dO, "dO"), (lse, "lse")):
+        _need(t, nm)
+    B, P, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if k.shape != (B, P, Hkv, D) or v.shape != k.shape or o.shape != q.shape or dO.shape != q.shape:
+        raise ValueError("q/k/v/o/dO shapes disagree")
+    if any(t.dtype != q.dtype for t in (k, v, o, dO)):
+        raise ValueError("q/k/v/o/dO dtypes disagree")
+    if lse.shape != (B, Hq, P) or lse.dtype != torch.float32:
+        raise ValueError("lse must be float32 [B, Hq, n*L]")
+    if P % n:
+        raise ValueError("sequence length is not a multiple of n")
+    L = P // n
+    if scale is None:
+        scale = D ** -0.5
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for t, ref, nm in ((dq, q, "dq"), (dk, k, "dk"), (dv, v, "dv")):
+        _need(t, nm)
+        if t.shape != ref.shape or t.dtype != ref.dtype:
+            raise ValueError(f"{nm} has the wrong shape or dtype")
+    need = hd_attn_bwd_workspace(B, L, n, Hq, mode)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _need(workspace, "workspace")
+    _check("hd_attn_bwd", lib().hd_attn_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), B, L, n, Hq, Hkv, D,
+        _MODES[mode], int(window), float(scale), _dt(q), _ptr(workspace), workspace.numel(), _ptr(dev_status),
+        _stream(stream)))
+    return dq, dk, dv
 
 
 def hd_attn_decode_workspace(B: int, n: int, Lmax: int, Hq: int, Hkv: int, D: int, mode="intra") -> int:

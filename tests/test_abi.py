@@ -87,3 +87,28 @@ def test_bad_arguments_rejected_on_host(L):
     # empty work is a no-op that succeeds without a device
     assert L.hd_final_stream_gather(None, None, 0, 4, 2, 8, hd.HD_F32, None) == hd.HD_OK
     assert L.hd_expand_embed(None, None, None, 0, 4, 2, 10, 8, hd.HD_F32, None, None) == hd.HD_OK
+
+
+def test_bwd_workspace_and_bad_arguments(L):
+    from stream_sequence_attention_b200 import hd
+    vp = ctypes.c_void_p
+    fake = vp(0x10000)
+    # two floats per (b, head, stream, token), tokens padded to 128 per stream
+    assert L.hd_attn_bwd_workspace(2, 100, 4, 8, hd.HD_INTRA) == 2 * 8 * 4 * 128 * 8
+    assert L.hd_attn_bwd_workspace(2, 100, 4, 8, hd.HD_CROSS) == 2 * 8 * 1 * 512 * 8
+    assert L.hd_attn_bwd_workspace(0, 100, 4, 8, hd.HD_CROSS) == 0
+    assert L.hd_attn_bwd_workspace(1, 8, 2, 2, 7) == 0
+
+    def bwd(*, q=fake, lse=fake, ws=fake, ws_bytes=1 << 20, Hq=2, Hkv=2, D=64, mode=0, scale=0.1, dt=1, B=1):
+        return L.hd_attn_bwd(q, fake, fake, fake, fake, lse, fake, fake, fake, B, 8, 2, Hq, Hkv, D, mode, 0, scale,
+                             dt, ws, ws_bytes, None, None)
+    assert bwd(Hq=3) == hd.HD_ERR_INVALID_ARG
+    assert bwd(D=96) == hd.HD_ERR_UNSUPPORTED
+    assert bwd(mode=5) == hd.HD_ERR_INVALID_ARG
+    assert bwd(scale=-1.0) == hd.HD_ERR_INVALID_ARG
+    assert bwd(lse=None) == hd.HD_ERR_INVALID_ARG
+    assert bwd(ws=None) == hd.HD_ERR_INVALID_ARG
+    assert bwd(ws=vp(0x10010)) == hd.HD_ERR_INVALID_ARG  # workspace not 256-byte aligned
+    assert bwd(q=vp(0x10008)) == hd.HD_ERR_INVALID_ARG
+    assert bwd(ws_bytes=16) == hd.HD_ERR_INVALID_ARG
+    assert bwd(B=0) == hd.HD_OK
