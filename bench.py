@@ -1,7 +1,7 @@
 """Benchmark of the Hidden Decoding hot path on B200; prints ONE JSON line.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload intra|cross|long|decode] [--no-extras]
+                    [--workload intra|cross|long|decode|mirror|bwd|bwd_cross] [--no-extras]
 
 Default workload (intra): n=4 streams, L=4096 tokens (nL=16384), batch 2,
 32 query / 8 KV heads, head_dim 128, bf16.  One step is one pass of the
@@ -10,8 +10,9 @@ Zipf(1.1) ids) -> hd_attn_fwd (intra-stream, causal) -> hd_final_stream_gather
 (final-stream rows of the expanded [B, nL, 4096] sequence).  The metric is
 useful attention TFLOP/s (visible pairs x 4 x head_dim per second of step
 time); the decode workload (batch 64, 32768 tokens per stream, both modes) is
-reported alongside in GB/s against HBM, and the cross-stream layer cost in
-TFLOP/s.
+reported alongside in GB/s against HBM, and the cross-stream layer, the
+KV-mirror layer and the backward (dQ, dK, dV; useful FLOPs = pairs x 10 x D)
+in TFLOP/s.
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
 on the launching stream, with an L2 flush (a 512 MiB write) between steps
@@ -44,6 +45,8 @@ WORKLOADS = {
     "long": dict(B=1, n=4, L=32768, Hq=64, Hkv=8, D=128, mode="intra", W=4096, V=152064, dm=4096),
     "decode": dict(B=64, n=4, T=32768, Hq=64, Hkv=8, D=128),
     "mirror": dict(B=2, n=4, L=4096, Hq=32, Hkv=8, D=128, mode="cross", W=0, V=152064, dm=4096, final=True),
+    "bwd": dict(B=2, n=4, L=4096, Hq=32, Hkv=8, D=128, mode="intra", W=0, bwd=True),
+    "bwd_cross": dict(B=2, n=4, L=4096, Hq=32, Hkv=8, D=128, mode="cross", W=0, bwd=True),
 }
 NAMES = {
     "intra": "bf16 prefill, intra-stream, n=4 L=4096 B=2 32q/8kv D=128",
@@ -51,6 +54,8 @@ NAMES = {
     "long": "long-context intra-stream W=4096, n=4 L=32768 B=1 64q/8kv D=128",
     "decode": "decode B=64 n=4 ctx=32768 64q/8kv D=128, intra+cross",
     "mirror": "bf16 KV-mirror layer: final-stream queries, cross-stream keys, n=4 L=4096 B=2 32q/8kv D=128",
+    "bwd": "bf16 attention backward (dQ, dK, dV), intra-stream, n=4 L=4096 B=2 32q/8kv D=128",
+    "bwd_cross": "bf16 attention backward (dQ, dK, dV), cross-stream, n=4 L=4096 B=2 32q/8kv D=128",
 }
 FLUSH_BYTES = 512 << 20
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
@@ -278,6 +283,62 @@ class Decode:
             self.h_o[m].copy_(self.o[m], non_blocking=True)
 
 
+class Backward:
+    """hd_attn_bwd on device-resident q, k, v, o, lse and dO (o and lse from
+    the library's forward of the same inputs)."""
+
+    def __init__(self, cfg, seed_base, torch, hd, synth):
+        self.cfg = c = cfg
+        self.torch, self.hd = torch, hd
+        P = c["n"] * c["L"]
+        self.q = synth.normal_device((c["B"], P, c["Hq"], c["D"]), seed_base + 3)
+        self.k = synth.normal_device((c["B"], P, c["Hkv"], c["D"]), seed_base + 4)
+        self.v = synth.normal_device((c["B"], P, c["Hkv"], c["D"]), seed_base + 5)
+        self.dO = synth.normal_device((c["B"], P, c["Hq"], c["D"]), seed_base + 6)
+        self.status = hd.new_status()
+        self.o, self.lse = hd.hd_attn_fwd(self.q, self.k, self.v, c["n"], c["mode"], c["W"], lse=True,
+                                          dev_status=self.status)
+        self.dq = torch.empty_like(self.q)
+        self.dk = torch.empty_like(self.k)
+        self.dv = torch.empty_like(self.v)
+        self.ws = torch.empty(hd.hd_attn_bwd_workspace(c["B"], c["L"], c["n"], c["Hq"], c["mode"]),
+                              dtype=torch.uint8, device="cuda")
+
+    def step(self, ev=None):
+        c = self.cfg
+        if ev is not None:
+            ev[0].record()
+        self.hd.hd_attn_bwd(self.q, self.k, self.v, self.o, self.dO, self.lse, c["n"], c["mode"], c["W"],
+                            dq=self.dq, dk=self.dk, dv=self.dv, workspace=self.ws, dev_status=self.status)
+        if ev is not None:
+            ev[1].record()
+
+    launches_per_step = 3  # lse/delta preparation, dK/dV, dQ
+
+    def e2e_buffers(self):
+        torch = self.torch
+        self.h_in = [torch.empty_like(t, device="cpu").pin_memory() for t in
+                     (self.q, self.k, self.v, self.o, self.dO, self.lse)]
+        for h, t in zip(self.h_in, (self.q, self.k, self.v, self.o, self.dO, self.lse)):
+            h.copy_(t)
+        self.h_out = [torch.empty_like(t, device="cpu").pin_memory() for t in (self.dq, self.dk, self.dv)]
+        bi = sum(h.numel() * h.element_size() for h in self.h_in)
+        bo = sum(h.numel() * h.element_size() for h in self.h_out)
+        return bi, bo
+
+    def e2e_step(self):
+        for t, h in zip((self.q, self.k, self.v, self.o, self.dO, self.lse), self.h_in):
+            t.copy_(h, non_blocking=True)
+        self.step()
+        for h, t in zip(self.h_out, (self.dq, self.dk, self.dv)):
+            h.copy_(t, non_blocking=True)
+
+    def flops(self):
+        from stream_sequence_attention_b200 import accounting as acc
+        c = self.cfg
+        return acc.attn_bwd_flops(c["B"], c["L"], c["n"], c["Hq"], c["D"], c["mode"], c["W"])
+
+
 def timed(torch, work, K, flush, dist=None, use_e2e=False):
     """Run K steps with per-step CUDA events (flush outside them).  Returns
     (per-step ms list, dominant-kernel ms list)."""
@@ -335,7 +396,12 @@ def run_ours(args, rank, world, dist):
     W = args.warmup if args.warmup is not None else 5
     W = max(W, 3)
     seed_base = rank_seed(wl, rank)
-    work = Decode(cfg, seed_base, torch, hd, synth) if wl == "decode" else Prefill(cfg, seed_base, torch, hd, synth)
+    if wl == "decode":
+        work = Decode(cfg, seed_base, torch, hd, synth)
+    elif cfg.get("bwd"):
+        work = Backward(cfg, seed_base, torch, hd, synth)
+    else:
+        work = Prefill(cfg, seed_base, torch, hd, synth)
     flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     flush = lambda: flush_buf.fill_(1)  # noqa: E731
 
@@ -375,6 +441,21 @@ def run_ours(args, rank, world, dist):
                 "peak_source": peaks["source"] + " hbm_gbs",
                 "traffic": recorded_traffic("decode_kernel", ["decode.cu"], "decode_intra")}
         e2e_value = world * nbytes / (e2e_ms * 1e-3) / 1e9
+        dtype = "bf16"
+    elif cfg.get("bwd"):
+        fl = work.flops()
+        value = world * fl / (ms_per_step * 1e-3) / 1e12
+        metric = "useful attn backward TFLOP/s at n=4 (%s)" % cfg["mode"]
+        unit = "TFLOP/s"
+        achieved = fl / (kern_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16"], "unit": "TFLOP/s",
+                "frac": round(achieved / peaks["bf16"], 4),
+                "kernel": "hd_attn_bwd (bwd_prep + attn_bwd_dkv_kernel<128> + attn_bwd_dq_kernel<128>)",
+                "peak_source": peaks["source"] + " bf16_tflops (burst)",
+                "flops_convention": "useful = visible pairs x 10 x D; the kernels execute 14 x D per pair",
+                "traffic": recorded_traffic("attn_bwd", ["attn_bwd_tc.cu", "attn_bwd_f32.cu", "hd_common.cuh"],
+                                            wl)}
+        e2e_value = world * fl / (e2e_ms * 1e-3) / 1e12
         dtype = "bf16"
     else:
         fl = work.flops()
@@ -451,6 +532,14 @@ def extras(torch, peaks, rank):
                                         "frac_bf16": round(tf / peaks["bf16"], 4)}
     del mi
     torch.cuda.empty_cache()
+    for wl in ("bwd", "bwd_cross"):
+        bw = Backward(WORKLOADS[wl], 7301 + rank, torch, hd, synth)
+        ms = time_fn(lambda: bw.step())
+        tf = bw.flops() / (ms * 1e-3) / 1e12
+        res[f"backward_{WORKLOADS[wl]['mode']}"] = {"ms": round(ms, 3), "TFLOP/s": round(tf, 1),
+                                                  "frac_bf16": round(tf / peaks["bf16"], 4)}
+        del bw
+        torch.cuda.empty_cache()
     return res
 
 
@@ -495,6 +584,19 @@ def oracle_sample_rate(wl, budget_s, seed=5):
     k = synth.normal((1, P, 1, D), seed + 2, dtype="bf16")
     v = synth.normal((1, P, 1, D), seed + 3, dtype="bf16")
     pk = np.arange(P)
+    if cfg.get("bwd"):
+        dO = synth.normal((1, P, 1, D), seed + 4, dtype="bf16")
+        t0 = time.perf_counter()
+        rows, pairs = 0, 0
+        while time.perf_counter() - t0 < budget_s:
+            p = int(g.integers(P))
+            keys = oracle.attn_bwd_query_rows(q, k, v, dO, n, mode, [(0, 0, p)], W, D ** -0.5)[0][0]
+            pairs += len(keys)
+            rows += 1
+        dt = time.perf_counter() - t0
+        return (pairs * 10 * D / dt / 1e12, "TFLOP/s",
+                f"{rows} uniformly sampled query rows of one (batch, head): each row's dQ and its dK/dV terms, "
+                f"{dt:.1f} s", threads)
     t0 = time.perf_counter()
     rows, pairs = 0, 0
     while time.perf_counter() - t0 < budget_s:
@@ -522,8 +624,12 @@ def run_reference(args):
         vals.append(v)
     wall = time.perf_counter() - t0
     value = statistics.mean(vals)
-    metric = ("decode GB/s vs HBM (intra+cross, B=64 n=4 ctx=32768)" if wl == "decode"
-              else "useful attn TFLOP/s at n=4 (%s)" % WORKLOADS[wl]["mode"])
+    if wl == "decode":
+        metric = "decode GB/s vs HBM (intra+cross, B=64 n=4 ctx=32768)"
+    elif WORKLOADS[wl].get("bwd"):
+        metric = "useful attn backward TFLOP/s at n=4 (%s)" % WORKLOADS[wl]["mode"]
+    else:
+        metric = "useful attn TFLOP/s at n=4 (%s)" % WORKLOADS[wl]["mode"]
     return {
         "impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus, "steps": K,
         "warmup": W, "ms_per_step": round(1000 * wall / K, 3), "higher_is_better": True, "scaling": "weak",

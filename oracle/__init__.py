@@ -39,6 +39,7 @@ from .hd_oracle import (  # noqa: F401
     attn_bwd,
     attn_bwd_dq_rows,
     attn_bwd_dkv_rows,
+    attn_bwd_query_rows,
     attn_final_stream,
     decode,
     decode_rows,

@@ -273,6 +273,25 @@ def attn_bwd_dkv_rows(q, k, v, dO, n, mode, rows, window=0, scale=None):
     return np.array(dks), np.array(dvs)
 
 
+def attn_bwd_query_rows(q, k, v, dO, n, mode, rows, window=0, scale=None):
+    """The terms of :func:`attn_bwd` that query row (b, h, p) contributes:
+    its dQ row, and over its visible keys p' the summands P[p,p'] dO[p] of dV
+    and scale dS[p,p'] q[p] of dK.  Summing the latter over every query row
+    (and the heads of a group) gives dK and dV.  Returns a list of
+    (keys, dq [D], dk_terms [len(keys), D], dv_terms [len(keys), D])."""
+    Hq, D = q.shape[2], q.shape[3]
+    G = Hq // k.shape[2]
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    out = []
+    for (b, h, p) in rows:
+        keys, kk, pr, ds = _bwd_row(q, k, v, dO, n, mode, b, h, p, G, window, scale)
+        qv = np.asarray(q[b, p, h, :], dtype=np.float64)
+        g = np.asarray(dO[b, p, h, :], dtype=np.float64)
+        out.append((keys, scale * (ds @ kk), scale * np.outer(ds, qv), np.outer(pr, g)))
+    return out
+
+
 def attn_rows(q, k, v, n, mode, rows, window=0, scale=None):
     """The same definition evaluated for selected output rows only.
 

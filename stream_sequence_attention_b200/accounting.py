@@ -76,3 +76,23 @@ def pairs_final_stream(L: int, n: int, mode: str, window: int = 0) -> int:
 
 def attn_flops_final_stream(B: int, L: int, n: int, Hq: int, D: int, mode: str, window: int = 0) -> int:
     return B * Hq * pairs_final_stream(L, n, mode, window) * 4 * D
+
+
+def attn_bwd_flops(B: int, L: int, n: int, Hq: int, D: int, mode: str, window: int = 0) -> int:
+    """Useful backward FLOPs: visible pairs x 10 x head_dim -- five products
+    per pair (recomputed scores, dP, dV, dK, dQ), 2 x head_dim each; 2.5x
+    the forward's useful FLOPs."""
+    return B * Hq * pairs_per_head(L, n, mode, window) * 10 * D
+
+
+def attn_bwd_exec_flops(B: int, L: int, n: int, Hq: int, D: int, mode: str, window: int = 0) -> int:
+    """Tensor-core FLOPs the bf16 backward executes on visible pairs: the
+    dK/dV pass forms S, dP, dV, dK and the dQ pass forms S, dP, dQ again, so
+    seven products per pair (full 128 x 128 tiles on the diagonal add more)."""
+    return B * Hq * pairs_per_head(L, n, mode, window) * 14 * D
+
+
+def attn_bwd_min_bytes(B: int, L: int, n: int, Hq: int, Hkv: int, D: int, esize: int = 2) -> int:
+    """Read q, k, v, o, dO and lse once, write dq, dk, dv once."""
+    P = n * L
+    return B * P * (D * esize * (3 * Hq + 2 * Hkv + 2 * Hkv + Hq) + 4 * Hq)

@@ -151,3 +151,20 @@ def test_bwd_row_functions_match_full_backward(mode, W):
     gk, gv = oracle.attn_bwd_dkv_rows(q, k, v, dO, n, mode, krows, W)
     np.testing.assert_allclose(gk, np.array([dK[b, p, g] for b, g, p in krows]), rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(gv, np.array([dV[b, p, g] for b, g, p in krows]), rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("mode,W", CASES)
+def test_bwd_query_row_terms_sum_to_full_backward(mode, W):
+    n, L, Hq, Hkv, D = 2, 6, 4, 2, 5
+    q, k, v, dO = _inputs(1, L, n, Hq, Hkv, D, 61)
+    dQ, dK, dV = oracle.attn_bwd(q, k, v, dO, n, mode, W)
+    P, G = n * L, Hq // Hkv
+    rows = [(0, h, p) for h in range(Hq) for p in range(P)]
+    sk = np.zeros_like(dK)
+    sv = np.zeros_like(dV)
+    for (b, h, p), (keys, dq, tk, tv) in zip(rows, oracle.attn_bwd_query_rows(q, k, v, dO, n, mode, rows, W)):
+        np.testing.assert_allclose(dq, dQ[b, p, h], rtol=1e-12, atol=1e-12)
+        sk[b, keys, h // G] += tk
+        sv[b, keys, h // G] += tv
+    np.testing.assert_allclose(sk, dK, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(sv, dV, rtol=1e-12, atol=1e-12)
