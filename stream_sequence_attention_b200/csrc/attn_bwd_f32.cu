@@ -19,59 +19,74 @@ namespace hd {
 
 // ------------------------------------------------------------ preparation
 
-// One warp per (b, p, h) row: delta = <dO, o> in float32 and lse in log2
-// units, stored stream-major; the warps past the last row write the padding.
+// Each row (b, p, h) is read by LPR lanes with 16-byte loads (a warp covers
+// 32/LPR rows): delta = <dO, o> in float32 and lse in log2 units, stored
+// stream-major.  Threads past the last row write the padding.
 template <int D, bool BF16>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const void* __restrict__ o, const void* __restrict__ dO,
-                                                       const float* __restrict__ lse, float2* __restrict__ ws,
+                                                       const float* __restrict__ lse, BwdWs ws,
                                                        const AttnGeom g, int Hq, int64_t rows, int64_t pad) {
-  constexpr int E = D / 32;
-  const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  constexpr int ES = BF16 ? 2 : 4;
+  constexpr int LPR = D * ES / 16;  // lanes per row
+  constexpr int RPW = 32 / LPR;     // rows per warp
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t w = tid >> 5;
   const int lane = threadIdx.x & 31;
   const int Lpad = bwd_lpad(g.Lq);
-  if (w < rows) {
+  const int64_t row_warps = (rows + RPW - 1) / RPW;
+  if (w < row_warps) {
+    const int64_t row = w * RPW + lane / LPR;
+    const int part = lane % LPR;
     float acc = 0.f;
-    const int64_t base = w * D + lane * E;
-    if (BF16) {
-      const __nv_bfloat16* a = static_cast<const __nv_bfloat16*>(o) + base;
-      const __nv_bfloat16* b = static_cast<const __nv_bfloat16*>(dO) + base;
+    if (row < rows) {
+      const uint4 a = reinterpret_cast<const uint4*>(o)[row * LPR + part];
+      const uint4 b = reinterpret_cast<const uint4*>(dO)[row * LPR + part];
+      if (BF16) {
+        const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
+        const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
 #pragma unroll
-      for (int e = 0; e < E; ++e) acc = fmaf(__bfloat162float(a[e]), __bfloat162float(b[e]), acc);
-    } else {
-      const float* a = static_cast<const float*>(o) + base;
-      const float* b = static_cast<const float*>(dO) + base;
-#pragma unroll
-      for (int e = 0; e < E; ++e) acc = fmaf(a[e], b[e], acc);
+        for (int e = 0; e < 4; ++e) {
+          const float2 fa = __bfloat1622float2(pa[e]), fb = __bfloat1622float2(pb[e]);
+          acc = fmaf(fa.x, fb.x, fmaf(fa.y, fb.y, acc));
+        }
+      } else {
+        acc = __uint_as_float(a.x) * __uint_as_float(b.x) + __uint_as_float(a.y) * __uint_as_float(b.y) +
+              __uint_as_float(a.z) * __uint_as_float(b.z) + __uint_as_float(a.w) * __uint_as_float(b.w);
+      }
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) {
-      // row w = (b*P + p)*Hq + h, p = i*ns + s
+    for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (part == 0 && row < rows) {
+      // row = (b*P + p)*Hq + h, p = i*ns + s
       const int64_t P = static_cast<int64_t>(g.ns) * g.Lq;
-      const int h = static_cast<int>(w % Hq);
-      const int64_t bp = w / Hq;
+      const int h = static_cast<int>(row % Hq);
+      const int64_t bp = row / Hq;
       const int b = static_cast<int>(bp / P);
       const int64_t p = bp - b * P;
       const int i = static_cast<int>(p / g.ns), s = static_cast<int>(p - static_cast<int64_t>(i) * g.ns);
       const float l2 = lse[(static_cast<int64_t>(b) * Hq + h) * P + p] * 1.4426950408889634f;
-      ws[((static_cast<int64_t>(b) * Hq + h) * g.ns + s) * Lpad + i] = make_float2(l2, acc);
+      const int64_t at = ((static_cast<int64_t>(b) * Hq + h) * g.ns + s) * Lpad + i;
+      ws.l2[at] = l2;
+      ws.delta[at] = acc;
     }
   } else {
     const int per = Lpad - g.Lq;
-    const int64_t e = (w - rows) * 32 + lane;
+    const int64_t e = (w - row_warps) * 32 + lane;
     if (per > 0 && e < pad) {
       const int64_t line = e / per;  // (b*Hq + h)*ns + s
       const int i = g.Lq + static_cast<int>(e - line * per);
-      ws[line * Lpad + i] = make_float2(INFINITY, 0.f);
+      ws.l2[line * Lpad + i] = INFINITY;
+      ws.delta[line * Lpad + i] = 0.f;
     }
   }
 }
 
-cudaError_t launch_bwd_prep(const void* o, const void* dO, const float* lse, float2* ws, const AttnGeom& g, int Hq,
+cudaError_t launch_bwd_prep(const void* o, const void* dO, const float* lse, BwdWs ws, const AttnGeom& g, int Hq,
                             int D, bool bf16, cudaStream_t st) {
   const int64_t rows = static_cast<int64_t>(g.B) * g.ns * g.Lq * Hq;
   const int64_t pad = static_cast<int64_t>(g.B) * Hq * g.ns * (bwd_lpad(g.Lq) - g.Lq);
-  const int64_t warps = rows + (pad + 31) / 32;
+  const int rpw = 32 / (D * (bf16 ? 2 : 4) / 16);
+  const int64_t warps = (rows + rpw - 1) / rpw + (pad + 31) / 32;
   const int64_t blocks = (warps * 32 + 255) / 256;
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
@@ -106,7 +121,7 @@ __device__ __forceinline__ float quad_sum(float x) {
 template <int D>
 __global__ void __launch_bounds__(kBwThreads) attn_bwd_dq_f32_kernel(
     const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
-    const float* __restrict__ dO, const float2* __restrict__ ws, float* __restrict__ dq, const AttnGeom g, int Hq,
+    const float* __restrict__ dO, const BwdWs ws, float* __restrict__ dq, const AttnGeom g, int Hq,
     int Hkv, int W, float sl2, float scale) {
   constexpr int DQ = D / 4;
   __shared__ __align__(16) float Ks[kBwTile][D];
@@ -130,7 +145,8 @@ __global__ void __launch_bounds__(kBwThreads) attn_bwd_dq_f32_kernel(
     dor[d] = dO[qrow + part * DQ + d];
     acc[d] = 0.f;
   }
-  const float2 ld = ws[((static_cast<int64_t>(b) * Hq + h) * g.ns + s) * bwd_lpad(g.Lq) + ic];
+  const int64_t lat = ((static_cast<int64_t>(b) * Hq + h) * g.ns + s) * bwd_lpad(g.Lq) + ic;
+  const float2 ld = make_float2(ws.l2[lat], ws.delta[lat]);
   const int hi = min(q0 + kBwRows - 1, g.Lq - 1);
   const int lo = W > 0 ? max(0, q0 - W + 1) : 0;
   const int64_t kv_stride = static_cast<int64_t>(g.ns) * Hkv * D;
@@ -177,7 +193,7 @@ __global__ void __launch_bounds__(kBwThreads) attn_bwd_dq_f32_kernel(
 template <int D>
 __global__ void __launch_bounds__(kBwThreads) attn_bwd_dkv_f32_kernel(
     const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
-    const float* __restrict__ dO, const float2* __restrict__ ws, float* __restrict__ dk, float* __restrict__ dv,
+    const float* __restrict__ dO, const BwdWs ws, float* __restrict__ dk, float* __restrict__ dv,
     const AttnGeom g, int Hq, int Hkv, int W, float sl2, float scale) {
   constexpr int DQ = D / 4;
   __shared__ __align__(16) float Qs[kBwTile][D];
@@ -223,7 +239,9 @@ __global__ void __launch_bounds__(kBwThreads) attn_bwd_dkv_f32_kernel(
         reinterpret_cast<float4*>(&Qs[c][0])[d4] = a;
         reinterpret_cast<float4*>(&Os[c][0])[d4] = bb;
       }
-      if (tid < kBwTile) Ls[tid] = (i0 + tid <= hi) ? ws[l_base + i0 + tid] : make_float2(INFINITY, 0.f);
+      if (tid < kBwTile)
+        Ls[tid] = (i0 + tid <= hi) ? make_float2(ws.l2[l_base + i0 + tid], ws.delta[l_base + i0 + tid])
+                                   : make_float2(INFINITY, 0.f);
       __syncthreads();
 #pragma unroll 4
       for (int c = 0; c < kBwTile; ++c) {
@@ -256,7 +274,7 @@ __global__ void __launch_bounds__(kBwThreads) attn_bwd_dkv_f32_kernel(
   }
 }
 
-cudaError_t launch_attn_bwd_f32(const float* q, const float* k, const float* v, const float* dO, const float2* ws,
+cudaError_t launch_attn_bwd_f32(const float* q, const float* k, const float* v, const float* dO, BwdWs ws,
                                 float* dq, float* dk, float* dv, const AttnGeom& g, int Hq, int Hkv, int D, int W,
                                 float scale, cudaStream_t st) {
   const int nb = (g.Lq + kBwRows - 1) / kBwRows;

@@ -47,7 +47,14 @@ constexpr int kThreads = 320;
 constexpr int kWarpTMA = 8;
 constexpr int kWarpMMA = 9;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kLdBytes = BT * 8;  // (lse2, delta) of one query tile
+constexpr int kLdBytes = BT * 8;  // lse2[128] then delta[128] of one query tile
+// One exponential in four of the dK/dV kernel's P tile on the FMA pipe (the
+// cubic of exp2_fma, relative error < 1e-4, below the bf16 rounding of P)
+// when nonzero, to offload the MUFU unit.
+#ifndef HD_BW_POLY_EXP
+#define HD_BW_POLY_EXP 0
+#endif
+constexpr bool kPolyExp = HD_BW_POLY_EXP != 0;
 
 template <int D>
 struct Tile {
@@ -96,7 +103,7 @@ struct LayQ {
 }  // namespace bw
 
 struct BwParams {
-  const float2* ws;  // (lse2, delta), stream-major, padded
+  BwdWs ws;  // lse2 and delta planes, stream-major, padded
   void* dq;
   void* dk;
   void* dv;
@@ -108,9 +115,12 @@ struct BwParams {
 };
 
 // dK/dV unit: key block ascending (causal: the first blocks see the most
-// query tiles), then (b, s, kvh).
+// query tiles), then (b, s, kvh).  Its tiles j = 0 .. G*nqt-1 walk the query
+// tiles from the last one down, the G heads of the group inside: the CTAs
+// that run the other key blocks of the same (b, s, kvh) at the same time
+// then read the same Q and dO tiles, which stay in L2.
 struct KvUnit {
-  int b, s, kvh, kblk, qt_lo, nqt;
+  int b, s, kvh, kblk, qt_lo, qt_hi, nqt;
 };
 __device__ __forceinline__ KvUnit kv_unit(int u, const BwParams& p) {
   const int per = p.B * p.ns * p.Hkv;
@@ -123,10 +133,12 @@ __device__ __forceinline__ KvUnit kv_unit(int u, const BwParams& p) {
   x.b = rem / p.ns;
   const int k0 = x.kblk * bw::BT;
   x.qt_lo = x.kblk;  // queries >= first key of the block
-  const int qt_hi = p.W > 0 ? min(p.nblk - 1, (k0 + bw::BT - 1 + p.W - 1) / bw::BT) : p.nblk - 1;
-  x.nqt = qt_hi - x.qt_lo + 1;
+  x.qt_hi = p.W > 0 ? min(p.nblk - 1, (k0 + bw::BT - 1 + p.W - 1) / bw::BT) : p.nblk - 1;
+  x.nqt = x.qt_hi - x.qt_lo + 1;
   return x;
 }
+__device__ __forceinline__ int kv_tile_qt(const KvUnit& x, int j, int G) { return x.qt_hi - j / G; }
+__device__ __forceinline__ int kv_tile_head(const KvUnit& x, int j, int G) { return x.kvh * G + j % G; }
 
 // dQ unit: query block descending (causal: the last blocks see the most key
 // tiles), then (b, s, h).
@@ -310,8 +322,8 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
         ++kv_issued;
         const int nt = G * x.nqt;
         for (int j = 0; j < nt; ++j, ++t) {
-          const int h = x.kvh * G + j / x.nqt;
-          const int qt = x.qt_lo + j % x.nqt;
+          const int h = kv_tile_head(x, j, G);
+          const int qt = kv_tile_qt(x, j, G);
           const int st = t % Lay::QST;
           const uint32_t ph = ((t / Lay::QST) & 1) ^ 1;
           if (!mbar_wait(bar(Lay::B_QEMPTY + st), ph, abort_flag)) { ok = false; break; }
@@ -320,9 +332,13 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
           for (int kb = 0; kb < T::KB; ++kb)
             tma_load_5d(sbase + Lay::Q_OFF + st * T::TILE + kb * T::BLK, &tmQ, bar(Lay::B_QFULL + st), kb * 64, h,
                         x.s, qt * bw::BT, x.b);
-          bulk_load(sbase + Lay::LD_OFF + st * bw::kLdBytes,
-                    p.ws + ((static_cast<int64_t>(x.b) * p.Hq + h) * p.ns + x.s) * p.Lpad + qt * bw::BT,
-                    bw::kLdBytes, bar(Lay::B_QFULL + st));
+          {
+            const int64_t at = ((static_cast<int64_t>(x.b) * p.Hq + h) * p.ns + x.s) * p.Lpad + qt * bw::BT;
+            bulk_load(sbase + Lay::LD_OFF + st * bw::kLdBytes, p.ws.l2 + at, bw::kLdBytes / 2,
+                      bar(Lay::B_QFULL + st));
+            bulk_load(sbase + Lay::LD_OFF + st * bw::kLdBytes + bw::kLdBytes / 2, p.ws.delta + at,
+                      bw::kLdBytes / 2, bar(Lay::B_QFULL + st));
+          }
           ++q_issued[st];
           if (!mbar_wait(bar(Lay::B_OEMPTY + st), ph, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(bar(Lay::B_OFULL + st), T::TILE);
@@ -418,7 +434,7 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
       const int jkey = k0 + r;  // this thread's key token
       for (int j = 0; j < nt; ++j, ++t) {
         const int st = t % Lay::QST;
-        const int q0 = (x.qt_lo + j % x.nqt) * bw::BT + 64 * ch;  // first query of this half
+        const int q0 = kv_tile_qt(x, j, G) * bw::BT + 64 * ch;  // first query of this half
         bool got = mbar_wait(bar(Lay::B_SFULL), t & 1, abort_flag);
         got = got && mbar_wait(bar(Lay::B_QFULL + st), (t / Lay::QST) & 1, abort_flag);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
@@ -426,14 +442,21 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
         uint32_t sv[64];
         tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
         tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        const float2* ld = reinterpret_cast<const float2*>(smem + Lay::LD_OFF + st * bw::kLdBytes) + 64 * ch;
+        // lse2 / delta of this half's 64 queries: 16-byte broadcast loads
+        // (every lane reads the same address), four columns per load.
+        const float4* l4 = reinterpret_cast<const float4*>(smem + Lay::LD_OFF + st * bw::kLdBytes) + 16 * ch;
+        const float4* d4 = reinterpret_cast<const float4*>(smem + Lay::LD_OFF + st * bw::kLdBytes + 512) + 16 * ch;
         tmem_wait_ld();
         const bool need_mask = (q0 < k0 + bw::BT - 1) || (p.W > 0 && q0 + 63 - k0 >= p.W);
         float pv[64];
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float a = fmaf(__uint_as_float(sv[c]), sl2, -ld[c].x);
-          pv[c] = ex2(a);
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 l = l4[c4];
+          pv[4 * c4 + 0] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 0]), sl2, -l.x));
+          pv[4 * c4 + 1] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 1]), sl2, -l.y));
+          pv[4 * c4 + 2] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 2]), sl2, -l.z));
+          const float a3 = fmaf(__uint_as_float(sv[4 * c4 + 3]), sl2, -l.w);
+          pv[4 * c4 + 3] = bw::kPolyExp ? exp2_fma(a3) : ex2(a3);
         }
         if (need_mask) {
 #pragma unroll
@@ -460,22 +483,18 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
         tmem_ld32(tDP, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
         tmem_ld32(tDP + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
         tmem_wait_ld();
-        {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
           uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int c = 2 * e;
-            pk[e] = pack_bf16x2(pv[c] * (__uint_as_float(sv[c]) - ld[c].y),
-                                pv[c + 1] * (__uint_as_float(sv[c + 1]) - ld[c + 1].y));
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const int c = 32 * half + 4 * e4;
+            const float4 d = d4[8 * half + e4];
+            pk[2 * e4] = pack_bf16x2(pv[c] * (__uint_as_float(sv[c]) - d.x), pv[c + 1] * (__uint_as_float(sv[c + 1]) - d.y));
+            pk[2 * e4 + 1] =
+                pack_bf16x2(pv[c + 2] * (__uint_as_float(sv[c + 2]) - d.z), pv[c + 3] * (__uint_as_float(sv[c + 3]) - d.w));
           }
-          tmem_st16(tDP, pk);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int c = 32 + 2 * e;
-            pk[e] = pack_bf16x2(pv[c] * (__uint_as_float(sv[c]) - ld[c].y),
-                                pv[c + 1] * (__uint_as_float(sv[c + 1]) - ld[c + 1].y));
-          }
-          tmem_st16(tDP + 16, pk);
+          tmem_st16(tDP + 16 * half, pk);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -678,7 +697,8 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
     for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++ul) {
       const QUnit x = q_unit(u, p);
       const int iq = x.qblk * bw::BT + r;  // this thread's query token
-      const float2 ld = p.ws[((static_cast<int64_t>(x.b) * p.Hq + x.h) * p.ns + x.s) * p.Lpad + iq];
+      const int64_t lat = ((static_cast<int64_t>(x.b) * p.Hq + x.h) * p.ns + x.s) * p.Lpad + iq;
+      const float2 ld = make_float2(p.ws.l2[lat], p.ws.delta[lat]);
       for (int j = 0; j < x.nkt; ++j, ++t) {
         const int k0 = (x.kt_lo + j) * bw::BT + 64 * ch;  // first key of this half
         const uint32_t tS = tmem + lane_addr + (t & 1) * 128 + 64 * ch;
@@ -771,7 +791,7 @@ static cudaError_t launch_bwd_tc_d(const CUtensorMap& mq, const CUtensorMap& mk,
   return cudaGetLastError();
 }
 
-cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, const void* dO, const float2* ws,
+cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, const void* dO, BwdWs ws,
                                void* dq, void* dk, void* dv, const AttnGeom& g, int Hq, int Hkv, int D, int W,
                                float scale, int32_t* status, int sms, cudaStream_t st) {
   CUtensorMap mq, mk, mv, mo;

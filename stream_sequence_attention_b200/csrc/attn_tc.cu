@@ -130,19 +130,6 @@ __device__ __forceinline__ TcUnit tc_unit(int u, const TcParams& p) {
   return x;
 }
 
-// 2^x on the FMA pipe for finite x <= 2^22: x = n + f, n = rint(x),
-// f in [-1/2, 1/2]; cubic for 2^f (coefficients from fit_exp2_poly.py);
-// 2^n by adding n to the exponent field.  Inputs below -127 are clamped.
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -127.0f);
-  const float t = x + 12582912.0f;  // 1.5 * 2^23: rint(x) lands in the low mantissa bits
-  const float f = x - (t - 12582912.0f);
-  float p = fmaf(0.0551713444f, f, 0.242610335f);
-  p = fmaf(p, f, 0.693260968f);
-  p = fmaf(p, f, 0.999928117f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 template <int D>
 __global__ void __launch_bounds__(tc::kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,

@@ -177,7 +177,7 @@ size_t hd_attn_bwd_workspace(int B, int L, int n, int Hq, hd_mode mode) {
   if (B < 1 || L < 1 || n < 1 || Hq < 1 || (mode != HD_INTRA && mode != HD_CROSS)) return 0;
   if (static_cast<int64_t>(n) * L > (1ll << 30)) return 0;
   const AttnGeom g = regular_geom(B, L, n, mode);
-  return static_cast<size_t>(B) * Hq * g.ns * bwd_lpad(g.Lq) * sizeof(float2);
+  return static_cast<size_t>(2 * bwd_plane(g, Hq)) * sizeof(float);
 }
 
 hd_status hd_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
@@ -192,7 +192,7 @@ hd_status hd_attn_bwd(const void* q, const void* k, const void* v, const void* o
   if (ws_bytes < hd_attn_bwd_workspace(B, L, n, Hq, mode)) return HD_ERR_INVALID_ARG;
   const AttnGeom g = regular_geom(B, L, n, mode);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  float2* ws = static_cast<float2*>(workspace);
+  const BwdWs ws = bwd_ws(workspace, g, Hq);
   const bool bf16 = dt == HD_BF16;
   cudaError_t e = launch_bwd_prep(o, dO, lse, ws, g, Hq, D, bf16, st);
   if (e != cudaSuccess) return HD_ERR_CUDA;

@@ -50,18 +50,28 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o,
                            cudaStream_t st);
 
 // Backward.  Regular geometry only (qstride 1, qoff 0, kv_stream -1, the
-// key streams equal the query streams).  The workspace holds, per
-// (b, query head, stream s, token i), the pair (lse * log2 e, delta =
-// <dO, o>) as float2 at ((b*Hq + h)*ns + s)*Lpad + i, with Lpad = Lq rounded
-// up to 128 and the padding rows set to (+inf, 0) so they contribute nothing.
+// key streams equal the query streams).  The workspace holds two float
+// planes, lse * log2 e and delta = <dO, o>, each indexed
+// ((b*Hq + h)*ns + s)*Lpad + i with Lpad = Lq rounded up to 128; the padding
+// rows are (+inf, 0) so they contribute nothing.  Separate planes let a
+// kernel fetch four consecutive tokens' values in one 16-byte load.
 constexpr int kBwdPad = 128;
 __host__ __device__ inline int bwd_lpad(int Lq) { return (Lq + kBwdPad - 1) / kBwdPad * kBwdPad; }
-cudaError_t launch_bwd_prep(const void* o, const void* dO, const float* lse, float2* ws, const AttnGeom& g, int Hq,
+struct BwdWs {
+  float* l2;
+  float* delta;
+};
+inline int64_t bwd_plane(const AttnGeom& g, int Hq) { return static_cast<int64_t>(g.B) * Hq * g.ns * bwd_lpad(g.Lq); }
+inline BwdWs bwd_ws(void* base, const AttnGeom& g, int Hq) {
+  float* p = static_cast<float*>(base);
+  return BwdWs{p, p + bwd_plane(g, Hq)};
+}
+cudaError_t launch_bwd_prep(const void* o, const void* dO, const float* lse, BwdWs ws, const AttnGeom& g, int Hq,
                             int D, bool bf16, cudaStream_t st);
-cudaError_t launch_attn_bwd_f32(const float* q, const float* k, const float* v, const float* dO, const float2* ws,
+cudaError_t launch_attn_bwd_f32(const float* q, const float* k, const float* v, const float* dO, BwdWs ws,
                                 float* dq, float* dk, float* dv, const AttnGeom& g, int Hq, int Hkv, int D, int W,
                                 float scale, cudaStream_t st);
-cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, const void* dO, const float2* ws,
+cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, const void* dO, BwdWs ws,
                                void* dq, void* dk, void* dv, const AttnGeom& g, int Hq, int Hkv, int D, int W,
                                float scale, int32_t* status, int sms, cudaStream_t st);
 
