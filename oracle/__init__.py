@@ -17,6 +17,8 @@ Sources (page "Hidden Decoding at Scale", WeLM blog):
     the attention forward  ->  :func:`attn_bwd`.
   * "Persistent KV and the KV-mirror Saving" (only the final stream runs
     through the mirrored layers)  ->  :func:`attn_final_stream`.
+  * "Multi-Stream Expansion and Training Objective" (the expanded sequence
+    runs with contiguous RoPE positions)  ->  :func:`rope`.
   * "Persistent KV and the KV-mirror Saving" (a KV cache kept for every
     stream) and "Inference Throughput" (the n streams of a token are processed
     together in one pass)  ->  :func:`decode`.
@@ -44,4 +46,6 @@ from .hd_oracle import (  # noqa: F401
     decode,
     decode_rows,
     pair_count,
+    rope,
+    rope_angles,
 )

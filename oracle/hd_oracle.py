@@ -19,6 +19,9 @@ Readings where the pages are silent (each listed in the design notes):
     token's stream s sees the new token's streams s' <= s in cross mode
     (causal in p), i.e. exactly the prefill row of that position.
   * lse is the natural-log log-sum-exp of the scaled visible scores.
+  * RoPE: the pages fix only the positions (contiguous over the expanded
+    sequence); the rotation is the standard rotary embedding with
+    theta_j = base^(-2j/rot_dim), in either pairing convention.
 """
 
 from __future__ import annotations
@@ -130,6 +133,51 @@ def final_stream_gather(h, n):
     for b in range(B):
         for i in range(L):
             out[b, i] = h[b, i * n + n - 1]
+    return out
+
+
+def rope_angles(positions, rot_dim, base):
+    """theta_j = base^(-2j/rot_dim), j < rot_dim/2; returns positions[:, None] * theta
+    in float64 (the rotary embedding of Su et al., "RoFormer")."""
+    j = np.arange(rot_dim // 2, dtype=np.float64)
+    theta = float(base) ** (-2.0 * j / rot_dim)
+    return np.asarray(positions, dtype=np.float64)[:, None] * theta[None, :]
+
+
+def rope(x, rot_dim, base=10000.0, layout="half", pos_base=0, pos_mult=0, pos0=None):
+    """Rotary position embedding over the expanded sequence, float64.
+
+    "Multi-Stream Expansion and Training Objective": the expanded sequence
+    runs with contiguous RoPE positions, so row r of sequence b sits at
+    position p = pos_base + pos_mult * pos0[b] + r (pos0 = None: 0); for a
+    prefill [B, nL, H, D] with pos_base = 0 that is p = i*n + s.  The first
+    rot_dim features are rotated pairwise by the angle p * theta_j:
+      layout "half":        pairs (j, j + rot_dim/2)
+      layout "interleaved": pairs (2j, 2j + 1)
+    (x_a, x_b) -> (x_a cos - x_b sin, x_a sin + x_b cos); features past
+    rot_dim are unchanged.  x: [B, P, H, D]; returns a new array.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    B, P, H, D = x.shape
+    if rot_dim % 2 or not 2 <= rot_dim <= D:
+        raise ValueError("rot_dim must be even and in [2, D]")
+    out = x.copy()
+    half = rot_dim // 2
+    for b in range(B):
+        start = pos_base + (pos_mult * int(pos0[b]) if pos0 is not None else 0)
+        ang = rope_angles(start + np.arange(P), rot_dim, base)  # [P, half]
+        c = np.cos(ang)[:, None, :]
+        s = np.sin(ang)[:, None, :]
+        if layout == "half":
+            xa, xb = x[b, :, :, :half], x[b, :, :, half:rot_dim]
+            out[b, :, :, :half] = xa * c - xb * s
+            out[b, :, :, half:rot_dim] = xa * s + xb * c
+        elif layout == "interleaved":
+            xa, xb = x[b, :, :, 0:rot_dim:2], x[b, :, :, 1:rot_dim:2]
+            out[b, :, :, 0:rot_dim:2] = xa * c - xb * s
+            out[b, :, :, 1:rot_dim:2] = xa * s + xb * c
+        else:
+            raise ValueError(layout)
     return out
 
 
