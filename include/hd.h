@@ -211,6 +211,38 @@ hd_status hd_attn_decode_noalloc(const void* q, const void* k_cache,
                                  float scale, hd_dtype in_dt, hd_dtype out_dt,
                                  int32_t* dev_status, void* stream);
 
+typedef enum {
+  HD_ROPE_HALF = 0,       /* pairs (j, j + rot_dim/2): the rotate-half form   */
+  HD_ROPE_INTERLEAVED = 1 /* pairs (2j, 2j + 1): the RoFormer paper's form    */
+} hd_rope_layout;
+
+/*
+ * Rotary position embedding over the expanded sequence ("Multi-Stream
+ * Expansion and Training Objective": the expanded sequence runs with
+ * contiguous RoPE positions), applied in place to q and k in one launch.
+ * The pages fix only the positions; the rotation is the standard rotary
+ * embedding.  Row r of sequence b sits at position
+ *   pos(b, r) = pos_base + pos_mult * pos0[b] + r      (pos0 NULL: 0)
+ * so a prefill of the expanded sequence (P = n*L, pos_base = 0) gives
+ * pos = i*n + s, and the decode rows of the new token ([B, n, H, D] with
+ * pos0 = ctx_len, pos_mult = n, pos_base = -n) give pos = (T-1)*n + s.
+ * The first rot_dim features rotate pairwise by pos * theta_j,
+ * theta_j = base^(-2j/rot_dim), j < rot_dim/2:
+ *   (x_a, x_b) -> (x_a cos - x_b sin, x_a sin + x_b cos);
+ * features past rot_dim are unchanged.
+ *
+ *   q    [B, P, Hq,  D]  element type `dt`, rotated in place (nullable)
+ *   k    [B, P, Hkv, D]  element type `dt`, rotated in place (nullable)
+ *   pos0 [B] int32 on the device (nullable)
+ * rot_dim % 8 == 0, 8 <= rot_dim <= D <= 256, D % 8 == 0, base finite and
+ * > 0, |pos| < 2^31 for every row.  Angles and their cos/sin are formed in
+ * float64; the rotation runs in float32 and rounds once to `dt`.
+ */
+hd_status hd_rope(void* q, void* k, const int32_t* pos0, int B, int P, int Hq,
+                  int Hkv, int D, int rot_dim, double base, int64_t pos_base,
+                  int64_t pos_mult, hd_rope_layout layout, hd_dtype dt,
+                  void* stream);
+
 /*
  * Final-stream gather ("Multi-Stream Expansion and Training Objective": only
  * the final stream E_n of each token feeds the shared LM head; Figure 1):

@@ -243,6 +243,38 @@ hd_status hd_attn_decode(const void* q, const void* k_cache, const void* v_cache
                                    static_cast<cudaStream_t>(stream)));
 }
 
+hd_status hd_rope(void* q, void* k, const int32_t* pos0, int B, int P, int Hq, int Hkv, int D, int rot_dim,
+                  double base, int64_t pos_base, int64_t pos_mult, hd_rope_layout layout, hd_dtype dt, void* stream) {
+  if (B < 0 || P < 0 || Hq < 0 || Hkv < 0 || !valid_dtype(dt)) return HD_ERR_INVALID_ARG;
+  if (layout != HD_ROPE_HALF && layout != HD_ROPE_INTERLEAVED) return HD_ERR_INVALID_ARG;
+  if (D % 8 || D < 8 || D > 2 * kRopeMaxPairs || rot_dim % 8 || rot_dim < 8 || rot_dim > D)
+    return HD_ERR_INVALID_ARG;
+  if (!std::isfinite(base) || !(base > 0.0)) return HD_ERR_INVALID_ARG;
+  const int heads = (q ? Hq : 0) + (k ? Hkv : 0);
+  if (B == 0 || P == 0 || heads == 0) return HD_OK;
+  if ((q && !aligned16(q)) || (k && !aligned16(k)) || (pos0 && (reinterpret_cast<uintptr_t>(pos0) & 3u)))
+    return HD_ERR_INVALID_ARG;
+  // Positions must stay within +-2^31: pos_base + pos_mult*pos0 + r for
+  // pos0 in int32 range is checked against the host-known parts only.
+  const int64_t lim = 1ll << 31;
+  if (pos_base <= -lim || pos_base + P >= lim || pos_mult < -lim || pos_mult > lim) return HD_ERR_INVALID_ARG;
+  RopeParams p;
+  p.q = q;
+  p.k = k;
+  p.pos0 = pos0;
+  p.B = B;
+  p.P = P;
+  p.Hq = q ? Hq : 0;
+  p.Hkv = k ? Hkv : 0;
+  p.D = D;
+  p.rot = rot_dim;
+  p.layout = layout;
+  p.pos_base = pos_base;
+  p.pos_mult = pos_mult;
+  for (int j = 0; j < rot_dim / 2; ++j) p.theta[j] = std::pow(base, -2.0 * j / rot_dim);
+  return cuda_status(launch_rope(p, dt == HD_BF16, static_cast<cudaStream_t>(stream)));
+}
+
 const char* hd_status_string(hd_status st) {
   switch (st) {
     case HD_OK: return "HD_OK";

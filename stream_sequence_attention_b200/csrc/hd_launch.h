@@ -75,6 +75,18 @@ cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, cons
                                void* dq, void* dk, void* dv, const AttnGeom& g, int Hq, int Hkv, int D, int W,
                                float scale, int32_t* status, int sms, cudaStream_t st);
 
+// Rotary embedding (rope.cu).  theta[j] = base^(-2j/rot), j < rot/2, from the host.
+constexpr int kRopeMaxPairs = 128;
+struct RopeParams {
+  void* q;
+  void* k;
+  const int32_t* pos0;
+  int B, P, Hq, Hkv, D, rot, layout;
+  int64_t pos_base, pos_mult;
+  double theta[kRopeMaxPairs];
+};
+cudaError_t launch_rope(const RopeParams& p, bool bf16, cudaStream_t st);
+
 // Decode work decomposition: units (one KV head of one sequence, and for
 // intra mode one stream), row groups of at most 32 query rows, token splits.
 struct DecPlan {

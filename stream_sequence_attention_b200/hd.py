@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libhd.so")
 HD_OK, HD_ERR_INVALID_ARG, HD_ERR_UNSUPPORTED, HD_ERR_CUDA, HD_ERR_TIMEOUT, HD_ERR_BAD_TOKEN = range(6)
 HD_F32, HD_BF16 = 0, 1
 HD_INTRA, HD_CROSS = 0, 1
+HD_ROPE_HALF, HD_ROPE_INTERLEAVED = 0, 1
 
 _MODES = {"intra": HD_INTRA, "cross": HD_CROSS, HD_INTRA: HD_INTRA, HD_CROSS: HD_CROSS}
 
@@ -33,6 +34,7 @@ EXPORTS = (
     "hd_attn_decode_workspace",
     "hd_attn_decode_noalloc",
     "hd_final_stream_gather",
+    "hd_rope",
     "hd_status_string",
     "hd_version",
 )
@@ -78,6 +80,8 @@ def lib() -> ctypes.CDLL:
         L.hd_attn_decode_noalloc.restype = i32
         L.hd_final_stream_gather.argtypes = [vp, vp, i32, i32, i32, i32, i32, vp]
         L.hd_final_stream_gather.restype = i32
+        L.hd_rope.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, ctypes.c_double, i64, i64, i32, i32, vp]
+        L.hd_rope.restype = i32
         L.hd_status_string.argtypes = [i32]
         L.hd_status_string.restype = ctypes.c_char_p
         L.hd_version.argtypes = []
@@ -162,6 +166,34 @@ def hd_final_stream_gather(h: torch.Tensor, n: int, out: torch.Tensor | None = N
     _check("hd_final_stream_gather", lib().hd_final_stream_gather(
         _ptr(h), _ptr(out), B, L, n, d, _dt(h), _stream(stream)))
     return out
+
+
+_ROPE_LAYOUTS = {"half": HD_ROPE_HALF, "interleaved": HD_ROPE_INTERLEAVED}
+
+
+def hd_rope(q: torch.Tensor | None, k: torch.Tensor | None = None, rot_dim: int | None = None,
+            base: float = 10000.0, pos_base: int = 0, pos_mult: int = 0, pos0: torch.Tensor | None = None,
+            layout: str = "half", stream=None):
+    """Rotary embedding in place on q [B, P, Hq, D] and k [B, P, Hkv, D]
+    (either may be None): row r of sequence b at position
+    pos_base + pos_mult * pos0[b] + r.  Returns (q, k)."""
+    ref = q if q is not None else k
+    if ref is None:
+        raise ValueError("q or k is required")
+    for t, nm in ((q, "q"), (k, "k"), (pos0, "pos0")):
+        if t is not None:
+            _need(t, nm)
+    B, P, _, D = ref.shape
+    Hq = q.shape[2] if q is not None else 0
+    Hkv = k.shape[2] if k is not None else 0
+    if q is not None and k is not None and (k.shape[:2] != q.shape[:2] or k.shape[3] != D or k.dtype != q.dtype):
+        raise ValueError("q and k disagree")
+    if pos0 is not None and (pos0.dtype != torch.int32 or pos0.shape != (B,)):
+        raise ValueError("pos0 must be int32 [B]")
+    _check("hd_rope", lib().hd_rope(
+        _ptr(q), _ptr(k), _ptr(pos0), B, P, Hq, Hkv, D, int(rot_dim or D), float(base), int(pos_base),
+        int(pos_mult), _ROPE_LAYOUTS[layout], _dt(ref), _stream(stream)))
+    return q, k
 
 
 def hd_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n: int, mode="intra", window: int = 0,

@@ -112,3 +112,22 @@ def test_bwd_workspace_and_bad_arguments(L):
     assert bwd(q=vp(0x10008)) == hd.HD_ERR_INVALID_ARG
     assert bwd(ws_bytes=16) == hd.HD_ERR_INVALID_ARG
     assert bwd(B=0) == hd.HD_OK
+
+
+def test_rope_bad_arguments(L):
+    from stream_sequence_attention_b200 import hd
+    vp = ctypes.c_void_p
+    fake = vp(0x10000)
+
+    def rope(*, q=fake, k=fake, D=128, rot=128, base=10000.0, layout=0, dt=1, B=1, P=4, pos_base=0):
+        return L.hd_rope(q, k, None, B, P, 4, 2, D, rot, base, pos_base, 0, layout, dt, None)
+    assert rope(rot=6) == hd.HD_ERR_INVALID_ARG          # not a multiple of 8
+    assert rope(rot=136) == hd.HD_ERR_INVALID_ARG        # > D
+    assert rope(D=260, rot=256) == hd.HD_ERR_INVALID_ARG  # D > 256
+    assert rope(base=0.0) == hd.HD_ERR_INVALID_ARG
+    assert rope(base=float("nan")) == hd.HD_ERR_INVALID_ARG
+    assert rope(layout=3) == hd.HD_ERR_INVALID_ARG
+    assert rope(q=vp(0x10008)) == hd.HD_ERR_INVALID_ARG
+    assert rope(pos_base=1 << 40) == hd.HD_ERR_INVALID_ARG
+    assert rope(B=0) == hd.HD_OK
+    assert rope(q=None, k=None) == hd.HD_OK
