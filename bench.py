@@ -1,7 +1,8 @@
 """Benchmark of the Hidden Decoding hot path on B200; prints ONE JSON line.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload intra|cross|long|decode|mirror|bwd|bwd_cross] [--no-extras]
+                    [--workload intra|cross|long|decode|mirror|bwd|bwd_cross|rope]
+                    [--no-extras]
 
 Default workload (intra): n=4 streams, L=4096 tokens (nL=16384), batch 2,
 32 query / 8 KV heads, head_dim 128, bf16.  One step is one pass of the
@@ -47,6 +48,7 @@ WORKLOADS = {
     "mirror": dict(B=2, n=4, L=4096, Hq=32, Hkv=8, D=128, mode="cross", W=0, V=152064, dm=4096, final=True),
     "bwd": dict(B=2, n=4, L=4096, Hq=32, Hkv=8, D=128, mode="intra", W=0, bwd=True),
     "bwd_cross": dict(B=2, n=4, L=4096, Hq=32, Hkv=8, D=128, mode="cross", W=0, bwd=True),
+    "rope": dict(B=2, n=4, L=4096, Hq=32, Hkv=8, D=128, rope=True),
 }
 NAMES = {
     "intra": "bf16 prefill, intra-stream, n=4 L=4096 B=2 32q/8kv D=128",
@@ -56,6 +58,7 @@ NAMES = {
     "mirror": "bf16 KV-mirror layer: final-stream queries, cross-stream keys, n=4 L=4096 B=2 32q/8kv D=128",
     "bwd": "bf16 attention backward (dQ, dK, dV), intra-stream, n=4 L=4096 B=2 32q/8kv D=128",
     "bwd_cross": "bf16 attention backward (dQ, dK, dV), cross-stream, n=4 L=4096 B=2 32q/8kv D=128",
+    "rope": "bf16 RoPE in place on q and k at positions i*n+s, n=4 L=4096 B=2 32q/8kv D=128",
 }
 FLUSH_BYTES = 512 << 20
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
@@ -339,6 +342,45 @@ class Backward:
         return acc.attn_bwd_flops(c["B"], c["L"], c["n"], c["Hq"], c["D"], c["mode"], c["W"])
 
 
+class Rope:
+    """hd_rope in place on device-resident q and k (one launch)."""
+
+    def __init__(self, cfg, seed_base, torch, hd, synth):
+        self.cfg = c = cfg
+        self.torch, self.hd = torch, hd
+        P = c["n"] * c["L"]
+        self.q = synth.normal_device((c["B"], P, c["Hq"], c["D"]), seed_base + 3)
+        self.k = synth.normal_device((c["B"], P, c["Hkv"], c["D"]), seed_base + 4)
+        self.status = hd.new_status()
+
+    def step(self, ev=None):
+        if ev is not None:
+            ev[0].record()
+        self.hd.hd_rope(self.q, self.k)
+        if ev is not None:
+            ev[1].record()
+
+    launches_per_step = 1
+
+    def nbytes(self):
+        return 2 * (self.q.numel() + self.k.numel()) * self.q.element_size()
+
+    def e2e_buffers(self):
+        torch = self.torch
+        self.h = [torch.empty_like(t, device="cpu").pin_memory() for t in (self.q, self.k)]
+        for h, t in zip(self.h, (self.q, self.k)):
+            h.copy_(t)
+        n = sum(h.numel() * h.element_size() for h in self.h)
+        return n, n
+
+    def e2e_step(self):
+        for t, h in zip((self.q, self.k), self.h):
+            t.copy_(h, non_blocking=True)
+        self.step()
+        for h, t in zip(self.h, (self.q, self.k)):
+            h.copy_(t, non_blocking=True)
+
+
 def timed(torch, work, K, flush, dist=None, use_e2e=False):
     """Run K steps with per-step CUDA events (flush outside them).  Returns
     (per-step ms list, dominant-kernel ms list)."""
@@ -400,6 +442,8 @@ def run_ours(args, rank, world, dist):
         work = Decode(cfg, seed_base, torch, hd, synth)
     elif cfg.get("bwd"):
         work = Backward(cfg, seed_base, torch, hd, synth)
+    elif cfg.get("rope"):
+        work = Rope(cfg, seed_base, torch, hd, synth)
     else:
         work = Prefill(cfg, seed_base, torch, hd, synth)
     flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
@@ -440,6 +484,17 @@ def run_ours(args, rank, world, dist):
                 "frac": round(achieved / peaks["hbm"], 4), "kernel": "decode_kernel (intra) + combine",
                 "peak_source": peaks["source"] + " hbm_gbs",
                 "traffic": recorded_traffic("decode_kernel", ["decode.cu"], "decode_intra")}
+        e2e_value = world * nbytes / (e2e_ms * 1e-3) / 1e9
+        dtype = "bf16"
+    elif cfg.get("rope"):
+        nbytes = work.nbytes()
+        value = world * nbytes / (ms_per_step * 1e-3) / 1e9
+        metric, unit = "RoPE GB/s vs HBM (q and k in place, n=4 L=4096 B=2 32q/8kv)", "GB/s"
+        achieved = nbytes / (kern_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm"], 4), "kernel": "rope_kernel<true>",
+                "peak_source": peaks["source"] + " hbm_gbs",
+                "traffic": recorded_traffic("rope_kernel", ["rope.cu"], wl)}
         e2e_value = world * nbytes / (e2e_ms * 1e-3) / 1e9
         dtype = "bf16"
     elif cfg.get("bwd"):
@@ -532,6 +587,12 @@ def extras(torch, peaks, rank):
                                         "frac_bf16": round(tf / peaks["bf16"], 4)}
     del mi
     torch.cuda.empty_cache()
+    rp = Rope(WORKLOADS["rope"], 7401 + rank, torch, hd, synth)
+    ms = time_fn(lambda: rp.step())
+    gbs = rp.nbytes() / (ms * 1e-3) / 1e9
+    res["rope"] = {"ms": round(ms, 3), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm"], 4)}
+    del rp
+    torch.cuda.empty_cache()
     for wl in ("bwd", "bwd_cross"):
         bw = Backward(WORKLOADS[wl], 7301 + rank, torch, hd, synth)
         ms = time_fn(lambda: bw.step())
@@ -578,6 +639,19 @@ def oracle_sample_rate(wl, budget_s, seed=5):
         # bytes each row's arithmetic reads from the cache: intra T, cross n*T entries of K and V
         per_row_bytes = 0.5 * (2 * T * D * 2) + 0.5 * (2 * n * T * D * 2)
         return rows * per_row_bytes / dt / 1e9, "GB/s", f"{rows} decode rows (one KV head, ctx {T}), {dt:.1f} s", threads
+    if cfg.get("rope"):
+        n, L, D, H = cfg["n"], cfg["L"], cfg["D"], cfg["Hq"] + cfg["Hkv"]
+        P = n * L
+        x = synth.normal((1, 256, H, D), seed + 1, dtype="bf16")
+        t0 = time.perf_counter()
+        rows = 0
+        while time.perf_counter() - t0 < budget_s:
+            oracle.rope(x, D, 10000.0, pos_base=int(g.integers(P - 256)))
+            rows += 256
+        dt = time.perf_counter() - t0
+        # bytes the GPU call moves for these rows: q and k read and written once (bf16)
+        return (rows * H * D * 2 * 2 / dt / 1e9, "GB/s",
+                f"{rows} positions x {H} heads in blocks of 256 consecutive positions, {dt:.1f} s", threads)
     n, L, D, mode, W = cfg["n"], cfg["L"], cfg["D"], cfg["mode"], cfg["W"]
     P = n * L
     q = synth.normal((1, P, 1, D), seed + 1, dtype="bf16")
@@ -628,6 +702,8 @@ def run_reference(args):
         metric = "decode GB/s vs HBM (intra+cross, B=64 n=4 ctx=32768)"
     elif WORKLOADS[wl].get("bwd"):
         metric = "useful attn backward TFLOP/s at n=4 (%s)" % WORKLOADS[wl]["mode"]
+    elif WORKLOADS[wl].get("rope"):
+        metric = "RoPE GB/s vs HBM (q and k in place, n=4 L=4096 B=2 32q/8kv)"
     else:
         metric = "useful attn TFLOP/s at n=4 (%s)" % WORKLOADS[wl]["mode"]
     return {

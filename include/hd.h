@@ -235,8 +235,9 @@ typedef enum {
  *   k    [B, P, Hkv, D]  element type `dt`, rotated in place (nullable)
  *   pos0 [B] int32 on the device (nullable)
  * rot_dim % 8 == 0, 8 <= rot_dim <= D <= 256, D % 8 == 0, base finite and
- * > 0, |pos| < 2^31 for every row.  Angles and their cos/sin are formed in
- * float64; the rotation runs in float32 and rounds once to `dt`.
+ * > 0, |pos| < 2^31 for every row.  The angle is reduced exactly (64-bit
+ * fixed-point turns), cos/sin and the rotation run in float32 (angle error
+ * < 2e-7 rad), and the result rounds once to `dt`.
  */
 hd_status hd_rope(void* q, void* k, const int32_t* pos0, int B, int P, int Hq,
                   int Hkv, int D, int rot_dim, double base, int64_t pos_base,

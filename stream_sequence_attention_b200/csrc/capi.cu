@@ -271,7 +271,13 @@ hd_status hd_rope(void* q, void* k, const int32_t* pos0, int B, int P, int Hq, i
   p.layout = layout;
   p.pos_base = pos_base;
   p.pos_mult = pos_mult;
-  for (int j = 0; j < rot_dim / 2; ++j) p.theta[j] = std::pow(base, -2.0 * j / rot_dim);
+  // theta_j / (2 pi) in turns, as a 64-bit binary fraction (long double:
+  // 64-bit mantissa); theta_j <= 1 so the fraction is below 1/(2 pi).
+  const long double two_pi = 6.283185307179586476925286766559005768L;
+  for (int j = 0; j < rot_dim / 2; ++j) {
+    const long double turns = powl(static_cast<long double>(base), -2.0L * j / rot_dim) / two_pi;
+    p.fturn[j] = static_cast<uint64_t>(ldexpl(turns, 64));
+  }
   return cuda_status(launch_rope(p, dt == HD_BF16, static_cast<cudaStream_t>(stream)));
 }
 

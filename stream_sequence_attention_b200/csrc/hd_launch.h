@@ -75,7 +75,8 @@ cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, cons
                                void* dq, void* dk, void* dv, const AttnGeom& g, int Hq, int Hkv, int D, int W,
                                float scale, int32_t* status, int sms, cudaStream_t st);
 
-// Rotary embedding (rope.cu).  theta[j] = base^(-2j/rot), j < rot/2, from the host.
+// Rotary embedding (rope.cu).  fturn[j] = theta_j / (2 pi) as a 64-bit
+// fixed-point fraction of a turn, theta_j = base^(-2j/rot), j < rot/2.
 constexpr int kRopeMaxPairs = 128;
 struct RopeParams {
   void* q;
@@ -83,7 +84,7 @@ struct RopeParams {
   const int32_t* pos0;
   int B, P, Hq, Hkv, D, rot, layout;
   int64_t pos_base, pos_mult;
-  double theta[kRopeMaxPairs];
+  uint64_t fturn[kRopeMaxPairs];
 };
 cudaError_t launch_rope(const RopeParams& p, bool bf16, cudaStream_t st);
 
