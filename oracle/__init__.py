@@ -19,6 +19,10 @@ Sources (page "Hidden Decoding at Scale", WeLM blog):
     through the mirrored layers)  ->  :func:`attn_final_stream`.
   * "Multi-Stream Expansion and Training Objective" (the expanded sequence
     runs with contiguous RoPE positions)  ->  :func:`rope`.
+  * "Persistent KV and the KV-mirror Saving" (stream parallelism: the
+    intra-stream KV sharded across ranks by stream)  ->  :func:`shard_streams`,
+    :func:`stream_interleave`, :func:`decode_rows_streams`,
+    :func:`combine_partials`.
   * "Persistent KV and the KV-mirror Saving" (a KV cache kept for every
     stream) and "Inference Throughput" (the n streams of a token are processed
     together in one pass)  ->  :func:`decode`.
@@ -45,6 +49,10 @@ from .hd_oracle import (  # noqa: F401
     attn_final_stream,
     decode,
     decode_rows,
+    decode_rows_streams,
+    shard_streams,
+    stream_interleave,
+    combine_partials,
     pair_count,
     rope,
     rope_angles,

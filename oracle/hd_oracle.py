@@ -435,6 +435,85 @@ def decode_rows(q, k_cache, v_cache, ctx_len, n, mode, rows, window=0, scale=Non
     return np.array(outs), np.array(lses)
 
 
+def shard_streams(n, R, r):
+    """Streams held by rank r of R under stream parallelism ("Persistent KV
+    and the KV-mirror Saving": the intra-stream KV is sharded across ranks by
+    stream): s = r, r + R, r + 2R, ...  (R must divide n)."""
+    if n % R:
+        raise ValueError("R must divide n")
+    return list(range(r, n, R))
+
+
+def stream_interleave(parts, n):
+    """Re-interleave per-rank stream shards into the expanded order.
+
+    parts: [R, B, (n/R)*L, ...] where rank r's local row i*(n/R) + l holds
+    token i of global stream s = r + R*l.  Returns [B, n*L, ...] with row
+    i*n + s.  A pure permutation."""
+    parts = np.asarray(parts)
+    R, B, PL = parts.shape[:3]
+    nl = n // R
+    L = PL // nl
+    out = np.empty((B, n * L) + parts.shape[3:], dtype=parts.dtype)
+    for r in range(R):
+        for l in range(nl):
+            s = r + R * l
+            for i in range(L):
+                out[:, i * n + s] = parts[r, :, i * nl + l]
+    return out
+
+
+def decode_rows_streams(q, k_cache, v_cache, ctx_len, n, streams, rows, window=0, scale=None):
+    """Cross-mode decode restricted to the cache streams in ``streams``.
+
+    q: [B, n, Hq, D] (all streams' queries of the new token); k_cache,
+    v_cache: [B, len(streams), Lmax, Hkv, D] holding global streams
+    ``streams`` in order.  For each (b, s, h): softmax over the keys of
+    :func:`decode_rows` (cross) that lie in those streams.  Returns
+    (O [R, D], lse [R]); a row with no such key gets O = 0 and lse = -inf.
+    """
+    Hq, D = q.shape[2], q.shape[3]
+    Hkv = k_cache.shape[3]
+    G = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    local = {s: l for l, s in enumerate(streams)}
+    outs, lses = [], []
+    for (b, s, h) in rows:
+        T = int(ctx_len[b])
+        kv = h // G
+        pk = _decode_keys(T, n, s, CROSS, window)
+        pk = pk[np.isin(pk % n, list(streams))]
+        if pk.size == 0:
+            outs.append(np.zeros(D))
+            lses.append(-np.inf)
+            continue
+        j, sl = pk // n, np.array([local[x] for x in pk % n])
+        kk = np.asarray(k_cache[b, sl, j, kv, :], dtype=np.float64)
+        vv = np.asarray(v_cache[b, sl, j, kv, :], dtype=np.float64)
+        qv = np.asarray(q[b, s, h, :], dtype=np.float64)
+        o, l = _softmax_weighted(scale * (kk @ qv)[None, :], vv)
+        outs.append(o[0])
+        lses.append(l[0])
+    return np.array(outs), np.array(lses)
+
+
+def combine_partials(o_parts, lse_parts):
+    """Merge softmax-weighted partial results over disjoint key sets:
+    O = sum_r exp(lse_r - LSE) O_r with LSE = log sum_r exp(lse_r).
+    o_parts [R, ..., D], lse_parts [R, ...] (-inf: empty part).
+    Returns (O, LSE); O = 0, LSE = -inf where every part is empty."""
+    o_parts = np.asarray(o_parts, dtype=np.float64)
+    lse_parts = np.asarray(lse_parts, dtype=np.float64)
+    m = lse_parts.max(axis=0)
+    safe = np.where(np.isfinite(m), m, 0.0)
+    w = np.where(np.isfinite(lse_parts), np.exp(lse_parts - safe), 0.0)
+    tot = w.sum(axis=0)
+    o = (w[..., None] * o_parts).sum(axis=0) / np.where(tot > 0, tot, 1.0)[..., None]
+    lse = np.where(tot > 0, safe + np.log(np.where(tot > 0, tot, 1.0)), -np.inf)
+    return o, lse
+
+
 def decode(q, k_cache, v_cache, ctx_len, n, mode, window=0, scale=None):
     """All rows of :func:`decode_rows`: returns (O [B, n, Hq, D], lse [B, n, Hq])."""
     B, _, Hq, D = q.shape
