@@ -211,8 +211,82 @@ hd_status hd_attn_decode_noalloc(const void* q, const void* k_cache,
                                  float scale, hd_dtype in_dt, hd_dtype out_dt,
                                  int32_t* dev_status, void* stream);
 
+/*
+ * Stream parallelism ("Persistent KV and the KV-mirror Saving": the
+ * intra-stream KV is sharded across ranks by stream).  With R ranks (R
+ * divides n), rank r holds the streams s = r + R*l, l < n/R, stored in the
+ * expanded order of its own streams: local row i*(n/R) + l is token i of
+ * global stream r + R*l.  Intra-stream layers need nothing new (call
+ * hd_attn_fwd / hd_attn_decode on the local tensors with n/R streams).  A
+ * cross-stream layer gathers every rank's K/V shard (a collective the caller
+ * runs, e.g. an NCCL all-gather into [R, ...]), restores the expanded order
+ * with hd_stream_interleave, and runs hd_attn_fwd_shard for the local
+ * queries; cross-stream decode runs hd_attn_decode_shard on every rank for
+ * all n stream queries against the local cache streams, gathers the
+ * partials, and merges them with hd_attn_combine.
+ */
+
+/*
+ *   out[b, i*n + r + R*l, :] = parts[r, b, i*(n/R) + l, :]
+ *   parts [R, B, (n/R)*L, row_elems], out [B, n*L, row_elems], type `dt`.
+ * row_elems*sizeof(dt) must be a multiple of 16 bytes.  Bit-exact copy.
+ */
+hd_status hd_stream_interleave(const void* parts, void* out, int R, int B, int L,
+                               int n, int64_t row_elems, hd_dtype dt, void* stream);
+
+/*
+ * Merge R partial attention results over disjoint key sets:
+ *   O[row] = sum_r w_r o_parts[r, row] / sum_r w_r,  w_r = exp(lse_parts[r, row] - M),
+ *   lse[row] = M + log sum_r w_r,  M = max_r lse_parts[r, row];
+ * a part with lse = -inf (no visible key) has weight 0; a row whose parts
+ * are all empty gets O = 0 and lse = -inf.
+ *   o_parts [R, rows, D] type `in_dt`;  lse_parts [R, rows] float32 (natural log);
+ *   o [rows, D] type `out_dt`;  lse [rows] float32 (nullable).  D % 4 == 0.
+ */
+hd_status hd_attn_combine(const void* o_parts, const float* lse_parts, void* o,
+                          float* lse, int R, int64_t rows, int D, hd_dtype in_dt,
+                          hd_dtype out_dt, void* stream);
+
+/*
+ * Cross-stream prefill attention of rank r's queries against every stream's
+ * keys: for local row i*(n/R) + l (global position p = i*n + r + R*l)
+ *   O = sum_{p' in vis(p)} softmax(scale <q, k[p']>) v[p']   (HD_CROSS rules)
+ *
+ *   q_loc [B, (n/R)*L, Hq, D]  element type `in_dt`
+ *   k, v  [B, n*L, Hkv, D]     all streams, expanded order (hd_stream_interleave)
+ *   o_loc [B, (n/R)*L, Hq, D]  element type `out_dt`
+ *   lse   [B, Hq, (n/R)*L]     float32, nullable
+ * Same kernels and argument rules as hd_attn_fwd (cross mode).
+ */
+hd_status hd_attn_fwd_shard(const void* q_loc, const void* k, const void* v, void* o_loc,
+                            float* lse, int B, int L, int n, int R, int r, int Hq,
+                            int Hkv, int D, int window, float scale, hd_dtype in_dt,
+                            hd_dtype out_dt, int32_t* dev_status, void* stream);
+
+/*
+ * Cross-stream decode restricted to rank r's cache streams: for every
+ * stream query s of the new token, the softmax over the visible keys (the
+ * HD_CROSS rules of hd_attn_decode) that lie in streams r + R*l only.
+ *
+ *   q            [B, n, Hq, D]           all n stream queries, `in_dt` (HD_BF16)
+ *   k/v_cache_loc [B, n/R, Lmax, Hkv, D] the local streams, `in_dt`
+ *   ctx_len      [B] int32 on the device
+ *   o            [B, n, Hq, D]           `out_dt`: the partial O (normalised over
+ *                                        this rank's keys; 0 where it has none)
+ *   lse          [B, n, Hq] float32 (required): log-sum-exp over this rank's
+ *                keys, -inf where it has none
+ *   workspace    >= hd_attn_decode_workspace(B, n, Lmax, Hq, Hkv, D, HD_CROSS)
+ * Merge the R ranks' (o, lse) with hd_attn_combine.
+ */
+hd_status hd_attn_decode_shard(const void* q, const void* k_cache_loc,
+                               const void* v_cache_loc, const int32_t* ctx_len, void* o,
+                               float* lse, int B, int n, int R, int r, int Lmax, int Hq,
+                               int Hkv, int D, int window, float scale, hd_dtype in_dt,
+                               hd_dtype out_dt, void* workspace, size_t ws_bytes,
+                               int32_t* dev_status, void* stream);
+
 typedef enum {
-  HD_ROPE_HALF = 0,       /* pairs (j, j + rot_dim/2): the rotate-half form   */
+  HD_ROPE_HALF = 0,      /* pairs (j, j + rot_dim/2): the rotate-half form   */
   HD_ROPE_INTERLEAVED = 1 /* pairs (2j, 2j + 1): the RoFormer paper's form    */
 } hd_rope_layout;
 

@@ -45,7 +45,8 @@ __global__ void __launch_bounds__(kF32Threads) attn_f32_kernel(
   const int q0 = qblk * kF32Rows;
   const int i = q0 + r;
   const bool row_ok = i < g.Lq;
-  const int pi = (row_ok ? i : g.Lq - 1) * g.qstride + g.qoff;  // key index of this query
+  const int qb = g.qoff + s * g.qsstride;  // key index offset of this query stream
+  const int pi = (row_ok ? i : g.Lq - 1) * g.qstride + qb;  // key index of this query
 
   float qr[DH], acc[DH];
   {
@@ -62,8 +63,8 @@ __global__ void __launch_bounds__(kF32Threads) attn_f32_kernel(
   float m = -INFINITY, l = 0.f;
 
   const int last = min(q0 + kF32Rows - 1, g.Lq - 1);
-  const int hi_tok = min(last * g.qstride + g.qoff, g.Lk - 1);
-  const int lo_tok = W > 0 ? max(0, q0 * g.qstride + g.qoff - W + 1) : 0;
+  const int hi_tok = min(last * g.qstride + qb, g.Lk - 1);
+  const int lo_tok = W > 0 ? max(0, q0 * g.qstride + qb - W + 1) : 0;
   const int64_t kv_row = static_cast<int64_t>(g.kv_ns) * Hkv * D;  // token stride in k/v
   const int64_t kv_base = (static_cast<int64_t>(b) * g.kv_ns * g.Lk * Hkv + static_cast<int64_t>(skv) * Hkv + kvh) * D;
   const float* kb = k + kv_base;

@@ -125,8 +125,9 @@ __device__ __forceinline__ TcUnit tc_unit(int u, const TcParams& p) {
   // window start of its first query.
   const int q0 = x.qblk * tc::BM;
   const int qlast = min(q0 + tc::BM - 1, p.g.Lq - 1);
-  x.t_hi = (qlast * p.g.qstride + p.g.qoff) / tc::BN;
-  x.t_lo = p.W > 0 ? max(0, q0 * p.g.qstride + p.g.qoff - p.W + 1) / tc::BN : 0;
+  const int qb = p.g.qoff + x.s * p.g.qsstride;  // key index offset of this query stream
+  x.t_hi = (qlast * p.g.qstride + qb) / tc::BN;
+  x.t_lo = p.W > 0 ? max(0, q0 * p.g.qstride + qb - p.W + 1) / tc::BN : 0;
   return x;
 }
 
@@ -340,9 +341,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       const bool paired = x.h1 >= 0;
       const int q0 = x.qblk * tc::BM;
       const int i = q0 + r;
-      const int pi = i * p.g.qstride + p.g.qoff;             // key index of this row's query
-      const int pfirst = q0 * p.g.qstride + p.g.qoff;         // ... of the block's first query
-      const int plast = (q0 + tc::BM - 1) * p.g.qstride + p.g.qoff;
+      const int qb = p.g.qoff + x.s * p.g.qsstride;
+      const int pi = i * p.g.qstride + qb;             // key index of this row's query
+      const int pfirst = q0 * p.g.qstride + qb;         // ... of the block's first query
+      const int plast = (q0 + tc::BM - 1) * p.g.qstride + qb;
       float m = -INFINITY, l = 0.f;
       const int nt = x.t_hi - x.t_lo + 1;
       for (int jj = 0; jj < nt; ++jj, ++sc) {

@@ -217,11 +217,12 @@ size_t hd_attn_decode_workspace(int B, int n, int Lmax, int Hq, int Hkv, int D, 
   return decode_workspace_bytes(decode_plan(B, n, Lmax, Hq, Hkv, mode == HD_CROSS, sms));
 }
 
-hd_status hd_attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* ctx_len,
-                         void* o, float* lse, int B, int n, int Lmax, int Hq, int Hkv, int D, hd_mode mode,
-                         int window, float scale, hd_dtype in_dt, hd_dtype out_dt, void* workspace,
-                         size_t ws_bytes, int32_t* dev_status, void* stream) {
-  if (B < 0 || n < 1 || Lmax < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || window < 0) return HD_ERR_INVALID_ARG;
+// Argument checks shared by the decode entry points; nc = cache streams.
+static hd_status check_decode_args(const void* q, const void* k_cache, const void* v_cache, const int32_t* ctx_len,
+                                   void* o, float* lse, int B, int n, int nc, int Lmax, int Hq, int Hkv, int D,
+                                   hd_mode mode, int window, float scale, hd_dtype in_dt, hd_dtype out_dt,
+                                   void* workspace) {
+  if (B < 0 || n < 1 || nc < 1 || Lmax < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || window < 0) return HD_ERR_INVALID_ARG;
   if (mode != HD_INTRA && mode != HD_CROSS) return HD_ERR_INVALID_ARG;
   if (!valid_dtype(in_dt) || !valid_dtype(out_dt) || !std::isfinite(scale) || !(scale > 0.f))
     return HD_ERR_INVALID_ARG;
@@ -233,6 +234,16 @@ hd_status hd_attn_decode(const void* q, const void* k_cache, const void* v_cache
       (reinterpret_cast<uintptr_t>(workspace) & 255u) || (reinterpret_cast<uintptr_t>(ctx_len) & 3u))
     return HD_ERR_INVALID_ARG;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return HD_ERR_INVALID_ARG;
+  return HD_OK;
+}
+
+hd_status hd_attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* ctx_len,
+                         void* o, float* lse, int B, int n, int Lmax, int Hq, int Hkv, int D, hd_mode mode,
+                         int window, float scale, hd_dtype in_dt, hd_dtype out_dt, void* workspace,
+                         size_t ws_bytes, int32_t* dev_status, void* stream) {
+  hd_status stt = check_decode_args(q, k_cache, v_cache, ctx_len, o, lse, B, n, n, Lmax, Hq, Hkv, D, mode, window,
+                                    scale, in_dt, out_dt, workspace);
+  if (stt != HD_OK || B == 0) return stt;
   const int sms = sm_count();
   if (sms <= 0) return HD_ERR_CUDA;
   const DecPlan pl = decode_plan(B, n, Lmax, Hq, Hkv, mode == HD_CROSS, sms);
@@ -241,6 +252,78 @@ hd_status hd_attn_decode(const void* q, const void* k_cache, const void* v_cache
   return cuda_status(launch_decode(q, k_cache, v_cache, ctx_len, o, lse, B, n, Lmax, Hq, Hkv, window, scale,
                                    mode == HD_CROSS, out_dt == HD_BF16, workspace, dev_status, sms,
                                    static_cast<cudaStream_t>(stream)));
+}
+
+static bool valid_shard(int n, int R, int r) { return R >= 1 && n >= 1 && n % R == 0 && r >= 0 && r < R; }
+
+hd_status hd_attn_decode_shard(const void* q, const void* k_cache_loc, const void* v_cache_loc,
+                               const int32_t* ctx_len, void* o, float* lse, int B, int n, int R, int r, int Lmax,
+                               int Hq, int Hkv, int D, int window, float scale, hd_dtype in_dt, hd_dtype out_dt,
+                               void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream) {
+  if (!valid_shard(n, R, r)) return HD_ERR_INVALID_ARG;
+  hd_status stt = check_decode_args(q, k_cache_loc, v_cache_loc, ctx_len, o, lse, B, n, n / R, Lmax, Hq, Hkv, D,
+                                    HD_CROSS, window, scale, in_dt, out_dt, workspace);
+  if (stt != HD_OK || B == 0) return stt;
+  if (!lse) return HD_ERR_INVALID_ARG;  // the partial is useless without its lse
+  const int sms = sm_count();
+  if (sms <= 0) return HD_ERR_CUDA;
+  const DecPlan pl = decode_plan(B, n, Lmax, Hq, Hkv, true, sms);
+  if (pl.units > 65535) return HD_ERR_UNSUPPORTED;
+  if (ws_bytes < decode_workspace_bytes(pl)) return HD_ERR_INVALID_ARG;
+  return cuda_status(launch_decode(q, k_cache_loc, v_cache_loc, ctx_len, o, lse, B, n, Lmax, Hq, Hkv, window, scale,
+                                   true, out_dt == HD_BF16, workspace, dev_status, sms,
+                                   static_cast<cudaStream_t>(stream), n / R, r, R));
+}
+
+hd_status hd_attn_fwd_shard(const void* q_loc, const void* k, const void* v, void* o_loc, float* lse, int B, int L,
+                            int n, int R, int r, int Hq, int Hkv, int D, int window, float scale, hd_dtype in_dt,
+                            hd_dtype out_dt, int32_t* dev_status, void* stream) {
+  if (!valid_shard(n, R, r)) return HD_ERR_INVALID_ARG;
+  hd_status stt = check_attn_args(q_loc, k, v, o_loc, lse, B, L, n, Hq, Hkv, D, HD_CROSS, window, scale, in_dt, out_dt);
+  if (stt != HD_OK || B == 0) return stt;
+  // Queries: the n/R local streams of L tokens; local stream l is global
+  // stream r + R*l, at position i*n + r + R*l of the single nL-key stream.
+  const int nl = n / R;
+  AttnGeom g;
+  g.B = B;
+  g.ns = nl;
+  g.Lq = L;
+  g.q_ns = nl;
+  g.kv_ns = 1;
+  g.Lk = n * L;
+  g.kv_stream = 0;
+  g.qstride = n;
+  g.qoff = r;
+  g.qsstride = R;
+  g.o_rows = nl * L;
+  g.o_ns = nl;
+  return run_attn(q_loc, k, v, o_loc, lse, g, Hq, Hkv, D, window, scale, in_dt, out_dt, dev_status, stream);
+}
+
+hd_status hd_stream_interleave(const void* parts, void* out, int R, int B, int L, int n, int64_t row_elems,
+                               hd_dtype dt, void* stream) {
+  if (B < 0 || L < 0 || !valid_shard(n, R, 0) || row_elems < 1 || !valid_dtype(dt)) return HD_ERR_INVALID_ARG;
+  const int64_t row_bytes = row_elems * esize(dt);
+  if (row_bytes % 16 || row_bytes > (1 << 30)) return HD_ERR_INVALID_ARG;
+  const int64_t rows = static_cast<int64_t>(B) * L * n;
+  if (rows == 0) return HD_OK;
+  if (!parts || !out || !aligned16(parts) || !aligned16(out)) return HD_ERR_INVALID_ARG;
+  const int sms = sm_count();
+  if (sms <= 0) return HD_ERR_CUDA;
+  return cuda_status(launch_stream_interleave(parts, out, rows, n, R, static_cast<int>(row_bytes), sms,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+hd_status hd_attn_combine(const void* o_parts, const float* lse_parts, void* o, float* lse, int R, int64_t rows,
+                          int D, hd_dtype in_dt, hd_dtype out_dt, void* stream) {
+  if (R < 1 || rows < 0 || D < 4 || D % 4 || !valid_dtype(in_dt) || !valid_dtype(out_dt)) return HD_ERR_INVALID_ARG;
+  if (rows == 0) return HD_OK;
+  if (!o_parts || !lse_parts || !o || (reinterpret_cast<uintptr_t>(o_parts) & 15u) ||
+      (reinterpret_cast<uintptr_t>(o) & 15u) || (reinterpret_cast<uintptr_t>(lse_parts) & 3u) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return HD_ERR_INVALID_ARG;
+  return cuda_status(launch_attn_combine(o_parts, lse_parts, o, lse, R, rows, D, in_dt == HD_BF16,
+                                         out_dt == HD_BF16, static_cast<cudaStream_t>(stream)));
 }
 
 hd_status hd_rope(void* q, void* k, const int32_t* pos0, int B, int P, int Hq, int Hkv, int D, int rot_dim,

@@ -10,6 +10,12 @@
 //   cross: (j, s') with p' = j*n + s' <= p = (T-1)*n + s  (and p-p' < W)
 // i.e. exactly the prefill row of position p.
 //
+// Under stream parallelism a rank's cache holds only nc of the n streams,
+// local stream l being global stream soff + sstride*l; in cross mode the
+// kernel then returns each query's softmax over the visible keys of those
+// streams (O = 0 and lse = -inf where there are none), to be merged across
+// ranks.  The whole cache is the case nc = n, soff = 0, sstride = 1.
+//
 // The step is HBM-bound (each cached K/V byte is read once per step), so the
 // design is about streaming: a work unit is one KV head of one sequence
 // (cross: all n*G query rows that share it -- the cache is read once and
@@ -52,6 +58,7 @@ struct DecParams {
   float* ws_lse;  // [nsplit][rows_total], log2 units
   int32_t* status;
   int B, n, Lmax, Hq, Hkv, W, cross, nsplit, rg_count;
+  int nc, soff, sstride;  // cache streams and their global stream ids
   float scale_log2;
 };
 
@@ -163,7 +170,7 @@ __global__ void __launch_bounds__(DecShape<MT>::kThreads, MT == 2 ? HD_DEC_MT2_C
   const int c_lo = base + split * chunk;
   const int c_hi = bad_T ? c_lo : min(T, c_lo + chunk);
   const int ntok_tiles = c_hi > c_lo ? (c_hi - c_lo + kTok - 1) / kTok : 0;
-  const int nstreams = p.cross ? p.n : 1;
+  const int nstreams = p.cross ? p.nc : 1;
   const int ntiles = ntok_tiles * nstreams;
 
   if (threadIdx.x == 0) {
@@ -297,7 +304,7 @@ __global__ void __launch_bounds__(DecShape<MT>::kThreads, MT == 2 ? HD_DEC_MT2_C
             bool vis;
             if (p.cross) {
               const int64_t pq = static_cast<int64_t>(T - 1) * p.n + srow[hh];
-              const int64_t pk = static_cast<int64_t>(j) * p.n + sp;
+              const int64_t pk = static_cast<int64_t>(j) * p.n + (p.soff + p.sstride * sp);
               vis = pk <= pq && (p.W <= 0 || pq - pk < p.W);
             } else {
               vis = j <= T - 1 && (p.W <= 0 || T - 1 - j < p.W);
@@ -469,6 +476,75 @@ __global__ void decode_combine_kernel(const float* __restrict__ ws_o, const floa
     lse[warp] = (M == -INFINITY) ? -INFINITY : (M + log2f(L)) * 0.69314718055994531f;
 }
 
+// One warp per row: merge R partial results over disjoint key sets (stream
+// parallelism: each rank's softmax over its own streams' keys).  o_parts
+// [R][rows][D] normalised within their part, lse_parts [R][rows] natural
+// log, -inf for a part with no visible key:
+//   O = sum_r e^(lse_r - M) O_r / sum_r e^(lse_r - M),  LSE = M + log sum_r e^(lse_r - M).
+template <bool IN_BF16>
+__global__ void attn_combine_kernel(const void* __restrict__ o_parts, const float* __restrict__ lse_parts,
+                                    void* __restrict__ o, float* __restrict__ lse, int R, int64_t rows, int D,
+                                    int out_bf16) {
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  float M = -INFINITY;
+  for (int r = 0; r < R; ++r) M = fmaxf(M, lse_parts[r * rows + row]);
+  float L = 0.f;
+  if (M != -INFINITY)
+    for (int r = 0; r < R; ++r) L += expf(lse_parts[r * rows + row] - M);  // exp(-inf) = 0
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  for (int c = lane; c < D / 4; c += 32) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (M != -INFINITY) {
+      for (int r = 0; r < R; ++r) {
+        const float lr = lse_parts[r * rows + row];
+        if (lr == -INFINITY) continue;
+        const float w = expf(lr - M) * inv;
+        const int64_t off = (r * rows + row) * D + 4 * c;
+        float4 v;
+        if (IN_BF16) {
+          const uint2 u = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(o_parts) + off);
+          const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+          const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+          v = make_float4(a.x, a.y, b.x, b.y);
+        } else {
+          v = *reinterpret_cast<const float4*>(static_cast<const float*>(o_parts) + off);
+        }
+        acc.x = fmaf(w, v.x, acc.x);
+        acc.y = fmaf(w, v.y, acc.y);
+        acc.z = fmaf(w, v.z, acc.z);
+        acc.w = fmaf(w, v.w, acc.w);
+      }
+    }
+    const int64_t off = row * D + 4 * c;
+    if (out_bf16) {
+      uint2 w2;
+      w2.x = pack_bf16x2(acc.x, acc.y);
+      w2.y = pack_bf16x2(acc.z, acc.w);
+      *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(o) + off) = w2;
+    } else {
+      *reinterpret_cast<float4*>(static_cast<float*>(o) + off) = acc;
+    }
+  }
+  if (lse && lane == 0) lse[row] = (M == -INFINITY) ? -INFINITY : M + logf(L);
+}
+
+cudaError_t launch_attn_combine(const void* o_parts, const float* lse_parts, void* o, float* lse, int R,
+                                int64_t rows, int D, bool in_bf16, bool out_bf16, cudaStream_t st) {
+  if (rows == 0) return cudaSuccess;
+  const int threads = 256;
+  const int64_t blocks = (rows * 32 + threads - 1) / threads;
+  if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
+  if (in_bf16)
+    attn_combine_kernel<true><<<static_cast<unsigned>(blocks), threads, 0, st>>>(o_parts, lse_parts, o, lse, R, rows,
+                                                                                 D, out_bf16 ? 1 : 0);
+  else
+    attn_combine_kernel<false><<<static_cast<unsigned>(blocks), threads, 0, st>>>(o_parts, lse_parts, o, lse, R,
+                                                                                  rows, D, out_bf16 ? 1 : 0);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------- host
 
 
@@ -514,10 +590,12 @@ size_t decode_workspace_bytes(const DecPlan& pl) {
 
 cudaError_t launch_decode(const void* q, const void* kc, const void* vc, const int32_t* ctx, void* o,
                           float* lse, int B, int n, int Lmax, int Hq, int Hkv, int W, float scale,
-                          bool cross, bool out_bf16, void* ws, int32_t* status, int sms, cudaStream_t st) {
+                          bool cross, bool out_bf16, void* ws, int32_t* status, int sms, cudaStream_t st,
+                          int nc, int soff, int sstride) {
   const DecPlan pl = decode_plan(B, n, Lmax, Hq, Hkv, cross, sms);
+  if (nc <= 0) nc = n;
   CUtensorMap mk, mv;
-  if (!encode_cache_view(&mk, kc, B, n, Lmax, Hkv) || !encode_cache_view(&mv, vc, B, n, Lmax, Hkv))
+  if (!encode_cache_view(&mk, kc, B, nc, Lmax, Hkv) || !encode_cache_view(&mv, vc, B, nc, Lmax, Hkv))
     return cudaErrorInvalidValue;
   DecParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -528,6 +606,9 @@ cudaError_t launch_decode(const void* q, const void* kc, const void* vc, const i
   p.status = status;
   p.B = B;
   p.n = n;
+  p.nc = nc;
+  p.soff = soff;
+  p.sstride = sstride;
   p.Lmax = Lmax;
   p.Hq = Hq;
   p.Hkv = Hkv;

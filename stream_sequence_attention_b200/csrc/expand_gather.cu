@@ -5,7 +5,12 @@
 // gather (same section; only the final stream feeds the LM head):
 //                                   out[b, i, :] = h[b, i*n + n-1, :]
 //
-// Both are row copies of R = d * elem_size bytes (a multiple of 16).  One
+// stream interleave (stream parallelism, "Persistent KV and the KV-mirror
+// Saving": the KV is sharded across ranks by stream; a cross-stream layer
+// gathers every rank's shard and restores the expanded order):
+//                                   out[b, i*n + r + R*l, :] = parts[r, b, i*(n/R) + l, :]
+//
+// All are row copies of R = d * elem_size bytes (a multiple of 16).  One
 // warp moves one row with 16-byte vector loads and stores; each lane keeps
 // kUnroll loads in flight before storing, and the grid is a multiple of the
 // SM count with warps striding over rows.
@@ -77,6 +82,24 @@ __global__ void __launch_bounds__(kCopyThreads) gather_kernel(
   }
 }
 
+// rows = B*L*n output rows, row (b*L + i)*n + s with s = r + R*l, from rank
+// part r (part_rows rows each) row (b*L + i)*(n/R) + l.
+__global__ void __launch_bounds__(kCopyThreads) stream_interleave_kernel(
+    const uint4* __restrict__ parts, uint4* __restrict__ out, int64_t rows, int n, int R, int64_t part_rows,
+    int nvec) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kCopyThreads + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kCopyThreads) >> 5;
+  const int nl = n / R;
+  for (int64_t r = warp; r < rows; r += nwarps) {
+    const int64_t tok = r / n;  // b*L + i
+    const int s = static_cast<int>(r - tok * n);
+    const int rk = s % R, l = s / R;
+    const uint4* src = parts + (static_cast<int64_t>(rk) * part_rows + tok * nl + l) * nvec;
+    warp_copy_row(src, out + r * nvec, nvec, lane);
+  }
+}
+
 static int copy_grid(int64_t rows, int sms) {
   const int64_t warps_per_cta = kCopyThreads / 32;
   int64_t want = (rows + warps_per_cta - 1) / warps_per_cta;
@@ -93,6 +116,14 @@ cudaError_t launch_expand(const void* tables, const int32_t* ids, void* out, int
   expand_kernel<<<copy_grid(rows, sms), kCopyThreads, 0, st>>>(
       static_cast<const uint4*>(tables), ids, static_cast<uint4*>(out), rows, n, V,
       row_bytes / 16, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_stream_interleave(const void* parts, void* out, int64_t rows, int n, int R, int row_bytes,
+                                     int sms, cudaStream_t st) {
+  if (rows == 0) return cudaSuccess;
+  stream_interleave_kernel<<<copy_grid(rows, sms), kCopyThreads, 0, st>>>(
+      static_cast<const uint4*>(parts), static_cast<uint4*>(out), rows, n, R, rows / R, row_bytes / 16);
   return cudaGetLastError();
 }
 

@@ -22,9 +22,9 @@ cudaError_t launch_gather(const void* h, void* out, int64_t rows, int n, int row
                           cudaStream_t st);
 // Geometry of one attention call, common to both attention kernels.  The
 // kernels walk query tokens i in [0, Lq) of ns query streams s.  Query token
-// i reads the key stream kv_stream (or s when kv_stream < 0), where it sits
-// at key index pos(i) = i*qstride + qoff; key j is visible iff j <= pos(i)
-// and, with a window W > 0, pos(i) - j < W.
+// i of stream s reads the key stream kv_stream (or s when kv_stream < 0),
+// where it sits at key index pos(i, s) = i*qstride + qoff + s*qsstride; key j
+// is visible iff j <= pos(i, s) and, with a window W > 0, pos(i, s) - j < W.
 //   q   [B, q_ns*Lq, Hq, D]    query (i, s) is row i*q_ns + s
 //   k,v [B, kv_ns*Lk, Hkv, D]  key (j, t) is row j*kv_ns + t
 //   o   [B, o_rows, Hq, D]     query (i, s) writes row i*o_ns + s
@@ -34,6 +34,7 @@ struct AttnGeom {
   int ns, Lq, q_ns;
   int kv_ns, Lk, kv_stream;
   int qstride, qoff;
+  int qsstride = 0;
   int o_rows, o_ns;
 };
 
@@ -88,6 +89,13 @@ struct RopeParams {
 };
 cudaError_t launch_rope(const RopeParams& p, bool bf16, cudaStream_t st);
 
+// Stream parallelism: re-interleave rank shards (copy rows of row_bytes),
+// and merge partial softmax results over disjoint key sets.
+cudaError_t launch_stream_interleave(const void* parts, void* out, int64_t rows, int n, int R, int row_bytes,
+                                     int sms, cudaStream_t st);
+cudaError_t launch_attn_combine(const void* o_parts, const float* lse_parts, void* o, float* lse, int R,
+                                int64_t rows, int D, bool in_bf16, bool out_bf16, cudaStream_t st);
+
 // Decode work decomposition: units (one KV head of one sequence, and for
 // intra mode one stream), row groups of at most 32 query rows, token splits.
 struct DecPlan {
@@ -96,8 +104,12 @@ struct DecPlan {
 };
 DecPlan decode_plan(int B, int n, int Lmax, int Hq, int Hkv, bool cross, int sms);
 size_t decode_workspace_bytes(const DecPlan& pl);
+// nc, soff, sstride: the cache holds nc streams, local stream l being global
+// stream soff + sstride*l (stream parallelism, cross mode); nc = 0 means the
+// whole cache (nc = n, soff = 0, sstride = 1).
 cudaError_t launch_decode(const void* q, const void* kc, const void* vc, const int32_t* ctx, void* o,
                           float* lse, int B, int n, int Lmax, int Hq, int Hkv, int W, float scale,
-                          bool cross, bool out_bf16, void* ws, int32_t* status, int sms, cudaStream_t st);
+                          bool cross, bool out_bf16, void* ws, int32_t* status, int sms, cudaStream_t st,
+                          int nc = 0, int soff = 0, int sstride = 1);
 
 }  // namespace hd

@@ -33,6 +33,10 @@ EXPORTS = (
     "hd_attn_decode",
     "hd_attn_decode_workspace",
     "hd_attn_decode_noalloc",
+    "hd_attn_decode_shard",
+    "hd_attn_fwd_shard",
+    "hd_stream_interleave",
+    "hd_attn_combine",
     "hd_final_stream_gather",
     "hd_rope",
     "hd_status_string",
@@ -80,6 +84,16 @@ def lib() -> ctypes.CDLL:
         L.hd_attn_decode_noalloc.restype = i32
         L.hd_final_stream_gather.argtypes = [vp, vp, i32, i32, i32, i32, i32, vp]
         L.hd_final_stream_gather.restype = i32
+        L.hd_attn_decode_shard.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, i32, f32,
+                                           i32, i32, vp, sz, vp, vp]
+        L.hd_attn_decode_shard.restype = i32
+        L.hd_attn_fwd_shard.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, i32, f32, i32, i32,
+                                        vp, vp]
+        L.hd_attn_fwd_shard.restype = i32
+        L.hd_stream_interleave.argtypes = [vp, vp, i32, i32, i32, i32, i64, i32, vp]
+        L.hd_stream_interleave.restype = i32
+        L.hd_attn_combine.argtypes = [vp, vp, vp, vp, i32, i64, i32, i32, i32, vp]
+        L.hd_attn_combine.restype = i32
         L.hd_rope.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, ctypes.c_double, i64, i64, i32, i32, vp]
         L.hd_rope.restype = i32
         L.hd_status_string.argtypes = [i32]
@@ -389,3 +403,112 @@ def hd_attn_decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torc
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(ctx_len), _ptr(out), _ptr(lse), B, n, Lmax, Hq, Hkv, D,
         _MODES[mode], int(window), float(scale), _dt(q), _dt(out), _ptr(dev_status), _stream(stream)))
     return (out, lse) if want_lse else out
+
+
+# ------------------------------------------------------- stream parallelism
+
+def hd_stream_interleave(parts: torch.Tensor, n: int, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """parts [R, B, (n/R)*L, ...] (rank r's streams r + R*l) -> out [B, n*L, ...]
+    in the expanded order."""
+    _need(parts, "parts")
+    R, B, PL = parts.shape[:3]
+    rest = tuple(parts.shape[3:])
+    if n % R or PL % (n // R):
+        raise ValueError("shard shapes do not match n")
+    L = PL // (n // R)
+    row = 1
+    for x in rest:
+        row *= x
+    if out is None:
+        out = torch.empty((B, n * L) + rest, dtype=parts.dtype, device=parts.device)
+    _need(out, "out")
+    if out.shape != (B, n * L) + rest or out.dtype != parts.dtype:
+        raise ValueError("out has the wrong shape or dtype")
+    _check("hd_stream_interleave", lib().hd_stream_interleave(
+        _ptr(parts), _ptr(out), R, B, L, n, row, _dt(parts), _stream(stream)))
+    return out
+
+
+def hd_attn_combine(o_parts: torch.Tensor, lse_parts: torch.Tensor, out: torch.Tensor | None = None,
+                    out_dtype=None, lse: torch.Tensor | bool | None = None, stream=None):
+    """Merge partial results over disjoint key sets: o_parts [R, ..., D],
+    lse_parts [R, ...] float32 -> O [..., D] (and lse [...] when asked)."""
+    _need(o_parts, "o_parts")
+    _need(lse_parts, "lse_parts")
+    R = o_parts.shape[0]
+    D = o_parts.shape[-1]
+    if lse_parts.shape != o_parts.shape[:-1] or lse_parts.dtype != torch.float32:
+        raise ValueError("lse_parts must be float32 with o_parts' shape minus the last dim")
+    rows = lse_parts[0].numel()
+    if out is None:
+        out = torch.empty(o_parts.shape[1:], dtype=out_dtype or o_parts.dtype, device=o_parts.device)
+    _need(out, "out")
+    want_lse = lse is True or isinstance(lse, torch.Tensor)
+    if lse is True:
+        lse = torch.empty(lse_parts.shape[1:], dtype=torch.float32, device=o_parts.device)
+    elif lse is False:
+        lse = None
+    _check("hd_attn_combine", lib().hd_attn_combine(
+        _ptr(o_parts), _ptr(lse_parts), _ptr(out), _ptr(lse), R, rows, D, _dt(o_parts), _dt(out), _stream(stream)))
+    return (out, lse) if want_lse else out
+
+
+def hd_attn_fwd_shard(q_loc: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n: int, R: int, r: int,
+                      window: int = 0, scale: float | None = None, out: torch.Tensor | None = None, out_dtype=None,
+                      lse: torch.Tensor | bool | None = None, dev_status: torch.Tensor | None = None, stream=None):
+    """Cross-stream attention of rank r's queries q_loc [B, (n/R)*L, Hq, D]
+    against all streams' k/v [B, n*L, Hkv, D] (expanded order)."""
+    for t, nm in ((q_loc, "q_loc"), (k, "k"), (v, "v")):
+        _need(t, nm)
+    B, PL, Hq, D = q_loc.shape
+    Hkv = k.shape[2]
+    if n % R or PL % (n // R):
+        raise ValueError("shard shapes do not match n")
+    L = PL // (n // R)
+    if k.shape != (B, n * L, Hkv, D) or v.shape != k.shape or k.dtype != q_loc.dtype or v.dtype != q_loc.dtype:
+        raise ValueError("q_loc/k/v shapes or dtypes disagree")
+    if scale is None:
+        scale = D ** -0.5
+    if out is None:
+        out = torch.empty(q_loc.shape, dtype=out_dtype or q_loc.dtype, device=q_loc.device)
+    _need(out, "out")
+    want_lse = lse is True or isinstance(lse, torch.Tensor)
+    if lse is True:
+        lse = torch.empty((B, Hq, PL), dtype=torch.float32, device=q_loc.device)
+    elif lse is False:
+        lse = None
+    _check("hd_attn_fwd_shard", lib().hd_attn_fwd_shard(
+        _ptr(q_loc), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, L, n, R, r, Hq, Hkv, D, int(window), float(scale),
+        _dt(q_loc), _dt(out), _ptr(dev_status), _stream(stream)))
+    return (out, lse) if want_lse else out
+
+
+def hd_attn_decode_shard(q: torch.Tensor, k_cache_loc: torch.Tensor, v_cache_loc: torch.Tensor,
+                         ctx_len: torch.Tensor, R: int, r: int, window: int = 0, scale: float | None = None,
+                         out: torch.Tensor | None = None, out_dtype=torch.float32, lse: torch.Tensor | None = None,
+                         workspace: torch.Tensor | None = None, dev_status: torch.Tensor | None = None, stream=None):
+    """Cross-stream decode of all n stream queries q [B, n, Hq, D] against
+    rank r's cache streams [B, n/R, Lmax, Hkv, D]: returns the partial
+    (O, lse) to be merged with :func:`hd_attn_combine`."""
+    for t, nm in ((q, "q"), (k_cache_loc, "k_cache_loc"), (v_cache_loc, "v_cache_loc"), (ctx_len, "ctx_len")):
+        _need(t, nm)
+    B, n, Hq, D = q.shape
+    _, nl, Lmax, Hkv, _ = k_cache_loc.shape
+    if n % R or nl != n // R or v_cache_loc.shape != k_cache_loc.shape:
+        raise ValueError("cache shard shapes do not match n / R")
+    if scale is None:
+        scale = D ** -0.5
+    if out is None:
+        out = torch.empty((B, n, Hq, D), dtype=out_dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, n, Hq), dtype=torch.float32, device=q.device)
+    _need(out, "out")
+    _need(lse, "lse")
+    if workspace is None:
+        workspace = torch.empty(max(hd_attn_decode_workspace(B, n, Lmax, Hq, Hkv, D, "cross"), 1),
+                                dtype=torch.uint8, device=q.device)
+    _check("hd_attn_decode_shard", lib().hd_attn_decode_shard(
+        _ptr(q), _ptr(k_cache_loc), _ptr(v_cache_loc), _ptr(ctx_len), _ptr(out), _ptr(lse), B, n, R, r, Lmax, Hq,
+        Hkv, D, int(window), float(scale), _dt(q), _dt(out), _ptr(workspace), workspace.numel(), _ptr(dev_status),
+        _stream(stream)))
+    return out, lse

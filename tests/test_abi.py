@@ -131,3 +131,25 @@ def test_rope_bad_arguments(L):
     assert rope(pos_base=1 << 40) == hd.HD_ERR_INVALID_ARG
     assert rope(B=0) == hd.HD_OK
     assert rope(q=None, k=None) == hd.HD_OK
+
+
+def test_stream_parallel_bad_arguments(L):
+    from stream_sequence_attention_b200 import hd
+    vp = ctypes.c_void_p
+    fake = vp(0x10000)
+    # R must divide n, 0 <= r < R
+    assert L.hd_attn_fwd_shard(fake, fake, fake, fake, None, 1, 8, 4, 3, 0, 2, 2, 128, 0, 0.1, 1, 1, None, None) \
+        == hd.HD_ERR_INVALID_ARG
+    assert L.hd_attn_fwd_shard(fake, fake, fake, fake, None, 1, 8, 4, 2, 2, 2, 2, 128, 0, 0.1, 1, 1, None, None) \
+        == hd.HD_ERR_INVALID_ARG
+    assert L.hd_attn_decode_shard(fake, fake, fake, fake, fake, fake, 1, 4, 3, 0, 8, 2, 2, 128, 0, 0.1, 1, 0,
+                                  fake, 1 << 20, None, None) == hd.HD_ERR_INVALID_ARG
+    # the decode partial needs its lse
+    assert L.hd_attn_decode_shard(fake, fake, fake, fake, fake, None, 1, 4, 2, 0, 8, 2, 2, 128, 0, 0.1, 1, 0,
+                                  fake, 1 << 20, None, None) == hd.HD_ERR_INVALID_ARG
+    assert L.hd_stream_interleave(fake, fake, 3, 1, 4, 4, 8, hd.HD_BF16, None) == hd.HD_ERR_INVALID_ARG
+    assert L.hd_stream_interleave(fake, fake, 2, 1, 4, 4, 4, hd.HD_BF16, None) == hd.HD_ERR_INVALID_ARG  # 8-byte rows
+    assert L.hd_stream_interleave(None, None, 2, 0, 4, 4, 8, hd.HD_BF16, None) == hd.HD_OK
+    assert L.hd_attn_combine(fake, fake, fake, None, 2, 10, 6, 0, 0, None) == hd.HD_ERR_INVALID_ARG  # D % 4
+    assert L.hd_attn_combine(fake, fake, fake, None, 0, 10, 8, 0, 0, None) == hd.HD_ERR_INVALID_ARG
+    assert L.hd_attn_combine(None, None, None, None, 2, 0, 8, 0, 0, None) == hd.HD_OK

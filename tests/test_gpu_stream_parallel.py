@@ -1,0 +1,133 @@
+"""GPU parity of the stream-parallel calls, with R ranks run one after
+another on one device: what an all-gather would deliver is the stack of the
+ranks' shards.  (Kernels of different ranks never wait on one another, so
+running them in sequence is exact.)  Checked against the float64 oracle:
+the re-interleave bit-exact, the cross-stream prefill rows of each rank, the
+per-rank decode partials (including ranks that see no key), and their merge
+= the full cross-stream decode; plus the merge kernel on its own."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from stream_sequence_attention_b200 import synth
+from tests.gpu_util import TOL_BF16, TOL_F32, dev, lib, max_abs, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def hd():
+    return lib()
+
+
+def _shard(x, n, R, r):
+    """Rank r's streams of x [B, n*L, ...] in local order (reshape, no oracle)."""
+    B, P = x.shape[:2]
+    L, nl = P // n, n // R
+    return np.ascontiguousarray(x.reshape((B, L, nl, R) + x.shape[2:])[:, :, :, r].reshape((B, L * nl) + x.shape[2:]))
+
+
+@pytest.mark.parametrize("R", [2, 4])
+def test_interleave_restores_the_expanded_order(hd, R):
+    n, B, L = 4, 2, 37
+    x = synth.normal((B, n * L, 8, 128), 1001, dtype="bf16")
+    parts = np.stack([_shard(x, n, R, r) for r in range(R)])
+    out = hd.hd_stream_interleave(dev(parts, "bf16"), n)
+    torch.cuda.synchronize()
+    want = oracle.stream_interleave(parts, n)
+    assert np.array_equal(want, x)
+    assert np.array_equal(out.float().cpu().numpy().view(np.uint32), want.astype(np.float32).view(np.uint32))
+
+
+@pytest.mark.parametrize("R,W,dtype", [(2, 0, "bf16"), (4, 0, "bf16"), (2, 150, "bf16"), (4, 0, "f32")])
+def test_cross_prefill_shards(hd, R, W, dtype):
+    n, B, L, Hq, Hkv, D = 4, 1, 150, 4, 2, 128
+    P = n * L
+    q = synth.normal((B, P, Hq, D), 1011, dtype=dtype)
+    k = synth.normal((B, P, Hkv, D), 1012, dtype=dtype)
+    v = synth.normal((B, P, Hkv, D), 1013, dtype=dtype)
+    ro, rl = oracle.attn(q, k, v, n, "cross", W)
+    kparts = dev(np.stack([_shard(k, n, R, r) for r in range(R)]), dtype)
+    vparts = dev(np.stack([_shard(v, n, R, r) for r in range(R)]), dtype)
+    kd, vd = hd.hd_stream_interleave(kparts, n), hd.hd_stream_interleave(vparts, n)
+    tol = TOL_BF16 if dtype == "bf16" else TOL_F32
+    for r in range(R):
+        o, lse = hd.hd_attn_fwd_shard(dev(_shard(q, n, R, r), dtype), kd, vd, n, R, r, W, lse=True,
+                                      out_dtype=torch.float32)
+        torch.cuda.synchronize()
+        assert max_abs(to_f64(o), _shard(ro, n, R, r)) <= tol
+        want_lse = _shard(np.transpose(rl, (0, 2, 1)), n, R, r)  # [B, P_loc, Hq]
+        assert max_abs(np.transpose(to_f64(lse), (0, 2, 1)), want_lse) <= 1e-3
+
+
+@pytest.mark.parametrize("R", [2, 4])
+def test_intra_prefill_shards_need_no_exchange(hd, R):
+    n, B, L, H, D = 4, 1, 130, 2, 128
+    q = synth.normal((B, n * L, H, D), 1021, dtype="bf16")
+    k = synth.normal((B, n * L, H, D), 1022, dtype="bf16")
+    v = synth.normal((B, n * L, H, D), 1023, dtype="bf16")
+    ro, _ = oracle.attn(q, k, v, n, "intra")
+    for r in range(R):
+        o = hd.hd_attn_fwd(*(dev(_shard(x, n, R, r), "bf16") for x in (q, k, v)), n // R, "intra")
+        torch.cuda.synchronize()
+        assert max_abs(to_f64(o), _shard(ro, n, R, r)) <= TOL_BF16
+
+
+@pytest.mark.parametrize("R,T,W", [(2, 300, 0), (4, 300, 0), (4, 1, 0), (2, 70, 64), (4, 2, 5)])
+def test_cross_decode_shards_and_merge(hd, R, T, W):
+    n, B, Lmax, Hq, Hkv, D = 4, 2, 320, 8, 2, 128
+    q = synth.normal((B, n, Hq, D), 1031, dtype="bf16")
+    kc = synth.normal((B, n, Lmax, Hkv, D), 1032, dtype="bf16")
+    vc = synth.normal((B, n, Lmax, Hkv, D), 1033, dtype="bf16")
+    ctx = np.array([T, max(1, T // 2)], dtype=np.int32)
+    ctx_d = dev(ctx, "i32")
+    rows = [(b, s, h) for b in range(B) for s in range(n) for h in range(Hq)]
+    # The all-gather of the ranks' stream queries restores q.
+    qparts = np.stack([q[:, r::R] for r in range(R)])
+    qd = hd.hd_stream_interleave(dev(qparts, "bf16"), n)
+    torch.cuda.synchronize()
+    assert np.array_equal(qd.float().cpu().numpy(), q)
+    o_parts, l_parts = [], []
+    for r in range(R):
+        st = oracle.shard_streams(n, R, r)
+        o, lse = hd.hd_attn_decode_shard(qd, dev(kc[:, st].copy(), "bf16"), dev(vc[:, st].copy(), "bf16"), ctx_d,
+                                         R, r, W)
+        torch.cuda.synchronize()
+        ro, rl = oracle.decode_rows_streams(q, kc[:, st], vc[:, st], ctx, n, st, rows, W)
+        got_o = to_f64(o).reshape(-1, D)
+        got_l = to_f64(lse).reshape(-1)
+        empty = np.isneginf(rl)
+        assert np.array_equal(np.isneginf(got_l), empty)
+        assert not got_o[empty].any()
+        assert max_abs(got_o, ro) <= TOL_BF16
+        assert max_abs(got_l[~empty], rl[~empty]) <= 1e-3
+        o_parts.append(o)
+        l_parts.append(lse)
+    if T == 1:
+        assert torch.isneginf(torch.stack(l_parts)).any()
+    om, lm = hd.hd_attn_combine(torch.stack(o_parts), torch.stack(l_parts), out_dtype=torch.float32, lse=True)
+    torch.cuda.synchronize()
+    fo, fl = oracle.decode_rows(q, kc, vc, ctx, n, "cross", rows, W)
+    assert max_abs(to_f64(om).reshape(-1, D), fo) <= TOL_BF16
+    assert max_abs(to_f64(lm).reshape(-1), fl) <= 1e-3
+
+
+@pytest.mark.parametrize("in_dt,out_dt", [("f32", "f32"), ("bf16", "bf16"), ("f32", "bf16")])
+def test_combine_kernel(hd, in_dt, out_dt):
+    R, rows, D = 3, 257, 64
+    o = synth.normal((R, rows, D), 1041, dtype=in_dt)
+    l = synth.normal((R, rows), 1042).astype(np.float32) * 4
+    l[0, :7] = -np.inf          # some empty parts
+    l[:, 10] = -np.inf          # a row with every part empty
+    wo, wl = oracle.combine_partials(o, l)
+    go, gl = hd.hd_attn_combine(dev(o, in_dt), dev(l, "f32"),
+                                out_dtype=torch.bfloat16 if out_dt == "bf16" else torch.float32, lse=True)
+    torch.cuda.synchronize()
+    tol = TOL_BF16 if out_dt == "bf16" else TOL_F32
+    assert max_abs(to_f64(go), wo) <= tol
+    gl = to_f64(gl)
+    assert np.array_equal(np.isneginf(gl), np.isneginf(wl))
+    fin = np.isfinite(wl)
+    assert max_abs(gl[fin], wl[fin]) <= 1e-5
