@@ -593,6 +593,7 @@ def extras(torch, peaks, rank):
     res["rope"] = {"ms": round(ms, 3), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm"], 4)}
     del rp
     torch.cuda.empty_cache()
+    res.update(stream_parallel_rank(torch, peaks, rank, time_fn))
     for wl in ("bwd", "bwd_cross"):
         bw = Backward(WORKLOADS[wl], 7301 + rank, torch, hd, synth)
         ms = time_fn(lambda: bw.step())
@@ -601,6 +602,61 @@ def extras(torch, peaks, rank):
                                                   "frac_bf16": round(tf / peaks["bf16"], 4)}
         del bw
         torch.cuda.empty_cache()
+    return res
+
+
+def stream_parallel_rank(torch, peaks, rank, time_fn, R=4):
+    """Rank 0's share of a stream-parallel step with R ranks, timed on one GPU:
+    the re-interleave of the all-gathered K/V shards and the local queries'
+    cross-stream attention (cross workload sizes), and the cross-stream decode
+    partial over the rank's cache streams plus the merge of R partials
+    (decode workload sizes).  The all-gathers themselves need R GPUs."""
+    from stream_sequence_attention_b200 import accounting as acc
+    from stream_sequence_attention_b200 import hd, synth
+
+    res = {}
+    c = WORKLOADS["cross"]
+    B, n, L, Hq, Hkv, D = c["B"], c["n"], c["L"], c["Hq"], c["Hkv"], c["D"]
+    nl = n // R
+    q_loc = synth.normal_device((B, L * nl, Hq, D), 7501 + rank)
+    kparts = synth.normal_device((R, B, L * nl, Hkv, D), 7502 + rank)
+    vparts = synth.normal_device((R, B, L * nl, Hkv, D), 7503 + rank)
+    k = torch.empty((B, n * L, Hkv, D), dtype=torch.bfloat16, device="cuda")
+    v = torch.empty_like(k)
+    o = torch.empty_like(q_loc)
+    ms_il = time_fn(lambda: (hd.hd_stream_interleave(kparts, n, out=k), hd.hd_stream_interleave(vparts, n, out=v)))
+    il_bytes = 2 * 2 * k.numel() * k.element_size()
+    ms_at = time_fn(lambda: hd.hd_attn_fwd_shard(q_loc, k, v, n, R, 0, out=o))
+    fl = B * Hq * acc.pairs_cross_shard(L, n, R, 0) * 4 * D
+    res[f"sp_R{R}_rank0_cross_prefill"] = {
+        "interleave_ms": round(ms_il, 3), "interleave_GB/s": round(il_bytes / (ms_il * 1e-3) / 1e9, 1),
+        "attn_ms": round(ms_at, 3), "attn_TFLOP/s": round(fl / (ms_at * 1e-3) / 1e12, 1),
+        "attn_frac_bf16": round(fl / (ms_at * 1e-3) / 1e12 / peaks["bf16"], 4),
+        "allgather_bytes_in_per_rank": (R - 1) * 2 * kparts[0].numel() * 2}
+    del q_loc, kparts, vparts, k, v, o
+    torch.cuda.empty_cache()
+    d = WORKLOADS["decode"]
+    B, n, T, Hq, Hkv, D = d["B"], d["n"], d["T"], d["Hq"], d["Hkv"], d["D"]
+    q = synth.normal_device((B, n, Hq, D), 7511 + rank)
+    kc = synth.normal_device((B, n // R, T, Hkv, D), 7512 + rank)
+    vc = synth.normal_device((B, n // R, T, Hkv, D), 7513 + rank)
+    ctx = torch.full((B,), T, dtype=torch.int32, device="cuda")
+    op = torch.empty((B, n, Hq, D), dtype=torch.float32, device="cuda")
+    lp = torch.empty((B, n, Hq), dtype=torch.float32, device="cuda")
+    ws = torch.empty(hd.hd_attn_decode_workspace(B, n, T, Hq, Hkv, D, "cross"), dtype=torch.uint8, device="cuda")
+    ms_dec = time_fn(lambda: hd.hd_attn_decode_shard(q, kc, vc, ctx, R, 0, out=op, lse=lp, workspace=ws))
+    dec_bytes = 2 * kc.numel() * 2 + q.numel() * 2 + op.numel() * 4
+    o_all = op.unsqueeze(0).expand(R, -1, -1, -1, -1).contiguous()
+    l_all = lp.unsqueeze(0).expand(R, -1, -1, -1).contiguous()
+    out = torch.empty((B, n, Hq, D), dtype=torch.bfloat16, device="cuda")
+    ms_cb = time_fn(lambda: hd.hd_attn_combine(o_all, l_all, out=out))
+    res[f"sp_R{R}_rank0_cross_decode"] = {
+        "partial_ms": round(ms_dec, 3), "partial_GB/s": round(dec_bytes / (ms_dec * 1e-3) / 1e9, 1),
+        "partial_frac_hbm": round(dec_bytes / (ms_dec * 1e-3) / 1e9 / peaks["hbm"], 4),
+        "merge_ms": round(ms_cb, 4),
+        "allgather_bytes_in_per_rank": (R - 1) * (q.numel() // R * 2 + op.numel() * 4 + lp.numel() * 4)}
+    del q, kc, vc, op, lp, ws, o_all, l_all, out
+    torch.cuda.empty_cache()
     return res
 
 

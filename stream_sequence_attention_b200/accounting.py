@@ -96,3 +96,16 @@ def attn_bwd_min_bytes(B: int, L: int, n: int, Hq: int, Hkv: int, D: int, esize:
     """Read q, k, v, o, dO and lse once, write dq, dk, dv once."""
     P = n * L
     return B * P * (D * esize * (3 * Hq + 2 * Hkv + 2 * Hkv + Hq) + 4 * Hq)
+
+
+def pairs_cross_shard(L: int, n: int, R: int, r: int, window: int = 0) -> int:
+    """Visible pairs per (batch, query head) of rank r's queries in a
+    cross-stream layer under stream parallelism: positions p = i*n + r + R*l
+    see every p' <= p (within the window)."""
+    nl = n // R
+    total = 0
+    for i in range(L):
+        for l in range(nl):
+            vis = i * n + r + R * l + 1
+            total += vis if window <= 0 else min(vis, window)
+    return total

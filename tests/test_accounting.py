@@ -41,3 +41,10 @@ def test_final_stream_pairs_match_enumeration(L, n, mode, W):
     pk = np.arange(n * L)
     want = sum(int(np.count_nonzero(oracle.visible(i * n + n - 1, pk, n, mode, W))) for i in range(L))
     assert acc.pairs_final_stream(L, n, mode, W) == want
+
+
+def test_cross_shard_pairs_sum_to_the_full_cross_layer():
+    from stream_sequence_attention_b200 import accounting as acc
+    for n, R, L, W in [(4, 2, 9, 0), (4, 4, 7, 5), (6, 3, 5, 0), (2, 1, 11, 3)]:
+        parts = [acc.pairs_cross_shard(L, n, R, r, W) for r in range(R)]
+        assert sum(parts) == acc.pairs_per_head(L, n, "cross", W)
