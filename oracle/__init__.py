@@ -42,6 +42,7 @@ from .hd_oracle import (  # noqa: F401
     final_stream_gather,
     attn,
     attn_rows,
+    attn_rows_block,
     attn_bwd,
     attn_bwd_dq_rows,
     attn_bwd_dkv_rows,

@@ -368,6 +368,27 @@ def attn_rows(q, k, v, n, mode, rows, window=0, scale=None):
     return np.array(outs), np.array(lses)
 
 
+def attn_rows_block(q, k, v, n, mode, b, h, p0, p1, window=0, scale=None):
+    """Rows p0 <= p < p1 of :func:`attn` for one (b, h), in float64: the same
+    per-row definition evaluated for a block of query rows at once (so the
+    score block fits in memory at full sizes).  Keys past p1 - 1 are never
+    visible to these rows and are not formed.  Inputs may be any array-likes
+    indexable as q[b, p, h, :].  Returns (O [p1-p0, D], lse [p1-p0])."""
+    Hq, D = q.shape[2], q.shape[3]
+    G = Hq // k.shape[2]
+    kv = h // G
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    pq = np.arange(p0, p1)
+    pk = np.arange(p1)
+    mask = visible(pq[:, None], pk[None, :], n, mode, window)
+    qq = np.asarray(q[b, p0:p1, h, :], dtype=np.float64)
+    kk = np.asarray(k[b, :p1, kv, :], dtype=np.float64)
+    vv = np.asarray(v[b, :p1, kv, :], dtype=np.float64)
+    s = np.where(mask, scale * (qq @ kk.T), -np.inf)
+    return _softmax_weighted(s, vv)
+
+
 def attn_final_stream(q_final, k, v, n, mode, window=0, scale=None):
     """Attention of the final-stream queries only ("Persistent KV and the
     KV-mirror Saving": in a mirrored layer only the final stream is run,

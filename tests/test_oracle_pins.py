@@ -416,3 +416,14 @@ def test_final_stream_cross_pair_count_equals_intra():
         pk = np.arange(n * L)
         pairs = sum(int(np.count_nonzero(oracle.visible(i * n + n - 1, pk, n, "cross"))) for i in range(L))
         assert pairs == n * L * (L + 1) // 2
+
+
+@pytest.mark.parametrize("mode,W", [("intra", 0), ("cross", 0), ("intra", 3), ("cross", 5)])
+def test_attn_rows_block_matches_full_attention(mode, W):
+    n, L, Hq, Hkv, D = 3, 11, 4, 2, 8
+    q, k, v = _qkv(2, n * L, Hq, Hkv, D, 77)
+    O, lse = oracle.attn(q, k, v, n, mode, W)
+    for b, h, p0, p1 in [(0, 0, 0, 33), (1, 3, 5, 17), (1, 2, 32, 33), (0, 1, 0, 1)]:
+        o, l = oracle.attn_rows_block(q, k, v, n, mode, b, h, p0, p1, W)
+        np.testing.assert_allclose(o, O[b, p0:p1, h], rtol=1e-13, atol=1e-13)
+        np.testing.assert_allclose(l, lse[b, h, p0:p1], rtol=1e-13, atol=1e-13)
