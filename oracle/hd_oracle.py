@@ -280,6 +280,42 @@ def _bwd_row(q, k, v, dO, n, mode, b, h, p, G, window, scale):
     return keys, kk, pr, ds
 
 
+def attn_bwd_blocked(q, k, v, dO, n, mode, b, kvh, window=0, scale=None, block=1024):
+    """:func:`attn_bwd` for one (b, KV head), its query heads' rows taken in
+    blocks so the float64 score blocks fit in memory at full sizes: for each
+    query head of the group and each block of query rows, form the rows' S,
+    P, dP and dS over their visible keys (all keys before the block's end),
+    write the rows' dQ and add their terms to dK and dV.  Inputs may be any
+    array-likes indexable as q[b, p, h, :].  Returns (dQ [P, G, D] for the
+    group's query heads, dK [P, D], dV [P, D])."""
+    P, Hq, D = q.shape[1], q.shape[2], q.shape[3]
+    G = Hq // k.shape[2]
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    kk_all = np.asarray(k[b, :, kvh, :], dtype=np.float64)
+    vv_all = np.asarray(v[b, :, kvh, :], dtype=np.float64)
+    dQ = np.zeros((P, G, D))
+    dK = np.zeros((P, D))
+    dV = np.zeros((P, D))
+    for g in range(G):
+        h = kvh * G + g
+        for p0 in range(0, P, block):
+            p1 = min(P, p0 + block)
+            mask = visible(np.arange(p0, p1)[:, None], np.arange(p1)[None, :], n, mode, window)
+            qq = np.asarray(q[b, p0:p1, h, :], dtype=np.float64)
+            gg = np.asarray(dO[b, p0:p1, h, :], dtype=np.float64)
+            kk, vv = kk_all[:p1], vv_all[:p1]
+            s = np.where(mask, scale * (qq @ kk.T), -np.inf)
+            e = np.exp(s - s.max(axis=-1, keepdims=True))
+            pr = e / e.sum(axis=-1, keepdims=True)
+            dp = gg @ vv.T
+            ds = pr * (dp - (pr * dp).sum(axis=-1, keepdims=True))
+            dQ[p0:p1, g] = scale * (ds @ kk)
+            dK[:p1] += scale * (ds.T @ qq)
+            dV[:p1] += pr.T @ gg
+    return dQ, dK, dV
+
+
 def attn_bwd_dq_rows(q, k, v, dO, n, mode, rows, window=0, scale=None):
     """dQ of :func:`attn_bwd` for selected (b, h, p), one row at a time:
     dQ[p] = scale * sum over p's visible keys of dS[p, p'] k[p'].

@@ -113,3 +113,45 @@ def test_long_context_rows_of_every_head_and_stream(hd):
             got = to_f64(o[0, pos, h])
             worst = max(worst, float(np.max(np.abs(got - ro))))
     assert worst <= TOL_BF16, worst
+
+
+@pytest.mark.parametrize("mode", ["intra", "cross"])
+def test_backward_every_row(hd, mode):
+    """dQ, dK, dV of the full-size backward workload (forward then backward
+    through the library) against the blocked float64 oracle, every row."""
+    B, n, L, Hq, Hkv, D = 2, 4, 4096, 32, 8, 128
+    P, G = n * L, Hq // Hkv
+    q = synth.normal_device((B, P, Hq, D), 1301)
+    k = synth.normal_device((B, P, Hkv, D), 1302)
+    v = synth.normal_device((B, P, Hkv, D), 1303)
+    dO = synth.normal_device((B, P, Hq, D), 1304)
+    st = hd.new_status()
+    o, lse = hd.hd_attn_fwd(q, k, v, n, mode, lse=True, dev_status=st)
+    dq, dk, dv = hd.hd_attn_bwd(q, k, v, o, dO, lse, n, mode, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    qh, kh, vh, gh = _host(q), _host(k), _host(v), _host(dO)
+    dqh, dkh, dvh = _host(dq), _host(dk), _host(dv)
+    del q, k, v, dO, o, lse, dq, dk, dv
+    torch.cuda.empty_cache()
+    if mode == "intra":
+        units = [(b, s, kvh) for b in range(B) for s in range(n) for kvh in range(Hkv)]
+    else:
+        units = [(b, None, kvh) for b in range(B) for kvh in range(Hkv)]
+
+    def one(u):
+        b, s, kvh = u
+        hs = slice(kvh * G, (kvh + 1) * G)
+        if s is None:
+            rq, rk, rv = oracle.attn_bwd_blocked(qh, kh, vh, gh, n, "cross", b, kvh)
+            gq, gk, gv = dqh[b, :, hs], dkh[b, :, kvh], dvh[b, :, kvh]
+        else:
+            sl = lambda x: x[b:b + 1, s::n]  # noqa: E731
+            rq, rk, rv = oracle.attn_bwd_blocked(sl(qh), sl(kh), sl(vh), sl(gh), 1, "intra", 0, kvh)
+            gq, gk, gv = dqh[b, s::n, hs], dkh[b, s::n, kvh], dvh[b, s::n, kvh]
+        return tuple(float(np.max(np.abs(g - r))) / max(1.0, float(np.max(np.abs(r))))
+                     for g, r in ((gq, rq), (gk, rk), (gv, rv)))
+
+    with _blas_one_thread(), cf.ThreadPoolExecutor(_workers()) as ex:
+        errs = np.array(list(ex.map(one, units)))
+    assert errs.max() <= TOL_BF16, (errs.max(axis=0), units[int(np.argmax(errs.max(axis=1)))])

@@ -168,3 +168,18 @@ def test_bwd_query_row_terms_sum_to_full_backward(mode, W):
         sv[b, keys, h // G] += tv
     np.testing.assert_allclose(sk, dK, rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(sv, dV, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("mode,W", CASES)
+def test_bwd_blocked_matches_full_backward(mode, W):
+    n, L, Hq, Hkv, D = 3, 9, 4, 2, 6
+    q, k, v, dO = _inputs(2, L, n, Hq, Hkv, D, 71)
+    dQ, dK, dV = oracle.attn_bwd(q, k, v, dO, n, mode, W)
+    G = Hq // Hkv
+    for b in range(2):
+        for kvh in range(Hkv):
+            for block in (1, 5, 64):
+                bq, bk, bv = oracle.attn_bwd_blocked(q, k, v, dO, n, mode, b, kvh, W, block=block)
+                np.testing.assert_allclose(bq, dQ[b, :, kvh * G:(kvh + 1) * G], rtol=1e-12, atol=1e-12)
+                np.testing.assert_allclose(bk, dK[b, :, kvh], rtol=1e-12, atol=1e-12)
+                np.testing.assert_allclose(bv, dV[b, :, kvh], rtol=1e-12, atol=1e-12)
