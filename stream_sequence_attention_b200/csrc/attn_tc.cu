@@ -39,6 +39,7 @@
 // (round to nearest integer, cubic for 2^f on [-1/2, 1/2], exponent add;
 // relative error < 1e-4, below the bf16 rounding of P) to offload MUFU.
 #include <cstdlib>
+#include <cstring>
 
 #include "hd_common.cuh"
 #include "hd_launch.h"
@@ -496,19 +497,32 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
 // ------------------------------------------------------------------- host
 
 // (D, H, ns, Ls, B) view of a [B, ns*Ls, H, D] bf16 tensor; box = 64 x 1 x 1 x 128 x 1.
-bool encode_stream_view(CUtensorMap* m, const void* ptr, int B, int Ls, int ns, int H, int D) {
+static bool make_stream_view(const TmapKey& k, CUtensorMap* m) {
   EncodeTiledFn enc = get_encode_tiled();
   if (!enc) return false;
-  const cuuint64_t dims[5] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)ns, (cuuint64_t)Ls, (cuuint64_t)B};
+  const cuuint64_t B = k.dims[0], Ls = k.dims[1], ns = k.dims[2], H = k.dims[3], D = k.dims[4];
+  const cuuint64_t dims[5] = {D, H, ns, Ls, B};
   const cuuint64_t e = 2;
-  const cuuint64_t strides[4] = {(cuuint64_t)D * e, (cuuint64_t)H * D * e, (cuuint64_t)ns * H * D * e,
-                                 (cuuint64_t)Ls * ns * H * D * e};
+  const cuuint64_t strides[4] = {D * e, H * D * e, ns * H * D * e, Ls * ns * H * D * e};
   const cuuint32_t box[5] = {64, 1, 1, (cuuint32_t)tc::BM, 1};
   const cuuint32_t es[5] = {1, 1, 1, 1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box, es,
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(k.ptr), dims, strides, box, es,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool encode_stream_view(CUtensorMap* m, const void* ptr, int B, int Ls, int ns, int H, int D) {
+  TmapKey k;
+  std::memset(&k, 0, sizeof(k));
+  k.ptr = ptr;
+  k.dims[0] = B;
+  k.dims[1] = Ls;
+  k.dims[2] = ns;
+  k.dims[3] = H;
+  k.dims[4] = D;
+  k.kind = 1;
+  return tmap_cached(k, m, make_stream_view);
 }
 
 int attn_tc_smem_bytes(int D) { return D == 64 ? tc::Layout<64>::ALLOC : tc::Layout<128>::ALLOC; }

@@ -27,6 +27,8 @@
 // an online softmax that only rescales O when the row max rises by more than
 // 2^8.  The four warps' partial (max, sum, O) are merged in shared memory and
 // written to the workspace, and a small combine kernel merges the splits.
+#include <cstring>
+
 #include "hd_common.cuh"
 #include "hd_launch.h"
 
@@ -549,18 +551,30 @@ cudaError_t launch_attn_combine(const void* o_parts, const float* lse_parts, voi
 
 
 // (D, Hkv, Lmax, n, B) view of the [B, n, Lmax, Hkv, D] cache; box 64 x 1 x 64 x 1 x 1.
-static bool encode_cache_view(CUtensorMap* m, const void* ptr, int B, int n, int Lmax, int Hkv) {
+static bool make_cache_view(const TmapKey& k, CUtensorMap* m) {
   EncodeTiledFn enc = get_encode_tiled();
   if (!enc) return false;
+  const cuuint64_t B = k.dims[0], n = k.dims[1], Lmax = k.dims[2], Hkv = k.dims[3];
   const cuuint64_t D = dec::kD, e = 2;
-  const cuuint64_t dims[5] = {D, (cuuint64_t)Hkv, (cuuint64_t)Lmax, (cuuint64_t)n, (cuuint64_t)B};
-  const cuuint64_t strides[4] = {D * e, (cuuint64_t)Hkv * D * e, (cuuint64_t)Lmax * Hkv * D * e,
-                                 (cuuint64_t)n * Lmax * Hkv * D * e};
+  const cuuint64_t dims[5] = {D, Hkv, Lmax, n, B};
+  const cuuint64_t strides[4] = {D * e, Hkv * D * e, Lmax * Hkv * D * e, n * Lmax * Hkv * D * e};
   const cuuint32_t box[5] = {64, 1, (cuuint32_t)dec::kTok, 1, 1};
   const cuuint32_t es[5] = {1, 1, 1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box, es,
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(k.ptr), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static bool encode_cache_view(CUtensorMap* m, const void* ptr, int B, int n, int Lmax, int Hkv) {
+  TmapKey k;
+  std::memset(&k, 0, sizeof(k));
+  k.ptr = ptr;
+  k.dims[0] = B;
+  k.dims[1] = n;
+  k.dims[2] = Lmax;
+  k.dims[3] = Hkv;
+  k.kind = 2;
+  return tmap_cached(k, m, make_cache_view);
 }
 
 DecPlan decode_plan(int B, int n, int Lmax, int Hq, int Hkv, bool cross, int sms) {

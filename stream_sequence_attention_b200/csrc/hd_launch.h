@@ -38,6 +38,17 @@ struct AttnGeom {
   int o_rows, o_ns;
 };
 
+// Cache of encoded TMA maps (tmap_cache.cu).  The key is zero-initialised
+// and compared bytewise: base pointer, the view's dimensions, and a kind tag
+// naming the view (box and layout).
+struct TmapKey {
+  const void* ptr;
+  int64_t dims[5];
+  int32_t kind;
+  int32_t pad;
+};
+bool tmap_cached(const TmapKey& key, CUtensorMap* out, bool (*make)(const TmapKey&, CUtensorMap*));
+
 // TMA view (D, H, ns, Ls, B) of a [B, ns*Ls, H, D] bf16 tensor with a
 // 64 x 1 x 1 x 128 x 1 box and 128-byte swizzle: one box is 128 tokens of one
 // stream and head, 64 features wide.
