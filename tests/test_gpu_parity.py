@@ -236,3 +236,24 @@ def test_decode_bad_ctx_len_reports_and_zeros(hd):
     torch.cuda.synchronize()
     assert int(st.item()) == hd.HD_ERR_INVALID_ARG
     assert not o.float().abs().sum().item()
+
+
+def test_same_buffers_under_different_shapes(hd):
+    """The tensor maps are cached by (pointer, shape): one allocation viewed
+    with two different geometries gives the right result for both."""
+    buf_q = torch.empty(2 * 4 * 160 * 4 * 128, dtype=torch.bfloat16, device="cuda")
+    buf_k = torch.empty(2 * 4 * 160 * 2 * 128, dtype=torch.bfloat16, device="cuda")
+    buf_v = torch.empty_like(buf_k)
+    for (B, n, L, Hq, Hkv, seed) in [(2, 4, 160, 4, 2, 61), (1, 2, 320, 8, 4, 62), (2, 4, 160, 4, 2, 63)]:
+        P = n * L
+        q, k, v = host_qkv(B, P, Hq, Hkv, 128, seed, "bf16")
+        qd = buf_q.view(B, P, Hq, 128)
+        kd = buf_k.view(B, P, Hkv, 128)
+        vd = buf_v.view(B, P, Hkv, 128)
+        qd.copy_(dev(q, "bf16"))
+        kd.copy_(dev(k, "bf16"))
+        vd.copy_(dev(v, "bf16"))
+        o = hd.hd_attn_fwd(qd, kd, vd, n, "cross", out_dtype=torch.float32)
+        torch.cuda.synchronize()
+        ro, _ = oracle.attn(q, k, v, n, "cross")
+        assert max_abs(to_f64(o), ro) <= TOL_BF16
