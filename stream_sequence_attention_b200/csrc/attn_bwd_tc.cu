@@ -36,6 +36,8 @@
 // producer, 9 MMA issuer.  Persistent, longest units first.  Every wait is
 // bounded (1 s), after which the kernel records HD_ERR_TIMEOUT, lets its
 // copies land, drains its MMAs and frees tensor memory.
+#include <cstdlib>
+
 #include "hd_common.cuh"
 #include "hd_launch.h"
 
@@ -112,6 +114,10 @@ struct BwParams {
   int nblk;  // 128-token blocks per stream
   float scale_log2, scale;
   int total_units;
+  // Test hook (environment HD_TEST_STALL_BWD=1): the MMA warp of CTA 0 of
+  // the dK/dV kernel never signals its S tiles, so the elementwise wait runs
+  // out and the kernel must take its timeout path.  0 in normal use.
+  int stall_first_s;
 };
 
 // dK/dV unit: key block ascending (causal: the first blocks see the most
@@ -368,7 +374,7 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
       auto issue_S = [&](int tt) {
         const int st = tt % Lay::QST;
         mma_rows_rows<D>(tS, sbase + Lay::K_OFF, sbase + Lay::Q_OFF + st * T::TILE);
-        tc_commit(bar(Lay::B_SFULL));
+        if (!(p.stall_first_s && blockIdx.x == 0)) tc_commit(bar(Lay::B_SFULL));
       };
       auto issue_dP = [&](int tt) {
         const int st = tt % Lay::QST;
@@ -814,6 +820,11 @@ cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, cons
   p.nblk = p.Lpad / bw::BT;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.scale = scale;
+  static const int stall = [] {
+    const char* e = getenv("HD_TEST_STALL_BWD");
+    return (e && e[0] == '1') ? 1 : 0;
+  }();
+  p.stall_first_s = stall;
   const int64_t kv_units = static_cast<int64_t>(p.nblk) * g.B * g.ns * Hkv;
   const int64_t q_units = static_cast<int64_t>(p.nblk) * g.B * g.ns * Hq;
   if (q_units <= 0) return cudaSuccess;

@@ -27,6 +27,7 @@
 // an online softmax that only rescales O when the row max rises by more than
 // 2^8.  The four warps' partial (max, sum, O) are merged in shared memory and
 // written to the workspace, and a small combine kernel merges the splits.
+#include <cstdlib>
 #include <cstring>
 
 #include "hd_common.cuh"
@@ -61,6 +62,10 @@ struct DecParams {
   int32_t* status;
   int B, n, Lmax, Hq, Hkv, W, cross, nsplit, rg_count;
   int nc, soff, sstride;  // cache streams and their global stream ids
+  // Test hook (environment HD_TEST_STALL_DECODE=1): the producer of CTA
+  // (0, 0) issues no loads, so its compute warps' waits run out and the
+  // kernel must take its timeout path.  0 in normal use.
+  int stall_first;
   float scale_log2;
 };
 
@@ -202,7 +207,7 @@ __global__ void __launch_bounds__(DecShape<MT>::kThreads, MT == 2 ? HD_DEC_MT2_C
   __syncthreads();
 
   if (warp == kCompute) {
-    if (lane == 0 && ntiles > 0) {
+    if (lane == 0 && ntiles > 0 && !(p.stall_first && blockIdx.x == 0 && blockIdx.y == 0)) {
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       int issued[kStages] = {};
@@ -631,6 +636,11 @@ cudaError_t launch_decode(const void* q, const void* kc, const void* vc, const i
   p.nsplit = pl.nsplit;
   p.rg_count = pl.rg_count;
   p.scale_log2 = scale * 1.4426950408889634f;
+  static const int stall = [] {
+    const char* e = getenv("HD_TEST_STALL_DECODE");
+    return (e && e[0] == '1') ? 1 : 0;
+  }();
+  p.stall_first = stall;
   if (pl.units > 65535) return cudaErrorInvalidValue;
   dim3 grid(pl.nsplit, pl.units);
   cudaError_t err;

@@ -44,3 +44,57 @@ def test_attention_wait_times_out_cleanly():
     out = json.loads(r.stdout.strip().splitlines()[-1])
     assert out["status"] == 4  # HD_ERR_TIMEOUT
     assert out["usable"]
+
+
+CHILD_BWD = r"""
+import json, sys, torch
+sys.path.insert(0, ROOT)
+from stream_sequence_attention_b200 import build, hd, synth
+build.build(); hd.lib()
+q = synth.normal_device((1, 2 * 256, 4, 128), 1)
+k = synth.normal_device((1, 2 * 256, 2, 128), 2)
+v = synth.normal_device((1, 2 * 256, 2, 128), 3)
+dO = synth.normal_device((1, 2 * 256, 4, 128), 4)
+o, lse = hd.hd_attn_fwd(q, k, v, 2, "intra", lse=True)
+st = hd.new_status()
+hd.hd_attn_bwd(q, k, v, o, dO, lse, 2, "intra", dev_status=st)
+torch.cuda.synchronize()
+status = int(st.item())
+h = synth.normal_device((1, 2 * 64, 16), 5)
+g = hd.hd_final_stream_gather(h, 2)
+torch.cuda.synchronize()
+print(json.dumps({"status": status, "usable": bool(torch.equal(g, h[:, 1::2]))}))
+"""
+
+CHILD_DEC = r"""
+import json, sys, torch
+sys.path.insert(0, ROOT)
+from stream_sequence_attention_b200 import build, hd, synth
+build.build(); hd.lib()
+q = synth.normal_device((2, 4, 16, 128), 1)
+kc = synth.normal_device((2, 4, 256, 2, 128), 2)
+vc = synth.normal_device((2, 4, 256, 2, 128), 3)
+ctx = torch.full((2,), 256, dtype=torch.int32, device="cuda")
+st = hd.new_status()
+hd.hd_attn_decode(q, kc, vc, ctx, "cross", dev_status=st)
+torch.cuda.synchronize()
+status = int(st.item())
+h = synth.normal_device((1, 2 * 64, 16), 5)
+g = hd.hd_final_stream_gather(h, 2)
+torch.cuda.synchronize()
+print(json.dumps({"status": status, "usable": bool(torch.equal(g, h[:, 1::2]))}))
+"""
+
+
+@pytest.mark.parametrize("var,child", [("HD_TEST_STALL_BWD", "bwd"), ("HD_TEST_STALL_DECODE", "dec")])
+def test_backward_and_decode_waits_time_out_cleanly(var, child):
+    """The same bounded-wait path in the dK/dV backward kernel (its MMA warp of
+    CTA 0 never signals S) and in the decode kernel (the producer of its first
+    CTA issues no loads)."""
+    env = dict(os.environ, **{var: "1"})
+    code = (CHILD_BWD if child == "bwd" else CHILD_DEC).replace("ROOT", repr(ROOT))
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=180)
+    assert r.returncode == 0, r.stderr[-2000:]
+    out = json.loads(r.stdout.strip().splitlines()[-1])
+    assert out["status"] == 4  # HD_ERR_TIMEOUT
+    assert out["usable"]
