@@ -439,9 +439,10 @@ class Rope:
             h.copy_(t, non_blocking=True)
 
 
-def timed(torch, work, K, flush, dist=None, use_e2e=False):
+def timed(torch, work, K, flush, dist=None, use_e2e=False, parts=None):
     """Run K steps with per-step CUDA events (flush outside them).  Returns
-    (per-step ms list, dominant-kernel ms list)."""
+    (per-step ms list, dominant-kernel ms list); with ``parts`` (a list) it
+    also receives per-step (ms before the dominant kernel, ms after it)."""
     st = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     en = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
@@ -461,6 +462,8 @@ def timed(torch, work, K, flush, dist=None, use_e2e=False):
         dist.barrier()
     steps = [a.elapsed_time(b) for a, b in zip(st, en)]
     kern = [] if use_e2e else [a.elapsed_time(b) for a, b in kev]
+    if parts is not None and not use_e2e:
+        parts.extend((a.elapsed_time(k0), k1.elapsed_time(b)) for a, (k0, k1), b in zip(st, kev, en))
     return steps, kern
 
 
@@ -516,7 +519,8 @@ def run_ours(args, rank, world, dist):
 
     clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", 0)))
     clocks.start()
-    steps, kern = timed(torch, work, K, flush, dist)
+    parts = []
+    steps, kern = timed(torch, work, K, flush, dist, parts=parts)
     clk = clocks.stop()
     if args.profile:
         return {"profile": True, "ms_per_step": sum(steps) / K, "kernel_ms": statistics.mean(kern)}, work, peaks
@@ -602,6 +606,20 @@ def run_ours(args, rank, world, dist):
         "gpu_launches": work.launches_per_step * K,
         "clocks": clk,
     })
+    if isinstance(work, Prefill):
+        # expand runs before the attention in the step, the gather after it
+        from stream_sequence_attention_b200 import accounting as acc
+        exp_ms = statistics.mean(p[0] for p in parts)
+        gat_ms = statistics.mean(p[1] for p in parts)
+        eb = acc.expand_bytes(cfg["B"], cfg["L"], cfg["n"], cfg["dm"])
+        gb = acc.gather_bytes(cfg["B"], cfg["L"], cfg["dm"])
+        uniq = int(torch.unique(work.ids).numel())
+        out["expand"] = {"ms": round(exp_ms, 4), "GB/s": round(eb / (exp_ms * 1e-3) / 1e9, 1),
+                         "frac_hbm": round(eb / (exp_ms * 1e-3) / 1e9 / peaks["hbm"], 4),
+                         "unique_rows_per_table": uniq, "rows_per_table": cfg["B"] * cfg["L"],
+                         "note": "Zipf(1.1) ids repeat rows; L2 hits on repeats can lift this figure above HBM"}
+        out["gather"] = {"ms": round(gat_ms, 4), "GB/s": round(gb / (gat_ms * 1e-3) / 1e9, 1),
+                         "frac_hbm": round(gb / (gat_ms * 1e-3) / 1e9 / peaks["hbm"], 4)}
     return out, work, peaks
 
 
