@@ -131,3 +131,44 @@ def test_combine_kernel(hd, in_dt, out_dt):
     assert np.array_equal(np.isneginf(gl), np.isneginf(wl))
     fin = np.isfinite(wl)
     assert max_abs(gl[fin], wl[fin]) <= 1e-5
+
+
+def test_orchestration_runs_end_to_end_on_one_rank(hd):
+    """StreamParallel's calls (NCCL all-gathers, re-interleave, shard kernels,
+    merge) in a one-rank NCCL group on this GPU: with R = 1 every layer must
+    equal the plain single-GPU result, here checked against the oracle."""
+    import os
+    import socket
+
+    import torch.distributed as dist
+
+    from stream_sequence_attention_b200 import stream_parallel as sp
+
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("nccl", rank=0, world_size=1)
+    try:
+        n, B, L, Hq, Hkv, D = 4, 1, 130, 4, 2, 128
+        view = sp.StreamParallel(n)
+        assert (view.R, view.r, view.streams) == (1, 0, [0, 1, 2, 3])
+        q, k, v = (synth.normal((B, n * L, H, D), 1051 + i, dtype="bf16") for i, H in enumerate((Hq, Hkv, Hkv)))
+        qd, kd, vd = dev(q, "bf16"), dev(k, "bf16"), dev(v, "bf16")
+        oc = view.cross_attention(qd, kd, vd, out_dtype=torch.float32)
+        oi = view.intra_attention(qd, kd, vd, out_dtype=torch.float32)
+        torch.cuda.synchronize()
+        assert max_abs(to_f64(oc), oracle.attn(q, k, v, n, "cross")[0]) <= TOL_BF16
+        assert max_abs(to_f64(oi), oracle.attn(q, k, v, n, "intra")[0]) <= TOL_BF16
+        Lmax, T = 200, 150
+        qd_ = synth.normal((2, n, 8, D), 1061, dtype="bf16")
+        kc = synth.normal((2, n, Lmax, Hkv, D), 1062, dtype="bf16")
+        vc = synth.normal((2, n, Lmax, Hkv, D), 1063, dtype="bf16")
+        ctx = np.array([T, 7], dtype=np.int32)
+        od = view.cross_decode(dev(qd_, "bf16"), dev(kc, "bf16"), dev(vc, "bf16"), dev(ctx, "i32"))
+        torch.cuda.synchronize()
+        ref, _ = oracle.decode(qd_, kc, vc, ctx, n, "cross")
+        assert max_abs(to_f64(od), ref) <= TOL_BF16
+    finally:
+        dist.destroy_process_group()
