@@ -91,11 +91,19 @@ def load_peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
 
 
+HOST_MARKER = b"// ------------------------------------------------------------------- host"
+
+
 def kernel_source_sha(names):
+    """Hash of the device part of the named sources (each file up to its
+    host-code marker): a recorded traffic figure stays valid across host-side
+    edits and turns stale when a kernel changes."""
     h = hashlib.sha256()
     for nm in names:
         with open(os.path.join(ROOT, "stream_sequence_attention_b200", "csrc", nm), "rb") as f:
-            h.update(f.read())
+            src = f.read()
+        cut = src.find(HOST_MARKER)
+        h.update(src if cut < 0 else src[:cut])
     return h.hexdigest()[:16]
 
 

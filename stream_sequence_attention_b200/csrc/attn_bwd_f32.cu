@@ -81,6 +81,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const void* __restrict__ 
   }
 }
 
+// ------------------------------------------------------------------- host
+
 cudaError_t launch_bwd_prep(const void* o, const void* dO, const float* lse, BwdWs ws, const AttnGeom& g, int Hq,
                             int D, bool bf16, cudaStream_t st) {
   const int64_t rows = static_cast<int64_t>(g.B) * g.ns * g.Lq * Hq;

@@ -100,6 +100,8 @@ __global__ void __launch_bounds__(kCopyThreads) stream_interleave_kernel(
   }
 }
 
+// ------------------------------------------------------------------- host
+
 static int copy_grid(int64_t rows, int sms) {
   const int64_t warps_per_cta = kCopyThreads / 32;
   int64_t want = (rows + warps_per_cta - 1) / warps_per_cta;

@@ -191,6 +191,8 @@ __global__ void __launch_bounds__(kRopeThreads) rope_kernel(const RopeParams p) 
   }
 }
 
+// ------------------------------------------------------------------- host
+
 cudaError_t launch_rope(const RopeParams& p, bool bf16, cudaStream_t st) {
   const int64_t rows = static_cast<int64_t>(p.B) * p.P;
   if (rows <= 0) return cudaSuccess;
