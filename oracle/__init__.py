@@ -45,6 +45,7 @@ from .hd_oracle import (  # noqa: F401
     attn_rows_block,
     attn_bwd,
     attn_bwd_blocked,
+    attn_bwd_final_stream,
     attn_bwd_dq_rows,
     attn_bwd_dkv_rows,
     attn_bwd_query_rows,

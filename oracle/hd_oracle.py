@@ -280,6 +280,43 @@ def _bwd_row(q, k, v, dO, n, mode, b, h, p, G, window, scale):
     return keys, kk, pr, ds
 
 
+def attn_bwd_final_stream(q_final, k, v, dO_final, n, mode, window=0, scale=None):
+    """Gradient of :func:`attn_final_stream` (the KV-mirror layers are trained
+    through too): the derivative of sum(dO_final * O_final), O_final the
+    final-stream queries' attention over every stream's keys.  Per (b, h),
+    with S = scale q_final k^T over the keys visible to position i*n + n-1:
+        dV = P^T dO,  dS = P * (dO V^T - rowsum(P * dO V^T)),
+        dQ = scale dS K,  dK = scale dS^T Q  (dK, dV summed over a GQA group).
+    Returns (dQ [B, L, Hq, D], dK [B, nL, Hkv, D], dV [B, nL, Hkv, D]); keys no
+    final-stream query sees get zero."""
+    q_final = np.asarray(q_final, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    dO_final = np.asarray(dO_final, dtype=np.float64)
+    B, L, Hq, D = q_final.shape
+    P, Hkv = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    mask = visible((np.arange(L) * n + n - 1)[:, None], np.arange(P)[None, :], n, mode, window)
+    dQ = np.zeros((B, L, Hq, D))
+    dK = np.zeros((B, P, Hkv, D))
+    dV = np.zeros((B, P, Hkv, D))
+    for b in range(B):
+        for h in range(Hq):
+            kv = h // G
+            s = np.where(mask, scale * (q_final[b, :, h, :] @ k[b, :, kv, :].T), -np.inf)
+            e = np.exp(s - s.max(axis=-1, keepdims=True))
+            pr = e / e.sum(axis=-1, keepdims=True)
+            g = dO_final[b, :, h, :]
+            dp = g @ v[b, :, kv, :].T
+            ds = pr * (dp - (pr * dp).sum(axis=-1, keepdims=True))
+            dV[b, :, kv, :] += pr.T @ g
+            dQ[b, :, h, :] = scale * (ds @ k[b, :, kv, :])
+            dK[b, :, kv, :] += scale * (ds.T @ q_final[b, :, h, :])
+    return dQ, dK, dV
+
+
 def attn_bwd_blocked(q, k, v, dO, n, mode, b, kvh, window=0, scale=None, block=1024):
     """:func:`attn_bwd` for one (b, KV head), its query heads' rows taken in
     blocks so the float64 score blocks fit in memory at full sizes: for each

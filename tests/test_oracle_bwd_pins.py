@@ -183,3 +183,45 @@ def test_bwd_blocked_matches_full_backward(mode, W):
                 np.testing.assert_allclose(bq, dQ[b, :, kvh * G:(kvh + 1) * G], rtol=1e-12, atol=1e-12)
                 np.testing.assert_allclose(bk, dK[b, :, kvh], rtol=1e-12, atol=1e-12)
                 np.testing.assert_allclose(bv, dV[b, :, kvh], rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("mode,W", CASES)
+def test_final_stream_bwd_is_the_full_bwd_with_only_final_rows(mode, W):
+    # The final-stream queries are the rows i*n + n-1 of the full layer: with
+    # those rows of q and dO and zero output gradient elsewhere, the full
+    # backward gives the same dK, dV and the same dQ on those rows.
+    n, L, Hq, Hkv, D = 3, 5, 4, 2, 6
+    q, k, v, dO = _inputs(2, L, n, Hq, Hkv, D, 81)
+    qf, gf = q[:, n - 1::n], dO[:, n - 1::n]
+    dO0 = np.zeros_like(dO)
+    dO0[:, n - 1::n] = gf
+    fq, fk, fv = oracle.attn_bwd(q, k, v, dO0, n, mode, W)
+    gq, gk, gv = oracle.attn_bwd_final_stream(qf, k, v, gf, n, mode, W)
+    np.testing.assert_allclose(gq, fq[:, n - 1::n], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(gk, fk, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(gv, fv, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("mode,W", CASES)
+def test_final_stream_bwd_matches_finite_differences(mode, W):
+    n, L, Hq, Hkv, D, h = 2, 3, 2, 1, 3, 1e-6
+    q, k, v, dO = _inputs(1, L, n, Hq, Hkv, D, 91)
+    qf, gf = q[:, n - 1::n].copy(), dO[:, n - 1::n]
+
+    def f(a, b_, c):
+        return float(np.sum(gf * oracle.attn_final_stream(a, b_, c, n, mode, W, 0.7)[0]))
+
+    got = oracle.attn_bwd_final_stream(qf, k, v, gf, n, mode, W, 0.7)
+    for which, x in enumerate((qf, k, v)):
+        args = [qf.copy(), k.copy(), v.copy()]
+        fd = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            i = it.multi_index
+            args[which][i] = x[i] + h
+            fp = f(*args)
+            args[which][i] = x[i] - h
+            fm = f(*args)
+            args[which][i] = x[i]
+            fd[i] = (fp - fm) / (2 * h)
+        np.testing.assert_allclose(got[which], fd, rtol=1e-6, atol=1e-7)
