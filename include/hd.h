@@ -139,6 +139,28 @@ hd_status hd_attn_bwd(const void* q, const void* k, const void* v, const void* o
                       int window, float scale, hd_dtype dt, void* workspace,
                       size_t ws_bytes, int32_t* dev_status, void* stream);
 
+/*
+ * Backward of hd_attn_fwd_final_stream (the KV-mirror layers are trained
+ * through too): the gradient of the final-stream queries' attention with
+ * respect to q_final and to every stream's k and v.  Same definition as
+ * hd_attn_bwd with the query rows at positions i*n + n-1.
+ *
+ *   q_final, o_final, dO_final, dq_final [B, L, Hq, D]  element type `dt`
+ *   k, v, dk, dv                         [B, n*L, Hkv, D] element type `dt`
+ *   lse_final [B, Hq, L] float32 from hd_attn_fwd_final_stream (required)
+ *   workspace: >= hd_attn_bwd_workspace(B, L, 1, Hq, HD_INTRA) bytes (L query
+ *              rows in one stream), 256-byte aligned.
+ * Keys no final-stream query sees (intra mode: the streams 0 .. n-2) get
+ * dk = dv = 0.  Same argument rules and kernels as hd_attn_bwd.
+ */
+hd_status hd_attn_bwd_final_stream(const void* q_final, const void* k, const void* v,
+                                   const void* o_final, const void* dO_final,
+                                   const float* lse_final, void* dq_final, void* dk,
+                                   void* dv, int B, int L, int n, int Hq, int Hkv, int D,
+                                   hd_mode mode, int window, float scale, hd_dtype dt,
+                                   void* workspace, size_t ws_bytes, int32_t* dev_status,
+                                   void* stream);
+
 /* Workspace bytes hd_attn_bwd needs for these sizes (0 on invalid sizes).
  * It holds two floats per (b, query head, position), padded per stream to a
  * multiple of 128 tokens. */

@@ -134,12 +134,14 @@ __global__ void __launch_bounds__(kBwThreads) attn_bwd_dq_f32_kernel(
   const int h = hs / g.ns, s = hs - h * g.ns;
   const int b = blockIdx.z;
   const int kvh = h / (Hq / Hkv);
+  const int skv = g.kv_stream >= 0 ? g.kv_stream : s;
   const int tid = threadIdx.x, r = tid >> 2, part = tid & 3;
   const int q0 = qblk * kBwRows;
   const int i = q0 + r;
   const bool row_ok = i < g.Lq;
   const int ic = row_ok ? i : g.Lq - 1;
-  const int64_t qrow = ((static_cast<int64_t>(b) * g.ns * g.Lq + static_cast<int64_t>(ic) * g.ns + s) * Hq + h) * D;
+  const int pic = ic * g.qstride + g.qoff;  // key index of this query
+  const int64_t qrow = ((static_cast<int64_t>(b) * g.q_ns * g.Lq + static_cast<int64_t>(ic) * g.q_ns + s) * Hq + h) * D;
   float qr[DQ], dor[DQ], acc[DQ];
 #pragma unroll
   for (int d = 0; d < DQ; ++d) {
@@ -149,10 +151,10 @@ __global__ void __launch_bounds__(kBwThreads) attn_bwd_dq_f32_kernel(
   }
   const int64_t lat = ((static_cast<int64_t>(b) * Hq + h) * g.ns + s) * bwd_lpad(g.Lq) + ic;
   const float2 ld = make_float2(ws.l2[lat], ws.delta[lat]);
-  const int hi = min(q0 + kBwRows - 1, g.Lq - 1);
-  const int lo = W > 0 ? max(0, q0 - W + 1) : 0;
-  const int64_t kv_stride = static_cast<int64_t>(g.ns) * Hkv * D;
-  const int64_t kv_base = (static_cast<int64_t>(b) * g.ns * g.Lq * Hkv + static_cast<int64_t>(s) * Hkv + kvh) * D;
+  const int hi = min(min(q0 + kBwRows - 1, g.Lq - 1) * g.qstride + g.qoff, g.Lk - 1);
+  const int lo = W > 0 ? max(0, q0 * g.qstride + g.qoff - W + 1) : 0;
+  const int64_t kv_stride = static_cast<int64_t>(g.kv_ns) * Hkv * D;
+  const int64_t kv_base = (static_cast<int64_t>(b) * g.kv_ns * g.Lk * Hkv + static_cast<int64_t>(skv) * Hkv + kvh) * D;
   for (int k0 = lo; k0 <= hi; k0 += kBwTile) {
     __syncthreads();
     for (int e = tid; e < kBwTile * (D / 4); e += kBwThreads) {
@@ -178,7 +180,7 @@ __global__ void __launch_bounds__(kBwThreads) attn_bwd_dq_f32_kernel(
       sd = quad_sum(sd);
       pd = quad_sum(pd);
       const int j = k0 + c;
-      const bool vis = j <= hi && j <= ic && (W <= 0 || ic - j < W);
+      const bool vis = j <= hi && j <= pic && (W <= 0 || pic - j < W);
       const float p = vis ? exp2f(sd - ld.x) : 0.f;
       const float ds = p * (pd - ld.y);
 #pragma unroll
@@ -202,16 +204,20 @@ __global__ void __launch_bounds__(kBwThreads) attn_bwd_dkv_f32_kernel(
   __shared__ __align__(16) float Os[kBwTile][D];
   __shared__ float2 Ls[kBwTile];
   const int kblk = blockIdx.x;  // causal: the first key blocks have the most queries
-  const int hs = blockIdx.y;    // kvh * ns + s
-  const int kvh = hs / g.ns, s = hs - kvh * g.ns;
+  const int kns = g.kv_stream >= 0 ? 1 : g.kv_ns;
+  const int hs = blockIdx.y;    // kvh * kns + key stream
+  const int kvh = hs / kns, ks = hs - kvh * kns;
+  const int skv = g.kv_stream >= 0 ? g.kv_stream : ks;  // stream of the K/V view
+  const int s = g.kv_stream >= 0 ? 0 : ks;              // query stream reading it
   const int b = blockIdx.z;
   const int G = Hq / Hkv;
   const int tid = threadIdx.x, r = tid >> 2, part = tid & 3;
   const int k0 = kblk * kBwRows;
   const int j = k0 + r;
-  const bool row_ok = j < g.Lq;
-  const int jc = row_ok ? j : g.Lq - 1;
-  const int64_t krow = ((static_cast<int64_t>(b) * g.ns * g.Lq + static_cast<int64_t>(jc) * g.ns + s) * Hkv + kvh) * D;
+  const bool row_ok = j < g.Lk;
+  const int jc = row_ok ? j : g.Lk - 1;
+  const int64_t krow =
+      ((static_cast<int64_t>(b) * g.kv_ns * g.Lk + static_cast<int64_t>(jc) * g.kv_ns + skv) * Hkv + kvh) * D;
   float kr[DQ], vr[DQ], ak[DQ], av[DQ];
 #pragma unroll
   for (int d = 0; d < DQ; ++d) {
@@ -220,13 +226,14 @@ __global__ void __launch_bounds__(kBwThreads) attn_bwd_dkv_f32_kernel(
     ak[d] = 0.f;
     av[d] = 0.f;
   }
-  const int lo = k0;
-  const int hi = W > 0 ? min(g.Lq - 1, k0 + kBwRows - 1 + W - 1) : g.Lq - 1;
+  // queries with k0 <= pos(i) (and pos(i) - (k0 + 63) < W), pos(i) = i*qstride + qoff
+  const int lo = k0 <= g.qoff ? 0 : (k0 - g.qoff + g.qstride - 1) / g.qstride;
+  const int hi = W > 0 ? min(g.Lq - 1, (k0 + kBwRows - 1 + W - 1 - g.qoff) / g.qstride) : g.Lq - 1;
   const int Lpad = bwd_lpad(g.Lq);
-  const int64_t q_stride = static_cast<int64_t>(g.ns) * Hq * D;
+  const int64_t q_stride = static_cast<int64_t>(g.q_ns) * Hq * D;
   for (int hh = 0; hh < G; ++hh) {
     const int h = kvh * G + hh;
-    const int64_t q_base = (static_cast<int64_t>(b) * g.ns * g.Lq * Hq + static_cast<int64_t>(s) * Hq + h) * D;
+    const int64_t q_base = (static_cast<int64_t>(b) * g.q_ns * g.Lq * Hq + static_cast<int64_t>(s) * Hq + h) * D;
     const int64_t l_base = ((static_cast<int64_t>(b) * Hq + h) * g.ns + s) * Lpad;
     for (int i0 = lo; i0 <= hi; i0 += kBwTile) {
       __syncthreads();
@@ -256,7 +263,8 @@ __global__ void __launch_bounds__(kBwThreads) attn_bwd_dkv_f32_kernel(
         sd = quad_sum(sd);
         pd = quad_sum(pd);
         const int i = i0 + c;
-        const bool vis = i <= hi && i >= jc && (W <= 0 || i - jc < W);
+        const int pi = i * g.qstride + g.qoff;
+        const bool vis = i <= hi && pi >= jc && (W <= 0 || pi - jc < W);
         const float2 l = Ls[c];
         const float p = vis ? exp2f(sd - l.x) : 0.f;
         const float ds = p * (pd - l.y);
@@ -280,8 +288,16 @@ cudaError_t launch_attn_bwd_f32(const float* q, const float* k, const float* v, 
                                 float* dq, float* dk, float* dv, const AttnGeom& g, int Hq, int Hkv, int D, int W,
                                 float scale, cudaStream_t st) {
   const int nb = (g.Lq + kBwRows - 1) / kBwRows;
+  const int nkb = (g.Lk + kBwRows - 1) / kBwRows;
+  const int kns = g.kv_stream >= 0 ? 1 : g.kv_ns;
   const float sl2 = scale * 1.4426950408889634f;
-  const dim3 gq(nb, Hq * g.ns, g.B), gk(nb, Hkv * g.ns, g.B);
+  const dim3 gq(nb, Hq * g.ns, g.B), gk(nkb, Hkv * kns, g.B);
+  if (g.kv_stream >= 0 && g.kv_ns > 1) {  // key streams no query reads: zero gradients
+    const size_t bytes = static_cast<size_t>(g.B) * g.kv_ns * g.Lk * Hkv * D * sizeof(float);
+    cudaError_t e = cudaMemsetAsync(dk, 0, bytes, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, bytes, st);
+    if (e != cudaSuccess) return e;
+  }
   if (D == 64) {
     attn_bwd_dq_f32_kernel<64><<<gq, kBwThreads, 0, st>>>(q, k, v, dO, ws, dq, g, Hq, Hkv, W, sl2, scale);
     attn_bwd_dkv_f32_kernel<64><<<gk, kBwThreads, 0, st>>>(q, k, v, dO, ws, dk, dv, g, Hq, Hkv, W, sl2, scale);

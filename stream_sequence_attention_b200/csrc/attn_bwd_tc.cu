@@ -110,8 +110,11 @@ struct BwParams {
   void* dk;
   void* dv;
   int32_t* status;
-  int B, ns, Lq, Lpad, Hq, Hkv, W;
-  int nblk;  // 128-token blocks per stream
+  AttnGeom g;  // query token i of stream s sits at key index i*qstride + qoff
+  int Lpad, Hq, Hkv, W;
+  int nqb;  // 128-token query blocks per query stream
+  int nkb;  // 128-token key blocks per key stream
+  int kns;  // key streams the dK/dV kernel walks
   float scale_log2, scale;
   int total_units;
   // Test hook (environment HD_TEST_STALL_BWD=1): the MMA warp of CTA 0 of
@@ -120,50 +123,63 @@ struct BwParams {
   int stall_first_s;
 };
 
+// Key index of query token i (of any query stream; the backward takes no
+// per-stream offset).
+__device__ __forceinline__ int bw_pos(const BwParams& p, int i) { return i * p.g.qstride + p.g.qoff; }
+
 // dK/dV unit: key block ascending (causal: the first blocks see the most
-// query tiles), then (b, s, kvh).  Its tiles j = 0 .. G*nqt-1 walk the query
-// tiles from the last one down, the G heads of the group inside: the CTAs
-// that run the other key blocks of the same (b, s, kvh) at the same time
-// then read the same Q and dO tiles, which stay in L2.
+// query tiles), then (b, key stream, kvh).  Its tiles j = 0 .. G*nqt-1 walk
+// the query tiles that see the block from the last one down, the G heads of
+// the group inside: the CTAs that run the other key blocks of the same
+// (b, stream, kvh) at the same time then read the same Q and dO tiles, which
+// stay in L2.  nqt = 0 when no query sees the block (its dK, dV are zero).
 struct KvUnit {
-  int b, s, kvh, kblk, qt_lo, qt_hi, nqt;
+  int b, skv, sq, kvh, kblk, qt_lo, qt_hi, nqt;
 };
 __device__ __forceinline__ KvUnit kv_unit(int u, const BwParams& p) {
-  const int per = p.B * p.ns * p.Hkv;
+  const int per = p.g.B * p.kns * p.Hkv;
   KvUnit x;
   x.kblk = u / per;
   int rem = u - x.kblk * per;
   x.kvh = rem % p.Hkv;
   rem /= p.Hkv;
-  x.s = rem % p.ns;
-  x.b = rem / p.ns;
+  const int ks = rem % p.kns;
+  x.b = rem / p.kns;
+  x.skv = p.g.kv_stream >= 0 ? p.g.kv_stream : ks;  // stream of the K/V view
+  x.sq = p.g.kv_stream >= 0 ? 0 : ks;               // query stream reading it
   const int k0 = x.kblk * bw::BT;
-  x.qt_lo = x.kblk;  // queries >= first key of the block
-  x.qt_hi = p.W > 0 ? min(p.nblk - 1, (k0 + bw::BT - 1 + p.W - 1) / bw::BT) : p.nblk - 1;
-  x.nqt = x.qt_hi - x.qt_lo + 1;
+  // queries with k0 <= pos(i) (and pos(i) - (k0 + 127) < W)
+  const int i_lo = k0 <= p.g.qoff ? 0 : (k0 - p.g.qoff + p.g.qstride - 1) / p.g.qstride;
+  const int i_hi = p.W > 0 ? min(p.g.Lq - 1, (k0 + bw::BT - 1 + p.W - 1 - p.g.qoff) / p.g.qstride) : p.g.Lq - 1;
+  x.qt_lo = i_lo / bw::BT;
+  x.qt_hi = i_hi / bw::BT;
+  x.nqt = i_lo <= i_hi ? x.qt_hi - x.qt_lo + 1 : 0;
   return x;
 }
 __device__ __forceinline__ int kv_tile_qt(const KvUnit& x, int j, int G) { return x.qt_hi - j / G; }
 __device__ __forceinline__ int kv_tile_head(const KvUnit& x, int j, int G) { return x.kvh * G + j % G; }
 
 // dQ unit: query block descending (causal: the last blocks see the most key
-// tiles), then (b, s, h).
+// tiles), then (b, query stream, h).
 struct QUnit {
-  int b, s, h, qblk, kt_lo, nkt;
+  int b, s, skv, h, qblk, kt_lo, nkt;
 };
 __device__ __forceinline__ QUnit q_unit(int u, const BwParams& p) {
-  const int per = p.B * p.ns * p.Hq;
+  const int per = p.g.B * p.g.ns * p.Hq;
   QUnit x;
   const int qi = u / per;
   int rem = u - qi * per;
-  x.qblk = p.nblk - 1 - qi;
+  x.qblk = p.nqb - 1 - qi;
   x.h = rem % p.Hq;
   rem /= p.Hq;
-  x.s = rem % p.ns;
-  x.b = rem / p.ns;
+  x.s = rem % p.g.ns;
+  x.b = rem / p.g.ns;
+  x.skv = p.g.kv_stream >= 0 ? p.g.kv_stream : x.s;
   const int q0 = x.qblk * bw::BT;
-  x.kt_lo = p.W > 0 ? max(0, q0 - p.W + 1) / bw::BT : 0;
-  x.nkt = x.qblk - x.kt_lo + 1;
+  const int qlast = min(q0 + bw::BT - 1, p.g.Lq - 1);
+  const int kt_hi = bw_pos(p, qlast) / bw::BT;
+  x.kt_lo = p.W > 0 ? max(0, bw_pos(p, q0) - p.W + 1) / bw::BT : 0;
+  x.nkt = kt_hi - x.kt_lo + 1;
   return x;
 }
 
@@ -320,9 +336,9 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
         mbar_arrive_expect_tx(bar(Lay::B_KVFULL), 2 * T::TILE);
 #pragma unroll
         for (int kb = 0; kb < T::KB; ++kb) {
-          tma_load_5d(sbase + Lay::K_OFF + kb * T::BLK, &tmK, bar(Lay::B_KVFULL), kb * 64, x.kvh, x.s,
+          tma_load_5d(sbase + Lay::K_OFF + kb * T::BLK, &tmK, bar(Lay::B_KVFULL), kb * 64, x.kvh, x.skv,
                       x.kblk * bw::BT, x.b);
-          tma_load_5d(sbase + Lay::V_OFF + kb * T::BLK, &tmV, bar(Lay::B_KVFULL), kb * 64, x.kvh, x.s,
+          tma_load_5d(sbase + Lay::V_OFF + kb * T::BLK, &tmV, bar(Lay::B_KVFULL), kb * 64, x.kvh, x.skv,
                       x.kblk * bw::BT, x.b);
         }
         ++kv_issued;
@@ -337,9 +353,9 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
 #pragma unroll
           for (int kb = 0; kb < T::KB; ++kb)
             tma_load_5d(sbase + Lay::Q_OFF + st * T::TILE + kb * T::BLK, &tmQ, bar(Lay::B_QFULL + st), kb * 64, h,
-                        x.s, qt * bw::BT, x.b);
+                        x.sq, qt * bw::BT, x.b);
           {
-            const int64_t at = ((static_cast<int64_t>(x.b) * p.Hq + h) * p.ns + x.s) * p.Lpad + qt * bw::BT;
+            const int64_t at = ((static_cast<int64_t>(x.b) * p.Hq + h) * p.g.ns + x.sq) * p.Lpad + qt * bw::BT;
             bulk_load(sbase + Lay::LD_OFF + st * bw::kLdBytes, p.ws.l2 + at, bw::kLdBytes / 2,
                       bar(Lay::B_QFULL + st));
             bulk_load(sbase + Lay::LD_OFF + st * bw::kLdBytes + bw::kLdBytes / 2, p.ws.delta + at,
@@ -351,7 +367,7 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
 #pragma unroll
           for (int kb = 0; kb < T::KB; ++kb)
             tma_load_5d(sbase + Lay::O_OFF + st * T::TILE + kb * T::BLK, &tmO, bar(Lay::B_OFULL + st), kb * 64, h,
-                        x.s, qt * bw::BT, x.b);
+                        x.sq, qt * bw::BT, x.b);
           ++o_issued[st];
         }
       }
@@ -385,6 +401,11 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
         const KvUnit x = kv_unit(u, p);
         const int nt = G * x.nqt;
         if (!mbar_wait(bar(Lay::B_KVFULL), ul & 1, abort_flag)) { ok = false; break; }
+        if (nt == 0) {  // no query sees this key block: nothing to accumulate
+          tc_commit(bar(Lay::B_ACCFULL));
+          tc_commit(bar(Lay::B_KVEMPTY));
+          continue;
+        }
         if (!mbar_wait(bar(Lay::B_QFULL + t % Lay::QST), (t / Lay::QST) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         issue_S(t);
@@ -453,7 +474,7 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
         const float4* l4 = reinterpret_cast<const float4*>(smem + Lay::LD_OFF + st * bw::kLdBytes) + 16 * ch;
         const float4* d4 = reinterpret_cast<const float4*>(smem + Lay::LD_OFF + st * bw::kLdBytes + 512) + 16 * ch;
         tmem_wait_ld();
-        const bool need_mask = (q0 < k0 + bw::BT - 1) || (p.W > 0 && q0 + 63 - k0 >= p.W);
+        const bool need_mask = (bw_pos(p, q0) < k0 + bw::BT - 1) || (p.W > 0 && bw_pos(p, q0 + 63) - k0 >= p.W);
         float pv[64];
 #pragma unroll
         for (int c4 = 0; c4 < 16; ++c4) {
@@ -467,8 +488,8 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
         if (need_mask) {
 #pragma unroll
           for (int c = 0; c < 64; ++c) {
-            const int i = q0 + c;
-            if (i < jkey || (p.W > 0 && i - jkey >= p.W)) pv[c] = 0.f;
+            const int pi = bw_pos(p, q0 + c);
+            if (pi < jkey || (p.W > 0 && pi - jkey >= p.W)) pv[c] = 0.f;
           }
         }
         {
@@ -511,14 +532,23 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
       const bool got = mbar_wait(bar(Lay::B_ACCFULL), ul & 1, abort_flag);
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
-      const bool row_ok = jkey < p.Lq;
-      const int64_t orow =
-          ((static_cast<int64_t>(x.b) * p.ns * p.Lq + static_cast<int64_t>(row_ok ? jkey : 0) * p.ns + x.s) * p.Hkv +
-           x.kvh) * D + ch * (D / 2);
-      acc_half_to_global<D>(tmem + lane_addr + 256 + ch * (D / 2), static_cast<__nv_bfloat16*>(p.dv) + orow, 1.f,
-                            row_ok);
-      acc_half_to_global<D>(tmem + lane_addr + 256 + D + ch * (D / 2), static_cast<__nv_bfloat16*>(p.dk) + orow,
-                            p.scale, row_ok);
+      const bool row_ok = jkey < p.g.Lk;
+      const int64_t orow = ((static_cast<int64_t>(x.b) * p.g.kv_ns * p.g.Lk +
+                             static_cast<int64_t>(row_ok ? jkey : 0) * p.g.kv_ns + x.skv) * p.Hkv + x.kvh) * D +
+                           ch * (D / 2);
+      if (nt == 0) {  // no query sees these keys
+        if (row_ok) {
+          uint4* a = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dv) + orow);
+          uint4* c = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dk) + orow);
+#pragma unroll
+          for (int e = 0; e < D / 16; ++e) a[e] = c[e] = make_uint4(0, 0, 0, 0);
+        }
+      } else {
+        acc_half_to_global<D>(tmem + lane_addr + 256 + ch * (D / 2), static_cast<__nv_bfloat16*>(p.dv) + orow, 1.f,
+                              row_ok);
+        acc_half_to_global<D>(tmem + lane_addr + 256 + D + ch * (D / 2), static_cast<__nv_bfloat16*>(p.dk) + orow,
+                              p.scale, row_ok);
+      }
       tc_fence_before();
       mbar_arrive(bar(Lay::B_ACCEMPTY));
     }
@@ -622,7 +652,7 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
 #pragma unroll
           for (int kb = 0; kb < T::KB; ++kb)
             tma_load_5d(sbase + Lay::K_OFF + ks * T::TILE + kb * T::BLK, &tmK, bar(Lay::B_KFULL + ks), kb * 64, kvh,
-                        x.s, kt * bw::BT, x.b);
+                        x.skv, kt * bw::BT, x.b);
           ++k_issued[ks];
           const int vs = t % Lay::VST;
           if (!mbar_wait(bar(Lay::B_VEMPTY + vs), ((t / Lay::VST) & 1) ^ 1, abort_flag)) { ok = false; break; }
@@ -630,7 +660,7 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
 #pragma unroll
           for (int kb = 0; kb < T::KB; ++kb)
             tma_load_5d(sbase + Lay::V_OFF + vs * T::TILE + kb * T::BLK, &tmV, bar(Lay::B_VFULL + vs), kb * 64, kvh,
-                        x.s, kt * bw::BT, x.b);
+                        x.skv, kt * bw::BT, x.b);
           ++v_issued[vs];
         }
       }
@@ -703,7 +733,8 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
     for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++ul) {
       const QUnit x = q_unit(u, p);
       const int iq = x.qblk * bw::BT + r;  // this thread's query token
-      const int64_t lat = ((static_cast<int64_t>(x.b) * p.Hq + x.h) * p.ns + x.s) * p.Lpad + iq;
+      const int64_t lat = ((static_cast<int64_t>(x.b) * p.Hq + x.h) * p.g.ns + x.s) * p.Lpad + iq;
+      const int piq = bw_pos(p, iq);  // key index of this thread's query
       const float2 ld = make_float2(p.ws.l2[lat], p.ws.delta[lat]);
       for (int j = 0; j < x.nkt; ++j, ++t) {
         const int k0 = (x.kt_lo + j) * bw::BT + 64 * ch;  // first key of this half
@@ -716,7 +747,8 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
         tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
         tmem_wait_ld();
         const int qfirst = x.qblk * bw::BT;
-        const bool need_mask = (k0 + 63 > qfirst) || (p.W > 0 && k0 < qfirst + bw::BT - 1 - p.W + 1);
+        const bool need_mask =
+            (k0 + 63 > bw_pos(p, qfirst)) || (p.W > 0 && k0 < bw_pos(p, qfirst + bw::BT - 1) - p.W + 1);
         float pv[64];
 #pragma unroll
         for (int c = 0; c < 64; ++c) pv[c] = ex2(fmaf(__uint_as_float(sv[c]), sl2, -ld.x));
@@ -724,7 +756,7 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
 #pragma unroll
           for (int c = 0; c < 64; ++c) {
             const int jk = k0 + c;
-            if (jk > iq || (p.W > 0 && iq - jk >= p.W)) pv[c] = 0.f;
+            if (jk > piq || (p.W > 0 && piq - jk >= p.W)) pv[c] = 0.f;
           }
         }
         got = mbar_wait(bar(Lay::B_DPFULL), t & 1, abort_flag);
@@ -756,10 +788,10 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
       const bool got = mbar_wait(bar(Lay::B_ACCFULL), ul & 1, abort_flag);
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
-      const bool row_ok = iq < p.Lq;
-      const int64_t orow =
-          ((static_cast<int64_t>(x.b) * p.ns * p.Lq + static_cast<int64_t>(row_ok ? iq : 0) * p.ns + x.s) * p.Hq +
-           x.h) * D + ch * (D / 2);
+      const bool row_ok = iq < p.g.Lq;
+      const int64_t orow = ((static_cast<int64_t>(x.b) * p.g.q_ns * p.g.Lq +
+                             static_cast<int64_t>(row_ok ? iq : 0) * p.g.q_ns + x.s) * p.Hq + x.h) * D +
+                           ch * (D / 2);
       acc_half_to_global<D>(tmem + lane_addr + 384 + ch * (D / 2), static_cast<__nv_bfloat16*>(p.dq) + orow, p.scale,
                             row_ok);
       tc_fence_before();
@@ -801,8 +833,8 @@ cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, cons
                                void* dq, void* dk, void* dv, const AttnGeom& g, int Hq, int Hkv, int D, int W,
                                float scale, int32_t* status, int sms, cudaStream_t st) {
   CUtensorMap mq, mk, mv, mo;
-  if (!encode_stream_view(&mq, q, g.B, g.Lq, g.ns, Hq, D) || !encode_stream_view(&mk, k, g.B, g.Lq, g.ns, Hkv, D) ||
-      !encode_stream_view(&mv, v, g.B, g.Lq, g.ns, Hkv, D) || !encode_stream_view(&mo, dO, g.B, g.Lq, g.ns, Hq, D))
+  if (!encode_stream_view(&mq, q, g.B, g.Lq, g.q_ns, Hq, D) || !encode_stream_view(&mk, k, g.B, g.Lk, g.kv_ns, Hkv, D) ||
+      !encode_stream_view(&mv, v, g.B, g.Lk, g.kv_ns, Hkv, D) || !encode_stream_view(&mo, dO, g.B, g.Lq, g.q_ns, Hq, D))
     return cudaErrorInvalidValue;
   BwParams p;
   p.ws = ws;
@@ -810,14 +842,14 @@ cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, cons
   p.dk = dk;
   p.dv = dv;
   p.status = status;
-  p.B = g.B;
-  p.ns = g.ns;
-  p.Lq = g.Lq;
+  p.g = g;
   p.Lpad = bwd_lpad(g.Lq);
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.W = W;
-  p.nblk = p.Lpad / bw::BT;
+  p.nqb = p.Lpad / bw::BT;
+  p.nkb = (g.Lk + bw::BT - 1) / bw::BT;
+  p.kns = g.kv_stream >= 0 ? 1 : g.kv_ns;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.scale = scale;
   static const int stall = [] {
@@ -825,10 +857,18 @@ cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, cons
     return (e && e[0] == '1') ? 1 : 0;
   }();
   p.stall_first_s = stall;
-  const int64_t kv_units = static_cast<int64_t>(p.nblk) * g.B * g.ns * Hkv;
-  const int64_t q_units = static_cast<int64_t>(p.nblk) * g.B * g.ns * Hq;
+  // Key streams no query reads (a single read stream of several) get zero
+  // gradients; the kernel writes the read stream's.
+  if (g.kv_stream >= 0 && g.kv_ns > 1) {
+    const size_t bytes = static_cast<size_t>(g.B) * g.kv_ns * g.Lk * Hkv * D * 2;
+    cudaError_t e = cudaMemsetAsync(dk, 0, bytes, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, bytes, st);
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t kv_units = static_cast<int64_t>(p.nkb) * g.B * p.kns * Hkv;
+  const int64_t q_units = static_cast<int64_t>(p.nqb) * g.B * g.ns * Hq;
   if (q_units <= 0) return cudaSuccess;
-  if (q_units > 0x7fffffff) return cudaErrorInvalidValue;
+  if (q_units > 0x7fffffff || kv_units > 0x7fffffff) return cudaErrorInvalidValue;
   if (D == 64) return launch_bwd_tc_d<64>(mq, mk, mv, mo, p, (int)kv_units, (int)q_units, sms, st);
   return launch_bwd_tc_d<128>(mq, mk, mv, mo, p, (int)kv_units, (int)q_units, sms, st);
 }

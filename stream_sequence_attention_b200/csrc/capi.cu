@@ -116,6 +116,33 @@ static AttnGeom regular_geom(int B, int L, int n, hd_mode mode) {
   return g;
 }
 
+// Queries: the L final-stream rows.  Intra: they read stream n-1 of the
+// interleaved K/V in place.  Cross: query i sits at position i*n + n-1 of the
+// single nL-position stream.
+static AttnGeom final_stream_geom(int B, int L, int n, hd_mode mode) {
+  AttnGeom g;
+  g.B = B;
+  g.ns = 1;
+  g.Lq = L;
+  g.q_ns = 1;
+  g.o_rows = L;
+  g.o_ns = 1;
+  if (mode == HD_INTRA) {
+    g.kv_ns = n;
+    g.Lk = L;
+    g.kv_stream = n - 1;
+    g.qstride = 1;
+    g.qoff = 0;
+  } else {
+    g.kv_ns = 1;
+    g.Lk = n * L;
+    g.kv_stream = -1;
+    g.qstride = n;
+    g.qoff = n - 1;
+  }
+  return g;
+}
+
 static hd_status run_attn(const void* q, const void* k, const void* v, void* o, float* lse, const AttnGeom& g,
                           int Hq, int Hkv, int D, int window, float scale, hd_dtype in_dt, hd_dtype out_dt,
                           int32_t* dev_status, void* stream) {
@@ -147,29 +174,7 @@ hd_status hd_attn_fwd_final_stream(const void* q_final, const void* k, const voi
                                    hd_dtype in_dt, hd_dtype out_dt, int32_t* dev_status, void* stream) {
   hd_status stt = check_attn_args(q_final, k, v, o, lse, B, L, n, Hq, Hkv, D, mode, window, scale, in_dt, out_dt);
   if (stt != HD_OK || B == 0) return stt;
-  // Queries: the L final-stream rows.  Intra: they read stream n-1 of the
-  // interleaved K/V in place.  Cross: query i sits at position i*n + n-1 of
-  // the single nL-position stream.
-  AttnGeom g;
-  g.B = B;
-  g.ns = 1;
-  g.Lq = L;
-  g.q_ns = 1;
-  g.o_rows = L;
-  g.o_ns = 1;
-  if (mode == HD_INTRA) {
-    g.kv_ns = n;
-    g.Lk = L;
-    g.kv_stream = n - 1;
-    g.qstride = 1;
-    g.qoff = 0;
-  } else {
-    g.kv_ns = 1;
-    g.Lk = n * L;
-    g.kv_stream = -1;
-    g.qstride = n;
-    g.qoff = n - 1;
-  }
+  const AttnGeom g = final_stream_geom(B, L, n, mode);
   return run_attn(q_final, k, v, o, lse, g, Hq, Hkv, D, window, scale, in_dt, out_dt, dev_status, stream);
 }
 
@@ -180,24 +185,22 @@ size_t hd_attn_bwd_workspace(int B, int L, int n, int Hq, hd_mode mode) {
   return static_cast<size_t>(2 * bwd_plane(g, Hq)) * sizeof(float);
 }
 
-hd_status hd_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
-                      void* dq, void* dk, void* dv, int B, int L, int n, int Hq, int Hkv, int D, hd_mode mode,
-                      int window, float scale, hd_dtype dt, void* workspace, size_t ws_bytes, int32_t* dev_status,
-                      void* stream) {
-  hd_status stt = check_attn_args(q, k, v, dq, nullptr, B, L, n, Hq, Hkv, D, mode, window, scale, dt, dt);
-  if (stt != HD_OK || B == 0) return stt;
+static hd_status run_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                              const float* lse, void* dq, void* dk, void* dv, const AttnGeom& g, int Hq, int Hkv,
+                              int D, int window, float scale, hd_dtype dt, void* workspace, size_t ws_bytes,
+                              int32_t* dev_status, void* stream) {
   if (!o || !dO || !lse || !dk || !dv || !workspace || !aligned16(o) || !aligned16(dO) || !aligned16(dk) ||
       !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return HD_ERR_INVALID_ARG;
-  if (ws_bytes < hd_attn_bwd_workspace(B, L, n, Hq, mode)) return HD_ERR_INVALID_ARG;
-  const AttnGeom g = regular_geom(B, L, n, mode);
+  if (ws_bytes < static_cast<size_t>(2 * bwd_plane(g, Hq)) * sizeof(float)) return HD_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const BwdWs ws = bwd_ws(workspace, g, Hq);
   const bool bf16 = dt == HD_BF16;
   cudaError_t e = launch_bwd_prep(o, dO, lse, ws, g, Hq, D, bf16, st);
   if (e != cudaSuccess) return HD_ERR_CUDA;
   if (!bf16) {
-    if (static_cast<int64_t>(Hq) * g.ns > 65535 || g.B > 65535) return HD_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(Hq) * g.ns > 65535 || static_cast<int64_t>(Hkv) * g.kv_ns > 65535 || g.B > 65535)
+      return HD_ERR_UNSUPPORTED;
     return cuda_status(launch_attn_bwd_f32(static_cast<const float*>(q), static_cast<const float*>(k),
                                            static_cast<const float*>(v), static_cast<const float*>(dO), ws,
                                            static_cast<float*>(dq), static_cast<float*>(dk), static_cast<float*>(dv),
@@ -207,6 +210,27 @@ hd_status hd_attn_bwd(const void* q, const void* k, const void* v, const void* o
   if (sms <= 0) return HD_ERR_CUDA;
   return cuda_status(
       launch_attn_bwd_tc(q, k, v, dO, ws, dq, dk, dv, g, Hq, Hkv, D, window, scale, dev_status, sms, st));
+}
+
+hd_status hd_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                      void* dq, void* dk, void* dv, int B, int L, int n, int Hq, int Hkv, int D, hd_mode mode,
+                      int window, float scale, hd_dtype dt, void* workspace, size_t ws_bytes, int32_t* dev_status,
+                      void* stream) {
+  hd_status stt = check_attn_args(q, k, v, dq, nullptr, B, L, n, Hq, Hkv, D, mode, window, scale, dt, dt);
+  if (stt != HD_OK || B == 0) return stt;
+  return run_attn_bwd(q, k, v, o, dO, lse, dq, dk, dv, regular_geom(B, L, n, mode), Hq, Hkv, D, window, scale, dt,
+                      workspace, ws_bytes, dev_status, stream);
+}
+
+hd_status hd_attn_bwd_final_stream(const void* q_final, const void* k, const void* v, const void* o_final,
+                                   const void* dO_final, const float* lse_final, void* dq_final, void* dk, void* dv,
+                                   int B, int L, int n, int Hq, int Hkv, int D, hd_mode mode, int window, float scale,
+                                   hd_dtype dt, void* workspace, size_t ws_bytes, int32_t* dev_status,
+                                   void* stream) {
+  hd_status stt = check_attn_args(q_final, k, v, dq_final, nullptr, B, L, n, Hq, Hkv, D, mode, window, scale, dt, dt);
+  if (stt != HD_OK || B == 0) return stt;
+  return run_attn_bwd(q_final, k, v, o_final, dO_final, lse_final, dq_final, dk, dv, final_stream_geom(B, L, n, mode),
+                      Hq, Hkv, D, window, scale, dt, workspace, ws_bytes, dev_status, stream);
 }
 
 size_t hd_attn_decode_workspace(int B, int n, int Lmax, int Hq, int Hkv, int D, hd_mode mode) {

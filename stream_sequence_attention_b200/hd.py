@@ -29,6 +29,7 @@ EXPORTS = (
     "hd_attn_fwd",
     "hd_attn_fwd_final_stream",
     "hd_attn_bwd",
+    "hd_attn_bwd_final_stream",
     "hd_attn_bwd_workspace",
     "hd_attn_decode",
     "hd_attn_decode_workspace",
@@ -72,6 +73,8 @@ def lib() -> ctypes.CDLL:
         L.hd_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, f32,
                                   i32, vp, sz, vp, vp]
         L.hd_attn_bwd.restype = i32
+        L.hd_attn_bwd_final_stream.argtypes = L.hd_attn_bwd.argtypes
+        L.hd_attn_bwd_final_stream.restype = i32
         L.hd_attn_bwd_workspace.argtypes = [i32, i32, i32, i32, i32]
         L.hd_attn_bwd_workspace.restype = sz
         L.hd_attn_decode.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, f32, i32, i32,
@@ -326,6 +329,48 @@ def hd_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tens
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), B, L, n, Hq, Hkv, D,
         _MODES[mode], int(window), float(scale), _dt(q), _ptr(workspace), workspace.numel(), _ptr(dev_status),
         _stream(stream)))
+    return dq, dk, dv
+
+
+def hd_attn_bwd_final_stream(q_final: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o_final: torch.Tensor,
+                             dO_final: torch.Tensor, lse_final: torch.Tensor, n: int, mode="intra", window: int = 0,
+                             scale: float | None = None, dq: torch.Tensor | None = None,
+                             dk: torch.Tensor | None = None, dv: torch.Tensor | None = None,
+                             workspace: torch.Tensor | None = None, dev_status: torch.Tensor | None = None,
+                             stream=None):
+    """Backward of :func:`hd_attn_fwd_final_stream`: returns (dq_final, dk, dv).
+
+    q_final/o_final/dO_final [B, L, Hq, D], k/v [B, n*L, Hkv, D] (one dtype),
+    lse_final [B, Hq, L] float32 from the forward."""
+    for t, nm in ((q_final, "q_final"), (k, "k"), (v, "v"), (o_final, "o_final"), (dO_final, "dO_final"),
+                  (lse_final, "lse_final")):
+        _need(t, nm)
+    B, L, Hq, D = q_final.shape
+    Hkv = k.shape[2]
+    if k.shape != (B, n * L, Hkv, D) or v.shape != k.shape or o_final.shape != q_final.shape or \
+            dO_final.shape != q_final.shape:
+        raise ValueError("q_final/k/v/o_final/dO_final shapes disagree")
+    if any(t.dtype != q_final.dtype for t in (k, v, o_final, dO_final)):
+        raise ValueError("dtypes disagree")
+    if lse_final.shape != (B, Hq, L) or lse_final.dtype != torch.float32:
+        raise ValueError("lse_final must be float32 [B, Hq, L]")
+    if scale is None:
+        scale = D ** -0.5
+    dq = torch.empty_like(q_final) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for t, ref, nm in ((dq, q_final, "dq"), (dk, k, "dk"), (dv, v, "dv")):
+        _need(t, nm)
+        if t.shape != ref.shape or t.dtype != ref.dtype:
+            raise ValueError(f"{nm} has the wrong shape or dtype")
+    need = hd_attn_bwd_workspace(B, L, 1, Hq, "intra")
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q_final.device)
+    _need(workspace, "workspace")
+    _check("hd_attn_bwd_final_stream", lib().hd_attn_bwd_final_stream(
+        _ptr(q_final), _ptr(k), _ptr(v), _ptr(o_final), _ptr(dO_final), _ptr(lse_final), _ptr(dq), _ptr(dk),
+        _ptr(dv), B, L, n, Hq, Hkv, D, _MODES[mode], int(window), float(scale), _dt(q_final), _ptr(workspace),
+        workspace.numel(), _ptr(dev_status), _stream(stream)))
     return dq, dk, dv
 
 

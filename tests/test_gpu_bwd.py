@@ -156,3 +156,55 @@ def test_bwd_full_size_sampled(hd, mode):
         worst = max(worst, max_abs(gk, rk) / max(1.0, float(np.max(np.abs(rk)))))
         worst = max(worst, max_abs(gv, rv) / max(1.0, float(np.max(np.abs(rv)))))
     assert worst <= TOL_BF16, worst
+
+
+FS_CASES = [
+    # dtype, mode, W, B, L, n, Hq, Hkv, D
+    ("bf16", "intra", 0, 2, 300, 4, 4, 2, 128),
+    ("bf16", "cross", 0, 1, 260, 4, 4, 1, 128),
+    ("bf16", "cross", 100, 1, 200, 3, 2, 2, 64),
+    ("bf16", "cross", 2, 1, 150, 4, 2, 2, 128),   # window < n: some keys seen by no query
+    ("f32", "intra", 0, 1, 130, 3, 2, 1, 64),
+    ("f32", "cross", 50, 1, 90, 2, 2, 2, 128),
+]
+
+
+@pytest.mark.parametrize("dtype,mode,W,B,L,n,Hq,Hkv,D", FS_CASES)
+def test_final_stream_bwd_matches_oracle(hd, dtype, mode, W, B, L, n, Hq, Hkv, D):
+    P = n * L
+    scale = D ** -0.5
+    qf = synth.normal((B, L, Hq, D), 1400 + L, dtype=dtype)
+    k = synth.normal((B, P, Hkv, D), 1401 + L, dtype=dtype)
+    v = synth.normal((B, P, Hkv, D), 1402 + L, dtype=dtype)
+    gf = synth.normal((B, L, Hq, D), 1403 + L, dtype=dtype)
+    of, lf = oracle.attn_final_stream(qf, k, v, n, mode, W, scale)
+    rq, rk, rv = oracle.attn_bwd_final_stream(qf, k, v, gf, n, mode, W, scale)
+    st = hd.new_status()
+    dk0 = torch.full(k.shape, 7.0, dtype=torch.bfloat16 if dtype == "bf16" else torch.float32, device="cuda")
+    dq, dk, dv = hd.hd_attn_bwd_final_stream(dev(qf, dtype), dev(k, dtype), dev(v, dtype), dev(_round(of, dtype), dtype),
+                                             dev(gf, dtype), dev(lf, "f32"), n, mode, W, scale, dk=dk0,
+                                             dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    tol = TOL_BF16 if dtype == "bf16" else TOL_F32
+    for name, got, ref in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+        err = max_abs(to_f64(got), ref)
+        assert err <= _bound(ref, tol), (name, err)
+    if mode == "intra":  # keys of streams 0..n-2 are seen by no final-stream query
+        assert not to_f64(dk)[:, np.arange(P) % n != n - 1].any()
+
+
+def test_final_stream_bwd_chain(hd):
+    """Forward and backward of the final-stream call through the library."""
+    B, L, n, Hq, Hkv, D = 1, 260, 4, 4, 2, 128
+    qf = synth.normal((B, L, Hq, D), 1501, dtype="bf16")
+    k = synth.normal((B, n * L, Hkv, D), 1502, dtype="bf16")
+    v = synth.normal((B, n * L, Hkv, D), 1503, dtype="bf16")
+    gf = synth.normal((B, L, Hq, D), 1504, dtype="bf16")
+    qd, kd, vd = dev(qf, "bf16"), dev(k, "bf16"), dev(v, "bf16")
+    for mode in ("intra", "cross"):
+        of, lf = hd.hd_attn_fwd_final_stream(qd, kd, vd, n, mode, lse=True)
+        grads = hd.hd_attn_bwd_final_stream(qd, kd, vd, of, dev(gf, "bf16"), lf, n, mode)
+        torch.cuda.synchronize()
+        for got, ref in zip(grads, oracle.attn_bwd_final_stream(qf, k, v, gf, n, mode)):
+            assert max_abs(to_f64(got), ref) <= _bound(ref, TOL_BF16)
