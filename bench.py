@@ -719,12 +719,24 @@ def stream_parallel_rank(torch, peaks, rank, time_fn, R=4):
     il_bytes = 2 * 2 * k.numel() * k.element_size()
     ms_at = time_fn(lambda: hd.hd_attn_fwd_shard(q_loc, k, v, n, R, 0, out=o))
     fl = B * Hq * acc.pairs_cross_shard(L, n, R, 0) * 4 * D
+    # The same rows straight from the gathered shards (no re-interleave), and
+    # the fused form that copies the R-1 other shards inside the kernel (here
+    # from this GPU's memory, so the copies compete for HBM, not NVLink).
+    ms_parts = time_fn(lambda: hd.hd_attn_fwd_parts(q_loc, kparts, vparts, n, R, 0, out=o))
+    kd = torch.empty_like(kparts)
+    vd = torch.empty_like(vparts)
+    flags = torch.empty(max(1, hd.hd_attn_peer_flags_bytes(B, L, n) // 8), dtype=torch.int64, device="cuda")
+    ms_fused = time_fn(lambda: hd.hd_attn_fwd_peer_gather(q_loc, list(kparts), list(vparts), kd, vd, n, R, 0,
+                                                          flags=flags, out=o))
+    tf = lambda ms: round(fl / (ms * 1e-3) / 1e12, 1)  # noqa: E731
     res[f"sp_R{R}_rank0_cross_prefill"] = {
         "interleave_ms": round(ms_il, 3), "interleave_GB/s": round(il_bytes / (ms_il * 1e-3) / 1e9, 1),
-        "attn_ms": round(ms_at, 3), "attn_TFLOP/s": round(fl / (ms_at * 1e-3) / 1e12, 1),
+        "attn_ms": round(ms_at, 3), "attn_TFLOP/s": tf(ms_at),
         "attn_frac_bf16": round(fl / (ms_at * 1e-3) / 1e12 / peaks["bf16"], 4),
+        "parts_ms": round(ms_parts, 3), "parts_TFLOP/s": tf(ms_parts),
+        "peer_gather_ms": round(ms_fused, 3), "peer_gather_TFLOP/s": tf(ms_fused),
         "allgather_bytes_in_per_rank": (R - 1) * 2 * kparts[0].numel() * 2}
-    del q_loc, kparts, vparts, k, v, o
+    del q_loc, kparts, vparts, k, v, o, kd, vd, flags
     torch.cuda.empty_cache()
     d = WORKLOADS["decode"]
     B, n, T, Hq, Hkv, D = d["B"], d["n"], d["T"], d["Hq"], d["Hkv"], d["D"]

@@ -307,6 +307,69 @@ hd_status hd_attn_decode_shard(const void* q, const void* k_cache_loc,
                                hd_dtype out_dt, void* workspace, size_t ws_bytes,
                                int32_t* dev_status, void* stream);
 
+/*
+ * Cross-stream prefill without the re-interleaved copy.  The operation is
+ * that of hd_attn_fwd_shard (rank r's queries, HD_CROSS rules over all n*L
+ * keys), with the keys and values given as the R ranks' shards:
+ *
+ *   k_parts[rho], v_parts[rho]  host arrays of R device pointers; rank rho's
+ *       shard [B, (n/R)*L, Hkv, D], whose row i*(n/R) + l holds token i of
+ *       global stream rho + R*l (e.g. the R slots of an all-gather).
+ *
+ * A 128-key tile of the expanded order is 128/R consecutive rows of every
+ * shard, so the kernel reads the shards where they lie.  bf16 input only;
+ * 1 <= R <= HD_MAX_RANKS, R divides n, n divides 128.  Other arguments and
+ * errors as hd_attn_fwd_shard.  The shards are read many times: they belong
+ * in this GPU's memory (for peers' memory use hd_attn_fwd_peer_gather).
+ */
+#define HD_MAX_RANKS 8
+hd_status hd_attn_fwd_parts(const void* q_loc, const void* const* k_parts,
+                            const void* const* v_parts, void* o_loc, float* lse, int B,
+                            int L, int n, int R, int r, int Hq, int Hkv, int D, int window,
+                            float scale, hd_dtype in_dt, hd_dtype out_dt,
+                            int32_t* dev_status, void* stream);
+
+/*
+ * hd_attn_fwd_parts with the exchange fused in.  k_src[rho], v_src[rho]
+ * (rho != r) are the other ranks' shards, normally peer memory (hd_ipc_open):
+ * a warp in every CTA copies each of them once into k_dst[rho], v_dst[rho]
+ * (this GPU, same shape), in key-tile order, while the attention runs; each
+ * key tile is read only after its own pieces have landed.  k_src[r],
+ * v_src[r] are this rank's shard, read in place (k_dst[r], v_dst[r] unused).
+ *   flags  device workspace of hd_attn_peer_flags_bytes(B, L, n) bytes,
+ *          zeroed by the call on `stream`.
+ * The launch is cooperative (all CTAs resident at once).  Ordering across
+ * ranks is the caller's: every shard must be complete before the call runs,
+ * and no rank may overwrite its shard before the other ranks' calls that
+ * read it have finished (e.g. one barrier collective per layer on `stream`
+ * with two shard buffers used in turn).  Results equal hd_attn_fwd_parts;
+ * k_dst/v_dst end up bit-identical to k_src/v_src.  A piece that never
+ * lands ends the waits after about one second with HD_ERR_TIMEOUT in
+ * *dev_status.
+ */
+size_t hd_attn_peer_flags_bytes(int B, int L, int n);
+hd_status hd_attn_fwd_peer_gather(const void* q_loc, const void* const* k_src,
+                                  const void* const* v_src, void* const* k_dst,
+                                  void* const* v_dst, void* flags, size_t flags_bytes,
+                                  void* o_loc, float* lse, int B, int L, int n, int R, int r,
+                                  int Hq, int Hkv, int D, int window, float scale,
+                                  hd_dtype in_dt, hd_dtype out_dt, int32_t* dev_status,
+                                  void* stream);
+
+/*
+ * CUDA IPC for the shards of hd_attn_fwd_peer_gather.
+ * hd_ipc_export: handle (HD_IPC_HANDLE_BYTES bytes, host) of the device
+ *   allocation that contains `ptr`, and ptr's byte offset in it.  Fails
+ *   (HD_ERR_CUDA) for memory that CUDA IPC cannot share.
+ * hd_ipc_open: in another process, map that allocation; *base is its start
+ *   (add the offset); peer access is enabled as needed.
+ * hd_ipc_close: unmap a base returned by hd_ipc_open.
+ */
+#define HD_IPC_HANDLE_BYTES 64
+hd_status hd_ipc_export(const void* ptr, void* handle, size_t* offset);
+hd_status hd_ipc_open(const void* handle, void** base);
+hd_status hd_ipc_close(void* base);
+
 typedef enum {
   HD_ROPE_HALF = 0,      /* pairs (j, j + rot_dim/2): the rotate-half form   */
   HD_ROPE_INTERLEAVED = 1 /* pairs (2j, 2j + 1): the RoFormer paper's form    */

@@ -40,6 +40,7 @@
 // relative error < 1e-4, below the bf16 rounding of P) to offload MUFU.
 #include <cstdlib>
 #include <cstring>
+#include <type_traits>
 
 #include "hd_common.cuh"
 #include "hd_launch.h"
@@ -52,6 +53,7 @@ constexpr int BN = 128;
 constexpr int kThreads = 320;
 constexpr int kWarpTMA = 8;
 constexpr int kWarpMMA = 9;
+constexpr int kWarpGather = 10;  // rank-shard form with gather only
 constexpr int KST = 3;
 constexpr int VST = 2;
 constexpr uint32_t kTmemCols = 512;
@@ -132,11 +134,92 @@ __device__ __forceinline__ TcUnit tc_unit(int u, const TcParams& p) {
   return x;
 }
 
-template <int D>
-__global__ void __launch_bounds__(tc::kThreads, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const TcParams p) {
+// Key/value sources.  NM == 1: one sequence in the expanded order (every
+// regular call).  NM == kPeerMaxRanks: the R rank shards of a stream-parallel
+// cross-stream layer.  Key tile [k0, k0 + 128) holds tokens k0/n .. k0/n +
+// 128/n - 1 of all n streams; in rank rho's shard (local stream l = global
+// stream rho + R*l at local row token*(n/R) + l) they are the contiguous rows
+// [k0/R, k0/R + 128/R).  So a tile is R boxes of 128/R rows, one per shard,
+// and shared-memory row c = rho*(128/R) + t holds key k0 + perm[c] with
+// perm[c] = (t / (n/R))*n + rho + R*(t mod (n/R)).  The MMAs do not depend on
+// the key order inside a tile (the same order feeds S and P V); only the
+// mask needs perm.
+struct PartsInfo {
+  int R, rows, self;
+  uint8_t perm[tc::BN];
+  // In-kernel gather (flags != nullptr): rank rho's shard (rho != self) is
+  // copied from src to dst in items of up to kPeerSub16 16-byte units,
+  // ordered key tile first; flags[b*nkt + kt] counts the finished items of
+  // key tile kt of sequence b, complete at per_flag.
+  const uint4* src_k[kPeerMaxRanks];
+  const uint4* src_v[kPeerMaxRanks];
+  uint4* dst_k[kPeerMaxRanks];
+  uint4* dst_v[kPeerMaxRanks];
+  unsigned long long* flags;
+  unsigned long long per_flag;
+  int64_t shard_rows;
+  int nkt, nsub, nitems, row16;
+  // Test hook (environment HD_TEST_STALL_GATHER=1): CTA 0 never publishes
+  // its first item, so a tile never becomes ready and the producer's wait
+  // must run out.  0 in normal use.
+  int stall_gather;
+};
+struct NoParts {};
+template <int NM>
+struct KvSrc {
+  CUtensorMap k[NM];
+  CUtensorMap v[NM];
+  std::conditional_t<(NM > 1), PartsInfo, NoParts> x;
+};
+
+// The gather warp: copies its share of the items (item w goes to CTA
+// w mod grid) with 16-byte loads, U in flight per lane, then publishes each.
+// It never waits on another CTA, so with every CTA resident (cooperative
+// launch) every flag is eventually published.
+template <int U>
+__device__ __forceinline__ void gather_items(const PartsInfo& x, int B, int lane, volatile int* abort) {
+  for (int w = blockIdx.x; w < x.nitems; w += gridDim.x) {
+    if (*abort) return;
+    int rem = w;
+    const int sub = rem % x.nsub;
+    rem /= x.nsub;
+    const int kind = rem & 1;
+    rem >>= 1;
+    const int rr = rem % (x.R - 1);
+    rem /= x.R - 1;
+    const int b = rem % B;
+    const int kt = rem / B;
+    const int rho = rr < x.self ? rr : rr + 1;
+    const int64_t r0 = static_cast<int64_t>(kt) * x.rows;
+    const int64_t r1 = min(r0 + x.rows, x.shard_rows);
+    const int64_t n16 = (r1 - r0) * x.row16;
+    const int64_t s0 = static_cast<int64_t>(sub) * kPeerSub16;
+    const int64_t s1 = min(s0 + kPeerSub16, n16);
+    const int64_t base = (static_cast<int64_t>(b) * x.shard_rows + r0) * x.row16;
+    const uint4* src = (kind ? x.src_v[rho] : x.src_k[rho]) + base;
+    uint4* dst = (kind ? x.dst_v[rho] : x.dst_k[rho]) + base;
+    for (int64_t i0 = s0 + lane; i0 < s1; i0 += 32 * U) {
+      uint4 t[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (i0 + 32 * u < s1) t[u] = __ldcs(src + i0 + 32 * u);
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (i0 + 32 * u < s1) dst[i0 + 32 * u] = t[u];
+    }
+    __threadfence();
+    __syncwarp();
+    if (lane == 0 && !(x.stall_gather && blockIdx.x == 0 && w == 0))
+      flag_publish(x.flags + static_cast<int64_t>(b) * x.nkt + kt);
+  }
+}
+
+template <int D, int NM>
+__global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ KvSrc<NM> kv,
+                   const TcParams p) {
   using Lay = tc::Layout<D>;
+  constexpr bool kParts = NM > 1;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -175,8 +258,14 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   }
   if (warp == tc::kWarpTMA && lane == 0) {
     tma_prefetch_desc(&tmQ);
-    tma_prefetch_desc(&tmK);
-    tma_prefetch_desc(&tmV);
+#pragma unroll
+    for (int i = 0; i < NM; ++i) {
+      if constexpr (kParts) {
+        if (i >= kv.x.R) break;
+      }
+      tma_prefetch_desc(&kv.k[i]);
+      tma_prefetch_desc(&kv.v[i]);
+    }
   }
   if (warp == tc::kWarpMMA) {
     tmem_alloc(smem_u32(tmem_slot), tc::kTmemCols);
@@ -190,6 +279,23 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   auto fail = [&]() {
     *abort_flag = 1;
     report(p.status, HD_ERR_TIMEOUT);
+  };
+  // One 128-key tile of K or V into the stage at `dst`.
+  auto load_kv_tile = [&](const CUtensorMap* maps, uint32_t dst, uint32_t full, const TcUnit& x, int skv, int kt) {
+    if constexpr (kParts) {
+#pragma unroll
+      for (int rho = 0; rho < NM; ++rho) {
+        if (rho >= kv.x.R) break;
+#pragma unroll
+        for (int kb = 0; kb < Lay::KB; ++kb)
+          tma_load_5d(dst + kb * Lay::BLK + rho * kv.x.rows * 128, &maps[rho], full, kb * 64, x.kvh, 0,
+                      kt * kv.x.rows, x.b);
+      }
+    } else {
+#pragma unroll
+      for (int kb = 0; kb < Lay::KB; ++kb)
+        tma_load_5d(dst + kb * Lay::BLK, &maps[0], full, kb * 64, x.kvh, skv, kt * tc::BN, x.b);
+    }
   };
 
   if (warp == tc::kWarpTMA) {
@@ -213,21 +319,23 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         ++q_issued;
         const int skv = p.g.kv_stream >= 0 ? p.g.kv_stream : x.s;
         for (int kt = x.t_lo; kt <= x.t_hi; ++kt, ++t) {
+          if constexpr (kParts) {
+            // Gathered shards: wait until every item of this key tile landed.
+            if (kv.x.flags &&
+                !flag_wait_ge(kv.x.flags + static_cast<int64_t>(x.b) * kv.x.nkt + kt, kv.x.per_flag, abort_flag)) {
+              ok = false;
+              break;
+            }
+          }
           const int ks = t % tc::KST;
           if (!mbar_wait(bar(Lay::B_KEMPTY + ks), ((t / tc::KST) & 1) ^ 1, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(bar(Lay::B_KFULL + ks), Lay::TILE);
-#pragma unroll
-          for (int kb = 0; kb < Lay::KB; ++kb)
-            tma_load_5d(sbase + Lay::K_OFF + ks * Lay::TILE + kb * Lay::BLK, &tmK, bar(Lay::B_KFULL + ks),
-                        kb * 64, x.kvh, skv, kt * tc::BN, x.b);
+          load_kv_tile(kv.k, sbase + Lay::K_OFF + ks * Lay::TILE, bar(Lay::B_KFULL + ks), x, skv, kt);
           ++k_issued[ks];
           const int vs = t % tc::VST;
           if (!mbar_wait(bar(Lay::B_VEMPTY + vs), ((t / tc::VST) & 1) ^ 1, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(bar(Lay::B_VFULL + vs), Lay::TILE);
-#pragma unroll
-          for (int kb = 0; kb < Lay::KB; ++kb)
-            tma_load_5d(sbase + Lay::V_OFF + vs * Lay::TILE + kb * Lay::BLK, &tmV, bar(Lay::B_VFULL + vs),
-                        kb * 64, x.kvh, skv, kt * tc::BN, x.b);
+          load_kv_tile(kv.v, sbase + Lay::V_OFF + vs * Lay::TILE, bar(Lay::B_VFULL + vs), x, skv, kt);
           ++v_issued[vs];
         }
       }
@@ -372,7 +480,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         if (need_mask) {
 #pragma unroll
           for (int c = 0; c < 128; ++c) {
-            const int j = k0 + c;
+            int j = k0 + c;
+            if constexpr (kParts) j = k0 + kv.x.perm[c];
             if (j > pi || (p.W > 0 && pi - j >= p.W)) sv[c] = __float_as_uint(-INFINITY);
           }
         }
@@ -484,6 +593,11 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       mbar_arrive(bar(Lay::B_OEMPTY + slot));
     }
     if (!ok) fail();
+  } else if (warp == tc::kWarpGather) {
+    // ------------------------------------------------------------- gather
+    if constexpr (kParts) {
+      if (kv.x.flags) gather_items<16>(kv.x, p.g.B, lane, abort_flag);
+    }
   }
 
   __syncthreads();
@@ -496,7 +610,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
 
 // ------------------------------------------------------------------- host
 
-// (D, H, ns, Ls, B) view of a [B, ns*Ls, H, D] bf16 tensor; box = 64 x 1 x 1 x 128 x 1.
+// (D, H, ns, Ls, B) view of a [B, ns*Ls, H, D] bf16 tensor; box = 64 x 1 x 1 x rows x 1
+// with rows = 128 (kind 1) or the key's `pad` (kind 3: one rank's part of a key tile).
 static bool make_stream_view(const TmapKey& k, CUtensorMap* m) {
   EncodeTiledFn enc = get_encode_tiled();
   if (!enc) return false;
@@ -504,7 +619,8 @@ static bool make_stream_view(const TmapKey& k, CUtensorMap* m) {
   const cuuint64_t dims[5] = {D, H, ns, Ls, B};
   const cuuint64_t e = 2;
   const cuuint64_t strides[4] = {D * e, H * D * e, ns * H * D * e, Ls * ns * H * D * e};
-  const cuuint32_t box[5] = {64, 1, 1, (cuuint32_t)tc::BM, 1};
+  const cuuint32_t rows = k.kind == 3 ? static_cast<cuuint32_t>(k.pad) : static_cast<cuuint32_t>(tc::BM);
+  const cuuint32_t box[5] = {64, 1, 1, rows, 1};
   const cuuint32_t es[5] = {1, 1, 1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(k.ptr), dims, strides, box, es,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -525,17 +641,26 @@ bool encode_stream_view(CUtensorMap* m, const void* ptr, int B, int Ls, int ns, 
   return tmap_cached(k, m, make_stream_view);
 }
 
+// One rank shard [B, rows, H, D] with a box of `box_rows` rows.
+static bool encode_shard_view(CUtensorMap* m, const void* ptr, int B, int64_t rows, int H, int D, int box_rows) {
+  TmapKey k;
+  std::memset(&k, 0, sizeof(k));
+  k.ptr = ptr;
+  k.dims[0] = B;
+  k.dims[1] = rows;
+  k.dims[2] = 1;
+  k.dims[3] = H;
+  k.dims[4] = D;
+  k.kind = 3;
+  k.pad = box_rows;
+  return tmap_cached(k, m, make_stream_view);
+}
+
 int attn_tc_smem_bytes(int D) { return D == 64 ? tc::Layout<64>::ALLOC : tc::Layout<128>::ALLOC; }
 
-cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o, float* lse, const AttnGeom& g,
-                           int Hq, int Hkv, int D, int W, float scale, bool out_bf16, int32_t* status, int sms,
-                           cudaStream_t st) {
-  CUtensorMap mq, mk, mv;
-  if (!encode_stream_view(&mq, q, g.B, g.Lq, g.q_ns, Hq, D) ||
-      !encode_stream_view(&mk, k, g.B, g.Lk, g.kv_ns, Hkv, D) ||
-      !encode_stream_view(&mv, v, g.B, g.Lk, g.kv_ns, Hkv, D))
-    return cudaErrorInvalidValue;
-  TcParams p;
+// Parameters common to both forms; false if the unit count overflows.
+static bool fill_params(TcParams& p, void* o, float* lse, const AttnGeom& g, int Hq, int Hkv, int W, float scale,
+                        bool out_bf16, int32_t* status) {
   p.o = o;
   p.lse = lse;
   p.status = status;
@@ -549,27 +674,128 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o,
   const int G = Hq / Hkv;
   p.npairs = (G + 1) / 2;
   const int64_t units = static_cast<int64_t>(p.nqb) * g.B * g.ns * Hkv * p.npairs;
-  if (units <= 0) return cudaSuccess;
-  if (units > 0x7fffffff) return cudaErrorInvalidValue;
+  if (units < 0 || units > 0x7fffffff) return false;
   p.total_units = static_cast<int>(units);
   static const int stall = [] {
     const char* e = getenv("HD_TEST_STALL_FIRST_S");
     return (e && e[0] == '1') ? 1 : 0;
   }();
   p.stall_first_s = stall;
-  const int grid = static_cast<int>(units < sms ? units : sms);
+  return true;
+}
+
+cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o, float* lse, const AttnGeom& g,
+                           int Hq, int Hkv, int D, int W, float scale, bool out_bf16, int32_t* status, int sms,
+                           cudaStream_t st) {
+  CUtensorMap mq;
+  KvSrc<1> kv;
+  if (!encode_stream_view(&mq, q, g.B, g.Lq, g.q_ns, Hq, D) ||
+      !encode_stream_view(&kv.k[0], k, g.B, g.Lk, g.kv_ns, Hkv, D) ||
+      !encode_stream_view(&kv.v[0], v, g.B, g.Lk, g.kv_ns, Hkv, D))
+    return cudaErrorInvalidValue;
+  TcParams p;
+  if (!fill_params(p, o, lse, g, Hq, Hkv, W, scale, out_bf16, status)) return cudaErrorInvalidValue;
+  if (p.total_units == 0) return cudaSuccess;
+  const int grid = p.total_units < sms ? p.total_units : sms;
   const int smem = attn_tc_smem_bytes(D);
   cudaError_t err;
   if (D == 64) {
-    err = cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    err = cudaFuncSetAttribute(attn_tc_kernel<64, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
-    attn_tc_kernel<64><<<grid, tc::kThreads, smem, st>>>(mq, mk, mv, p);
+    attn_tc_kernel<64, 1><<<grid, tc::kThreads, smem, st>>>(mq, kv, p);
   } else {
-    err = cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    err = cudaFuncSetAttribute(attn_tc_kernel<128, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
-    attn_tc_kernel<128><<<grid, tc::kThreads, smem, st>>>(mq, mk, mv, p);
+    attn_tc_kernel<128, 1><<<grid, tc::kThreads, smem, st>>>(mq, kv, p);
   }
   return cudaGetLastError();
+}
+
+int64_t parts_flag_count(int B, int n, int L) {
+  return static_cast<int64_t>(B) * ((static_cast<int64_t>(n) * L + tc::BN - 1) / tc::BN);
+}
+
+template <int D>
+static cudaError_t launch_parts_kernel(const CUtensorMap& mq, const KvSrc<kPeerMaxRanks>& kv, const TcParams& p,
+                                       int grid, bool cooperative, cudaStream_t st) {
+  const int smem = attn_tc_smem_bytes(D);
+  cudaError_t err =
+      cudaFuncSetAttribute(attn_tc_kernel<D, kPeerMaxRanks>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(tc::kThreads + 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeCooperative;
+  at[0].val.cooperative = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = cooperative ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, attn_tc_kernel<D, kPeerMaxRanks>, mq, kv, p);
+}
+
+cudaError_t launch_attn_tc_parts(const void* q, const PartsArgs& a, void* o, float* lse, const AttnGeom& g, int n,
+                                 int Hq, int Hkv, int D, int W, float scale, bool out_bf16, int32_t* status, int sms,
+                                 cudaStream_t st) {
+  const int R = a.R;
+  if (R < 1 || R > kPeerMaxRanks || n % R || tc::BN % n || a.self < 0 || a.self >= R) return cudaErrorInvalidValue;
+  const int nl = n / R;
+  const int L = g.Lq;
+  const int rows = tc::BN / R;
+  const int64_t shard_rows = static_cast<int64_t>(nl) * L;
+  const bool gather = R > 1 && a.k_dst[0 == a.self ? 1 : 0] != nullptr;
+  CUtensorMap mq;
+  if (!encode_stream_view(&mq, q, g.B, g.Lq, g.q_ns, Hq, D)) return cudaErrorInvalidValue;
+  KvSrc<kPeerMaxRanks> kv;
+  std::memset(&kv, 0, sizeof(kv));
+  PartsInfo& x = kv.x;
+  for (int rho = 0; rho < R; ++rho) {
+    const bool copied = gather && rho != a.self;
+    const void* ks = copied ? a.k_dst[rho] : a.k_src[rho];
+    const void* vs = copied ? a.v_dst[rho] : a.v_src[rho];
+    if (!encode_shard_view(&kv.k[rho], ks, g.B, shard_rows, Hkv, D, rows) ||
+        !encode_shard_view(&kv.v[rho], vs, g.B, shard_rows, Hkv, D, rows))
+      return cudaErrorInvalidValue;
+    x.src_k[rho] = static_cast<const uint4*>(a.k_src[rho]);
+    x.src_v[rho] = static_cast<const uint4*>(a.v_src[rho]);
+    x.dst_k[rho] = static_cast<uint4*>(a.k_dst[rho]);
+    x.dst_v[rho] = static_cast<uint4*>(a.v_dst[rho]);
+  }
+  x.R = R;
+  x.rows = rows;
+  x.self = a.self;
+  for (int c = 0; c < tc::BN; ++c) {
+    const int rho = c / rows, t = c % rows;
+    x.perm[c] = static_cast<uint8_t>((t / nl) * n + rho + R * (t % nl));
+  }
+  x.shard_rows = shard_rows;
+  x.nkt = static_cast<int>((static_cast<int64_t>(n) * L + tc::BN - 1) / tc::BN);
+  x.row16 = Hkv * D * 2 / 16;
+  const int64_t tile16 = static_cast<int64_t>(rows) * x.row16;
+  x.nsub = static_cast<int>((tile16 + kPeerSub16 - 1) / kPeerSub16);
+  x.flags = gather ? a.flags : nullptr;
+  x.per_flag = static_cast<unsigned long long>(2 * (R - 1)) * x.nsub;
+  const int64_t items = gather ? static_cast<int64_t>(x.nkt) * g.B * (R - 1) * 2 * x.nsub : 0;
+  if (items > 0x7fffffff) return cudaErrorInvalidValue;
+  x.nitems = static_cast<int>(items);
+  static const int stall = [] {
+    const char* e = getenv("HD_TEST_STALL_GATHER");
+    return (e && e[0] == '1') ? 1 : 0;
+  }();
+  x.stall_gather = stall;
+  TcParams p;
+  if (!fill_params(p, o, lse, g, Hq, Hkv, W, scale, out_bf16, status)) return cudaErrorInvalidValue;
+  if (p.total_units == 0) return cudaSuccess;
+  if (gather) {
+    if (!a.flags) return cudaErrorInvalidValue;
+    cudaError_t err = cudaMemsetAsync(a.flags, 0, parts_flag_count(g.B, n, L) * sizeof(unsigned long long), st);
+    if (err != cudaSuccess) return err;
+  }
+  const int grid = p.total_units < sms ? p.total_units : sms;
+  // A producer may wait for an item of any CTA: all CTAs must be resident.
+  return D == 64 ? launch_parts_kernel<64>(mq, kv, p, grid, gather, st)
+                 : launch_parts_kernel<128>(mq, kv, p, grid, gather, st);
 }
 
 }  // namespace hd

@@ -1,6 +1,7 @@
 // C ABI of the library (include/hd.h): argument checks, the mode -> stream
 // view mapping, and dispatch to the kernels.  Nothing here allocates device
-// memory or synchronises.
+// memory or synchronises (the IPC calls only map and unmap other processes'
+// allocations).
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -278,6 +279,25 @@ hd_status hd_attn_decode(const void* q, const void* k_cache, const void* v_cache
                                    static_cast<cudaStream_t>(stream)));
 }
 
+// Geometry of rank r's queries in a stream-parallel cross-stream layer.
+static AttnGeom shard_geom(int B, int L, int n, int R, int r) {
+  const int nl = n / R;
+  AttnGeom g;
+  g.B = B;
+  g.ns = nl;
+  g.Lq = L;
+  g.q_ns = nl;
+  g.kv_ns = 1;
+  g.Lk = n * L;
+  g.kv_stream = 0;
+  g.qstride = n;
+  g.qoff = r;
+  g.qsstride = R;
+  g.o_rows = nl * L;
+  g.o_ns = nl;
+  return g;
+}
+
 static bool valid_shard(int n, int R, int r) { return R >= 1 && n >= 1 && n % R == 0 && r >= 0 && r < R; }
 
 hd_status hd_attn_decode_shard(const void* q, const void* k_cache_loc, const void* v_cache_loc,
@@ -305,23 +325,114 @@ hd_status hd_attn_fwd_shard(const void* q_loc, const void* k, const void* v, voi
   if (!valid_shard(n, R, r)) return HD_ERR_INVALID_ARG;
   hd_status stt = check_attn_args(q_loc, k, v, o_loc, lse, B, L, n, Hq, Hkv, D, HD_CROSS, window, scale, in_dt, out_dt);
   if (stt != HD_OK || B == 0) return stt;
-  // Queries: the n/R local streams of L tokens; local stream l is global
-  // stream r + R*l, at position i*n + r + R*l of the single nL-key stream.
-  const int nl = n / R;
-  AttnGeom g;
-  g.B = B;
-  g.ns = nl;
-  g.Lq = L;
-  g.q_ns = nl;
-  g.kv_ns = 1;
-  g.Lk = n * L;
-  g.kv_stream = 0;
-  g.qstride = n;
-  g.qoff = r;
-  g.qsstride = R;
-  g.o_rows = nl * L;
-  g.o_ns = nl;
-  return run_attn(q_loc, k, v, o_loc, lse, g, Hq, Hkv, D, window, scale, in_dt, out_dt, dev_status, stream);
+  return run_attn(q_loc, k, v, o_loc, lse, shard_geom(B, L, n, R, r), Hq, Hkv, D, window, scale, in_dt, out_dt,
+                  dev_status, stream);
+}
+
+// Shared checks of the rank-shard calls; *pa gets the shard pointers.
+static hd_status parts_args(const void* q_loc, const void* const* k_src, const void* const* v_src, void* o_loc,
+                            float* lse, int B, int L, int n, int R, int r, int Hq, int Hkv, int D, int window,
+                            float scale, hd_dtype in_dt, hd_dtype out_dt, PartsArgs* pa) {
+  if (!valid_shard(n, R, r) || R > kPeerMaxRanks || 128 % n) return HD_ERR_INVALID_ARG;
+  if (!k_src || !v_src) return HD_ERR_INVALID_ARG;
+  // q_loc doubles as the k/v placeholder of the common checks; the shards are checked below.
+  hd_status stt = check_attn_args(q_loc, q_loc, q_loc, o_loc, lse, B, L, n, Hq, Hkv, D, HD_CROSS, window, scale,
+                                  in_dt, out_dt);
+  if (stt != HD_OK) return stt;
+  if (in_dt != HD_BF16) return HD_ERR_UNSUPPORTED;
+  std::memset(pa, 0, sizeof(*pa));
+  pa->R = R;
+  pa->self = r;
+  for (int rho = 0; rho < R; ++rho) {
+    if (B > 0 && (!k_src[rho] || !v_src[rho] || !aligned16(k_src[rho]) || !aligned16(v_src[rho])))
+      return HD_ERR_INVALID_ARG;
+    pa->k_src[rho] = k_src[rho];
+    pa->v_src[rho] = v_src[rho];
+  }
+  return HD_OK;
+}
+
+hd_status hd_attn_fwd_parts(const void* q_loc, const void* const* k_parts, const void* const* v_parts, void* o_loc,
+                            float* lse, int B, int L, int n, int R, int r, int Hq, int Hkv, int D, int window,
+                            float scale, hd_dtype in_dt, hd_dtype out_dt, int32_t* dev_status, void* stream) {
+  PartsArgs pa;
+  hd_status stt = parts_args(q_loc, k_parts, v_parts, o_loc, lse, B, L, n, R, r, Hq, Hkv, D, window, scale, in_dt,
+                             out_dt, &pa);
+  if (stt != HD_OK || B == 0) return stt;
+  const int sms = sm_count();
+  if (sms <= 0) return HD_ERR_CUDA;
+  return cuda_status(launch_attn_tc_parts(q_loc, pa, o_loc, lse, shard_geom(B, L, n, R, r), n, Hq, Hkv, D, window,
+                                          scale, out_dt == HD_BF16, dev_status, sms,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+size_t hd_attn_peer_flags_bytes(int B, int L, int n) {
+  if (B < 0 || L < 0 || n < 1) return 0;
+  return static_cast<size_t>(parts_flag_count(B, n, L)) * sizeof(unsigned long long);
+}
+
+hd_status hd_attn_fwd_peer_gather(const void* q_loc, const void* const* k_src, const void* const* v_src,
+                                  void* const* k_dst, void* const* v_dst, void* flags, size_t flags_bytes,
+                                  void* o_loc, float* lse, int B, int L, int n, int R, int r, int Hq, int Hkv, int D,
+                                  int window, float scale, hd_dtype in_dt, hd_dtype out_dt, int32_t* dev_status,
+                                  void* stream) {
+  PartsArgs pa;
+  hd_status stt = parts_args(q_loc, k_src, v_src, o_loc, lse, B, L, n, R, r, Hq, Hkv, D, window, scale, in_dt,
+                             out_dt, &pa);
+  if (stt != HD_OK || B == 0) return stt;
+  if (R > 1) {
+    if (!k_dst || !v_dst || !flags || (reinterpret_cast<uintptr_t>(flags) & 7u) ||
+        flags_bytes < hd_attn_peer_flags_bytes(B, L, n))
+      return HD_ERR_INVALID_ARG;
+    for (int rho = 0; rho < R; ++rho) {
+      if (rho == r) continue;
+      if (!k_dst[rho] || !v_dst[rho] || !aligned16(k_dst[rho]) || !aligned16(v_dst[rho])) return HD_ERR_INVALID_ARG;
+      pa.k_dst[rho] = k_dst[rho];
+      pa.v_dst[rho] = v_dst[rho];
+    }
+    pa.flags = static_cast<unsigned long long*>(flags);
+  }
+  const int sms = sm_count();
+  if (sms <= 0) return HD_ERR_CUDA;
+  return cuda_status(launch_attn_tc_parts(q_loc, pa, o_loc, lse, shard_geom(B, L, n, R, r), n, Hq, Hkv, D, window,
+                                          scale, out_dt == HD_BF16, dev_status, sms,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+static_assert(sizeof(cudaIpcMemHandle_t) == HD_IPC_HANDLE_BYTES, "IPC handle size");
+
+hd_status hd_ipc_export(const void* ptr, void* handle, size_t* offset) {
+  if (!ptr || !handle || !offset) return HD_ERR_INVALID_ARG;
+  using RangeFn = CUresult (*)(CUdeviceptr*, size_t*, CUdeviceptr);
+  static RangeFn range = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<RangeFn>(p);
+    return static_cast<RangeFn>(nullptr);
+  }();
+  if (!range) return HD_ERR_CUDA;
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  if (range(&base, &size, reinterpret_cast<CUdeviceptr>(ptr)) != CUDA_SUCCESS) return HD_ERR_CUDA;
+  cudaIpcMemHandle_t h;
+  if (cudaIpcGetMemHandle(&h, reinterpret_cast<void*>(base)) != cudaSuccess) return HD_ERR_CUDA;
+  std::memcpy(handle, &h, sizeof(h));
+  *offset = static_cast<size_t>(reinterpret_cast<CUdeviceptr>(ptr) - base);
+  return HD_OK;
+}
+
+hd_status hd_ipc_open(const void* handle, void** base) {
+  if (!handle || !base) return HD_ERR_INVALID_ARG;
+  cudaIpcMemHandle_t h;
+  std::memcpy(&h, handle, sizeof(h));
+  return cuda_status(cudaIpcOpenMemHandle(base, h, cudaIpcMemLazyEnablePeerAccess));
+}
+
+hd_status hd_ipc_close(void* base) {
+  if (!base) return HD_ERR_INVALID_ARG;
+  return cuda_status(cudaIpcCloseMemHandle(base));
 }
 
 hd_status hd_stream_interleave(const void* parts, void* out, int R, int B, int L, int n, int64_t row_elems,

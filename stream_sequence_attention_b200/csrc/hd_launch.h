@@ -61,6 +61,28 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o,
                            int Hq, int Hkv, int D, int W, float scale, bool out_bf16, int32_t* status, int sms,
                            cudaStream_t st);
 
+// Cross-stream prefill of one rank's queries (geometry as for the shard
+// call) with the keys/values held as R rank shards [B, (n/R)*L, Hkv, D]
+// instead of one interleaved sequence.  n must divide 128 (a 128-key tile is
+// 128/R rows of every shard).  Without gather (k_dst == nullptr) every shard
+// is read where it lies.  With gather, shard rho != self is copied once from
+// k_src[rho] to k_dst[rho] inside the kernel (overlapped with the attention,
+// published per (batch, key tile) through `flags`) and read from k_dst.
+constexpr int kPeerMaxRanks = 8;
+constexpr int kPeerSub16 = 1024;  // 16-byte units per gather item (16 KiB)
+struct PartsArgs {
+  int R, self;
+  const void* k_src[kPeerMaxRanks];
+  const void* v_src[kPeerMaxRanks];
+  void* k_dst[kPeerMaxRanks];  // all nullptr: no gather
+  void* v_dst[kPeerMaxRanks];
+  unsigned long long* flags;   // [B * key tiles], zeroed by the launcher
+};
+int64_t parts_flag_count(int B, int n, int L);
+cudaError_t launch_attn_tc_parts(const void* q, const PartsArgs& a, void* o, float* lse, const AttnGeom& g, int n,
+                                 int Hq, int Hkv, int D, int W, float scale, bool out_bf16, int32_t* status, int sms,
+                                 cudaStream_t st);
+
 // Backward.  Regular geometry only (qstride 1, qoff 0, kv_stream -1, the
 // key streams equal the query streams).  The workspace holds two float
 // planes, lse * log2 e and delta = <dO, o>, each indexed

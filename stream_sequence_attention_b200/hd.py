@@ -36,6 +36,12 @@ EXPORTS = (
     "hd_attn_decode_noalloc",
     "hd_attn_decode_shard",
     "hd_attn_fwd_shard",
+    "hd_attn_fwd_parts",
+    "hd_attn_fwd_peer_gather",
+    "hd_attn_peer_flags_bytes",
+    "hd_ipc_export",
+    "hd_ipc_open",
+    "hd_ipc_close",
     "hd_stream_interleave",
     "hd_attn_combine",
     "hd_final_stream_gather",
@@ -93,6 +99,20 @@ def lib() -> ctypes.CDLL:
         L.hd_attn_fwd_shard.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, i32, f32, i32, i32,
                                         vp, vp]
         L.hd_attn_fwd_shard.restype = i32
+        L.hd_attn_fwd_parts.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, i32, f32, i32, i32,
+                                        vp, vp]
+        L.hd_attn_fwd_parts.restype = i32
+        L.hd_attn_fwd_peer_gather.argtypes = [vp, vp, vp, vp, vp, vp, sz, vp, vp, i32, i32, i32, i32, i32, i32, i32,
+                                              i32, i32, f32, i32, i32, vp, vp]
+        L.hd_attn_fwd_peer_gather.restype = i32
+        L.hd_attn_peer_flags_bytes.argtypes = [i32, i32, i32]
+        L.hd_attn_peer_flags_bytes.restype = sz
+        L.hd_ipc_export.argtypes = [vp, vp, ctypes.POINTER(sz)]
+        L.hd_ipc_export.restype = i32
+        L.hd_ipc_open.argtypes = [vp, ctypes.POINTER(vp)]
+        L.hd_ipc_open.restype = i32
+        L.hd_ipc_close.argtypes = [vp]
+        L.hd_ipc_close.restype = i32
         L.hd_stream_interleave.argtypes = [vp, vp, i32, i32, i32, i32, i64, i32, vp]
         L.hd_stream_interleave.restype = i32
         L.hd_attn_combine.argtypes = [vp, vp, vp, vp, i32, i64, i32, i32, i32, vp]
@@ -526,6 +546,127 @@ def hd_attn_fwd_shard(q_loc: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n: 
         _ptr(q_loc), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, L, n, R, r, Hq, Hkv, D, int(window), float(scale),
         _dt(q_loc), _dt(out), _ptr(dev_status), _stream(stream)))
     return (out, lse) if want_lse else out
+
+
+HD_MAX_RANKS = 8
+HD_IPC_HANDLE_BYTES = 64
+
+
+def _shard_list(parts, R: int, name: str, shape=None, dtype=None, allow_addr: bool = False):
+    """R shard addresses from a list (tensors, or device addresses if
+    allow_addr) or from one tensor [R, ...]; checks the tensors' shape/dtype."""
+    if isinstance(parts, torch.Tensor):
+        _need(parts, name)
+        if parts.shape[0] != R:
+            raise ValueError(f"{name} must hold R = {R} shards")
+        parts = [parts[i] for i in range(R)]
+    parts = list(parts)
+    if len(parts) != R:
+        raise ValueError(f"{name} must hold R = {R} shards")
+    addrs = []
+    for i, t in enumerate(parts):
+        if isinstance(t, torch.Tensor):
+            _need(t, f"{name}[{i}]")
+            if shape is not None and (tuple(t.shape) != tuple(shape) or t.dtype != dtype):
+                raise ValueError(f"{name}[{i}] must be {tuple(shape)} {dtype}, got {tuple(t.shape)} {t.dtype}")
+            addrs.append(t.data_ptr())
+        elif allow_addr and isinstance(t, int):
+            addrs.append(t)
+        elif allow_addr and t is None:
+            addrs.append(0)
+        else:
+            raise TypeError(f"{name}[{i}] must be a CUDA tensor" + (" or a device address" if allow_addr else ""))
+    return (ctypes.c_void_p * R)(*[a or None for a in addrs])
+
+
+def _parts_common(q_loc, n, R, Hkv, scale, out, out_dtype, lse):
+    _need(q_loc, "q_loc")
+    B, PL, Hq, D = q_loc.shape
+    if R < 1 or n % R or PL % (n // R):
+        raise ValueError("shard shapes do not match n")
+    L = PL // (n // R)
+    if scale is None:
+        scale = D ** -0.5
+    if out is None:
+        out = torch.empty(q_loc.shape, dtype=out_dtype or q_loc.dtype, device=q_loc.device)
+    _need(out, "out")
+    want_lse = lse is True or isinstance(lse, torch.Tensor)
+    if lse is True:
+        lse = torch.empty((B, Hq, PL), dtype=torch.float32, device=q_loc.device)
+    elif lse is False:
+        lse = None
+    return B, L, Hq, D, (B, (n // R) * L, Hkv, D), scale, out, lse, want_lse
+
+
+def hd_attn_fwd_parts(q_loc: torch.Tensor, k_parts, v_parts, n: int, R: int, r: int, window: int = 0,
+                      scale: float | None = None, out: torch.Tensor | None = None, out_dtype=None,
+                      lse: torch.Tensor | bool | None = None, dev_status: torch.Tensor | None = None, stream=None):
+    """Cross-stream attention of rank r's queries q_loc [B, (n/R)*L, Hq, D]
+    against the R ranks' shards (a list of R tensors [B, (n/R)*L, Hkv, D], or
+    one tensor [R, B, (n/R)*L, Hkv, D] such as an all-gather output), read in
+    place."""
+    first = k_parts[0]
+    Hkv = first.shape[-2]
+    B, L, Hq, D, sh, scale, out, lse, want_lse = _parts_common(q_loc, n, R, Hkv, scale, out, out_dtype, lse)
+    ka = _shard_list(k_parts, R, "k_parts", sh, q_loc.dtype)
+    va = _shard_list(v_parts, R, "v_parts", sh, q_loc.dtype)
+    _check("hd_attn_fwd_parts", lib().hd_attn_fwd_parts(
+        _ptr(q_loc), ka, va, _ptr(out), _ptr(lse), B, L, n, R, r, Hq, Hkv, D, int(window), float(scale),
+        _dt(q_loc), _dt(out), _ptr(dev_status), _stream(stream)))
+    return (out, lse) if want_lse else out
+
+
+def hd_attn_peer_flags_bytes(B: int, L: int, n: int) -> int:
+    return int(lib().hd_attn_peer_flags_bytes(B, L, n))
+
+
+def hd_attn_fwd_peer_gather(q_loc: torch.Tensor, k_src, v_src, k_dst, v_dst, n: int, R: int, r: int,
+                            flags: torch.Tensor | None = None, window: int = 0, scale: float | None = None,
+                            out: torch.Tensor | None = None, out_dtype=None, lse: torch.Tensor | bool | None = None,
+                            dev_status: torch.Tensor | None = None, stream=None):
+    """hd_attn_fwd_parts with the exchange inside the kernel: k_src/v_src are
+    R shards (entry r a local tensor; the others tensors or peer device
+    addresses from :func:`hd_ipc_open`), copied once into the local k_dst/
+    v_dst shards (entry r unused) while the attention runs."""
+    if not isinstance(k_src[r], torch.Tensor) or not isinstance(v_src[r], torch.Tensor):
+        raise TypeError("k_src[r] and v_src[r] must be this rank's local shard tensors")
+    Hkv = k_src[r].shape[-2]
+    B, L, Hq, D, sh, scale, out, lse, want_lse = _parts_common(q_loc, n, R, Hkv, scale, out, out_dtype, lse)
+    ks = _shard_list(k_src, R, "k_src", sh, q_loc.dtype, allow_addr=True)
+    vs = _shard_list(v_src, R, "v_src", sh, q_loc.dtype, allow_addr=True)
+    kd = _shard_list(k_dst, R, "k_dst", sh, q_loc.dtype, allow_addr=True)
+    vd = _shard_list(v_dst, R, "v_dst", sh, q_loc.dtype, allow_addr=True)
+    nb = hd_attn_peer_flags_bytes(B, L, n)
+    if flags is None:
+        flags = torch.empty(max(1, nb // 8), dtype=torch.int64, device=q_loc.device)
+    _need(flags, "flags")
+    _check("hd_attn_fwd_peer_gather", lib().hd_attn_fwd_peer_gather(
+        _ptr(q_loc), ks, vs, kd, vd, _ptr(flags), flags.numel() * flags.element_size(), _ptr(out), _ptr(lse), B, L,
+        n, R, r, Hq, Hkv, D, int(window), float(scale), _dt(q_loc), _dt(out), _ptr(dev_status), _stream(stream)))
+    return (out, lse) if want_lse else out
+
+
+def hd_ipc_export(t: torch.Tensor):
+    """(handle bytes, byte offset) of the device allocation holding t."""
+    _need(t, "t")
+    h = ctypes.create_string_buffer(HD_IPC_HANDLE_BYTES)
+    off = ctypes.c_size_t(0)
+    _check("hd_ipc_export", lib().hd_ipc_export(_ptr(t), h, ctypes.byref(off)))
+    return h.raw, int(off.value)
+
+
+def hd_ipc_open(handle: bytes) -> int:
+    """Map another process's allocation; returns its base device address."""
+    if len(handle) != HD_IPC_HANDLE_BYTES:
+        raise ValueError("bad IPC handle")
+    base = ctypes.c_void_p(0)
+    _check("hd_ipc_open", lib().hd_ipc_open(ctypes.create_string_buffer(handle, HD_IPC_HANDLE_BYTES),
+                                            ctypes.byref(base)))
+    return int(base.value)
+
+
+def hd_ipc_close(base: int) -> None:
+    _check("hd_ipc_close", lib().hd_ipc_close(ctypes.c_void_p(base)))
 
 
 def hd_attn_decode_shard(q: torch.Tensor, k_cache_loc: torch.Tensor, v_cache_loc: torch.Tensor,

@@ -8,9 +8,15 @@ of global stream r + R*l.  Per layer:
 
 * intra-stream attention and decode touch only a rank's own streams: the
   library's regular calls on the local tensors with n/R streams, no exchange;
-* a cross-stream prefill layer all-gathers K and V (NCCL into local HBM),
-  restores the expanded order with ``hd_stream_interleave`` and runs
-  ``hd_attn_fwd_shard`` for the local queries;
+* a cross-stream prefill layer all-gathers K and V (NCCL into local HBM)
+  and runs ``hd_attn_fwd_parts`` for the local queries, which reads the
+  gathered shards where they lie (a key tile is 128/R rows of every shard);
+  ``hd_stream_interleave`` + ``hd_attn_fwd_shard`` cover the shapes that call
+  does not take (float32, n not dividing 128, more than 8 ranks);
+* or, with :class:`PeerShards`, the exchange runs inside the attention
+  kernel: each rank exports its K/V shard buffers by CUDA IPC, and
+  ``hd_attn_fwd_peer_gather`` copies the peers' shards into local memory
+  tile by tile while it computes;
 * cross-stream decode all-gathers the n stream queries of the new token,
   runs ``hd_attn_decode_shard`` (every query against the local cache
   streams), all-gathers the partial (O, lse) and merges them with
@@ -71,8 +77,16 @@ class StreamParallel:
         v = hd.hd_stream_interleave(all_gather_shards(v_loc, self.group), self.n)
         return k, v
 
+    def parts_supported(self, dtype) -> bool:
+        """Whether hd_attn_fwd_parts takes this layer (else the re-interleave path)."""
+        return dtype == torch.bfloat16 and 128 % self.n == 0 and self.R <= hd.HD_MAX_RANKS
+
     def cross_attention(self, q_loc, k_loc, v_loc, window: int = 0, scale=None, **kw):
         """Cross-stream layer: all-gather K/V, then the local queries' rows."""
+        if self.parts_supported(q_loc.dtype):
+            kp = all_gather_shards(k_loc, self.group)
+            vp = all_gather_shards(v_loc, self.group)
+            return hd.hd_attn_fwd_parts(q_loc, kp, vp, self.n, self.R, self.r, window, scale, **kw)
         k, v = self.gather_kv(k_loc, v_loc)
         return hd.hd_attn_fwd_shard(q_loc, k, v, self.n, self.R, self.r, window, scale, **kw)
 
@@ -92,3 +106,109 @@ class StreamParallel:
         lse_all = all_gather_shards(lse_part, self.group)
         o = hd.hd_attn_combine(o_all, lse_all, out_dtype=q_loc.dtype)  # [B, n, Hq, D]
         return o[:, self.r::self.R].contiguous()
+
+
+class PeerShards:
+    """K/V shard buffers of one cross-stream prefill layer shape, shared
+    between the ranks of ``view`` by CUDA IPC, for ``hd_attn_fwd_peer_gather``.
+
+    Each rank owns ``buffers`` pairs (K, V) of [B, (n/R)*L, Hkv, D] that the
+    other ranks map; a layer writes its shard into the next pair (``stage``),
+    all ranks pass a barrier (``fence``), and the kernel pulls the peers'
+    shards over NVLink into local slots while it computes (``attend``).  With
+    two pairs used in turn, one barrier per layer also keeps a rank from
+    overwriting a pair before the peers' kernels that read it have finished:
+    a rank passes the next barrier only after its previous kernel.
+
+    ``fence`` is a device-side barrier on the current stream for NCCL groups
+    (a one-element all-reduce); for other backends it synchronises the device
+    and calls ``dist.barrier``.  Call ``close`` on every rank before the
+    buffers go away.
+    """
+
+    def __init__(self, view: StreamParallel, B: int, L: int, Hkv: int, D: int, dtype=torch.bfloat16,
+                 buffers: int = 2, device=None):
+        if not view.parts_supported(dtype):
+            raise ValueError("PeerShards needs bf16, n dividing 128 and at most HD_MAX_RANKS ranks")
+        self.view = view
+        self.shape = (B, view.n_loc * L, Hkv, D)
+        self.dtype = dtype
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        self.own = [(torch.empty(self.shape, dtype=dtype, device=dev), torch.empty(self.shape, dtype=dtype, device=dev))
+                    for _ in range(buffers)]
+        def export(t):
+            handle, off = hd.hd_ipc_export(t)
+            return handle, off, t.data_ptr() - off  # the exporter's allocation base identifies it
+
+        mine = [(export(k), export(v)) for k, v in self.own]
+        every = [None] * view.R
+        dist.all_gather_object(every, mine, group=view.group)
+        # Buffers may share one allocation (the caching allocator splits
+        # segments): map each exported allocation once.
+        self._bases = {}
+        # src[i][rho] = (k address, v address) of rank rho's pair i
+        self.src = []
+        for i in range(buffers):
+            row = []
+            for rho in range(view.R):
+                if rho == view.r:
+                    row.append(self.own[i])
+                    continue
+                pair = []
+                for handle, off, owner_base in every[rho][i]:
+                    key = (rho, owner_base)
+                    if key not in self._bases:
+                        self._bases[key] = hd.hd_ipc_open(handle)
+                    pair.append(self._bases[key] + off)
+                row.append(tuple(pair))
+            self.src.append(row)
+        self.k_dst = torch.empty((view.R,) + self.shape, dtype=dtype, device=dev)
+        self.v_dst = torch.empty_like(self.k_dst)
+        nb = hd.hd_attn_peer_flags_bytes(B, L, view.n)
+        self.flags = torch.empty(max(1, nb // 8), dtype=torch.int64, device=dev)
+        self._tok = torch.zeros(1, dtype=torch.float32, device=dev)
+        self.turn = 0
+        self.staged = None
+
+    def fence(self):
+        if dist.get_backend(self.view.group) == "nccl":
+            dist.all_reduce(self._tok, group=self.view.group)
+        else:
+            torch.cuda.synchronize()
+            dist.barrier(group=self.view.group)
+
+    def stage(self, k_loc: torch.Tensor | None = None, v_loc: torch.Tensor | None = None) -> int:
+        """Take the next buffer pair, copy k_loc/v_loc into it (None: the caller
+        wrote ``own[i]`` directly) and return its index."""
+        i = self.turn
+        self.turn = (self.turn + 1) % len(self.own)
+        if k_loc is not None:
+            self.own[i][0].copy_(k_loc)
+        if v_loc is not None:
+            self.own[i][1].copy_(v_loc)
+        self.staged = i
+        return i
+
+    def attend(self, q_loc, window: int = 0, scale=None, **kw):
+        """The fused gather + attention of the local queries on the staged pair."""
+        if self.staged is None:
+            raise RuntimeError("stage() a buffer pair first")
+        row = self.src[self.staged]
+        ks = [self.own[self.staged][0] if rho == self.view.r else row[rho][0] for rho in range(self.view.R)]
+        vs = [self.own[self.staged][1] if rho == self.view.r else row[rho][1] for rho in range(self.view.R)]
+        return hd.hd_attn_fwd_peer_gather(q_loc, ks, vs, self.k_dst, self.v_dst, self.view.n, self.view.R,
+                                          self.view.r, flags=self.flags, window=window, scale=scale, **kw)
+
+    def cross_attention(self, q_loc, k_loc, v_loc, window: int = 0, scale=None, **kw):
+        """stage + fence + attend."""
+        self.stage(k_loc, v_loc)
+        self.fence()
+        return self.attend(q_loc, window, scale, **kw)
+
+    def close(self):
+        """Unmap the peers' buffers (after a barrier, so no rank still reads)."""
+        self.fence()
+        torch.cuda.synchronize()
+        for base in self._bases.values():
+            hd.hd_ipc_close(base)
+        self._bases = {}

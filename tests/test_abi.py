@@ -153,3 +153,44 @@ def test_stream_parallel_bad_arguments(L):
     assert L.hd_attn_combine(fake, fake, fake, None, 2, 10, 6, 0, 0, None) == hd.HD_ERR_INVALID_ARG  # D % 4
     assert L.hd_attn_combine(fake, fake, fake, None, 0, 10, 8, 0, 0, None) == hd.HD_ERR_INVALID_ARG
     assert L.hd_attn_combine(None, None, None, None, 2, 0, 8, 0, 0, None) == hd.HD_OK
+
+
+def test_rank_shard_calls_bad_arguments(L):
+    from stream_sequence_attention_b200 import hd
+    vp = ctypes.c_void_p
+    fake = vp(0x10000)
+    arr = lambda *p: (vp * len(p))(*p)  # noqa: E731
+    k4, v4 = arr(fake, fake, fake, fake), arr(fake, fake, fake, fake)
+
+    def parts(k, v, B=1, L_=8, n=4, R=4, r=0, in_dt=hd.HD_BF16):
+        return L.hd_attn_fwd_parts(fake, k, v, fake, None, B, L_, n, R, r, 2, 2, 128, 0, 0.1, in_dt, hd.HD_BF16,
+                                   None, None)
+
+    assert parts(k4, v4, B=0) == hd.HD_OK
+    assert parts(k4, v4, n=6, R=3) == hd.HD_ERR_INVALID_ARG            # n must divide 128
+    assert parts(k4, v4, R=3) == hd.HD_ERR_INVALID_ARG                 # R must divide n
+    assert parts(k4, v4, r=4) == hd.HD_ERR_INVALID_ARG
+    assert parts(k4, v4, n=16, R=16) == hd.HD_ERR_INVALID_ARG          # more ranks than supported
+    assert parts(k4, v4, in_dt=hd.HD_F32) == hd.HD_ERR_UNSUPPORTED     # tensor-core path only
+    assert parts(arr(fake, None, fake, fake), v4) == hd.HD_ERR_INVALID_ARG
+    assert parts(k4, arr(fake, fake, vp(0x10008), fake)) == hd.HD_ERR_INVALID_ARG  # 16-byte alignment
+    assert parts(None, v4) == hd.HD_ERR_INVALID_ARG
+    # one flag word per (sequence, 128-key tile)
+    assert L.hd_attn_peer_flags_bytes(2, 4096, 4) == 2 * 128 * 8
+    assert L.hd_attn_peer_flags_bytes(1, 150, 4) == 5 * 8
+    assert L.hd_attn_peer_flags_bytes(-1, 150, 4) == 0
+
+    def gather(kd, vd, flags=fake, nbytes=1 << 20, R=4):
+        return L.hd_attn_fwd_peer_gather(fake, k4, v4, kd, vd, flags, nbytes, fake, None, 1, 8, 4, R, 0, 2, 2, 128,
+                                         0, 0.1, hd.HD_BF16, hd.HD_BF16, None, None)
+
+    assert gather(k4, v4, nbytes=7) == hd.HD_ERR_INVALID_ARG           # flags smaller than one word per tile
+    assert gather(k4, v4, flags=None) == hd.HD_ERR_INVALID_ARG
+    assert gather(k4, v4, flags=vp(0x10004)) == hd.HD_ERR_INVALID_ARG  # 8-byte alignment
+    assert gather(None, v4) == hd.HD_ERR_INVALID_ARG
+    assert gather(arr(None, fake, None, fake), v4) == hd.HD_ERR_INVALID_ARG  # a peer's slot missing
+    # IPC helpers reject null arguments without touching CUDA
+    off = ctypes.c_size_t(0)
+    assert L.hd_ipc_export(None, ctypes.create_string_buffer(64), ctypes.byref(off)) == hd.HD_ERR_INVALID_ARG
+    assert L.hd_ipc_open(None, None) == hd.HD_ERR_INVALID_ARG
+    assert L.hd_ipc_close(None) == hd.HD_ERR_INVALID_ARG

@@ -161,6 +161,12 @@ def test_orchestration_runs_end_to_end_on_one_rank(hd):
         torch.cuda.synchronize()
         assert max_abs(to_f64(oc), oracle.attn(q, k, v, n, "cross")[0]) <= TOL_BF16
         assert max_abs(to_f64(oi), oracle.attn(q, k, v, n, "intra")[0]) <= TOL_BF16
+        ps = sp.PeerShards(view, B, L, Hkv, D)
+        for _ in range(3):  # cycles both buffer pairs
+            op = ps.cross_attention(qd, kd, vd, out_dtype=torch.float32)
+        torch.cuda.synchronize()
+        ps.close()
+        assert max_abs(to_f64(op), oracle.attn(q, k, v, n, "cross")[0]) <= TOL_BF16
         Lmax, T = 200, 150
         qd_ = synth.normal((2, n, 8, D), 1061, dtype="bf16")
         kc = synth.normal((2, n, Lmax, Hkv, D), 1062, dtype="bf16")
@@ -172,3 +178,107 @@ def test_orchestration_runs_end_to_end_on_one_rank(hd):
         assert max_abs(to_f64(od), ref) <= TOL_BF16
     finally:
         dist.destroy_process_group()
+
+
+# (n, R, L, Hq, Hkv, D, W): ragged tails, GQA, windows, every rank count that
+# divides n up to the 8-rank limit (128/R rows of each shard per key tile).
+PARTS_CASES = [
+    (4, 1, 150, 4, 2, 128, 0),
+    (4, 2, 150, 4, 2, 128, 0),
+    (4, 4, 150, 4, 2, 128, 0),
+    (4, 2, 150, 4, 2, 128, 150),
+    (8, 8, 70, 2, 1, 128, 0),
+    (8, 2, 95, 4, 4, 64, 0),
+    (2, 2, 300, 6, 2, 128, 37),
+    (16, 4, 40, 2, 2, 128, 0),
+]
+
+
+def _parts_inputs(n, R, L, Hq, Hkv, D, seed):
+    B, P = 2, n * L
+    q = synth.normal((B, P, Hq, D), seed, dtype="bf16")
+    k = synth.normal((B, P, Hkv, D), seed + 1, dtype="bf16")
+    v = synth.normal((B, P, Hkv, D), seed + 2, dtype="bf16")
+    return q, k, v
+
+
+@pytest.mark.parametrize("n,R,L,Hq,Hkv,D,W", PARTS_CASES)
+def test_parts_prefill_reads_shards_in_place(hd, n, R, L, Hq, Hkv, D, W):
+    q, k, v = _parts_inputs(n, R, L, Hq, Hkv, D, 1071)
+    ro, rl = oracle.attn(q, k, v, n, "cross", W)
+    kp = dev(np.stack([_shard(k, n, R, r) for r in range(R)]), "bf16")
+    vp = [dev(_shard(v, n, R, r), "bf16") for r in range(R)]  # list form for v, stacked form for k
+    for r in range(R):
+        st = hd.new_status()
+        o, lse = hd.hd_attn_fwd_parts(dev(_shard(q, n, R, r), "bf16"), kp, vp, n, R, r, W, lse=True,
+                                      out_dtype=torch.float32, dev_status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        assert max_abs(to_f64(o), _shard(ro, n, R, r)) <= TOL_BF16
+        want_lse = _shard(np.transpose(rl, (0, 2, 1)), n, R, r)
+        assert max_abs(np.transpose(to_f64(lse), (0, 2, 1)), want_lse) <= 1e-3
+
+
+@pytest.mark.parametrize("n,R,L,Hq,Hkv,D,W", [c for c in PARTS_CASES if c[1] > 1] + [PARTS_CASES[0]])
+def test_peer_gather_copies_and_attends(hd, n, R, L, Hq, Hkv, D, W):
+    """The fused form with every 'peer' shard in local memory: the same
+    kernel code as with peer pointers.  Run twice with different data through
+    the same destination slots and flags (the flags are reset by the call)."""
+    for rep in range(2):
+        q, k, v = _parts_inputs(n, R, L, Hq, Hkv, D, 1081 + 10 * rep)
+        ro, _ = oracle.attn(q, k, v, n, "cross", W)
+        ks = [dev(_shard(k, n, R, r), "bf16") for r in range(R)]
+        vs = [dev(_shard(v, n, R, r), "bf16") for r in range(R)]
+        for r in range(R):
+            kd = [torch.full_like(ks[0], 7.0) for _ in range(R)]
+            vd = [torch.full_like(vs[0], 7.0) for _ in range(R)]
+            st = hd.new_status()
+            o = hd.hd_attn_fwd_peer_gather(dev(_shard(q, n, R, r), "bf16"), ks, vs, kd, vd, n, R, r, window=W,
+                                           out_dtype=torch.float32, dev_status=st)
+            torch.cuda.synchronize()
+            assert int(st.item()) == 0
+            assert max_abs(to_f64(o), _shard(ro, n, R, r)) <= TOL_BF16
+            for rho in range(R):
+                if rho == r:
+                    assert bool((kd[rho] == 7.0).all()) and bool((vd[rho] == 7.0).all())  # own slot untouched
+                else:
+                    assert torch.equal(kd[rho].view(torch.int16), ks[rho].view(torch.int16))
+                    assert torch.equal(vd[rho].view(torch.int16), vs[rho].view(torch.int16))
+
+
+def test_parts_at_full_size_sampled_rows(hd):
+    """The cross-stream prefill workload (n=4, L=4096, batch 2, 32/8 heads)
+    as rank 0 of 4: the fused gather form, sampled rows of every head against
+    the oracle, and the copies bit-exact."""
+    n, R, r, B, L, Hq, Hkv, D = 4, 4, 0, 2, 4096, 32, 8, 128
+    nl = n // R
+    g = synth.rng(1091)
+    ql = synth.normal_device((B, nl * L, Hq, D), 1092)
+    ks = [synth.normal_device((B, nl * L, Hkv, D), 1093 + i) for i in range(R)]
+    vs = [synth.normal_device((B, nl * L, Hkv, D), 1103 + i) for i in range(R)]
+    kd = [torch.zeros_like(ks[0]) for _ in range(R)]
+    vd = [torch.zeros_like(vs[0]) for _ in range(R)]
+    st = hd.new_status()
+    o = hd.hd_attn_fwd_peer_gather(ql, ks, vs, kd, vd, n, R, r, out_dtype=torch.float32, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    for rho in range(1, R):
+        assert torch.equal(kd[rho].view(torch.int16), ks[rho].view(torch.int16))
+        assert torch.equal(vd[rho].view(torch.int16), vs[rho].view(torch.int16))
+    # the expanded order: position i*n + s holds shard s % R, local row i*nl + s // R
+    kx = torch.stack(ks).view(R, B, L, nl, Hkv, D).permute(1, 2, 3, 0, 4, 5).reshape(B, n * L, Hkv, D)
+    vx = torch.stack(vs).view(R, B, L, nl, Hkv, D).permute(1, 2, 3, 0, 4, 5).reshape(B, n * L, Hkv, D)
+    toks = sorted({0, L - 1, *g.integers(0, L, size=3).tolist()})
+    rows_loc = [i * nl + l for i in toks for l in range(nl)]
+    worst = 0.0
+    for b in range(B):
+        kh, vh = to_f64(kx[b:b + 1]), to_f64(vx[b:b + 1])
+        for h in range(Hq):
+            qh = np.zeros((1, n * L, 1, D))
+            pos = [i * n + r + R * l for i in toks for l in range(nl)]
+            qh[0, pos, 0] = to_f64(ql[b, rows_loc, h])
+            kvh = h // (Hq // Hkv)
+            ro, _ = oracle.attn_rows(qh, kh[:, :, kvh:kvh + 1], vh[:, :, kvh:kvh + 1], n, "cross",
+                                     [(0, 0, p) for p in pos])
+            worst = max(worst, float(np.max(np.abs(to_f64(o[b, rows_loc, h]) - ro))))
+    assert worst <= TOL_BF16, worst

@@ -86,13 +86,40 @@ print(json.dumps({"status": status, "usable": bool(torch.equal(g, h[:, 1::2]))})
 """
 
 
-@pytest.mark.parametrize("var,child", [("HD_TEST_STALL_BWD", "bwd"), ("HD_TEST_STALL_DECODE", "dec")])
-def test_backward_and_decode_waits_time_out_cleanly(var, child):
+CHILD_GATHER = r"""
+import json, sys, torch
+sys.path.insert(0, ROOT)
+from stream_sequence_attention_b200 import build, hd, synth
+build.build(); hd.lib()
+n, R, r, L = 4, 2, 0, 300
+q = synth.normal_device((1, 2 * L, 4, 128), 1)
+ks = [synth.normal_device((1, 2 * L, 2, 128), 2 + i) for i in range(R)]
+vs = [synth.normal_device((1, 2 * L, 2, 128), 4 + i) for i in range(R)]
+kd = [torch.empty_like(ks[0]) for _ in range(R)]
+vd = [torch.empty_like(vs[0]) for _ in range(R)]
+st = hd.new_status()
+hd.hd_attn_fwd_peer_gather(q, ks, vs, kd, vd, n, R, r, dev_status=st)
+torch.cuda.synchronize()
+status = int(st.item())
+h = synth.normal_device((1, 2 * 64, 16), 5)
+g = hd.hd_final_stream_gather(h, 2)
+torch.cuda.synchronize()
+print(json.dumps({"status": status, "usable": bool(torch.equal(g, h[:, 1::2]))}))
+"""
+
+CHILDREN = {"bwd": CHILD_BWD, "dec": CHILD_DEC, "gather": CHILD_GATHER}
+
+
+@pytest.mark.parametrize("var,child", [("HD_TEST_STALL_BWD", "bwd"), ("HD_TEST_STALL_DECODE", "dec"),
+                                       ("HD_TEST_STALL_GATHER", "gather")])
+def test_backward_decode_and_gather_waits_time_out_cleanly(var, child):
     """The same bounded-wait path in the dK/dV backward kernel (its MMA warp of
-    CTA 0 never signals S) and in the decode kernel (the producer of its first
-    CTA issues no loads)."""
+    CTA 0 never signals S), in the decode kernel (the producer of its first
+    CTA issues no loads), and in the fused peer-gather attention (CTA 0 never
+    publishes its first copied piece, so the first key tile never becomes
+    ready for any CTA)."""
     env = dict(os.environ, **{var: "1"})
-    code = (CHILD_BWD if child == "bwd" else CHILD_DEC).replace("ROOT", repr(ROOT))
+    code = CHILDREN[child].replace("ROOT", repr(ROOT))
     r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=180)
     assert r.returncode == 0, r.stderr[-2000:]
     out = json.loads(r.stdout.strip().splitlines()[-1])
