@@ -127,36 +127,55 @@ class ClockSampler:
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
+    INTERVAL_MS = 20
+
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.lines = []
+        self.lines = []  # (arrival time, line)
 
     def start(self):
+        """Start sampling; returns once the first sample has arrived (at most
+        a few seconds), so that a short timed region still gets samples."""
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", str(self.INTERVAL_MS)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
         except OSError:
             self.proc = None
+            return
+        t0 = time.monotonic()
+        while not self.lines and self.proc.poll() is None and time.monotonic() - t0 < 5.0:
+            time.sleep(0.005)
+
+    def mark(self):
+        """Call right before the timed region."""
+        self.t_begin = time.monotonic()
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
 
     def stop(self):
+        """Call right after the timed region.  Keeps the samples that arrived
+        within one interval of it."""
         if self.proc is None:
             return None
+        t_end = time.monotonic()
+        time.sleep(2 * self.INTERVAL_MS / 1000)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
+        slack = self.INTERVAL_MS / 1000
+        t_begin = getattr(self, "t_begin", t_end)
+        window = [ln for (t, ln) in self.lines if t_begin - slack <= t <= t_end + slack]
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
+        for line in window:
             f = [x.strip() for x in line.split(",")]
             if len(f) < 9:
                 continue
@@ -527,6 +546,7 @@ def run_ours(args, rank, world, dist):
 
     clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", 0)))
     clocks.start()
+    clocks.mark()
     parts = []
     steps, kern = timed(torch, work, K, flush, dist, parts=parts)
     clk = clocks.stop()

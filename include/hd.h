@@ -240,11 +240,13 @@ hd_status hd_attn_decode_noalloc(const void* q, const void* k_cache,
  * expanded order of its own streams: local row i*(n/R) + l is token i of
  * global stream r + R*l.  Intra-stream layers need nothing new (call
  * hd_attn_fwd / hd_attn_decode on the local tensors with n/R streams).  A
- * cross-stream layer gathers every rank's K/V shard (a collective the caller
- * runs, e.g. an NCCL all-gather into [R, ...]), restores the expanded order
- * with hd_stream_interleave, and runs hd_attn_fwd_shard for the local
- * queries; cross-stream decode runs hd_attn_decode_shard on every rank for
- * all n stream queries against the local cache streams, gathers the
+ * cross-stream prefill layer either gathers every rank's K/V shard (a
+ * collective the caller runs, e.g. an NCCL all-gather into [R, ...]) and runs
+ * hd_attn_fwd_parts on the gathered shards as they lie (or, for shapes that
+ * call does not take, hd_stream_interleave + hd_attn_fwd_shard), or runs
+ * hd_attn_fwd_peer_gather, whose kernel pulls the peers' shards itself while
+ * it computes.  Cross-stream decode runs hd_attn_decode_shard on every rank
+ * for all n stream queries against the local cache streams, gathers the
  * partials, and merges them with hd_attn_combine.
  */
 
