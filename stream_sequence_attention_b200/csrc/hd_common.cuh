@@ -127,40 +127,6 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
-// ------------------------------------------------- flags between CTAs
-
-// Publish data written with ordinary stores (by the calling warp, whose
-// lanes fenced and synchronised before) to readers in other CTAs that read
-// it through the tensor-memory-access (async) proxy: flag += 1, release.
-__device__ __forceinline__ void flag_publish(unsigned long long* f) {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-  asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(f) : "memory");
-}
-
-// Wait until *f >= target (acquire), then order later TMA reads after it.
-// Bounded like mbar_wait.
-__device__ __forceinline__ bool flag_wait_ge(const unsigned long long* f, unsigned long long target,
-                                             volatile int* abort) {
-  auto ready = [&]() {
-    unsigned long long v;
-    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(f) : "memory");
-    return v >= target;
-  };
-  bool ok = ready();
-  if (!ok) {
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 1;; ++it) {
-      if (ready()) { ok = true; break; }
-      if ((it & 15) == 0) {
-        if (*abort) return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
-      }
-    }
-  }
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-  return ok;
-}
-
 // ----------------------------------------------------------------- tcgen05
 
 // Tensor-memory allocation (whole warp).  Writes the base address to *slot.
