@@ -613,6 +613,25 @@ cudaError_t launch_decode(const void* q, const void* kc, const void* vc, const i
                           int nc, int soff, int sstride) {
   const DecPlan pl = decode_plan(B, n, Lmax, Hq, Hkv, cross, sms);
   if (nc <= 0) nc = n;
+#ifndef HD_DECODE_CROSS_TC
+#define HD_DECODE_CROSS_TC 1
+#endif
+  if (HD_DECODE_CROSS_TC && decode_tc_supported(n, Hq, Hkv, dec::kD, cross)) {
+    // Cross mode on the tensor-core kernel; its split count stays within the
+    // plan the workspace was sized for.
+    const size_t o_bytes = static_cast<size_t>(pl.nsplit) * pl.rows_total * dec::kD * sizeof(float);
+    float* ws_o = static_cast<float*>(ws);
+    float* ws_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + ((o_bytes + 255) & ~static_cast<size_t>(255)));
+    const int ns = decode_tc_nsplit(B * Hkv, Lmax, pl.nsplit, sms);
+    cudaError_t err = launch_decode_tc(q, kc, vc, ctx, ws_o, ws_lse, B, n, Lmax, Hq, Hkv, W, scale, ns, status, st,
+                                       nc, soff, sstride);
+    if (err != cudaSuccess) return err;
+    const int rows = static_cast<int>(pl.rows_total);
+    const int threads = 256;
+    const int blocks = (rows * 32 + threads - 1) / threads;
+    decode_combine_kernel<<<blocks, threads, 0, st>>>(ws_o, ws_lse, o, lse, rows, ns, out_bf16 ? 1 : 0);
+    return cudaGetLastError();
+  }
   CUtensorMap mk, mv;
   if (!encode_cache_view(&mk, kc, B, nc, Lmax, Hkv) || !encode_cache_view(&mv, vc, B, nc, Lmax, Hkv))
     return cudaErrorInvalidValue;

@@ -137,6 +137,14 @@ struct DecPlan {
 };
 DecPlan decode_plan(int B, int n, int Lmax, int Hq, int Hkv, bool cross, int sms);
 size_t decode_workspace_bytes(const DecPlan& pl);
+// Cross-stream decode on tcgen05 (decode_tc.cu): n*G <= 32 query rows per KV
+// head, D = 128.  Writes nsplit partials to the split workspace (the same
+// format as the warp-MMA decode kernel).
+bool decode_tc_supported(int n, int Hq, int Hkv, int D, bool cross);
+int decode_tc_nsplit(int units, int Lmax, int cap, int sms);
+cudaError_t launch_decode_tc(const void* q, const void* kc, const void* vc, const int32_t* ctx, float* ws_o,
+                             float* ws_lse, int B, int n, int Lmax, int Hq, int Hkv, int W, float scale, int nsplit,
+                             int32_t* status, cudaStream_t st, int nc, int soff, int sstride);
 // nc, soff, sstride: the cache holds nc streams, local stream l being global
 // stream soff + sstride*l (stream parallelism, cross mode); nc = 0 means the
 // whole cache (nc = n, soff = 0, sstride = 1).

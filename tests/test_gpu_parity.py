@@ -176,6 +176,11 @@ DECODE_CASES = [
     (2, 3, 200, 6, 3, [199, 64], "cross", 70),
     (1, 1, 129, 4, 4, [129], "intra", 0),
     (2, 8, 100, 16, 2, [100, 3], "cross", 0),        # 64 query rows: two row groups
+    # tensor-core cross decode (n*G <= 32 rows): many splits of one KV head,
+    # a window across split boundaries, one stream with 32 heads per group
+    (1, 4, 5000, 8, 1, [4999], "cross", 0),
+    (1, 2, 3000, 32, 2, [2999], "cross", 1000),
+    (2, 1, 700, 32, 1, [700, 333], "cross", 0),
 ]
 
 
