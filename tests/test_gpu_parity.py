@@ -181,6 +181,7 @@ DECODE_CASES = [
     (1, 4, 5000, 8, 1, [4999], "cross", 0),
     (1, 2, 3000, 32, 2, [2999], "cross", 1000),
     (2, 1, 700, 32, 1, [700, 333], "cross", 0),
+    (2, 4, 70, 8, 1, [70, 5], "cross", 0),             # cache shorter than one 128-token box
 ]
 
 
