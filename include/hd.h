@@ -246,8 +246,9 @@ hd_status hd_attn_decode_noalloc(const void* q, const void* k_cache,
  * call does not take, hd_stream_interleave + hd_attn_fwd_shard), or runs
  * hd_attn_fwd_peer_gather, whose kernel pulls the peers' shards itself while
  * it computes.  Cross-stream decode runs hd_attn_decode_shard on every rank
- * for all n stream queries against the local cache streams, gathers the
- * partials, and merges them with hd_attn_combine.
+ * for all n stream queries against the local cache streams, then either
+ * gathers the partials and merges them with hd_attn_combine, or merges its own
+ * stream rows straight from the ranks' partials with hd_attn_combine_streams.
  */
 
 /*
@@ -308,6 +309,23 @@ hd_status hd_attn_decode_shard(const void* q, const void* k_cache_loc,
                                int Hkv, int D, int window, float scale, hd_dtype in_dt,
                                hd_dtype out_dt, void* workspace, size_t ws_bytes,
                                int32_t* dev_status, void* stream);
+
+/*
+ * The merge of hd_attn_combine for rank r's own stream queries, with the
+ * exchange fused in: each rank's partial is read where it lies (another
+ * GPU's memory through hd_ipc_open, or local), and only rank r's rows:
+ *   o_loc[b, l, h] = merge over rho of (o_parts[rho], lse_parts[rho]) at row
+ *                    (b, r + R*l, h)     (the hd_attn_combine formula)
+ *   o_parts[rho]   [B, n, Hq, D] `in_dt`: rank rho's hd_attn_decode_shard o
+ *   lse_parts[rho] [B, n, Hq] float32: its lse
+ *   o_loc          [B, n/R, Hq, D] `out_dt`;  lse_loc [B, n/R, Hq] float32, nullable
+ * (host arrays of R device pointers).  1 <= R <= HD_MAX_RANKS, R divides n,
+ * D % 4 == 0.  The caller orders the peers' writes of their partials before
+ * the call (e.g. a barrier collective on `stream`).
+ */
+hd_status hd_attn_combine_streams(const void* const* o_parts, const float* const* lse_parts,
+                                  void* o_loc, float* lse_loc, int B, int n, int Hq, int D,
+                                  int R, int r, hd_dtype in_dt, hd_dtype out_dt, void* stream);
 
 /*
  * Cross-stream prefill without the re-interleaved copy.  The operation is

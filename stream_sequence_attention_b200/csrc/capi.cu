@@ -399,6 +399,24 @@ hd_status hd_attn_fwd_peer_gather(const void* q_loc, const void* const* k_src, c
                                           static_cast<cudaStream_t>(stream)));
 }
 
+hd_status hd_attn_combine_streams(const void* const* o_parts, const float* const* lse_parts, void* o_loc,
+                                  float* lse_loc, int B, int n, int Hq, int D, int R, int r, hd_dtype in_dt,
+                                  hd_dtype out_dt, void* stream) {
+  if (B < 0 || Hq < 1 || D < 4 || D % 4 || !valid_shard(n, R, r) || R > kPeerMaxRanks || !valid_dtype(in_dt) ||
+      !valid_dtype(out_dt))
+    return HD_ERR_INVALID_ARG;
+  if (B == 0) return HD_OK;
+  if (!o_parts || !lse_parts || !o_loc || !aligned16(o_loc) || (lse_loc && (reinterpret_cast<uintptr_t>(lse_loc) & 3u)))
+    return HD_ERR_INVALID_ARG;
+  for (int rho = 0; rho < R; ++rho)
+    if (!o_parts[rho] || !lse_parts[rho] || !aligned16(o_parts[rho]) ||
+        (reinterpret_cast<uintptr_t>(lse_parts[rho]) & 3u))
+      return HD_ERR_INVALID_ARG;
+  return cuda_status(launch_attn_combine_streams(o_parts, lse_parts, o_loc, lse_loc, R, B, n, Hq, D, r,
+                                                 in_dt == HD_BF16, out_dt == HD_BF16,
+                                                 static_cast<cudaStream_t>(stream)));
+}
+
 static_assert(sizeof(cudaIpcMemHandle_t) == HD_IPC_HANDLE_BYTES, "IPC handle size");
 
 hd_status hd_ipc_export(const void* ptr, void* handle, size_t* offset) {

@@ -128,6 +128,11 @@ cudaError_t launch_stream_interleave(const void* parts, void* out, int64_t rows,
                                      int sms, cudaStream_t st);
 cudaError_t launch_attn_combine(const void* o_parts, const float* lse_parts, void* o, float* lse, int R,
                                 int64_t rows, int D, bool in_bf16, bool out_bf16, cudaStream_t st);
+// The same merge for rank r's own stream rows only, each part given by its
+// own pointer ([B, n, Hq, D] and [B, n, Hq]; peer memory allowed).
+cudaError_t launch_attn_combine_streams(const void* const* o_parts, const float* const* lse_parts, void* o,
+                                        float* lse, int R, int B, int n, int Hq, int D, int r, bool in_bf16,
+                                        bool out_bf16, cudaStream_t st);
 
 // Decode work decomposition: units (one KV head of one sequence, and for
 // intra mode one stream), row groups of at most 32 query rows, token splits.

@@ -36,6 +36,7 @@ EXPORTS = (
     "hd_attn_decode_noalloc",
     "hd_attn_decode_shard",
     "hd_attn_fwd_shard",
+    "hd_attn_combine_streams",
     "hd_attn_fwd_parts",
     "hd_attn_fwd_peer_gather",
     "hd_attn_peer_flags_bytes",
@@ -99,6 +100,8 @@ def lib() -> ctypes.CDLL:
         L.hd_attn_fwd_shard.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, i32, f32, i32, i32,
                                         vp, vp]
         L.hd_attn_fwd_shard.restype = i32
+        L.hd_attn_combine_streams.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp]
+        L.hd_attn_combine_streams.restype = i32
         L.hd_attn_fwd_parts.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, i32, f32, i32, i32,
                                         vp, vp]
         L.hd_attn_fwd_parts.restype = i32
@@ -613,6 +616,36 @@ def hd_attn_fwd_parts(q_loc: torch.Tensor, k_parts, v_parts, n: int, R: int, r: 
     _check("hd_attn_fwd_parts", lib().hd_attn_fwd_parts(
         _ptr(q_loc), ka, va, _ptr(out), _ptr(lse), B, L, n, R, r, Hq, Hkv, D, int(window), float(scale),
         _dt(q_loc), _dt(out), _ptr(dev_status), _stream(stream)))
+    return (out, lse) if want_lse else out
+
+
+def hd_attn_combine_streams(o_parts, lse_parts, n: int, R: int, r: int, out: torch.Tensor | None = None,
+                            out_dtype=None, lse: torch.Tensor | bool | None = None, like: torch.Tensor | None = None,
+                            stream=None):
+    """Merge the R ranks' cross-stream decode partials for rank r's own
+    stream queries.  o_parts / lse_parts: R tensors [B, n, Hq, D] / [B, n, Hq]
+    (or a stacked tensor), or device addresses of peers' buffers; ``like``
+    (or the first tensor among the parts) gives B, Hq, D and the dtype."""
+    ref = like
+    if ref is None:
+        ref = next((t for t in o_parts if isinstance(t, torch.Tensor)), None)
+    if ref is None:
+        raise TypeError("give `like` when every part is a device address")
+    B, nn, Hq, D = ref.shape
+    if nn != n or R < 1 or n % R:
+        raise ValueError("partials must be [B, n, Hq, D] with R dividing n")
+    oa = _shard_list(o_parts, R, "o_parts", ref.shape, ref.dtype, allow_addr=True)
+    la = _shard_list(lse_parts, R, "lse_parts", (B, n, Hq), torch.float32, allow_addr=True)
+    if out is None:
+        out = torch.empty((B, n // R, Hq, D), dtype=out_dtype or ref.dtype, device=ref.device)
+    _need(out, "out")
+    want_lse = lse is True or isinstance(lse, torch.Tensor)
+    if lse is True:
+        lse = torch.empty((B, n // R, Hq), dtype=torch.float32, device=ref.device)
+    elif lse is False:
+        lse = None
+    _check("hd_attn_combine_streams", lib().hd_attn_combine_streams(
+        oa, la, _ptr(out), _ptr(lse), B, n, Hq, D, R, r, _dt(ref), _dt(out), _stream(stream)))
     return (out, lse) if want_lse else out
 
 

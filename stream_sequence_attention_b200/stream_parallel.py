@@ -20,7 +20,9 @@ of global stream r + R*l.  Per layer:
 * cross-stream decode all-gathers the n stream queries of the new token,
   runs ``hd_attn_decode_shard`` (every query against the local cache
   streams), all-gathers the partial (O, lse) and merges them with
-  ``hd_attn_combine``.
+  ``hd_attn_combine``; or, with :class:`PeerDecode`, each rank merges its own
+  stream rows straight from the ranks' exported partials
+  (``hd_attn_combine_streams``).
 
 Every rank takes the same collective steps in the same order.  This module
 is host-side plumbing: the arithmetic runs in the library's kernels and the
@@ -136,32 +138,10 @@ class PeerShards:
         dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
         self.own = [(torch.empty(self.shape, dtype=dtype, device=dev), torch.empty(self.shape, dtype=dtype, device=dev))
                     for _ in range(buffers)]
-        def export(t):
-            handle, off = hd.hd_ipc_export(t)
-            return handle, off, t.data_ptr() - off  # the exporter's allocation base identifies it
-
-        mine = [(export(k), export(v)) for k, v in self.own]
-        every = [None] * view.R
-        dist.all_gather_object(every, mine, group=view.group)
-        # Buffers may share one allocation (the caching allocator splits
-        # segments): map each exported allocation once.
-        self._bases = {}
-        # src[i][rho] = (k address, v address) of rank rho's pair i
-        self.src = []
-        for i in range(buffers):
-            row = []
-            for rho in range(view.R):
-                if rho == view.r:
-                    row.append(self.own[i])
-                    continue
-                pair = []
-                for handle, off, owner_base in every[rho][i]:
-                    key = (rho, owner_base)
-                    if key not in self._bases:
-                        self._bases[key] = hd.hd_ipc_open(handle)
-                    pair.append(self._bases[key] + off)
-                row.append(tuple(pair))
-            self.src.append(row)
+        self._peers = _PeerMap(view, [t for pair in self.own for t in pair])
+        # src[i][rho] = (k, v) of rank rho's pair i: this rank's tensors, or peer addresses
+        self.src = [[(self._peers.ref(rho, 2 * i, self.own[i][0]), self._peers.ref(rho, 2 * i + 1, self.own[i][1]))
+                     for rho in range(view.R)] for i in range(buffers)]
         self.k_dst = torch.empty((view.R,) + self.shape, dtype=dtype, device=dev)
         self.v_dst = torch.empty_like(self.k_dst)
         nb = hd.hd_attn_peer_flags_bytes(B, L, view.n)
@@ -171,11 +151,7 @@ class PeerShards:
         self.staged = None
 
     def fence(self):
-        if dist.get_backend(self.view.group) == "nccl":
-            dist.all_reduce(self._tok, group=self.view.group)
-        else:
-            torch.cuda.synchronize()
-            dist.barrier(group=self.view.group)
+        _fence(self.view, self._tok)
 
     def stage(self, k_loc: torch.Tensor | None = None, v_loc: torch.Tensor | None = None) -> int:
         """Take the next buffer pair, copy k_loc/v_loc into it (None: the caller
@@ -194,8 +170,8 @@ class PeerShards:
         if self.staged is None:
             raise RuntimeError("stage() a buffer pair first")
         row = self.src[self.staged]
-        ks = [self.own[self.staged][0] if rho == self.view.r else row[rho][0] for rho in range(self.view.R)]
-        vs = [self.own[self.staged][1] if rho == self.view.r else row[rho][1] for rho in range(self.view.R)]
+        ks = [row[rho][0] for rho in range(self.view.R)]
+        vs = [row[rho][1] for rho in range(self.view.R)]
         return hd.hd_attn_fwd_peer_gather(q_loc, ks, vs, self.k_dst, self.v_dst, self.view.n, self.view.R,
                                           self.view.r, flags=self.flags, window=window, scale=scale, **kw)
 
@@ -209,6 +185,114 @@ class PeerShards:
         """Unmap the peers' buffers (after a barrier, so no rank still reads)."""
         self.fence()
         torch.cuda.synchronize()
+        self._peers.close()
+
+
+class PeerDecode:
+    """Stream-parallel cross-stream decode with the partials' exchange fused
+    into the merge: each rank writes its partial (O, lse) for all n stream
+    queries into buffers the other ranks map by CUDA IPC, all ranks pass a
+    barrier, and ``hd_attn_combine_streams`` reads the R partials of this
+    rank's own stream rows where they lie.  Two buffer sets are used in turn,
+    so one barrier per step also keeps a rank from overwriting a set that a
+    peer still reads.  The n stream queries themselves are still gathered
+    with a collective (``cross_decode``), or passed in whole (``partial``)."""
+
+    def __init__(self, view: StreamParallel, B: int, Hq: int, D: int, buffers: int = 2, device=None):
+        if view.R > hd.HD_MAX_RANKS:
+            raise ValueError("PeerDecode supports at most HD_MAX_RANKS ranks")
+        self.view = view
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        n = view.n
+        self.own = [(torch.empty((B, n, Hq, D), dtype=torch.float32, device=dev),
+                     torch.empty((B, n, Hq), dtype=torch.float32, device=dev)) for _ in range(buffers)]
+        self._peers = _PeerMap(view, [t for pair in self.own for t in pair])
+        self.src = [[(self._peers.ref(rho, 2 * i, self.own[i][0]), self._peers.ref(rho, 2 * i + 1, self.own[i][1]))
+                     for rho in range(view.R)] for i in range(buffers)]
+        self._tok = torch.zeros(1, dtype=torch.float32, device=dev)
+        self.turn = 0
+        self.staged = None
+
+    def fence(self):
+        _fence(self.view, self._tok)
+
+    def partial(self, q, kc_loc, vc_loc, ctx_len, window: int = 0, scale=None, workspace=None, dev_status=None):
+        """This rank's partial for all n stream queries q [B, n, Hq, D] against
+        its cache streams, written into the next buffer set."""
+        i = self.turn
+        self.turn = (self.turn + 1) % len(self.own)
+        o, lse = self.own[i]
+        hd.hd_attn_decode_shard(q, kc_loc, vc_loc, ctx_len, self.view.R, self.view.r, window, scale, out=o, lse=lse,
+                                workspace=workspace, dev_status=dev_status)
+        self.staged = i
+        return i
+
+    def merge(self, out_dtype=torch.bfloat16, out=None):
+        """O [B, n/R, Hq, D] of this rank's stream queries from the R partials."""
+        if self.staged is None:
+            raise RuntimeError("partial() first")
+        row = self.src[self.staged]
+        return hd.hd_attn_combine_streams([row[rho][0] for rho in range(self.view.R)],
+                                          [row[rho][1] for rho in range(self.view.R)], self.view.n, self.view.R,
+                                          self.view.r, out=out, out_dtype=out_dtype, like=self.own[self.staged][0])
+
+    def cross_decode(self, q_loc, kc_loc, vc_loc, ctx_len, window: int = 0, scale=None, workspace=None):
+        """All-gather the stream queries, partial, barrier, fused merge."""
+        q = hd.hd_stream_interleave(all_gather_shards(q_loc, self.view.group), self.view.n)
+        self.partial(q, kc_loc, vc_loc, ctx_len, window, scale, workspace)
+        self.fence()
+        return self.merge(out_dtype=q_loc.dtype)
+
+    def close(self):
+        self.fence()
+        torch.cuda.synchronize()
+        self._peers.close()
+
+
+def _fence(view: StreamParallel, tok: torch.Tensor):
+    """Barrier of the view's ranks on the current stream (NCCL: a one-element
+    all-reduce; other backends: synchronise the device, then dist.barrier)."""
+    if dist.get_backend(view.group) == "nccl":
+        dist.all_reduce(tok, group=view.group)
+    else:
+        torch.cuda.synchronize()
+        dist.barrier(group=view.group)
+
+
+class _PeerMap:
+    """CUDA IPC mapping of every rank's copy of a list of device tensors.
+    ``ref(rho, j, mine)`` is rank rho's tensor j: ``mine`` for this rank, else
+    the device address of the peer's tensor in this process."""
+
+    def __init__(self, view: StreamParallel, tensors):
+        def export(t):
+            handle, off = hd.hd_ipc_export(t)
+            return handle, off, t.data_ptr() - off  # the exporter's allocation base identifies it
+
+        mine = [export(t) for t in tensors]
+        every = [None] * view.R
+        dist.all_gather_object(every, mine, group=view.group)
+        # Tensors may share one allocation (the caching allocator splits
+        # segments): map each exported allocation once.
+        self._bases = {}
+        self.addr = []
+        for rho in range(view.R):
+            row = []
+            for handle, off, owner_base in every[rho]:
+                if rho == view.r:
+                    row.append(None)
+                    continue
+                key = (rho, owner_base)
+                if key not in self._bases:
+                    self._bases[key] = hd.hd_ipc_open(handle)
+                row.append(self._bases[key] + off)
+            self.addr.append(row)
+        self.r = view.r
+
+    def ref(self, rho: int, j: int, mine):
+        return mine if rho == self.r else self.addr[rho][j]
+
+    def close(self):
         for base in self._bases.values():
             hd.hd_ipc_close(base)
         self._bases = {}

@@ -194,3 +194,23 @@ def test_rank_shard_calls_bad_arguments(L):
     assert L.hd_ipc_export(None, ctypes.create_string_buffer(64), ctypes.byref(off)) == hd.HD_ERR_INVALID_ARG
     assert L.hd_ipc_open(None, None) == hd.HD_ERR_INVALID_ARG
     assert L.hd_ipc_close(None) == hd.HD_ERR_INVALID_ARG
+
+
+def test_combine_streams_bad_arguments(L):
+    from stream_sequence_attention_b200 import hd
+    vp = ctypes.c_void_p
+    fake = vp(0x10000)
+    arr = lambda *p: (vp * len(p))(*p)  # noqa: E731
+    o2, l2 = arr(fake, fake), arr(fake, fake)
+
+    def call(o, l, B=2, n=4, Hq=8, D=128, R=2, r=0, out=fake):
+        return L.hd_attn_combine_streams(o, l, out, None, B, n, Hq, D, R, r, hd.HD_F32, hd.HD_BF16, None)
+
+    assert call(o2, l2, B=0) == hd.HD_OK
+    assert call(o2, l2, R=3) == hd.HD_ERR_INVALID_ARG          # R must divide n
+    assert call(o2, l2, r=2) == hd.HD_ERR_INVALID_ARG
+    assert call(o2, l2, D=6) == hd.HD_ERR_INVALID_ARG          # D % 4
+    assert call(arr(fake, None), l2) == hd.HD_ERR_INVALID_ARG
+    assert call(o2, arr(fake, vp(0x10002))) == hd.HD_ERR_INVALID_ARG  # lse alignment
+    assert call(o2, l2, out=vp(0x10008)) == hd.HD_ERR_INVALID_ARG     # 16-byte output
+    assert call(None, l2) == hd.HD_ERR_INVALID_ARG

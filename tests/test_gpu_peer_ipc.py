@@ -5,7 +5,9 @@ hd_attn_fwd_peer_gather that reads the other process's buffers through the
 mapped addresses.  The processes take turns on the GPU (a host barrier
 between their launches), so no kernel ever runs beside the other process's;
 no kernel waits on anything outside its own launch.  Three layers cycle the
-two buffer pairs.  Each rank's rows are checked against the float64 oracle."""
+two buffer pairs.  Then the cross-stream decode with the partials' exchange
+fused into the merge (PeerDecode): three steps cycle its two buffer sets.
+Each rank's rows are checked against the float64 oracle."""
 
 import json
 import os
@@ -58,6 +60,31 @@ for layer in range(3):
     ro, _ = oracle.attn(q, k, v, n, "cross")
     errs.append([int(st.item()), max_abs(to_f64(o), shard(ro))])
 ps.close()
+# Cross-stream decode: each rank's partial over its cache streams, merged
+# for its own stream rows from both processes' exported partials.
+Lmax, T, Hd = 300, 257, 8
+pdec = sp.PeerDecode(view, B, Hd, D)
+for step in range(3):
+    qd = synth.normal((B, n, Hd, D), 1501 + 10 * step, dtype="bf16")
+    kc = synth.normal((B, n, Lmax, Hkv, D), 1502 + 10 * step, dtype="bf16")
+    vc = synth.normal((B, n, Lmax, Hkv, D), 1503 + 10 * step, dtype="bf16")
+    ctx = np.array([T, T // 3], dtype=np.int32)
+    st = hd.new_status()
+    for turn in range(R):
+        if turn == rank:
+            pdec.partial(dev(qd, "bf16"), dev(kc[:, rank::R].copy(), "bf16"), dev(vc[:, rank::R].copy(), "bf16"),
+                         dev(ctx, "i32"), dev_status=st)
+            torch.cuda.synchronize()
+        dist.barrier()
+    pdec.fence()
+    for turn in range(R):
+        if turn == rank:
+            od = pdec.merge(out_dtype=torch.float32)
+            torch.cuda.synchronize()
+        dist.barrier()
+    ref, _ = oracle.decode(qd, kc, vc, ctx, n, "cross")
+    errs.append([int(st.item()), max_abs(to_f64(od), ref[:, rank::R])])
+pdec.close()
 dist.destroy_process_group()
 print(json.dumps({"rank": rank, "errs": errs}))
 """

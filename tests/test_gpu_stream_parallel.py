@@ -112,6 +112,16 @@ def test_cross_decode_shards_and_merge(hd, R, T, W):
     fo, fl = oracle.decode_rows(q, kc, vc, ctx, n, "cross", rows, W)
     assert max_abs(to_f64(om).reshape(-1, D), fo) <= TOL_BF16
     assert max_abs(to_f64(lm).reshape(-1), fl) <= 1e-3
+    # The fused form: each rank merges only its own stream rows, reading the
+    # R partials through their own pointers.
+    fo4 = fo.reshape(B, n, Hq, D)
+    fl3 = fl.reshape(B, n, Hq)
+    for r in range(R):
+        ol, ll = hd.hd_attn_combine_streams(o_parts, l_parts, n, R, r, out_dtype=torch.float32, lse=True)
+        torch.cuda.synchronize()
+        assert ol.shape == (B, n // R, Hq, D)
+        assert max_abs(to_f64(ol), fo4[:, r::R]) <= TOL_BF16
+        assert max_abs(to_f64(ll), fl3[:, r::R]) <= 1e-3
 
 
 @pytest.mark.parametrize("in_dt,out_dt", [("f32", "f32"), ("bf16", "bf16"), ("f32", "bf16")])
@@ -176,6 +186,12 @@ def test_orchestration_runs_end_to_end_on_one_rank(hd):
         torch.cuda.synchronize()
         ref, _ = oracle.decode(qd_, kc, vc, ctx, n, "cross")
         assert max_abs(to_f64(od), ref) <= TOL_BF16
+        pdec = sp.PeerDecode(view, 2, 8, D)
+        for _ in range(3):  # cycles both buffer sets
+            op = pdec.cross_decode(dev(qd_, "bf16"), dev(kc, "bf16"), dev(vc, "bf16"), dev(ctx, "i32"))
+        torch.cuda.synchronize()
+        pdec.close()
+        assert max_abs(to_f64(op), ref) <= TOL_BF16
     finally:
         dist.destroy_process_group()
 
