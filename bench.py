@@ -773,12 +773,18 @@ def stream_parallel_rank(torch, peaks, rank, time_fn, R=4):
     l_all = lp.unsqueeze(0).expand(R, -1, -1, -1).contiguous()
     out = torch.empty((B, n, Hq, D), dtype=torch.bfloat16, device="cuda")
     ms_cb = time_fn(lambda: hd.hd_attn_combine(o_all, l_all, out=out))
+    # The fused merge of rank 0's own stream rows from R partials read through
+    # their own pointers (here R local copies; on R GPUs, peers' memory).
+    o_list = [op] + [op.clone() for _ in range(R - 1)]
+    l_list = [lp] + [lp.clone() for _ in range(R - 1)]
+    out_loc = torch.empty((B, n // R, Hq, D), dtype=torch.bfloat16, device="cuda")
+    ms_cs = time_fn(lambda: hd.hd_attn_combine_streams(o_list, l_list, n, R, 0, out=out_loc))
     res[f"sp_R{R}_rank0_cross_decode"] = {
         "partial_ms": round(ms_dec, 3), "partial_GB/s": round(dec_bytes / (ms_dec * 1e-3) / 1e9, 1),
         "partial_frac_hbm": round(dec_bytes / (ms_dec * 1e-3) / 1e9 / peaks["hbm"], 4),
-        "merge_ms": round(ms_cb, 4),
+        "merge_ms": round(ms_cb, 4), "merge_own_rows_ms": round(ms_cs, 4),
         "allgather_bytes_in_per_rank": (R - 1) * (q.numel() // R * 2 + op.numel() * 4 + lp.numel() * 4)}
-    del q, kc, vc, op, lp, ws, o_all, l_all, out
+    del q, kc, vc, op, lp, ws, o_all, l_all, out, o_list, l_list, out_loc
     torch.cuda.empty_cache()
     return res
 
