@@ -357,7 +357,8 @@ hd_status hd_attn_fwd_parts(const void* q_loc, const void* const* k_parts,
  * key tile is read only after its own pieces have landed.  k_src[r],
  * v_src[r] are this rank's shard, read in place (k_dst[r], v_dst[r] unused).
  *   flags  device workspace of hd_attn_peer_flags_bytes(B, L, n) bytes,
- *          zeroed by the call on `stream`.
+ *          zeroed by the call on `stream`; calls that may run at the same
+ *          time need separate flags (and separate k_dst/v_dst).
  * The launch is cooperative (all CTAs resident at once).  Ordering across
  * ranks is the caller's: every shard must be complete before the call runs,
  * and no rank may overwrite its shard before the other ranks' calls that
