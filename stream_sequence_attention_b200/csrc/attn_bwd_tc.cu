@@ -136,6 +136,21 @@ __device__ __forceinline__ int bw_pos(const BwParams& p, int i) { return i * p.g
 struct KvUnit {
   int b, skv, sq, kvh, kblk, qt_lo, qt_hi, nqt;
 };
+// Unit schedule of a CTA: rounds of gridDim.x units in the longest-first
+// order, walked forwards in even rounds and backwards in odd ones, so that
+// every CTA gets a similar total.  The k-th unit of this CTA, -1 when the
+// rounds are exhausted, -2 when round k has none for it.
+#ifndef HD_TC_SNAKE
+#define HD_TC_SNAKE 1
+#endif
+__device__ __forceinline__ int bw_unit_of(int k, int total) {
+  const int base = k * static_cast<int>(gridDim.x);
+  if (base >= total) return -1;
+  const int c = (HD_TC_SNAKE && (k & 1)) ? static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x)
+                                         : static_cast<int>(blockIdx.x);
+  return base + c < total ? base + c : -2;
+}
+
 __device__ __forceinline__ KvUnit kv_unit(int u, const BwParams& p) {
   const int per = p.g.B * p.kns * p.Hkv;
   KvUnit x;
@@ -330,7 +345,9 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
       int t = 0, ul = 0, kv_issued = 0;
       int q_issued[Lay::QST] = {}, o_issued[Lay::QST] = {};
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++ul) {
+      for (int k = 0, u = bw_unit_of(0, p.total_units); ok && u != -1;
+           ul += (u >= 0), u = bw_unit_of(++k, p.total_units)) {
+        if (u < 0) continue;  // round k has no unit for this CTA
         const KvUnit x = kv_unit(u, p);
         if (!mbar_wait(bar(Lay::B_KVEMPTY), (ul & 1) ^ 1, abort_flag)) { ok = false; break; }
         mbar_arrive_expect_tx(bar(Lay::B_KVFULL), 2 * T::TILE);
@@ -397,7 +414,9 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
         mma_rows_rows<D>(tDP, sbase + Lay::V_OFF, sbase + Lay::O_OFF + st * T::TILE);
         tc_commit(bar(Lay::B_DPFULL));
       };
-      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++ul) {
+      for (int k = 0, u = bw_unit_of(0, p.total_units); ok && u != -1;
+           ul += (u >= 0), u = bw_unit_of(++k, p.total_units)) {
+        if (u < 0) continue;  // round k has no unit for this CTA
         const KvUnit x = kv_unit(u, p);
         const int nt = G * x.nqt;
         if (!mbar_wait(bar(Lay::B_KVFULL), ul & 1, abort_flag)) { ok = false; break; }
@@ -454,7 +473,9 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
     const float sl2 = p.scale_log2;
     int t = 0, ul = 0;
     bool ok = true;
-    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++ul) {
+    for (int k = 0, u = bw_unit_of(0, p.total_units); ok && u != -1;
+         ul += (u >= 0), u = bw_unit_of(++k, p.total_units)) {
+      if (u < 0) continue;  // round k has no unit for this CTA
       const KvUnit x = kv_unit(u, p);
       const int nt = G * x.nqt;
       const int k0 = x.kblk * bw::BT;
@@ -631,7 +652,9 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
       int t = 0, ul = 0, q_issued = 0;
       int k_issued[Lay::KST] = {}, v_issued[Lay::VST] = {};
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++ul) {
+      for (int k = 0, u = bw_unit_of(0, p.total_units); ok && u != -1;
+           ul += (u >= 0), u = bw_unit_of(++k, p.total_units)) {
+        if (u < 0) continue;  // round k has no unit for this CTA
         const QUnit x = q_unit(u, p);
         const int kvh = x.h / G;
         if (!mbar_wait(bar(Lay::B_QEMPTY), (ul & 1) ^ 1, abort_flag)) { ok = false; break; }
@@ -698,7 +721,9 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
         tc_commit(bar(Lay::B_VEMPTY + vs));
         return true;
       };
-      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++ul) {
+      for (int k = 0, u = bw_unit_of(0, p.total_units); ok && u != -1;
+           ul += (u >= 0), u = bw_unit_of(++k, p.total_units)) {
+        if (u < 0) continue;  // round k has no unit for this CTA
         const QUnit x = q_unit(u, p);
         const int nt = x.nkt;
         if (!mbar_wait(bar(Lay::B_QFULL), ul & 1, abort_flag)) { ok = false; break; }
@@ -730,7 +755,9 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
     const float sl2 = p.scale_log2;
     int t = 0, ul = 0;
     bool ok = true;
-    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++ul) {
+    for (int k = 0, u = bw_unit_of(0, p.total_units); ok && u != -1;
+         ul += (u >= 0), u = bw_unit_of(++k, p.total_units)) {
+      if (u < 0) continue;  // round k has no unit for this CTA
       const QUnit x = q_unit(u, p);
       const int iq = x.qblk * bw::BT + r;  // this thread's query token
       const int64_t lat = ((static_cast<int64_t>(x.b) * p.Hq + x.h) * p.g.ns + x.s) * p.Lpad + iq;

@@ -109,6 +109,23 @@ struct TcUnit {
   int b, s, kvh, qblk, h0, h1, t_lo, t_hi;  // h1 < 0: only one head in this unit
 };
 
+// Unit schedule of a CTA: rounds of gridDim.x units in the longest-first
+// order, walked forwards in even rounds and backwards in odd ones, so that
+// every CTA gets a similar total (with a plain stride the first CTAs would
+// always take the longest unit of each round).  Returns the k-th unit of
+// this CTA, -1 when the rounds are exhausted, -2 when round k has none for
+// it.  Every role walks the same sequence.
+#ifndef HD_TC_SNAKE
+#define HD_TC_SNAKE 1
+#endif
+__device__ __forceinline__ int tc_unit_of(int k, int total) {
+  const int base = k * static_cast<int>(gridDim.x);
+  if (base >= total) return -1;
+  const int c = (HD_TC_SNAKE && (k & 1)) ? static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x)
+                                         : static_cast<int>(blockIdx.x);
+  return base + c < total ? base + c : -2;
+}
+
 __device__ __forceinline__ TcUnit tc_unit(int u, const TcParams& p) {
   const int G = p.Hq / p.Hkv;
   const int per = p.g.B * p.g.ns * p.Hkv * p.npairs;
@@ -338,7 +355,10 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
       int t = 0, ul = 0, q_issued = 0;
       int k_issued[tc::KST] = {}, v_issued[tc::VST] = {};
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++ul) {
+      for (int k = 0; ok; ++k) {
+        const int u = tc_unit_of(k, p.total_units);
+        if (u == -1) break;
+        if (u < 0) continue;
         const TcUnit x = tc_unit(u, p);
         if (!mbar_wait(bar(Lay::B_QEMPTY), (ul & 1) ^ 1, abort_flag)) { ok = false; break; }
         mbar_arrive_expect_tx(bar(Lay::B_QFULL), Lay::TILE * (x.h1 >= 0 ? 2 : 1));
@@ -372,6 +392,7 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
           load_kv_tile(kv.v, sbase + Lay::V_OFF + vs * Lay::TILE, bar(Lay::B_VFULL + vs), x, skv, kt);
           ++v_issued[vs];
         }
+        ++ul;
       }
       if (!ok) {
         fail();
@@ -415,7 +436,10 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
       int ts[2] = {0, 0};  // P_h V MMAs issued per head slot
       int us[2] = {0, 0};  // units per head slot
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++ul) {
+      for (int k = 0; ok; ++k) {
+        const int u = tc_unit_of(k, p.total_units);
+        if (u == -1) break;
+        if (u < 0) continue;
         const TcUnit x = tc_unit(u, p);
         const int nslot = x.h1 >= 0 ? 2 : 1;
         const int nt = x.t_hi - x.t_lo + 1;
@@ -461,6 +485,7 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
         }
         us[0]++;
         if (nslot == 2) us[1]++;
+        ++ul;
       }
       if (!ok) fail();
       // Drain: every MMA issued above has completed before TMEM is freed.
@@ -477,7 +502,10 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
     const float sl2 = p.scale_log2;
     int sc = 0, uc = 0, oc = 0;
     bool ok = true;
-    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
+    for (int k = 0; ok; ++k) {
+      const int u = tc_unit_of(k, p.total_units);
+      if (u == -1) break;
+      if (u < 0) continue;
       const TcUnit x = tc_unit(u, p);
       const int h = slot ? x.h1 : x.h0;
       if (h < 0) continue;  // uniform across the warpgroup
