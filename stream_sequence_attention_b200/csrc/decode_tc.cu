@@ -66,7 +66,13 @@ constexpr int MX_OFF = P_OFF + 2 * 2 * kRBlk;       // [2 groups][4 warps][32 ro
 constexpr int LS_OFF = MX_OFF + 2 * 4 * kN * 4;     // [2 groups][4 warps][32 rows] float
 constexpr int ML_OFF = LS_OFF + 2 * 4 * kN * 4;     // [2 groups][32 rows] float (running max)
 constexpr int BAR_OFF = ML_OFF + 2 * kN * 4;
-constexpr int B_KFULL = 0, B_VFULL = B_KFULL + kStages, B_EMPTY = B_VFULL + kStages, B_QFULL = B_EMPTY + kStages,
+// B_EMPTY: a stage's K half is free (S of its tile done); B_VEMPTY: its V
+// half is free (P V done).  With HD_DTC_SPLIT_EMPTY=0 both halves wait for P V.
+#ifndef HD_DTC_SPLIT_EMPTY
+#define HD_DTC_SPLIT_EMPTY 1
+#endif
+constexpr int B_KFULL = 0, B_VFULL = B_KFULL + kStages, B_EMPTY = B_VFULL + kStages, B_VEMPTY = B_EMPTY + kStages,
+              B_QFULL = B_VEMPTY + kStages,
               B_SFULL = B_QFULL + 1, B_PFULL = B_SFULL + 2, B_PVDONE = B_PFULL + 2, B_MX = B_PVDONE + 2,
               B_LS = B_MX + 2, B_DRAIN = B_LS + 1, NBAR = B_DRAIN + 1;
 constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
@@ -155,6 +161,7 @@ __global__ void __launch_bounds__(dtc::kThreads, 1)
       mbar_init(bar(B_KFULL + i), 1);
       mbar_init(bar(B_VFULL + i), 1);
       mbar_init(bar(B_EMPTY + i), 1);
+      mbar_init(bar(B_VEMPTY + i), 1);
     }
     mbar_init(bar(B_QFULL), 256);
     for (int i = 0; i < 2; ++i) {
@@ -200,6 +207,8 @@ __global__ void __launch_bounds__(dtc::kThreads, 1)
         for (int hh = 0; hh < 2; ++hh)
           tma_load_5d(sbase + K_OFF + st * kTile + hh * kBlk, &tmK, bar(B_KFULL + st), hh * 64, kvh, j0, sp, b);
         ++k_issued[st];
+        if (HD_DTC_SPLIT_EMPTY &&
+            !mbar_wait(bar(B_VEMPTY + st), ((t / kStages) & 1) ^ 1, abort_flag)) { ok = false; break; }
         mbar_arrive_expect_tx(bar(B_VFULL + st), kTile);
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh)
@@ -231,6 +240,7 @@ __global__ void __launch_bounds__(dtc::kThreads, 1)
                  kk > 0 ? 1u : 0u);
         }
         tc_commit(bar(B_SFULL + (t & 1)));
+        if (HD_DTC_SPLIT_EMPTY) tc_commit(bar(B_EMPTY + t % kStages));
       };
       bool ok = mbar_wait(bar(B_QFULL), 0, abort_flag);
       if (ok && ntiles > 0) {
@@ -268,7 +278,7 @@ __global__ void __launch_bounds__(dtc::kThreads, 1)
           mma_ss(tmem + (2 + g) * kN, adesc, bdesc, idO, (t > 1 || kk > 0) ? 1u : 0u);
         }
         tc_commit(bar(B_PVDONE + g));
-        tc_commit(bar(B_EMPTY + st));
+        tc_commit(bar(HD_DTC_SPLIT_EMPTY ? B_VEMPTY + st : B_EMPTY + st));
       }
       if (!ok) fail();
       tc_commit(bar(B_DRAIN));
