@@ -520,13 +520,16 @@ bool decode_tc_supported(int n, int Hq, int Hkv, int D, bool cross) {
   return cross && D == dtc::kD && n * (Hq / Hkv) <= dtc::kN;
 }
 
-// Splits per unit: at least ~4 waves of one CTA per SM, the count whose
+// Splits per unit: at least ~2 waves of one CTA per SM, the count whose
 // last wave is fullest, never more than the workspace was sized for.
 int decode_tc_nsplit(int units, int Lmax, int cap, int sms) {
   int max_ns = (Lmax + dtc::kTok - 1) / dtc::kTok;
   if (max_ns > cap) max_ns = cap;
   if (max_ns < 1) max_ns = 1;
-  int lo = (4 * sms + units - 1) / units;
+#ifndef HD_DTC_MIN_WAVES
+#define HD_DTC_MIN_WAVES 2
+#endif
+  int lo = (HD_DTC_MIN_WAVES * sms + units - 1) / units;
   if (lo < 1) lo = 1;
   if (lo > max_ns) lo = max_ns;
   int best = lo;
