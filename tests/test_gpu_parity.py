@@ -110,7 +110,7 @@ ATTN_CASES = [
 @pytest.mark.parametrize("out_f32", [False, True])
 def test_attn_fwd_matches_oracle(hd, dtype, B, n, L, Hq, Hkv, D, mode, W, out_f32):
     if dtype == "f32" and not out_f32:
-        pytest.skip("fp32 inputs are judged on fp32 output")
+        pytest.skip("fp32 inputs are compared on fp32 output")
     P = n * L
     q, k, v = host_qkv(B, P, Hq, Hkv, D, 50 + L + W, dtype)
     scale = D ** -0.5
