@@ -1,0 +1,102 @@
+"""Seeded random sweep of the attention calls against the float64 oracle.
+
+Beyond the hand-picked cases of the other GPU tests: shapes drawn from a
+fixed generator (stream count n, tokens per stream L including ragged tails,
+query/KV heads with every GQA ratio, head dim 64 or 128, window or none, mode,
+input dtype), each case run through the forward, the final-stream forward,
+decode and the backward.  Sizes stay small enough for the oracle to finish in
+seconds; the same seeds give the same cases on every run."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from stream_sequence_attention_b200 import synth
+from tests.gpu_util import TOL_BF16, TOL_F32, dev, lib, max_abs, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def hd():
+    return lib()
+
+
+def _case(seed):
+    g = np.random.default_rng(seed)
+    n = int(g.choice([1, 2, 3, 4, 5, 8]))
+    L = int(g.integers(1, 300 // n + 40))
+    Hkv = int(g.choice([1, 2, 3]))
+    G = int(g.choice([1, 2, 3, 4, 8]))
+    D = int(g.choice([64, 128]))
+    mode = str(g.choice(["intra", "cross"]))
+    W = 0 if g.random() < 0.5 else int(g.integers(1, max(2, (L if mode == "intra" else n * L))))
+    dt = "bf16" if g.random() < 0.75 else "f32"
+    return n, L, Hkv * G, Hkv, D, mode, W, dt
+
+
+SEEDS = list(range(9000, 9048))
+
+
+@pytest.mark.parametrize("seed", SEEDS)
+def test_forward_and_final_stream(hd, seed):
+    n, L, Hq, Hkv, D, mode, W, dt = _case(seed)
+    B, P = 2, n * L
+    q = synth.normal((B, P, Hq, D), seed, dtype=dt)
+    k = synth.normal((B, P, Hkv, D), seed + 1, dtype=dt)
+    v = synth.normal((B, P, Hkv, D), seed + 2, dtype=dt)
+    tol = TOL_BF16 if dt == "bf16" else TOL_F32
+    st = hd.new_status()
+    o, lse = hd.hd_attn_fwd(dev(q, dt), dev(k, dt), dev(v, dt), n, mode, W, lse=True, out_dtype=torch.float32,
+                            dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ro, rl = oracle.attn(q, k, v, n, mode, W)
+    assert max_abs(to_f64(o), ro) <= tol, (n, L, Hq, Hkv, D, mode, W, dt)
+    assert max_abs(to_f64(lse), rl) <= (1e-3 if dt == "bf16" else 1e-4)
+    qf = np.ascontiguousarray(q.reshape(B, L, n, Hq, D)[:, :, n - 1])
+    of = hd.hd_attn_fwd_final_stream(dev(qf, dt), dev(k, dt), dev(v, dt), n, mode, W, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    rf, _ = oracle.attn_final_stream(qf, k, v, n, mode, W)
+    assert max_abs(to_f64(of), rf) <= tol
+
+
+@pytest.mark.parametrize("seed", SEEDS[:24])
+def test_backward(hd, seed):
+    n, L, Hq, Hkv, D, mode, W, dt = _case(seed)
+    B, P = 1, n * L
+    q = synth.normal((B, P, Hq, D), seed + 10, dtype=dt)
+    k = synth.normal((B, P, Hkv, D), seed + 11, dtype=dt)
+    v = synth.normal((B, P, Hkv, D), seed + 12, dtype=dt)
+    dO = synth.normal((B, P, Hq, D), seed + 13, dtype=dt)
+    qd, kd, vd, gd = dev(q, dt), dev(k, dt), dev(v, dt), dev(dO, dt)
+    st = hd.new_status()
+    o, lse = hd.hd_attn_fwd(qd, kd, vd, n, mode, W, lse=True, dev_status=st)
+    dq, dk, dv = hd.hd_attn_bwd(qd, kd, vd, o, gd, lse, n, mode, W, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    rq, rk, rv = oracle.attn_bwd(q, k, v, dO, n, mode, W)
+    tol = TOL_BF16 if dt == "bf16" else TOL_F32
+    for got, ref in ((dq, rq), (dk, rk), (dv, rv)):
+        assert max_abs(to_f64(got), ref) <= tol * max(1.0, float(np.max(np.abs(ref)))), (n, L, Hq, Hkv, D, mode, W)
+
+
+@pytest.mark.parametrize("seed", SEEDS[:32])
+def test_decode(hd, seed):
+    n, L, Hq, Hkv, D, mode, W, dt = _case(seed)
+    D = 128  # the decode kernels take head dim 128
+    B, Lmax = 3, L + 7
+    q = synth.normal((B, n, Hq, D), seed + 20, dtype="bf16")
+    kc = synth.normal((B, n, Lmax, Hkv, D), seed + 21, dtype="bf16")
+    vc = synth.normal((B, n, Lmax, Hkv, D), seed + 22, dtype="bf16")
+    g = np.random.default_rng(seed + 23)
+    ctx = g.integers(1, Lmax + 1, size=B).astype(np.int32)
+    st = hd.new_status()
+    o, lse = hd.hd_attn_decode(dev(q, "bf16"), dev(kc, "bf16"), dev(vc, "bf16"), dev(ctx, "i32"), mode, W,
+                               out_dtype=torch.float32, lse=True, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ro, rl = oracle.decode(q, kc, vc, ctx, n, mode, W)
+    assert max_abs(to_f64(o), ro) <= TOL_BF16, (n, Lmax, Hq, Hkv, mode, W, ctx.tolist())
+    assert max_abs(to_f64(lse), rl) <= 1e-3
