@@ -100,3 +100,48 @@ def test_decode(hd, seed):
     ro, rl = oracle.decode(q, kc, vc, ctx, n, mode, W)
     assert max_abs(to_f64(o), ro) <= TOL_BF16, (n, Lmax, Hq, Hkv, mode, W, ctx.tolist())
     assert max_abs(to_f64(lse), rl) <= 1e-3
+
+
+def _shard(x, n, R, r):
+    """Rank r's streams of x [B, n*L, ...] in local order (reshape, no oracle)."""
+    B, P = x.shape[:2]
+    L, nl = P // n, n // R
+    return np.ascontiguousarray(x.reshape((B, L, nl, R) + x.shape[2:])[:, :, :, r].reshape((B, L * nl) + x.shape[2:]))
+
+
+@pytest.mark.parametrize("seed", list(range(9100, 9116)))
+def test_rank_shard_prefill(hd, seed):
+    """hd_attn_fwd_parts and hd_attn_fwd_peer_gather for a random rank of a
+    random stream-parallel layout (R | n, n | 128), against the oracle."""
+    g = np.random.default_rng(seed)
+    n = int(g.choice([1, 2, 4, 8]))
+    R = int(g.choice([d for d in (1, 2, 4, 8) if n % d == 0]))
+    r = int(g.integers(0, R))
+    L = int(g.integers(1, 400 // n + 20))
+    Hkv = int(g.choice([1, 2]))
+    Hq = Hkv * int(g.choice([1, 2, 3, 4]))
+    D = int(g.choice([64, 128]))
+    W = 0 if g.random() < 0.6 else int(g.integers(1, n * L + 1))
+    B, P = 2, n * L
+    q = synth.normal((B, P, Hq, D), seed, dtype="bf16")
+    k = synth.normal((B, P, Hkv, D), seed + 1, dtype="bf16")
+    v = synth.normal((B, P, Hkv, D), seed + 2, dtype="bf16")
+    ro, _ = oracle.attn(q, k, v, n, "cross", W)
+    want = _shard(ro, n, R, r)
+    ks = [dev(_shard(k, n, R, rho), "bf16") for rho in range(R)]
+    vs = [dev(_shard(v, n, R, rho), "bf16") for rho in range(R)]
+    ql = dev(_shard(q, n, R, r), "bf16")
+    st = hd.new_status()
+    o1 = hd.hd_attn_fwd_parts(ql, ks, vs, n, R, r, W, out_dtype=torch.float32, dev_status=st)
+    kd = [torch.zeros_like(ks[0]) for _ in range(R)]
+    vd = [torch.zeros_like(vs[0]) for _ in range(R)]
+    o2 = hd.hd_attn_fwd_peer_gather(ql, ks, vs, kd, vd, n, R, r, window=W, out_dtype=torch.float32, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    case = (n, R, r, L, Hq, Hkv, D, W)
+    assert max_abs(to_f64(o1), want) <= TOL_BF16, case
+    assert max_abs(to_f64(o2), want) <= TOL_BF16, case
+    for rho in range(R):
+        if rho != r:
+            assert torch.equal(kd[rho].view(torch.int16), ks[rho].view(torch.int16)), case
+            assert torch.equal(vd[rho].view(torch.int16), vs[rho].view(torch.int16)), case
