@@ -109,8 +109,9 @@ ATTN_CASES = [
 @pytest.mark.parametrize("dtype,B,n,L,Hq,Hkv,D,mode,W", ATTN_CASES)
 @pytest.mark.parametrize("out_f32", [False, True])
 def test_attn_fwd_matches_oracle(hd, dtype, B, n, L, Hq, Hkv, D, mode, W, out_f32):
-    if dtype == "f32" and not out_f32:
-        pytest.skip("fp32 inputs are compared on fp32 output")
+    """Every case with float32 and bf16 output.  bf16 output is held to the
+    bf16 bound whatever the input type (its rounding alone is up to 2^-9 of
+    |O|)."""
     P = n * L
     q, k, v = host_qkv(B, P, Hq, Hkv, D, 50 + L + W, dtype)
     scale = D ** -0.5
@@ -119,7 +120,7 @@ def test_attn_fwd_matches_oracle(hd, dtype, B, n, L, Hq, Hkv, D, mode, W, out_f3
                             out_dtype=torch.float32 if out_f32 else None, lse=True, dev_status=st)
     torch.cuda.synchronize()
     ro, rl = oracle.attn(q, k, v, n, mode, W, scale)
-    tol = TOL_F32 if dtype == "f32" else TOL_BF16
+    tol = TOL_F32 if (dtype == "f32" and out_f32) else TOL_BF16
     err = max_abs(to_f64(o), ro)
     assert err <= tol, f"max-abs {err}"
     assert max_abs(to_f64(lse), rl) <= (TOL_F32 if dtype == "f32" else 1e-3)
