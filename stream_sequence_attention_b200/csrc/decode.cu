@@ -622,7 +622,7 @@ cudaError_t launch_decode(const void* q, const void* kc, const void* vc, const i
     const size_t o_bytes = static_cast<size_t>(pl.nsplit) * pl.rows_total * dec::kD * sizeof(float);
     float* ws_o = static_cast<float*>(ws);
     float* ws_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + ((o_bytes + 255) & ~static_cast<size_t>(255)));
-    const int ns = decode_tc_nsplit(B * Hkv, Lmax, pl.nsplit, sms);
+    const int ns = decode_tc_nsplit(pl.units, Lmax, pl.nsplit, sms);
     cudaError_t err = launch_decode_tc(q, kc, vc, ctx, ws_o, ws_lse, B, n, Lmax, Hq, Hkv, W, scale, ns, status, st,
                                        nc, soff, sstride);
     if (err != cudaSuccess) return err;

@@ -4,10 +4,11 @@
 // ("Hidden Decoding at Scale", "Persistent KV and the KV-mirror Saving" and
 // "Inference Throughput": the n stream queries of a new token read every
 // stream's cache.)  In cross mode the n*G query rows of one KV head (n
-// streams x G heads of the group, at most 32) share every cached key, so a
-// unit is one (sequence, KV head) with all its rows, and its token range is
-// split across CTAs as in the warp-MMA kernel; the partial results go to the
-// same workspace and the same split-merge kernel.
+// streams x G heads of the group) share every cached key, so a unit is one
+// (sequence, KV head) with its rows -- up to 32 per unit, more rows making
+// more row groups -- and its token range is split across CTAs as in the
+// warp-MMA kernel; the partial results go to the same workspace and the same
+// split-merge kernel.
 //
 // Each cached K/V byte is read once per step, so the kernel is meant to run
 // at the HBM rate.  The warp-level MMA form reads every K, V and Q fragment
@@ -133,9 +134,15 @@ __global__ void __launch_bounds__(dtc::kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.Hq / p.Hkv;
-  const int R = p.n * G;  // query rows of the unit (<= kN)
-  const int kvh = blockIdx.y % p.Hkv;
-  const int b = blockIdx.y / p.Hkv;
+  // Unit = (sequence, KV head, row group): rows [r0, r0 + R) of the n*G
+  // query rows that share the KV head, at most kN per group (each group
+  // streams the cache once).
+  const int rg_count = (p.n * G + kN - 1) / kN;
+  const int rg = blockIdx.y % rg_count;
+  const int kvh = (blockIdx.y / rg_count) % p.Hkv;
+  const int b = blockIdx.y / rg_count / p.Hkv;
+  const int r0 = rg * kN;
+  const int R = min(kN, p.n * G - r0);
   const int split = blockIdx.x;
   const int rows_total = p.B * p.n * p.Hq;
 
@@ -298,7 +305,7 @@ __global__ void __launch_bounds__(dtc::kThreads, 1)
         const int r = e >> 4, c = e & 15;
         uint4 val = make_uint4(0, 0, 0, 0);
         if (r < R) {
-          const int s = r / G, h = kvh * G + (r - s * G);
+          const int s = (r0 + r) / G, h = kvh * G + (r0 + r - s * G);
           val = reinterpret_cast<const uint4*>(p.q + ((static_cast<int64_t>(b) * p.n + s) * p.Hq + h) * kD)[c];
         }
         *reinterpret_cast<uint4*>(smem + Q_OFF + (c >> 3) * kRBlk + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = val;
@@ -345,13 +352,17 @@ __global__ void __launch_bounds__(dtc::kThreads, 1)
         // Key p' = j*n + (its global stream) is visible to row r (stream
         // r div G, position (T-1)*n + r div G) iff, with dk = p' - (T-1)*n,
         // dk <= r div G and (W = 0 or r div G - dk < W), i.e. r >= dk*G and
-        // (W = 0 or r < (W + dk)*G); keys of the next split (j >= c_hi) are
-        // not this CTA's.  Rows r >= R are padding.
+        // (W = 0 or r < (W + dk)*G) for the unit's row r; keys of the next
+        // split (j >= c_hi) are not this CTA's.  Rows >= R are padding.
         const int j = j0 + key;
         const int64_t dk = static_cast<int64_t>(j) * p.n + (p.soff + p.sstride * sp) - pq_base;
-        const int rlo = j >= c_hi ? kN : dk <= 0 ? 0 : dk >= kN ? kN : static_cast<int>(dk) * G;
+        // In this group's row numbering r = r' - r0 (all in 64 bits, clamped).
+        const int64_t big = static_cast<int64_t>(1) << 40;
+        const int64_t lo_g = j >= c_hi ? big : dk <= 0 ? 0 : dk * G;
         const int64_t x = static_cast<int64_t>(p.W) + dk;
-        const int rhi = p.W <= 0 ? kN : x <= 0 ? 0 : x >= kN ? kN : static_cast<int>(x) * G;
+        const int64_t hi_g = p.W <= 0 ? big : x <= 0 ? 0 : x * G;
+        const int rlo = static_cast<int>(min(max(lo_g - r0, static_cast<int64_t>(0)), static_cast<int64_t>(kN)));
+        const int rhi = static_cast<int>(min(max(hi_g - r0, static_cast<int64_t>(0)), static_cast<int64_t>(kN)));
 #pragma unroll
         for (int r = 0; r < kN; ++r)
           if (r < rlo || r >= rhi) sv[r] = __float_as_uint(-INFINITY);
@@ -466,7 +477,7 @@ __global__ void __launch_bounds__(dtc::kThreads, 1)
           const float L = w0 * L0 + w1 * L1;
           const float inv = L > 0.f ? 1.f / L : 0.f;
           const float ov = (w0 * __uint_as_float(o0[e]) + w1 * __uint_as_float(o1[e])) * inv;
-          const int s = r / G, h = kvh * G + (r - s * G);
+          const int s = (r0 + r) / G, h = kvh * G + (r0 + r - s * G);
           const int64_t row = (static_cast<int64_t>(b) * p.n + s) * p.Hq + h;
           p.ws_o[(static_cast<int64_t>(split) * rows_total + row) * kD + d] = ov;
           if (d == r) p.ws_lse[static_cast<int64_t>(split) * rows_total + row] = L > 0.f ? M + __log2f(L) : -INFINITY;
@@ -517,7 +528,10 @@ static bool encode_cache_view128(CUtensorMap* m, const void* ptr, int B, int n, 
 }
 
 bool decode_tc_supported(int n, int Hq, int Hkv, int D, bool cross) {
-  return cross && D == dtc::kD && n * (Hq / Hkv) <= dtc::kN;
+  (void)n;
+  (void)Hq;
+  (void)Hkv;
+  return cross && D == dtc::kD;
 }
 
 // Splits per unit: at least ~2 waves of one CTA per SM, the count whose
@@ -574,7 +588,7 @@ cudaError_t launch_decode_tc(const void* q, const void* kc, const void* vc, cons
     return (e && e[0] == '1') ? 1 : 0;
   }();
   p.stall_first = stall;
-  const int64_t units = static_cast<int64_t>(B) * Hkv;
+  const int64_t units = static_cast<int64_t>(B) * Hkv * ((n * (Hq / Hkv) + dtc::kN - 1) / dtc::kN);
   if (units > 65535 || units < 1) return cudaErrorInvalidValue;
   cudaError_t err = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dtc::kAlloc);
   if (err != cudaSuccess) return err;

@@ -142,9 +142,9 @@ struct DecPlan {
 };
 DecPlan decode_plan(int B, int n, int Lmax, int Hq, int Hkv, bool cross, int sms);
 size_t decode_workspace_bytes(const DecPlan& pl);
-// Cross-stream decode on tcgen05 (decode_tc.cu): n*G <= 32 query rows per KV
-// head, D = 128.  Writes nsplit partials to the split workspace (the same
-// format as the warp-MMA decode kernel).
+// Cross-stream decode on tcgen05 (decode_tc.cu), D = 128: the n*G query rows
+// of a KV head in groups of at most 32.  Writes nsplit partials to the split
+// workspace (the same format as the warp-MMA decode kernel).
 bool decode_tc_supported(int n, int Hq, int Hkv, int D, bool cross);
 int decode_tc_nsplit(int units, int Lmax, int cap, int sms);
 cudaError_t launch_decode_tc(const void* q, const void* kc, const void* vc, const int32_t* ctx, float* ws_o,
