@@ -361,7 +361,8 @@ hd_status hd_attn_fwd_parts(const void* q_loc, const void* const* k_parts,
  *          time need separate flags (and separate k_dst/v_dst).
  * The launch is cooperative (all CTAs resident at once); where the GPU cannot
  * host them together (e.g. shared with other work) the call returns
- * HD_ERR_CUDA and launches nothing.  Ordering across
+ * HD_ERR_CUDA without running the attention (only the flags were zeroed).
+ * Ordering across
  * ranks is the caller's: every shard must be complete before the call runs,
  * and no rank may overwrite its shard before the other ranks' calls that
  * read it have finished (e.g. one barrier collective per layer on `stream`
