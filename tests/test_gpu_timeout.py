@@ -107,15 +107,17 @@ torch.cuda.synchronize()
 print(json.dumps({"status": status, "usable": bool(torch.equal(g, h[:, 1::2]))}))
 """
 
-CHILDREN = {"bwd": CHILD_BWD, "dec": CHILD_DEC, "gather": CHILD_GATHER}
+CHILDREN = {"bwd": CHILD_BWD, "dec": CHILD_DEC, "dec_intra": CHILD_DEC.replace('"cross"', '"intra"'),
+            "gather": CHILD_GATHER}
 
 
 @pytest.mark.parametrize("var,child", [("HD_TEST_STALL_BWD", "bwd"), ("HD_TEST_STALL_DECODE", "dec"),
-                                       ("HD_TEST_STALL_GATHER", "gather")])
+                                       ("HD_TEST_STALL_DECODE", "dec_intra"), ("HD_TEST_STALL_GATHER", "gather")])
 def test_backward_decode_and_gather_waits_time_out_cleanly(var, child):
     """The same bounded-wait path in the dK/dV backward kernel (its MMA warp of
-    CTA 0 never signals S), in the decode kernel (the producer of its first
-    CTA issues no loads), and in the fused peer-gather attention (CTA 0 never
+    CTA 0 never signals S), in both decode kernels (cross mode: the tcgen05
+    kernel; intra mode: the warp-MMA kernel; the producer of the first CTA
+    issues no loads), and in the fused peer-gather attention (CTA 0 never
     publishes its first copied piece, so the first key tile never becomes
     ready for any CTA)."""
     env = dict(os.environ, **{var: "1"})
