@@ -298,3 +298,29 @@ def test_parts_at_full_size_sampled_rows(hd):
                                      [(0, 0, p) for p in pos])
             worst = max(worst, float(np.max(np.abs(to_f64(o[b, rows_loc, h]) - ro))))
     assert worst <= TOL_BF16, worst
+
+
+@pytest.mark.parametrize("in_dt,out_dt,R", [("f32", "f32", 2), ("bf16", "bf16", 4), ("f32", "bf16", 8),
+                                            ("bf16", "f32", 2)])
+def test_combine_streams_kernel(hd, in_dt, out_dt, R):
+    """The own-rows merge on random partials (some parts and some rows empty),
+    each part through its own pointer, against the oracle's merge."""
+    B, n, Hq, D = 3, 8, 5, 64
+    o = [synth.normal((B, n, Hq, D), 1601 + i, dtype=in_dt) for i in range(R)]
+    lse = [synth.normal((B, n, Hq), 1611 + i).astype(np.float32) * 3 for i in range(R)]
+    lse[0][0, :, :2] = -np.inf          # empty parts
+    for i in range(R):
+        lse[i][1, 3, 4] = -np.inf       # a row with every part empty
+    wo, wl = oracle.combine_partials(np.stack(o), np.stack(lse))
+    tol = TOL_BF16 if out_dt == "bf16" else TOL_F32
+    for r in range(R):
+        go, gl = hd.hd_attn_combine_streams([dev(x, in_dt) for x in o], [dev(x, "f32") for x in lse], n, R, r,
+                                            out_dtype=torch.bfloat16 if out_dt == "bf16" else torch.float32,
+                                            lse=True)
+        torch.cuda.synchronize()
+        assert max_abs(to_f64(go), wo[:, r::R]) <= tol
+        gl = to_f64(gl)
+        want = wl[:, r::R]
+        assert np.array_equal(np.isneginf(gl), np.isneginf(want))
+        fin = np.isfinite(want)
+        assert max_abs(gl[fin], want[fin]) <= 1e-5
