@@ -931,7 +931,9 @@ def main():
             print(json.dumps(out), flush=True)
         return
     if rank == 0:
-        if not args.no_extras and args.workload != "decode":
+        # The side measurements are single-GPU figures (the N = 1 run reports
+        # them); with several ranks they would only hold the other GPUs idle.
+        if not args.no_extras and args.workload != "decode" and world == 1:
             out["also"] = extras(torch, peaks, rank)
         v, unit, sample, threads = oracle_sample_rate(args.workload, 15.0)
         out["cpu_baseline"] = {"value": v, "unit": unit, "cores": threads, "kind": "oracle", "sample": sample}
