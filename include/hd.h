@@ -337,7 +337,9 @@ hd_status hd_attn_combine_streams(const void* const* o_parts, const float* const
  *       global stream rho + R*l (e.g. the R slots of an all-gather).
  *
  * A 128-key tile of the expanded order is 128/R consecutive rows of every
- * shard, so the kernel reads the shards where they lie.  bf16 input only;
+ * shard, so the kernel reads the shards where they lie (fastest when they
+ * lie at one stride, e.g. one [R, ...] tensor: then a key tile is one TMA box
+ * per 64 features instead of one per rank).  bf16 input only;
  * 1 <= R <= HD_MAX_RANKS, R divides n, n divides 128.  Other arguments and
  * errors as hd_attn_fwd_shard.  The shards are read many times: they belong
  * in this GPU's memory (for peers' memory use hd_attn_fwd_peer_gather).
@@ -355,7 +357,11 @@ hd_status hd_attn_fwd_parts(const void* q_loc, const void* const* k_parts,
  * a warp in every CTA copies each of them once into k_dst[rho], v_dst[rho]
  * (this GPU, same shape), in key-tile order, while the attention runs; each
  * key tile is read only after its own pieces have landed.  k_src[r],
- * v_src[r] are this rank's shard, read in place (k_dst[r], v_dst[r] unused).
+ * v_src[r] are this rank's shard: read in place when k_dst[r] or v_dst[r]
+ * is NULL, else copied there as well.  When the R slots the attention reads
+ * lie at one stride in memory (e.g. k_dst/v_dst are the R slots of one
+ * [R, B, (n/R)*L, Hkv, D] tensor, own slot included), each key tile is one
+ * TMA box per 64 features instead of one per rank.
  *   flags  device workspace of hd_attn_peer_flags_bytes(B, L, n) bytes,
  *          zeroed by the call on `stream`; calls that may run at the same
  *          time need separate flags (and separate k_dst/v_dst).

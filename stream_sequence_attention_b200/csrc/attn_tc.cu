@@ -197,11 +197,16 @@ __device__ __forceinline__ bool flag_wait_ge(const unsigned long long* f, unsign
 // mask needs perm.
 struct PartsInfo {
   int R, rows, self;
+  // The R shards lie at one stride in memory (kv.k[0]/kv.v[0] then view them
+  // as one 5-D tensor (D, H, rows, B, R): a tile is one box per 64 features).
+  int stacked;
   uint8_t perm[tc::BN];
-  // In-kernel gather (flags != nullptr): rank rho's shard (rho != self) is
-  // copied from src to dst in items of up to kPeerSub16 16-byte units,
-  // ordered key tile first; flags[b*nkt + kt] counts the finished items of
-  // key tile kt of sequence b, complete at per_flag.
+  // In-kernel gather (flags != nullptr): the shards of ngath ranks (the
+  // others, and this rank's own when gself) are copied from src to dst in
+  // items of up to kPeerSub16 16-byte units, ordered key tile first;
+  // flags[b*nkt + kt] counts the finished items of key tile kt of sequence
+  // b, complete at per_flag.
+  int ngath, gself;
   const uint4* src_k[kPeerMaxRanks];
   const uint4* src_v[kPeerMaxRanks];
   uint4* dst_k[kPeerMaxRanks];
@@ -236,11 +241,11 @@ __device__ __forceinline__ void gather_items(const PartsInfo& x, int B, int lane
     rem /= x.nsub;
     const int kind = rem & 1;
     rem >>= 1;
-    const int rr = rem % (x.R - 1);
-    rem /= x.R - 1;
+    const int rr = rem % x.ngath;
+    rem /= x.ngath;
     const int b = rem % B;
     const int kt = rem / B;
-    const int rho = rr < x.self ? rr : rr + 1;
+    const int rho = x.gself ? rr : (rr < x.self ? rr : rr + 1);
     const int64_t r0 = static_cast<int64_t>(kt) * x.rows;
     const int64_t r1 = min(r0 + x.rows, x.shard_rows);
     const int64_t n16 = (r1 - r0) * x.row16;
@@ -312,7 +317,7 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
 #pragma unroll
     for (int i = 0; i < NM; ++i) {
       if constexpr (kParts) {
-        if (i >= kv.x.R) break;
+        if (i >= (kv.x.stacked ? 1 : kv.x.R)) break;
       }
       tma_prefetch_desc(&kv.k[i]);
       tma_prefetch_desc(&kv.v[i]);
@@ -334,13 +339,20 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
   // One 128-key tile of K or V into the stage at `dst`.
   auto load_kv_tile = [&](const CUtensorMap* maps, uint32_t dst, uint32_t full, const TcUnit& x, int skv, int kt) {
     if constexpr (kParts) {
-#pragma unroll
-      for (int rho = 0; rho < NM; ++rho) {
-        if (rho >= kv.x.R) break;
+      if (kv.x.stacked) {
+        // One box covers the tile's rows of every rank, rank-major.
 #pragma unroll
         for (int kb = 0; kb < Lay::KB; ++kb)
-          tma_load_5d(dst + kb * Lay::BLK + rho * kv.x.rows * 128, &maps[rho], full, kb * 64, x.kvh, 0,
-                      kt * kv.x.rows, x.b);
+          tma_load_5d(dst + kb * Lay::BLK, &maps[0], full, kb * 64, x.kvh, kt * kv.x.rows, x.b, 0);
+      } else {
+#pragma unroll
+        for (int rho = 0; rho < NM; ++rho) {
+          if (rho >= kv.x.R) break;
+#pragma unroll
+          for (int kb = 0; kb < Lay::KB; ++kb)
+            tma_load_5d(dst + kb * Lay::BLK + rho * kv.x.rows * 128, &maps[rho], full, kb * 64, x.kvh, 0,
+                        kt * kv.x.rows, x.b);
+        }
       }
     } else {
 #pragma unroll
@@ -703,6 +715,49 @@ bool encode_stream_view(CUtensorMap* m, const void* ptr, int B, int Ls, int ns, 
   return tmap_cached(k, m, make_stream_view);
 }
 
+// R rank shards [B, rows, H, D] at a stride of `step` bytes, viewed as the 5-D
+// tensor (D, H, rows, B, R) with a box of 64 x 1 x box_rows x 1 x R.
+static bool make_stacked_view(const TmapKey& k, CUtensorMap* m) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) return false;
+  const cuuint64_t B = k.dims[0], rows = k.dims[1], R = k.dims[2], H = k.dims[3], D = k.dims[4];
+  const cuuint64_t e = 2;
+  const cuuint64_t dims[5] = {D, H, rows, B, R};
+  const cuuint64_t strides[4] = {D * e, H * D * e, rows * H * D * e, static_cast<cuuint64_t>(k.extra)};
+  const cuuint32_t box[5] = {64, 1, static_cast<cuuint32_t>(k.pad), 1, static_cast<cuuint32_t>(R)};
+  const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(k.ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static bool encode_stacked_view(CUtensorMap* m, const void* ptr, int B, int64_t rows, int R, int H, int D,
+                                int box_rows, int64_t step) {
+  TmapKey k;
+  std::memset(&k, 0, sizeof(k));
+  k.ptr = ptr;
+  k.dims[0] = B;
+  k.dims[1] = rows;
+  k.dims[2] = R;
+  k.dims[3] = H;
+  k.dims[4] = D;
+  k.kind = 5;
+  k.pad = box_rows;
+  k.extra = step;
+  return tmap_cached(k, m, make_stacked_view);
+}
+
+// Stride of R addresses in arithmetic progression (a positive multiple of 16
+// bytes, at least `min_step`), or 0.
+static int64_t stack_step(const void* const* a, int R, int64_t min_step) {
+  if (R < 2) return 0;
+  const int64_t d = reinterpret_cast<intptr_t>(a[1]) - reinterpret_cast<intptr_t>(a[0]);
+  if (d < min_step || d % 16 || d >= (static_cast<int64_t>(1) << 40)) return 0;
+  for (int i = 2; i < R; ++i)
+    if (reinterpret_cast<intptr_t>(a[i]) - reinterpret_cast<intptr_t>(a[i - 1]) != d) return 0;
+  return d;
+}
+
 // One rank shard [B, rows, H, D] with a box of `box_rows` rows.
 static bool encode_shard_view(CUtensorMap* m, const void* ptr, int B, int64_t rows, int H, int D, int box_rows) {
   TmapKey k;
@@ -807,26 +862,42 @@ cudaError_t launch_attn_tc_parts(const void* q, const PartsArgs& a, void* o, flo
   const int rows = tc::BN / R;
   const int64_t shard_rows = static_cast<int64_t>(nl) * L;
   const bool gather = R > 1 && a.k_dst[0 == a.self ? 1 : 0] != nullptr;
+  const bool gself = gather && a.k_dst[a.self] != nullptr && a.v_dst[a.self] != nullptr;
   CUtensorMap mq;
   if (!encode_stream_view(&mq, q, g.B, g.Lq, g.q_ns, Hq, D)) return cudaErrorInvalidValue;
   KvSrc<kPeerMaxRanks> kv;
   std::memset(&kv, 0, sizeof(kv));
   PartsInfo& x = kv.x;
+  // The shards the attention reads: the copies where the kernel gathers them.
+  const void* rk[kPeerMaxRanks];
+  const void* rv[kPeerMaxRanks];
   for (int rho = 0; rho < R; ++rho) {
-    const bool copied = gather && rho != a.self;
-    const void* ks = copied ? a.k_dst[rho] : a.k_src[rho];
-    const void* vs = copied ? a.v_dst[rho] : a.v_src[rho];
-    if (!encode_shard_view(&kv.k[rho], ks, g.B, shard_rows, Hkv, D, rows) ||
-        !encode_shard_view(&kv.v[rho], vs, g.B, shard_rows, Hkv, D, rows))
-      return cudaErrorInvalidValue;
+    const bool copied = gather && (rho != a.self || gself);
+    rk[rho] = copied ? a.k_dst[rho] : a.k_src[rho];
+    rv[rho] = copied ? a.v_dst[rho] : a.v_src[rho];
     x.src_k[rho] = static_cast<const uint4*>(a.k_src[rho]);
     x.src_v[rho] = static_cast<const uint4*>(a.v_src[rho]);
     x.dst_k[rho] = static_cast<uint4*>(a.k_dst[rho]);
     x.dst_v[rho] = static_cast<uint4*>(a.v_dst[rho]);
   }
+  const int64_t shard_bytes = static_cast<int64_t>(g.B) * shard_rows * Hkv * D * 2;
+  const int64_t sk = stack_step(rk, R, shard_bytes), sv = stack_step(rv, R, shard_bytes);
+  x.stacked = sk > 0 && sv > 0;
+  if (x.stacked) {
+    if (!encode_stacked_view(&kv.k[0], rk[0], g.B, shard_rows, R, Hkv, D, rows, sk) ||
+        !encode_stacked_view(&kv.v[0], rv[0], g.B, shard_rows, R, Hkv, D, rows, sv))
+      return cudaErrorInvalidValue;
+  } else {
+    for (int rho = 0; rho < R; ++rho)
+      if (!encode_shard_view(&kv.k[rho], rk[rho], g.B, shard_rows, Hkv, D, rows) ||
+          !encode_shard_view(&kv.v[rho], rv[rho], g.B, shard_rows, Hkv, D, rows))
+        return cudaErrorInvalidValue;
+  }
   x.R = R;
   x.rows = rows;
   x.self = a.self;
+  x.ngath = gather ? (gself ? R : R - 1) : 0;
+  x.gself = gself ? 1 : 0;
   for (int c = 0; c < tc::BN; ++c) {
     const int rho = c / rows, t = c % rows;
     x.perm[c] = static_cast<uint8_t>((t / nl) * n + rho + R * (t % nl));
@@ -837,8 +908,8 @@ cudaError_t launch_attn_tc_parts(const void* q, const PartsArgs& a, void* o, flo
   const int64_t tile16 = static_cast<int64_t>(rows) * x.row16;
   x.nsub = static_cast<int>((tile16 + kPeerSub16 - 1) / kPeerSub16);
   x.flags = gather ? a.flags : nullptr;
-  x.per_flag = static_cast<unsigned long long>(2 * (R - 1)) * x.nsub;
-  const int64_t items = gather ? static_cast<int64_t>(x.nkt) * g.B * (R - 1) * 2 * x.nsub : 0;
+  x.per_flag = static_cast<unsigned long long>(2 * x.ngath) * x.nsub;
+  const int64_t items = gather ? static_cast<int64_t>(x.nkt) * g.B * x.ngath * 2 * x.nsub : 0;
   if (items > 0x7fffffff) return cudaErrorInvalidValue;
   x.nitems = static_cast<int>(items);
   static const int stall = [] {

@@ -385,7 +385,15 @@ hd_status hd_attn_fwd_peer_gather(const void* q_loc, const void* const* k_src, c
         flags_bytes < hd_attn_peer_flags_bytes(B, L, n))
       return HD_ERR_INVALID_ARG;
     for (int rho = 0; rho < R; ++rho) {
-      if (rho == r) continue;
+      if (rho == r) {
+        // Optional: given both, the own shard is copied there too.
+        if (k_dst[rho] && v_dst[rho]) {
+          if (!aligned16(k_dst[rho]) || !aligned16(v_dst[rho])) return HD_ERR_INVALID_ARG;
+          pa.k_dst[rho] = k_dst[rho];
+          pa.v_dst[rho] = v_dst[rho];
+        }
+        continue;
+      }
       if (!k_dst[rho] || !v_dst[rho] || !aligned16(k_dst[rho]) || !aligned16(v_dst[rho])) return HD_ERR_INVALID_ARG;
       pa.k_dst[rho] = k_dst[rho];
       pa.v_dst[rho] = v_dst[rho];

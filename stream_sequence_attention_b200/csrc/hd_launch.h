@@ -46,6 +46,7 @@ struct TmapKey {
   int64_t dims[5];
   int32_t kind;
   int32_t pad;
+  int64_t extra;  // kind-specific (the rank stride of a stacked shard view)
 };
 bool tmap_cached(const TmapKey& key, CUtensorMap* out, bool (*make)(const TmapKey&, CUtensorMap*));
 
@@ -74,8 +75,8 @@ struct PartsArgs {
   int R, self;
   const void* k_src[kPeerMaxRanks];
   const void* v_src[kPeerMaxRanks];
-  void* k_dst[kPeerMaxRanks];  // all nullptr: no gather
-  void* v_dst[kPeerMaxRanks];
+  void* k_dst[kPeerMaxRanks];  // all nullptr: no gather; [self] optional (then
+  void* v_dst[kPeerMaxRanks];  // the own shard is copied there as well)
   unsigned long long* flags;   // [B * key tiles], zeroed by the launcher
 };
 int64_t parts_flag_count(int B, int n, int L);

@@ -128,20 +128,34 @@ def test_rank_shard_prefill(hd, seed):
     v = synth.normal((B, P, Hkv, D), seed + 2, dtype="bf16")
     ro, _ = oracle.attn(q, k, v, n, "cross", W)
     want = _shard(ro, n, R, r)
-    ks = [dev(_shard(k, n, R, rho), "bf16") for rho in range(R)]
-    vs = [dev(_shard(v, n, R, rho), "bf16") for rho in range(R)]
+    # Shards either as the slots of one [R, ...] tensor (one stride: the
+    # stacked view) or as separate tensors with gaps between them.
+    stacked = bool(g.random() < 0.5)
+    if stacked:
+        kstk = dev(np.stack([_shard(k, n, R, rho) for rho in range(R)]), "bf16")
+        vstk = dev(np.stack([_shard(v, n, R, rho) for rho in range(R)]), "bf16")
+        ks, vs = list(kstk), list(vstk)
+    else:
+        ks, vs, gaps = [], [], []
+        for rho in range(R):
+            ks.append(dev(_shard(k, n, R, rho), "bf16"))
+            gaps.append(torch.empty(4096 * (rho + 1), dtype=torch.uint8, device="cuda"))
+            vs.append(dev(_shard(v, n, R, rho), "bf16"))
     ql = dev(_shard(q, n, R, r), "bf16")
     st = hd.new_status()
     o1 = hd.hd_attn_fwd_parts(ql, ks, vs, n, R, r, W, out_dtype=torch.float32, dev_status=st)
-    kd = [torch.zeros_like(ks[0]) for _ in range(R)]
-    vd = [torch.zeros_like(vs[0]) for _ in range(R)]
+    own_slot = bool(g.random() < 0.7)
+    kdt = torch.zeros((R,) + tuple(ks[0].shape), dtype=torch.bfloat16, device="cuda")
+    vdt = torch.zeros_like(kdt)
+    kd = [None if (rho == r and not own_slot) else kdt[rho] for rho in range(R)]
+    vd = [None if (rho == r and not own_slot) else vdt[rho] for rho in range(R)]
     o2 = hd.hd_attn_fwd_peer_gather(ql, ks, vs, kd, vd, n, R, r, window=W, out_dtype=torch.float32, dev_status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
-    case = (n, R, r, L, Hq, Hkv, D, W)
+    case = (n, R, r, L, Hq, Hkv, D, W, stacked, own_slot)
     assert max_abs(to_f64(o1), want) <= TOL_BF16, case
     assert max_abs(to_f64(o2), want) <= TOL_BF16, case
     for rho in range(R):
-        if rho != r:
+        if R > 1 and (rho != r or own_slot):
             assert torch.equal(kd[rho].view(torch.int16), ks[rho].view(torch.int16)), case
             assert torch.equal(vd[rho].view(torch.int16), vs[rho].view(torch.int16)), case

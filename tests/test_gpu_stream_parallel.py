@@ -254,12 +254,18 @@ def test_peer_gather_copies_and_attends(hd, n, R, L, Hq, Hkv, D, W):
             torch.cuda.synchronize()
             assert int(st.item()) == 0
             assert max_abs(to_f64(o), _shard(ro, n, R, r)) <= TOL_BF16
-            for rho in range(R):
-                if rho == r:
-                    assert bool((kd[rho] == 7.0).all()) and bool((vd[rho] == 7.0).all())  # own slot untouched
-                else:
+            for rho in range(R):  # every slot given: the own shard is copied as well
+                if R > 1:
                     assert torch.equal(kd[rho].view(torch.int16), ks[rho].view(torch.int16))
                     assert torch.equal(vd[rho].view(torch.int16), vs[rho].view(torch.int16))
+            if R > 1:  # own slot not given: the own shard is read in place
+                kd2 = [None if rho == r else torch.full_like(ks[0], 7.0) for rho in range(R)]
+                vd2 = [None if rho == r else torch.full_like(vs[0], 7.0) for rho in range(R)]
+                o2 = hd.hd_attn_fwd_peer_gather(dev(_shard(q, n, R, r), "bf16"), ks, vs, kd2, vd2, n, R, r,
+                                                window=W, out_dtype=torch.float32, dev_status=st)
+                torch.cuda.synchronize()
+                assert int(st.item()) == 0
+                assert max_abs(to_f64(o2), _shard(ro, n, R, r)) <= TOL_BF16
 
 
 def test_parts_at_full_size_sampled_rows(hd):
