@@ -117,7 +117,9 @@ class PeerShards:
     Each rank owns ``buffers`` pairs (K, V) of [B, (n/R)*L, Hkv, D] that the
     other ranks map; a layer writes its shard into the next pair (``stage``),
     all ranks pass a barrier (``fence``), and the kernel pulls the peers'
-    shards over NVLink into local slots while it computes (``attend``).  With
+    shards over NVLink into local slots while it computes (``attend``); its
+    own shard is copied into its slot too, so that the R local slots (one
+    [R, ...] tensor) are read with one TMA box per 64 features.  With
     two pairs used in turn, one barrier per layer also keeps a rank from
     overwriting a pair before the peers' kernels that read it have finished:
     a rank passes the next barrier only after its previous kernel.
