@@ -660,7 +660,10 @@ def hd_attn_fwd_peer_gather(q_loc: torch.Tensor, k_src, v_src, k_dst, v_dst, n: 
     """hd_attn_fwd_parts with the exchange inside the kernel: k_src/v_src are
     R shards (entry r a local tensor; the others tensors or peer device
     addresses from :func:`hd_ipc_open`), copied once into the local k_dst/
-    v_dst shards (entry r unused) while the attention runs."""
+    v_dst shards while the attention runs.  Entry r of k_dst/v_dst may be
+    None (this rank's shard is then read in place) or a slot (the shard is
+    copied too; when all R slots lie at one stride, as the slots of one
+    [R, ...] tensor do, a key tile is one TMA box per 64 features)."""
     if not isinstance(k_src[r], torch.Tensor) or not isinstance(v_src[r], torch.Tensor):
         raise TypeError("k_src[r] and v_src[r] must be this rank's local shard tensors")
     Hkv = k_src[r].shape[-2]
