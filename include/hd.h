@@ -12,10 +12,14 @@
  *    position p = i*n + s of the expanded sequence (the page's t = (i-1)n + k).
  *    The final stream is s = n-1.
  *  - All tensors are dense, row-major (last index fastest), on the current
- *    CUDA device, owned by the caller.  Base pointers must be 16-byte aligned.
- *  - The library allocates no device memory (the decode workspace is passed
- *    in) and never synchronises: every call is enqueued on `stream` (a
- *    cudaStream_t; NULL = legacy default stream) and returns at once.
+ *    CUDA device, owned by the caller.  Base pointers must be 16-byte aligned
+ *    (int32 token ids: 4-byte aligned).
+ *  - The library allocates no device memory and never synchronises: every
+ *    call is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and returns at once.  Scratch memory is passed in by the caller
+ *    (the decode and backward workspaces), except for
+ *    hd_attn_decode_noalloc, which uses a fixed scratch array that is part
+ *    of the library's own device image (see that call).
  *  - Host-side argument errors return a status synchronously and launch
  *    nothing.  Problems found on the device (a token id out of range, a
  *    pipeline wait that ran out of time) are written to `*dev_status` (a
@@ -54,7 +58,7 @@ typedef enum {
  * eq. S_t = E_k(x_i)):   out[b, i*n + s, :] = tables[s, ids[b, i], :]
  *
  *   tables  [n, V, d]   element type `dt`
- *   ids     [B, L]      int32, each in [0, V)
+ *   ids     [B, L]      int32, each in [0, V); 4-byte aligned
  *   out     [B, n*L, d] element type `dt`
  * d*sizeof(dt) must be a multiple of 16 bytes.  A row whose id is out of
  * range is written as zeros and HD_ERR_BAD_TOKEN is recorded in *dev_status.
@@ -220,7 +224,10 @@ size_t hd_attn_decode_workspace(int B, int n, int Lmax, int Hq, int Hkv, int D,
  *    exceeds HD_DECODE_NOALLOC_SCRATCH_BYTES return HD_ERR_UNSUPPORTED and
  *    launch nothing; use hd_attn_decode with a workspace for those.
  *  - The first call on a device looks up the scratch's device address for
- *    that device; make that first call before any stream capture.
+ *    that device; make that first call before any stream capture.  The
+ *    address is kept for the life of the process: the call assumes each
+ *    device keeps one primary context throughout (no cudaDeviceReset
+ *    between calls, which would leave the kept address stale).
  *  - All calls share the one scratch array.  Calls whose kernels can overlap
  *    on the GPU (different streams with no ordering between them) race on it
  *    and give wrong results; order them on one stream or with events.

@@ -59,7 +59,9 @@ hd_status hd_expand_embed(const void* tables, const int32_t* ids, void* out, int
   if (row_bytes % 16 || row_bytes > (1 << 30)) return HD_ERR_INVALID_ARG;
   const int64_t rows = static_cast<int64_t>(B) * L * n;
   if (rows == 0) return HD_OK;
-  if (!tables || !ids || !out || !aligned16(tables) || !aligned16(out) || !aligned16(ids))
+  // The kernel reads ids one int32 at a time: 4-byte alignment suffices
+  // (a view such as ids[:, 1:] is accepted).
+  if (!tables || !ids || !out || !aligned16(tables) || !aligned16(out) || (reinterpret_cast<uintptr_t>(ids) & 3u))
     return HD_ERR_INVALID_ARG;
   const int sms = sm_count();
   if (sms <= 0) return HD_ERR_CUDA;

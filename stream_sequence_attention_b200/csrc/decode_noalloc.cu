@@ -12,7 +12,10 @@
 // (every GPU that loads the library keeps it until the process exits).  Its
 // device address is looked up once per device with cudaGetSymbolAddress, with
 // that device current, the first time the entry point runs on it; that first
-// call should therefore be made before any stream capture begins.  Every call
+// call should therefore be made before any stream capture begins.  The address
+// is kept for the life of the process, which assumes the device keeps one
+// primary context throughout (a cudaDeviceReset between calls would leave the
+// kept address stale).  Every call
 // shares the one array: two calls whose kernels overlap on the GPU (different
 // streams, no ordering between them) race on it.  Nothing in it needs to start
 // at zero: each call writes every partial it later reads.

@@ -267,17 +267,22 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe for finite x <= 2^22: x = n + f, n = rint(x),
-// f in [-1/2, 1/2]; cubic for 2^f (coefficients from csrc/fit_exp2_poly.py);
-// 2^n by adding n to the exponent field.  Inputs below -127 are clamped.
+// 2^x on the FMA pipe for x <= 2^22: x = n + f, n = rint(x), f in
+// [-1/2, 1/2]; cubic for 2^f (coefficients from csrc/fit_exp2_poly.py); 2^n
+// by adding n to the exponent field.  The cubic can come out just below 1
+// (biased exponent 126), so n must stay >= -126 or the exponent add borrows
+// into the sign bit: inputs are clamped to -126, and every x < -126
+// (-inf included) returns 0, as the flush-to-zero MUFU form does.
 __device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -127.0f);
+  const bool under = x < -126.0f;
+  x = fmaxf(x, -126.0f);
   const float t = x + 12582912.0f;  // 1.5 * 2^23: rint(x) lands in the low mantissa bits
   const float f = x - (t - 12582912.0f);
   float p = fmaf(0.0551713444f, f, 0.242610335f);
   p = fmaf(p, f, 0.693260968f);
   p = fmaf(p, f, 0.999928117f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+  const float r = __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+  return under ? 0.0f : r;
 }
 
 // Per-warpgroup register re-allocation (all four warps of a warpgroup must

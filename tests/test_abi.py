@@ -61,6 +61,9 @@ def test_bad_arguments_rejected_on_host(L):
     fake = vp(0x10000)  # never dereferenced: every call below fails validation first
     # n = 0
     assert L.hd_expand_embed(fake, fake, fake, 1, 4, 0, 10, 8, hd.HD_BF16, None, None) == hd.HD_ERR_INVALID_ARG
+    # ids not int32-aligned (a 4-byte offset is allowed; 2 bytes is not)
+    assert L.hd_expand_embed(fake, vp(0x10002), fake, 1, 4, 2, 10, 8, hd.HD_BF16, None, None) \
+        == hd.HD_ERR_INVALID_ARG
     # row bytes not a multiple of 16 (d = 4 bf16)
     assert L.hd_expand_embed(fake, fake, fake, 1, 4, 2, 10, 4, hd.HD_BF16, None, None) == hd.HD_ERR_INVALID_ARG
     # Hq % Hkv != 0

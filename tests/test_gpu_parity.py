@@ -39,6 +39,22 @@ def test_expand_bit_exact(hd, dtype, n, B, L, V, d):
     assert int(st.item()) == 0
 
 
+def test_expand_ids_at_a_four_byte_offset(hd):
+    """ids need only int32 alignment: a view starting one token in (ids[:, 1:]
+    of one sequence) is accepted and expands bit-exactly."""
+    n, V, d = 3, 50, 64
+    tables = synth.normal((n, V, d), 35, std=0.02, dtype="bf16")
+    ids = synth.ids_uniform(1, 41, V, 36)
+    ids_d = dev(ids, "i32")[:, 1:]
+    assert ids_d.is_contiguous() and ids_d.data_ptr() % 16 == 4
+    st = hd.new_status()
+    out = hd.hd_expand_embed(dev(tables, "bf16"), ids_d, dev_status=st)
+    torch.cuda.synchronize()
+    ref = oracle.expand(tables, ids[:, 1:])
+    assert np.array_equal(out.float().cpu().numpy().view(np.uint32), ref.astype(np.float32).view(np.uint32))
+    assert int(st.item()) == 0
+
+
 def test_expand_bad_token_zero_row_and_status(hd):
     n, V, d = 2, 16, 64
     tables = synth.normal((n, V, d), 33, std=0.02, dtype="bf16")

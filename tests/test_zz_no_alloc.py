@@ -3,9 +3,11 @@ callers that cannot give the library device memory.
 
 Run last (file name) so a stop-at-first-failure run has covered everything
 else first; it also passes alone in a fresh process.  The new entry point is
-called through the C ABI twice in a row and checked against hd_attn_decode
-(caller-provided workspace) within the bf16 parity bound of the other tests;
-sizes needing more scratch than the fixed maximum are refused on the host.
+called through the C ABI twice in a row.  It runs the same kernels on the
+same work plan as hd_attn_decode (caller-provided workspace), only with
+another scratch address, so both results must be bit-identical; they are
+also checked against the float64 oracle within the bf16 parity bound.  Sizes
+needing more scratch than the fixed maximum are refused on the host.
 """
 
 import ctypes
@@ -14,8 +16,9 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from stream_sequence_attention_b200 import synth
-from tests.gpu_util import TOL_BF16, lib
+from tests.gpu_util import TOL_BF16, lib, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -44,6 +47,7 @@ def test_noalloc_matches_workspace_decode_twice(mode, window):
     vc = synth.normal_device((B, n, Lmax, Hkv, D), 503)
     ctx = torch.tensor([1000, 1, 517, 64], dtype=torch.int32, device="cuda")
     ref, ref_lse = hd.hd_attn_decode(q, kc, vc, ctx, mode, window, out_dtype=torch.float32, lse=True)
+    oo, ol = oracle.decode(to_f64(q), to_f64(kc), to_f64(vc), ctx.cpu().numpy(), n, mode, window)
     for call in range(2):
         o = torch.full((B, n, Hq, D), float("nan"), dtype=torch.float32, device="cuda")
         lse = torch.full((B, n, Hq), float("nan"), dtype=torch.float32, device="cuda")
@@ -51,8 +55,11 @@ def test_noalloc_matches_workspace_decode_twice(mode, window):
         torch.cuda.synchronize()
         assert code == hd.HD_OK, hd.status_string(code)
         assert int(st.item()) == 0
-        assert float((o - ref).abs().max()) <= TOL_BF16, call
-        assert float((lse - ref_lse).abs().max()) <= 1e-3, call
+        # same kernels, same plan, same summation order: bit-identical
+        assert torch.equal(o, ref), call
+        assert torch.equal(lse, ref_lse), call
+        assert float(np.abs(to_f64(o) - oo).max()) <= TOL_BF16, call
+        assert float(np.abs(to_f64(lse) - ol).max()) <= 1e-3, call
 
 
 def test_noalloc_refuses_sizes_beyond_the_scratch():
@@ -83,4 +90,4 @@ def test_noalloc_after_other_work_on_the_device():
             o = hd.hd_attn_decode_noalloc(q, kc, vc, ctx, mode, out_dtype=torch.float32)
             torch.cuda.synchronize()
             assert np.isfinite(o.cpu().numpy()).all()
-            assert float((o - ref).abs().max()) <= TOL_BF16
+            assert torch.equal(o, ref)
