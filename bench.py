@@ -652,8 +652,10 @@ def run_ours(args, rank, world, dist):
 
 
 def extras(torch, peaks, rank):
-    """Side measurements on one GPU: decode GB/s (both modes) and the
-    cross-stream prefill layer."""
+    """Side measurements on one GPU: decode GB/s (both modes), the
+    cross-stream prefill layer, the KV-mirror layer, the long-context
+    workload (expand, windowed intra attention, gather), RoPE, rank 0's
+    stream-parallel share and the backward."""
     from stream_sequence_attention_b200 import hd, synth
 
     res = {}
@@ -697,6 +699,53 @@ def extras(torch, peaks, rank):
     res["mirror_final_stream_cross"] = {"ms": round(ms, 3), "TFLOP/s": round(tf, 1),
                                         "frac_bf16": round(tf / peaks["bf16"], 4)}
     del mi
+    torch.cuda.empty_cache()
+    # Long-context workload: expand over 4 tables of 152064 x 4096 with
+    # Zipf(1.1) ids -> intra-stream attention with a 4096-token window ->
+    # final-stream gather, n=4 L=32768 B=1 64q/8kv D=128; each part timed.
+    from stream_sequence_attention_b200 import accounting as acc
+    lc = Prefill(WORKLOADS["long"], 7601 + rank, torch, hd, synth)
+    c = WORKLOADS["long"]
+    ms_e = time_fn(lambda: hd.hd_expand_embed(lc.tables, lc.ids, lc.x, dev_status=lc.status))
+    ms_a = time_fn(lambda: hd.hd_attn_fwd(lc.q, lc.k, lc.v, c["n"], c["mode"], c["W"], out=lc.o,
+                                          dev_status=lc.status))
+    ms_g = time_fn(lambda: hd.hd_final_stream_gather(lc.x, c["n"], out=lc.g))
+    torch.cuda.synchronize()
+    if int(lc.status.item()) != 0:
+        raise RuntimeError(f"device status {hd.status_string(int(lc.status.item()))}")
+    tf = lc.flops() / (ms_a * 1e-3) / 1e12
+    eb = acc.expand_bytes(c["B"], c["L"], c["n"], c["dm"])
+    gb = acc.gather_bytes(c["B"], c["L"], c["dm"])
+    res["long_context"] = {
+        "workload": NAMES["long"] + ", expand 4 x 152064 x 4096 Zipf(1.1) ids, final-stream gather",
+        "attn_ms": round(ms_a, 3), "attn_TFLOP/s": round(tf, 1), "attn_frac_bf16": round(tf / peaks["bf16"], 4),
+        "expand_ms": round(ms_e, 4), "expand_GB/s": round(eb / (ms_e * 1e-3) / 1e9, 1),
+        "expand_unique_rows_per_table": int(torch.unique(lc.ids).numel()), "expand_rows_per_table": c["B"] * c["L"],
+        "gather_ms": round(ms_g, 4), "gather_GB/s": round(gb / (ms_g * 1e-3) / 1e9, 1),
+        "gather_frac_hbm": round(gb / (ms_g * 1e-3) / 1e9 / peaks["hbm"], 4),
+        "step_ms": round(ms_e + ms_a + ms_g, 3),
+        "repeats": 10, "l2": "flushed before each timed launch"}
+    del lc
+    torch.cuda.empty_cache()
+    # RoPE fused into the attention (intra workload): hd_rope on q and k then
+    # hd_attn_fwd, against hd_attn_fwd_rope (k rotated in place, q rotated
+    # inside the attention kernel).  Repeated rotation of the same buffers
+    # changes the values, not the work.
+    c = WORKLOADS["intra"]
+    B, P = c["B"], c["n"] * c["L"]
+    rq = synth.normal_device((B, P, c["Hq"], c["D"]), 7701 + rank)
+    rk = synth.normal_device((B, P, c["Hkv"], c["D"]), 7702 + rank)
+    rv = synth.normal_device((B, P, c["Hkv"], c["D"]), 7703 + rank)
+    ro = torch.empty_like(rq)
+    rws = torch.empty(hd.hd_attn_rope_workspace(c["L"], c["n"], c["D"]), dtype=torch.uint8, device="cuda")
+    ms_sep = time_fn(lambda: (hd.hd_rope(rq, rk), hd.hd_attn_fwd(rq, rk, rv, c["n"], "intra", out=ro)))
+    ms_fused = time_fn(lambda: hd.hd_attn_fwd_rope(rq, rk, rv, c["n"], "intra", out=ro, workspace=rws))
+    fl = acc.attn_flops(B, c["L"], c["n"], c["Hq"], c["D"], "intra", 0)
+    res["rope_fused_intra"] = {"separate_ms": round(ms_sep, 3), "fused_ms": round(ms_fused, 3),
+                               "fused_attn_TFLOP/s": round(fl / (ms_fused * 1e-3) / 1e12, 1),
+                               "note": "separate = hd_rope(q, k) + hd_attn_fwd; fused = hd_attn_fwd_rope "
+                                       "(table + rope(k) + attention with q rotated in the kernel)"}
+    del rq, rk, rv, ro, rws
     torch.cuda.empty_cache()
     rp = Rope(WORKLOADS["rope"], 7401 + rank, torch, hd, synth)
     ms = time_fn(lambda: rp.step())

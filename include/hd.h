@@ -441,6 +441,36 @@ hd_status hd_rope(void* q, void* k, const int32_t* pos0, int B, int P, int Hq,
                   void* stream);
 
 /*
+ * hd_attn_fwd with the rotary embedding of hd_rope fused in ("Multi-Stream
+ * Expansion and Training Objective": the expanded sequence runs with
+ * contiguous RoPE positions; "Stream-Factorized Attention", Figure 2):
+ *   O = hd_attn_fwd(rope(q), rope(k), v)
+ * with rope as hd_rope at the contiguous positions of the expanded sequence
+ * (row p of a sequence at position p = i*n + s; pos_base = 0, pos_mult = 0).
+ *   q     [B, n*L, Hq, D]  bf16, read only: its rows are rotated inside the
+ *                          attention kernel, as its tiles arrive, and never
+ *                          written back
+ *   k     [B, n*L, Hkv, D] bf16, rotated IN PLACE (on return k holds rope(k),
+ *                          the keys a cache of this layer keeps)
+ *   v, o, lse, mode, window, scale: as hd_attn_fwd (out_dt bf16 or f32)
+ *   rot_dim, base, layout: as hd_rope; rot_dim <= D, and a multiple of 16
+ *                          (HD_ROPE_HALF) or of 8 (HD_ROPE_INTERLEAVED)
+ *   workspace: device scratch of at least hd_attn_rope_workspace(L, n,
+ *              rot_dim) bytes (the cos/sin table of the n*L positions),
+ *              256-byte aligned, owned by the caller, no initialisation
+ *              needed, dead after the call completes.
+ * in_dt must be HD_BF16 (HD_ERR_UNSUPPORTED otherwise).  Three launches on
+ * `stream`: the cos/sin table, the rotation of k, the attention.
+ */
+size_t hd_attn_rope_workspace(int L, int n, int rot_dim);
+hd_status hd_attn_fwd_rope(const void* q, void* k, const void* v, void* o,
+                           float* lse, int B, int L, int n, int Hq, int Hkv, int D,
+                           hd_mode mode, int window, float scale, int rot_dim,
+                           double base, hd_rope_layout layout, void* workspace,
+                           size_t ws_bytes, hd_dtype in_dt, hd_dtype out_dt,
+                           int32_t* dev_status, void* stream);
+
+/*
  * Final-stream gather ("Multi-Stream Expansion and Training Objective": only
  * the final stream E_n of each token feeds the shared LM head; Figure 1):
  *   out[b, i, :] = h[b, i*n + n-1, :]

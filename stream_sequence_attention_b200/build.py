@@ -48,10 +48,13 @@ def _stale() -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    if not force and not _stale():
+def build(force: bool = False, verbose: bool = False, extra=(), out: str | None = None) -> str:
+    """Build libhd.so (or, with ``out``, a library at that path, e.g. a
+    diagnostic build with extra -D switches; always rebuilt)."""
+    target = out or LIB
+    if out is None and not force and not _stale():
         return LIB
-    tmp = LIB + ".tmp"
+    tmp = target + ".tmp"
     cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, *extra, "-o", tmp, *sources()]
     if verbose:
         print(" ".join(cmd), flush=True)
@@ -60,8 +63,8 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
         raise RuntimeError(f"nvcc failed ({r.returncode}):\n{r.stdout}\n{r.stderr}")
     if verbose and (r.stdout or r.stderr):
         print(r.stdout, r.stderr, sep="\n")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, target)
+    return target
 
 
 if __name__ == "__main__":

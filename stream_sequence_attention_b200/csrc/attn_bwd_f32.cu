@@ -66,7 +66,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const void* __restrict__ 
       const int i = static_cast<int>(p / g.ns), s = static_cast<int>(p - static_cast<int64_t>(i) * g.ns);
       const float l2 = lse[(static_cast<int64_t>(b) * Hq + h) * P + p] * 1.4426950408889634f;
       const int64_t at = ((static_cast<int64_t>(b) * Hq + h) * g.ns + s) * Lpad + i;
-      ws.l2[at] = l2;
+      ws.nl2[at] = -l2;
       ws.delta[at] = acc;
     }
   } else {
@@ -75,7 +75,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const void* __restrict__ 
     if (per > 0 && e < pad) {
       const int64_t line = e / per;  // (b*Hq + h)*ns + s
       const int i = g.Lq + static_cast<int>(e - line * per);
-      ws.l2[line * Lpad + i] = INFINITY;
+      ws.nl2[line * Lpad + i] = -INFINITY;
       ws.delta[line * Lpad + i] = 0.f;
     }
   }
@@ -150,7 +150,7 @@ __global__ void __launch_bounds__(kBwThreads) attn_bwd_dq_f32_kernel(
     acc[d] = 0.f;
   }
   const int64_t lat = ((static_cast<int64_t>(b) * Hq + h) * g.ns + s) * bwd_lpad(g.Lq) + ic;
-  const float2 ld = make_float2(ws.l2[lat], ws.delta[lat]);
+  const float2 ld = make_float2(ws.nl2[lat], ws.delta[lat]);
   const int hi = min(min(q0 + kBwRows - 1, g.Lq - 1) * g.qstride + g.qoff, g.Lk - 1);
   const int lo = W > 0 ? max(0, q0 * g.qstride + g.qoff - W + 1) : 0;
   const int64_t kv_stride = static_cast<int64_t>(g.kv_ns) * Hkv * D;
@@ -181,7 +181,7 @@ __global__ void __launch_bounds__(kBwThreads) attn_bwd_dq_f32_kernel(
       pd = quad_sum(pd);
       const int j = k0 + c;
       const bool vis = j <= hi && j <= pic && (W <= 0 || pic - j < W);
-      const float p = vis ? exp2f(sd - ld.x) : 0.f;
+      const float p = vis ? exp2f(sd + ld.x) : 0.f;
       const float ds = p * (pd - ld.y);
 #pragma unroll
       for (int d = 0; d < DQ; ++d) acc[d] = fmaf(ds, Ks[c][part * DQ + d], acc[d]);
@@ -249,7 +249,7 @@ __global__ void __launch_bounds__(kBwThreads) attn_bwd_dkv_f32_kernel(
         reinterpret_cast<float4*>(&Os[c][0])[d4] = bb;
       }
       if (tid < kBwTile)
-        Ls[tid] = (i0 + tid <= hi) ? make_float2(ws.l2[l_base + i0 + tid], ws.delta[l_base + i0 + tid])
+        Ls[tid] = (i0 + tid <= hi) ? make_float2(ws.nl2[l_base + i0 + tid], ws.delta[l_base + i0 + tid])
                                    : make_float2(INFINITY, 0.f);
       __syncthreads();
 #pragma unroll 4
@@ -266,7 +266,7 @@ __global__ void __launch_bounds__(kBwThreads) attn_bwd_dkv_f32_kernel(
         const int pi = i * g.qstride + g.qoff;
         const bool vis = i <= hi && pi >= jc && (W <= 0 || pi - jc < W);
         const float2 l = Ls[c];
-        const float p = vis ? exp2f(sd - l.x) : 0.f;
+        const float p = vis ? exp2f(sd + l.x) : 0.f;
         const float ds = p * (pd - l.y);
 #pragma unroll
         for (int d = 0; d < DQ; ++d) {

@@ -6,9 +6,9 @@
 // the forward: q/k/v/dO [B, ns*Ls, H, D] are read through 5-D TMA maps
 // (D, H, ns, Ls, B), so intra mode (ns = n) and cross mode (ns = 1, Ls = nL)
 // are the same kernels and keys of other streams are never loaded.  P is
-// recomputed from the forward's lse; per-row (lse*log2e, delta = <dO, O>)
+// recomputed from the forward's lse; per-row (-lse*log2e, delta = <dO, O>)
 // come from the preparation kernel, stream-major and padded to 128 tokens
-// with (+inf, 0) so padded queries contribute nothing.
+// with (-inf, 0) so padded queries contribute nothing.
 //
 // Two kernels, each owning its output (no atomics):
 //
@@ -49,7 +49,7 @@ constexpr int kThreads = 320;
 constexpr int kWarpTMA = 8;
 constexpr int kWarpMMA = 9;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kLdBytes = BT * 8;  // lse2[128] then delta[128] of one query tile
+constexpr int kLdBytes = BT * 8;  // -lse2[128] then delta[128] of one query tile
 // One exponential in four of the dK/dV kernel's P tile on the FMA pipe (the
 // cubic of exp2_fma, relative error < 1e-4, below the bf16 rounding of P)
 // when nonzero, to offload the MUFU unit.
@@ -57,6 +57,14 @@ constexpr int kLdBytes = BT * 8;  // lse2[128] then delta[128] of one query tile
 #define HD_BW_POLY_EXP 0
 #endif
 constexpr bool kPolyExp = HD_BW_POLY_EXP != 0;
+// Elementwise arithmetic as packed f32x2 operations (exponents of P for a
+// whole tile first, then the exponentials; dS = P (dP - delta) in pairs)
+// when nonzero.
+#ifndef HD_BW_PACKED
+#define HD_BW_PACKED 1
+#endif
+constexpr bool kPacked = HD_BW_PACKED != 0;
+
 
 template <int D>
 struct Tile {
@@ -105,7 +113,7 @@ struct LayQ {
 }  // namespace bw
 
 struct BwParams {
-  BwdWs ws;  // lse2 and delta planes, stream-major, padded
+  BwdWs ws;  // -lse2 and delta planes, stream-major, padded
   void* dq;
   void* dk;
   void* dv;
@@ -373,7 +381,7 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
                         x.sq, qt * bw::BT, x.b);
           {
             const int64_t at = ((static_cast<int64_t>(x.b) * p.Hq + h) * p.g.ns + x.sq) * p.Lpad + qt * bw::BT;
-            bulk_load(sbase + Lay::LD_OFF + st * bw::kLdBytes, p.ws.l2 + at, bw::kLdBytes / 2,
+            bulk_load(sbase + Lay::LD_OFF + st * bw::kLdBytes, p.ws.nl2 + at, bw::kLdBytes / 2,
                       bar(Lay::B_QFULL + st));
             bulk_load(sbase + Lay::LD_OFF + st * bw::kLdBytes + bw::kLdBytes / 2, p.ws.delta + at,
                       bw::kLdBytes / 2, bar(Lay::B_QFULL + st));
@@ -497,14 +505,30 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
         tmem_wait_ld();
         const bool need_mask = (bw_pos(p, q0) < k0 + bw::BT - 1) || (p.W > 0 && bw_pos(p, q0 + 63) - k0 >= p.W);
         float pv[64];
+        if constexpr (bw::kPacked) {
+          const uint64_t s2 = pack_f32x2(sl2, sl2);
 #pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
-          const float4 l = l4[c4];
-          pv[4 * c4 + 0] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 0]), sl2, -l.x));
-          pv[4 * c4 + 1] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 1]), sl2, -l.y));
-          pv[4 * c4 + 2] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 2]), sl2, -l.z));
-          const float a3 = fmaf(__uint_as_float(sv[4 * c4 + 3]), sl2, -l.w);
-          pv[4 * c4 + 3] = bw::kPolyExp ? exp2_fma(a3) : ex2(a3);
+          for (int c4 = 0; c4 < 16; ++c4) {
+            const float4 l = l4[c4];
+            unpack_f32x2(fma_f32x2(pack_f32x2(__uint_as_float(sv[4 * c4]), __uint_as_float(sv[4 * c4 + 1])), s2,
+                                   pack_f32x2(l.x, l.y)),
+                         pv[4 * c4], pv[4 * c4 + 1]);
+            unpack_f32x2(fma_f32x2(pack_f32x2(__uint_as_float(sv[4 * c4 + 2]), __uint_as_float(sv[4 * c4 + 3])), s2,
+                                   pack_f32x2(l.z, l.w)),
+                         pv[4 * c4 + 2], pv[4 * c4 + 3]);
+          }
+#pragma unroll
+          for (int c = 0; c < 64; ++c) pv[c] = (bw::kPolyExp && (c & 3) == 3) ? exp2_fma(pv[c]) : ex2(pv[c]);
+        } else {
+#pragma unroll
+          for (int c4 = 0; c4 < 16; ++c4) {
+            const float4 l = l4[c4];
+            pv[4 * c4 + 0] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 0]), sl2, l.x));
+            pv[4 * c4 + 1] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 1]), sl2, l.y));
+            pv[4 * c4 + 2] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 2]), sl2, l.z));
+            const float a3 = fmaf(__uint_as_float(sv[4 * c4 + 3]), sl2, l.w);
+            pv[4 * c4 + 3] = bw::kPolyExp ? exp2_fma(a3) : ex2(a3);
+          }
         }
         if (need_mask) {
 #pragma unroll
@@ -538,9 +562,21 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
           for (int e4 = 0; e4 < 8; ++e4) {
             const int c = 32 * half + 4 * e4;
             const float4 d = d4[8 * half + e4];
-            pk[2 * e4] = pack_bf16x2(pv[c] * (__uint_as_float(sv[c]) - d.x), pv[c + 1] * (__uint_as_float(sv[c + 1]) - d.y));
-            pk[2 * e4 + 1] =
-                pack_bf16x2(pv[c + 2] * (__uint_as_float(sv[c + 2]) - d.z), pv[c + 3] * (__uint_as_float(sv[c + 3]) - d.w));
+            if constexpr (bw::kPacked) {
+              pk[2 * e4] = pack_bf16x2_of(
+                  mul_f32x2(pack_f32x2(pv[c], pv[c + 1]),
+                            sub_f32x2(pack_f32x2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
+                                      pack_f32x2(d.x, d.y))));
+              pk[2 * e4 + 1] = pack_bf16x2_of(
+                  mul_f32x2(pack_f32x2(pv[c + 2], pv[c + 3]),
+                            sub_f32x2(pack_f32x2(__uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3])),
+                                      pack_f32x2(d.z, d.w))));
+            } else {
+              pk[2 * e4] =
+                  pack_bf16x2(pv[c] * (__uint_as_float(sv[c]) - d.x), pv[c + 1] * (__uint_as_float(sv[c + 1]) - d.y));
+              pk[2 * e4 + 1] = pack_bf16x2(pv[c + 2] * (__uint_as_float(sv[c + 2]) - d.z),
+                                           pv[c + 3] * (__uint_as_float(sv[c + 3]) - d.w));
+            }
           }
           tmem_st16(tDP + 16 * half, pk);
         }
@@ -762,7 +798,7 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
       const int iq = x.qblk * bw::BT + r;  // this thread's query token
       const int64_t lat = ((static_cast<int64_t>(x.b) * p.Hq + x.h) * p.g.ns + x.s) * p.Lpad + iq;
       const int piq = bw_pos(p, iq);  // key index of this thread's query
-      const float2 ld = make_float2(p.ws.l2[lat], p.ws.delta[lat]);
+      const float2 ld = make_float2(p.ws.nl2[lat], p.ws.delta[lat]);
       for (int j = 0; j < x.nkt; ++j, ++t) {
         const int k0 = (x.kt_lo + j) * bw::BT + 64 * ch;  // first key of this half
         const uint32_t tS = tmem + lane_addr + (t & 1) * 128 + 64 * ch;
@@ -777,8 +813,18 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
         const bool need_mask =
             (k0 + 63 > bw_pos(p, qfirst)) || (p.W > 0 && k0 < bw_pos(p, qfirst + bw::BT - 1) - p.W + 1);
         float pv[64];
+        if constexpr (bw::kPacked) {
+          const uint64_t s2 = pack_f32x2(sl2, sl2), l2 = pack_f32x2(ld.x, ld.x);
 #pragma unroll
-        for (int c = 0; c < 64; ++c) pv[c] = ex2(fmaf(__uint_as_float(sv[c]), sl2, -ld.x));
+          for (int c = 0; c < 32; ++c)
+            unpack_f32x2(fma_f32x2(pack_f32x2(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1])), s2, l2),
+                         pv[2 * c], pv[2 * c + 1]);
+#pragma unroll
+          for (int c = 0; c < 64; ++c) pv[c] = ex2(pv[c]);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) pv[c] = ex2(fmaf(__uint_as_float(sv[c]), sl2, ld.x));
+        }
         if (need_mask) {
 #pragma unroll
           for (int c = 0; c < 64; ++c) {
@@ -794,17 +840,21 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
         tmem_wait_ld();
         {
           uint32_t pk[16];
+          const uint64_t d2 = pack_f32x2(ld.y, ld.y);
+          auto ds_pair = [&](int c) -> uint32_t {
+            if constexpr (bw::kPacked)
+              return pack_bf16x2_of(mul_f32x2(
+                  pack_f32x2(pv[c], pv[c + 1]),
+                  sub_f32x2(pack_f32x2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), d2)));
+            else
+              return pack_bf16x2(pv[c] * (__uint_as_float(sv[c]) - ld.y),
+                                 pv[c + 1] * (__uint_as_float(sv[c + 1]) - ld.y));
+          };
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int c = 2 * e;
-            pk[e] = pack_bf16x2(pv[c] * (__uint_as_float(sv[c]) - ld.y), pv[c + 1] * (__uint_as_float(sv[c + 1]) - ld.y));
-          }
+          for (int e = 0; e < 16; ++e) pk[e] = ds_pair(2 * e);
           tmem_st16(tS, pk);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int c = 32 + 2 * e;
-            pk[e] = pack_bf16x2(pv[c] * (__uint_as_float(sv[c]) - ld.y), pv[c + 1] * (__uint_as_float(sv[c + 1]) - ld.y));
-          }
+          for (int e = 0; e < 16; ++e) pk[e] = ds_pair(32 + 2 * e);
           tmem_st16(tS + 16, pk);
         }
         tmem_wait_st();

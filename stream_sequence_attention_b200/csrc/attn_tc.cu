@@ -50,11 +50,21 @@ namespace hd {
 namespace tc {
 constexpr int BM = 128;
 constexpr int BN = 128;
-constexpr int kThreads = 320;
+// MMA issuers: one warp issuing for both head slots (1), or one warp per head
+// slot (2), so that a head's P V and next S never wait behind the other
+// head's issue order.
+#ifndef HD_TC_ISSUERS
+#define HD_TC_ISSUERS 1
+#endif
+constexpr int kIssuers = HD_TC_ISSUERS;
+static_assert(kIssuers == 1 || kIssuers == 2, "one or two MMA issuers");
+// Warps: two softmax warpgroups (0-7), the TMA producer (8), the MMA
+// issuer(s) (9, and 10 with two), and in the rank-shard form with gather the
+// gather warp after them.
+constexpr int kThreads = 32 * (9 + kIssuers);
 constexpr int kWarpTMA = 8;
 constexpr int kWarpMMA = 9;
-constexpr int kWarpGather = 10;  // rank-shard form with gather only
-constexpr int KST = 3;
+constexpr int kWarpGather = 9 + kIssuers;  // rank-shard form with gather only
 constexpr int VST = 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -69,25 +79,56 @@ constexpr int kPolyEvery = HD_TC_POLY_EVERY;
 #define HD_TC_PINGPONG 0
 #endif
 constexpr bool kPingPong = HD_TC_PINGPONG != 0;
+// Epilogue: O / l leaves through shared memory, one TMA store per warp and
+// 128-byte column chunk (1), or as per-thread global stores (0).
+#ifndef HD_TC_TMA_STORE
+#define HD_TC_TMA_STORE 1
+#endif
+constexpr bool kTmaStore = HD_TC_TMA_STORE != 0;
+// Softmax arithmetic per tile: the exponents of the whole row first, as
+// packed f32x2 FMAs, then the exponentials (1); or exponent and exponential
+// column pair by column pair (0).
+#ifndef HD_TC_SPLIT
+#define HD_TC_SPLIT 1
+#endif
+constexpr bool kSplit = HD_TC_SPLIT != 0;
+// Diagnostic build only: per-role clock counters (see hd_tc_trace_fetch).
+#ifndef HD_TC_TRACE
+#define HD_TC_TRACE 0
+#endif
+constexpr bool kTrace = HD_TC_TRACE != 0;
 
 template <int D>
 struct Layout {
   static constexpr int KB = D / 64;     // 128-byte column blocks per row
   static constexpr int BLK = BM * 128;  // bytes of one 128-row x 128-byte block
   static constexpr int TILE = BLK * KB; // bytes of a 128-row tile
+  // K stages: 3, or 2 at D = 128 when the epilogue's staging (32 KB) takes
+  // the third stage's shared memory.
+  static constexpr int KST = (kTmaStore && D == 128) ? 2 : 3;
   static constexpr int Q_OFF = 0;       // head slots 0 and 1
   static constexpr int K_OFF = Q_OFF + 2 * TILE;
   static constexpr int V_OFF = K_OFF + KST * TILE;
-  static constexpr int BAR_OFF = V_OFF + VST * TILE;
+  // Epilogue staging: one 128-row x 128-byte block per head slot (each warp
+  // owns its 32 rows, 4 KB).
+  static constexpr int O_OFF = V_OFF + VST * TILE;
+  static constexpr int BAR_OFF = O_OFF + (kTmaStore ? 2 * BLK : 0);
   static constexpr int B_QFULL = 0, B_QEMPTY = 1, B_KFULL = 2, B_KEMPTY = B_KFULL + KST,
                        B_VFULL = B_KEMPTY + KST, B_VEMPTY = B_VFULL + VST, B_SFULL = B_VEMPTY + VST,
                        B_PFULL = B_SFULL + 2, B_ODONE = B_PFULL + 2, B_OEMPTY = B_ODONE + 2,
-                       B_ORD = B_OEMPTY + 2, B_DRAIN = B_ORD + 2, NBAR = B_DRAIN + 1;
+                       B_ORD = B_OEMPTY + 2, B_DRAIN = B_ORD + 2, B_QROT = B_DRAIN + 1, NBAR = B_QROT + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int ALLOC = BYTES + 1024;
 };
 }  // namespace tc
+
+#if HD_TC_TRACE
+// Per-CTA clock counters of the diagnostic build: kTraceSlots per CTA.
+constexpr int kTraceCtas = 1024;
+constexpr int kTraceSlots = 20;
+__device__ unsigned long long g_tc_trace[kTraceCtas * kTraceSlots];
+#endif
 
 struct TcParams {
   void* o;
@@ -99,6 +140,11 @@ struct TcParams {
   int out_bf16;
   int nqb, npairs;
   int total_units;
+  // Rotary embedding of the query rows inside the kernel (nullptr: q is
+  // used as given).  rope_tab[pos * rope_half + j] = (cos, sin) of
+  // pos * theta_j for positions pos = i * q_ns + s of the expanded sequence.
+  const float2* rope_tab;
+  int rope_half, rope_layout;
   // Test hook (environment HD_TEST_STALL_FIRST_S=1): the MMA warp of CTA 0
   // never signals its first S tile, so the softmax wait runs out and the
   // kernel must take its timeout path.  0 in normal use.
@@ -270,10 +316,79 @@ __device__ __forceinline__ void gather_items(const PartsInfo& x, int B, int lane
   }
 }
 
-template <int D, int NM>
+// Rotary embedding of one query row in place in a 128-byte-swizzled Q tile
+// (row r at qrow; 64-feature blocks blk bytes apart): pairs (j, j + half) or
+// (2j, 2j + 1), j < half, (a, b) -> (a cos - b sin, a sin + b cos) with
+// (cos, sin) of pair j at t4[j / 2] (two pairs per float4).
+__device__ __forceinline__ void rope_rotate_row(uint8_t* qrow, int blk, int r, const float4* t4, int half,
+                                             int layout) {
+  // 16-byte unit holding features f .. f+7 (f a multiple of 8) of the
+  // row: 128-byte swizzle within each 64-feature block.
+  auto unit = [&](int f) -> uint4* {
+    return reinterpret_cast<uint4*>(qrow + (f >> 6) * blk + ((((f & 63) >> 3) ^ (r & 7)) << 4));
+  };
+#pragma unroll 1
+  for (int qtr = 0; qtr < 4; ++qtr) {
+    float4 cs[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      if (16 * qtr + 2 * c < half) cs[c] = __ldg(t4 + 8 * qtr + c);
+    // pair 16*qtr + j of this quarter
+    auto cs_of = [&](int j) -> float2 {
+      const float4 c4 = cs[j >> 1];
+      return (j & 1) ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y);
+    };
+    if (16 * qtr >= half) {
+    } else if (layout == HD_ROPE_HALF) {
+      // pairs (j, j + half), (a, b) -> (a cos - b sin, a sin + b cos):
+      // the units at features j and j + half, j = 16*qtr + 8w
+#pragma unroll
+      for (int w = 0; w < 2; ++w) {
+        const int f = 16 * qtr + 8 * w;
+        if (f < half) {
+          uint4* pa = unit(f);
+          uint4* pb = unit(f + half);
+          const uint4 ua = *pa, ub = *pb;
+          uint32_t wa[4] = {ua.x, ua.y, ua.z, ua.w}, wb[4] = {ub.x, ub.y, ub.z, ub.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 fa = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wa[e]));
+            const float2 fb = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wb[e]));
+            const float2 t0 = cs_of(8 * w + 2 * e), t1 = cs_of(8 * w + 2 * e + 1);
+            wa[e] = pack_bf16x2(fmaf(fa.x, t0.x, -fb.x * t0.y), fmaf(fa.y, t1.x, -fb.y * t1.y));
+            wb[e] = pack_bf16x2(fmaf(fa.x, t0.y, fb.x * t0.x), fmaf(fa.y, t1.y, fb.y * t1.x));
+          }
+          *pa = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+          *pb = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+        }
+      }
+    } else {
+      // pairs (2j, 2j + 1): unit 4*qtr + w holds pairs 16*qtr + 4w .. + 3
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        if (16 * qtr + 4 * w < half) {
+          uint4* pa = unit(32 * qtr + 8 * w);
+          const uint4 ua = *pa;
+          uint32_t wa[4] = {ua.x, ua.y, ua.z, ua.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 fa = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wa[e]));
+            const float2 t = cs_of(4 * w + e);
+            wa[e] = pack_bf16x2(fmaf(fa.x, t.x, -fa.y * t.y), fmaf(fa.x, t.y, fa.y * t.x));
+          }
+          *pa = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+        }
+      }
+    }
+  }
+}
+
+// ROPE: the query rows are rotated in the Q tile at the start of each unit
+// (a separate instantiation, so the other forms carry none of its code).
+template <int D, int NM, bool ROPE = false>
 __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ KvSrc<NM> kv,
-                   const TcParams p) {
+                   const __grid_constant__ CUtensorMap tmO, const TcParams p) {
   using Lay = tc::Layout<D>;
   constexpr bool kParts = NM > 1;
   extern __shared__ uint8_t smem_raw[];
@@ -290,14 +405,15 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(Lay::B_QFULL), 1);
-    mbar_init(bar(Lay::B_QEMPTY), 1);
-    for (int i = 0; i < tc::KST; ++i) {
+    // Stages are released by every MMA issuer.
+    mbar_init(bar(Lay::B_QEMPTY), tc::kIssuers);
+    for (int i = 0; i < Lay::KST; ++i) {
       mbar_init(bar(Lay::B_KFULL + i), 1);
-      mbar_init(bar(Lay::B_KEMPTY + i), 1);
+      mbar_init(bar(Lay::B_KEMPTY + i), tc::kIssuers);
     }
     for (int i = 0; i < tc::VST; ++i) {
       mbar_init(bar(Lay::B_VFULL + i), 1);
-      mbar_init(bar(Lay::B_VEMPTY + i), 1);
+      mbar_init(bar(Lay::B_VEMPTY + i), tc::kIssuers);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(Lay::B_SFULL + i), 1);
@@ -307,13 +423,16 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
     }
     mbar_init(bar(Lay::B_ORD + 0), 128);
     mbar_init(bar(Lay::B_ORD + 1), 128);
-    mbar_init(bar(Lay::B_DRAIN), 1);
+    mbar_init(bar(Lay::B_QROT + 0), 128);
+    mbar_init(bar(Lay::B_QROT + 1), 128);
+    mbar_init(bar(Lay::B_DRAIN), tc::kIssuers);
     *abort_flag = 0;
     *no_abort = 0;
     fence_barrier_init();
   }
   if (warp == tc::kWarpTMA && lane == 0) {
     tma_prefetch_desc(&tmQ);
+    if (tc::kTmaStore) tma_prefetch_desc(&tmO);
 #pragma unroll
     for (int i = 0; i < NM; ++i) {
       if constexpr (kParts) {
@@ -361,11 +480,13 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
     }
   };
 
+  if (warp >= 8) {
+  // Producer, MMA issuer, gather (each warp its own role).
   if (warp == tc::kWarpTMA) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int t = 0, ul = 0, q_issued = 0;
-      int k_issued[tc::KST] = {}, v_issued[tc::VST] = {};
+      int k_issued[Lay::KST] = {}, v_issued[tc::VST] = {};
       bool ok = true;
       for (int k = 0; ok; ++k) {
         const int u = tc_unit_of(k, p.total_units);
@@ -393,8 +514,8 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
               break;
             }
           }
-          const int ks = t % tc::KST;
-          if (!mbar_wait(bar(Lay::B_KEMPTY + ks), ((t / tc::KST) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          const int ks = t % Lay::KST;
+          if (!mbar_wait(bar(Lay::B_KEMPTY + ks), ((t / Lay::KST) & 1) ^ 1, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(bar(Lay::B_KFULL + ks), Lay::TILE);
           load_kv_tile(kv.k, sbase + Lay::K_OFF + ks * Lay::TILE, bar(Lay::B_KFULL + ks), x, skv, kt);
           ++k_issued[ks];
@@ -410,68 +531,105 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
         fail();
         // Let every copy already issued land before the CTA can exit.
         if (q_issued) mbar_wait(bar(Lay::B_QFULL), (q_issued - 1) & 1, no_abort);
-        for (int i = 0; i < tc::KST; ++i)
+        for (int i = 0; i < Lay::KST; ++i)
           if (k_issued[i]) mbar_wait(bar(Lay::B_KFULL + i), (k_issued[i] - 1) & 1, no_abort);
         for (int i = 0; i < tc::VST; ++i)
           if (v_issued[i]) mbar_wait(bar(Lay::B_VFULL + i), (v_issued[i] - 1) & 1, no_abort);
       }
     }
-  } else if (warp == tc::kWarpMMA) {
+  } else if (warp >= tc::kWarpMMA && warp < tc::kWarpMMA + tc::kIssuers) {
     // ---------------------------------------------------------------- MMA
-    // Issue order per tile t (heads 0, 1):  PV_0(t) S_0(t+1) PV_1(t) S_1(t+1).
-    // S_h(t+1) overwrites the columns P_h(t) occupies; tcgen05.mma from one
-    // thread executes in issue order, so PV_h(t) has read P_h(t) by then.
+    // With one issuer the order per tile t is PV_0(t) S_0(t+1) PV_1(t)
+    // S_1(t+1); with two, each issues PV_h(t) S_h(t+1) for its own head
+    // slot h.  S_h(t+1) overwrites the columns P_h(t) occupies; tcgen05.mma
+    // from one thread executes in issue order, so PV_h(t) has read P_h(t) by
+    // then.  Each issuer releases every Q/K/V stage once (its commit, or a
+    // plain arrive when it has no head in the unit).
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(tc::BM, tc::BN, false, false);
       constexpr uint32_t idO = idesc_bf16_f32(tc::BM, D, false, true);
+      const int me = warp - tc::kWarpMMA;  // issuer index
       auto issue_S = [&](int h, int kst) {
-        const uint32_t qbase = sbase + Lay::Q_OFF + h * Lay::TILE;
-        const uint32_t kbase = sbase + Lay::K_OFF + kst * Lay::TILE;
+        // Descriptors once per tile; the K-steps add their byte offset / 16.
+        const uint64_t qd = smem_desc_sw128(sbase + Lay::Q_OFF + h * Lay::TILE, 16, 1024);
+        const uint64_t kd = smem_desc_sw128(sbase + Lay::K_OFF + kst * Lay::TILE, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * Lay::BLK + (kk & 3) * 32;
-          mma_ss(tmem + h * 128, smem_desc_sw128(qbase + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
-                 idS, kk > 0 ? 1u : 0u);
+          const uint32_t off16 = ((kk >> 2) * Lay::BLK + (kk & 3) * 32) >> 4;
+          mma_ss(tmem + h * 128, qd + off16, kd + off16, idS, kk > 0 ? 1u : 0u);
         }
         if (!(p.stall_first_s && blockIdx.x == 0)) tc_commit(bar(Lay::B_SFULL + h));
       };
       auto issue_PV = [&](int h, int vst, bool acc) {
-        const uint32_t vbase = sbase + Lay::V_OFF + vst * Lay::TILE;
+        // V tile is MN-major (D contiguous): 16 keys = 16 rows of 128 B.
+        const uint64_t vd = smem_desc_sw128(sbase + Lay::V_OFF + vst * Lay::TILE, Lay::BLK, 1024);
 #pragma unroll
-        for (int kk = 0; kk < tc::BN / 16; ++kk) {
-          // V tile is MN-major (D contiguous): 16 keys = 16 rows of 128 B.
-          const uint64_t bdesc = smem_desc_sw128(vbase + kk * 2048, Lay::BLK, 1024);
-          mma_ts(tmem + 256 + h * 128, tmem + h * 128 + kk * 8, bdesc, idO, (acc || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < tc::BN / 16; ++kk)
+          mma_ts(tmem + 256 + h * 128, tmem + h * 128 + kk * 8, vd + ((kk * 2048) >> 4), idO,
+                 (acc || kk > 0) ? 1u : 0u);
       };
       int t = 0, ul = 0;
       int ts[2] = {0, 0};  // P_h V MMAs issued per head slot
       int us[2] = {0, 0};  // units per head slot
       bool ok = true;
+      // Diagnostic counters (HD_TC_TRACE): waiting for P, for Q/K/V/O, total.
+      unsigned long long mw[3] = {0, 0, 0};
+      const long long mt0 = tc::kTrace ? clock64() : 0;
+      auto timed_wait = [&](int which, uint32_t b, uint32_t par) {
+        if constexpr (tc::kTrace) {
+          const long long t0 = clock64();
+          const bool r = mbar_wait(b, par, abort_flag);
+          mw[which] += static_cast<unsigned long long>(clock64() - t0);
+          return r;
+        } else {
+          return mbar_wait(b, par, abort_flag);
+        }
+      };
       for (int k = 0; ok; ++k) {
         const int u = tc_unit_of(k, p.total_units);
         if (u == -1) break;
         if (u < 0) continue;
         const TcUnit x = tc_unit(u, p);
-        const int nslot = x.h1 >= 0 ? 2 : 1;
+        // Head slots this issuer serves in this unit: [h_lo, h_hi).
+        const int h_lo = tc::kIssuers == 2 ? me : 0;
+        const int h_hi = tc::kIssuers == 2 ? (me == 0 || x.h1 >= 0 ? me + 1 : me) : (x.h1 >= 0 ? 2 : 1);
+        const bool mine = h_hi > h_lo;
+        auto release = [&](uint32_t b) {
+          if (mine)
+            tc_commit(b);
+          else
+            mbar_arrive(b);
+        };
         const int nt = x.t_hi - x.t_lo + 1;
-        if (!mbar_wait(bar(Lay::B_QFULL), ul & 1, abort_flag)) { ok = false; break; }
+        if (!timed_wait(1, bar(Lay::B_QFULL), ul & 1)) { ok = false; break; }
+        if constexpr (ROPE) {
+          // The softmax warps rotate their query rows in place first.
+          for (int h = h_lo; h < h_hi; ++h)
+            if (!timed_wait(1, bar(Lay::B_QROT + h), us[h] & 1)) { ok = false; break; }
+          if (!ok) break;
+        }
         {
-          const int ks = t % tc::KST;
-          if (!mbar_wait(bar(Lay::B_KFULL + ks), (t / tc::KST) & 1, abort_flag)) { ok = false; break; }
+          const int ks = t % Lay::KST;
+          if (!timed_wait(1, bar(Lay::B_KFULL + ks), (t / Lay::KST) & 1)) { ok = false; break; }
           tc_fence_after();
-          for (int h = 0; h < nslot; ++h) issue_S(h, ks);
-          tc_commit(bar(Lay::B_KEMPTY + ks));
-          if (nt == 1) tc_commit(bar(Lay::B_QEMPTY));
+          for (int h = h_lo; h < h_hi; ++h) issue_S(h, ks);
+          release(bar(Lay::B_KEMPTY + ks));
+          if (nt == 1) release(bar(Lay::B_QEMPTY));
         }
         for (int jj = 0; ok && jj < nt; ++jj, ++t) {
           const int vs = t % tc::VST;
-          if (!mbar_wait(bar(Lay::B_VFULL + vs), (t / tc::VST) & 1, abort_flag)) { ok = false; break; }
+          if (!timed_wait(1, bar(Lay::B_VFULL + vs), (t / tc::VST) & 1)) { ok = false; break; }
           const bool nxt = jj + 1 < nt;
-          const int ksn = (t + 1) % tc::KST;
-          for (int h = 0; h < nslot; ++h) {
-            if (!mbar_wait(bar(Lay::B_PFULL + h), ts[h] & 1, abort_flag)) { ok = false; break; }
-            if (jj == 0 && us[h] > 0 && !mbar_wait(bar(Lay::B_OEMPTY + h), (us[h] - 1) & 1, abort_flag)) {
+          const int ksn = (t + 1) % Lay::KST;
+          // An issuer with no head in the unit still sees each stage full
+          // before it releases it.
+          if (!mine && nxt && !timed_wait(1, bar(Lay::B_KFULL + ksn), ((t + 1) / Lay::KST) & 1)) {
+            ok = false;
+            break;
+          }
+          for (int h = h_lo; h < h_hi; ++h) {
+            if (!timed_wait(0, bar(Lay::B_PFULL + h), ts[h] & 1)) { ok = false; break; }
+            if (jj == 0 && us[h] > 0 && !timed_wait(1, bar(Lay::B_OEMPTY + h), (us[h] - 1) & 1)) {
               ok = false;
               break;
             }
@@ -479,7 +637,7 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
             issue_PV(h, vs, jj > 0);
             ++ts[h];
             if (nxt) {
-              if (h == 0 && !mbar_wait(bar(Lay::B_KFULL + ksn), ((t + 1) / tc::KST) & 1, abort_flag)) {
+              if (h == h_lo && !timed_wait(1, bar(Lay::B_KFULL + ksn), ((t + 1) / Lay::KST) & 1)) {
                 ok = false;
                 break;
               }
@@ -489,22 +647,32 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
             }
           }
           if (!ok) break;
-          tc_commit(bar(Lay::B_VEMPTY + vs));
+          release(bar(Lay::B_VEMPTY + vs));
           if (nxt) {
-            tc_commit(bar(Lay::B_KEMPTY + ksn));
-            if (jj + 1 == nt - 1) tc_commit(bar(Lay::B_QEMPTY));
+            release(bar(Lay::B_KEMPTY + ksn));
+            if (jj + 1 == nt - 1) release(bar(Lay::B_QEMPTY));
           }
         }
-        us[0]++;
-        if (nslot == 2) us[1]++;
+        for (int h = h_lo; h < h_hi; ++h) us[h]++;
         ++ul;
       }
       if (!ok) fail();
       // Drain: every MMA issued above has completed before TMEM is freed.
       tc_commit(bar(Lay::B_DRAIN));
       mbar_wait(bar(Lay::B_DRAIN), 0, no_abort);
+#if HD_TC_TRACE
+      mw[2] = static_cast<unsigned long long>(clock64() - mt0);
+      if (blockIdx.x < kTraceCtas)
+        for (int c = 0; c < 3; ++c) g_tc_trace[blockIdx.x * kTraceSlots + 12 + 3 * me + c] = mw[c];
+#endif
     }
-  } else if (warp < 8) {
+  } else if (warp == tc::kWarpGather) {
+    // ------------------------------------------------------------- gather
+    if constexpr (kParts) {
+      if (kv.x.flags) gather_items<16>(kv.x, p.g.B, lane, abort_flag);
+    }
+  }
+  } else {
     // ------------------------------------------------- softmax + epilogue
     const int slot = warp >> 2;
     const int r = threadIdx.x & 127;  // tensor-memory lane
@@ -514,24 +682,56 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
     const float sl2 = p.scale_log2;
     int sc = 0, uc = 0, oc = 0;
     bool ok = true;
+    bool stored = false;  // this warp has TMA stores in flight (lane 0)
+    // Diagnostic counters (HD_TC_TRACE): wait for S, load + max, exponents
+    // to P published, row sum, epilogue, tiles.
+    unsigned long long tr[6] = {0, 0, 0, 0, 0, 0};
+    long long tmark = tc::kTrace ? clock64() : 0;
+    auto tick = [&](int i) {
+      if constexpr (tc::kTrace) {
+        const long long t = clock64();
+        tr[i] += static_cast<unsigned long long>(t - tmark);
+        tmark = t;
+      }
+    };
+    int uall = 0;  // units of this CTA so far (phases of B_QFULL)
     for (int k = 0; ok; ++k) {
       const int u = tc_unit_of(k, p.total_units);
       if (u == -1) break;
       if (u < 0) continue;
+      const int ucur = uall++;
       const TcUnit x = tc_unit(u, p);
       const int h = slot ? x.h1 : x.h0;
       if (h < 0) continue;  // uniform across the warpgroup
       const bool paired = x.h1 >= 0;
       const int q0 = x.qblk * tc::BM;
       const int i = q0 + r;
-      const int qb = p.g.qoff + x.s * p.g.qsstride;
+      const int qb = p.g.qoff + x.s * p.g.qsstride;  // key index offset of this query stream
       const int pi = i * p.g.qstride + qb;             // key index of this row's query
       const int pfirst = q0 * p.g.qstride + qb;         // ... of the block's first query
       const int plast = (q0 + tc::BM - 1) * p.g.qstride + qb;
       float m = -INFINITY, l = 0.f;
       const int nt = x.t_hi - x.t_lo + 1;
+      if constexpr (ROPE) {
+        // Rotary embedding of this thread's query row, in the Q tile itself
+        // (position i*q_ns + s; "Multi-Stream Expansion and Training
+        // Objective": contiguous positions over the expanded sequence).  The
+        // cos/sin pairs are fetched before the tile lands.
+        const bool rok = i < p.g.Lq;
+        const int half = p.rope_half;
+        // (cos, sin) pairs of the row, 16 pairs (8 float4) at a time.
+        const float4* t4 =
+            reinterpret_cast<const float4*>(p.rope_tab + (static_cast<int64_t>(i) * p.g.q_ns + x.s) * half);
+        const bool got = mbar_wait(bar(Lay::B_QFULL), ucur & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        if (rok) rope_rotate_row(smem + Lay::Q_OFF + slot * Lay::TILE + r * 128, Lay::BLK, r, t4, half, p.rope_layout);
+        // The tensor core reads the tile through the async proxy.
+        fence_proxy_async_smem();
+        mbar_arrive(bar(Lay::B_QROT + slot));
+      }
       for (int jj = 0; jj < nt; ++jj, ++sc) {
         const int k0 = (x.t_lo + jj) * tc::BN;
+        if (tc::kTrace) tmark = clock64();
         bool got = mbar_wait(bar(Lay::B_SFULL + slot), sc & 1, abort_flag);
         // Ping-pong: the two warpgroups take turns for the softmax arithmetic
         // (slot 0 first), so each runs alone on the SM sub-partitions while
@@ -543,6 +743,7 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
             got = mbar_wait(bar(Lay::B_ORD + 0), (oc - 1) & 1, abort_flag);
         }
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        tick(0);
         tc_fence_after();
         uint32_t sv[128];
         tmem_ld32(sS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
@@ -578,17 +779,35 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
           resc = true;
         }
         const float nmu = (m == -INFINITY) ? 0.f : -m;
+        tick(1);
         // P = 2^(s*scale - m) as bf16 pairs, written over the S columns 16 at
         // a time (column 16j of P holds S columns 32j.. already consumed).
         float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if constexpr (tc::kSplit) {
+          const uint64_t s2 = pack_f32x2(sl2, sl2), n2 = pack_f32x2(nmu, nmu);
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            float a0, a1;
+            unpack_f32x2(fma_f32x2(pack_f32x2(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1])), s2, n2),
+                         a0, a1);
+            sv[2 * c] = __float_as_uint(a0);
+            sv[2 * c + 1] = __float_as_uint(a1);
+          }
+        }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int c = 16 * j + e;
-            const float a0 = fmaf(__uint_as_float(sv[2 * c]), sl2, nmu);
-            const float a1 = fmaf(__uint_as_float(sv[2 * c + 1]), sl2, nmu);
+            float a0, a1;
+            if constexpr (tc::kSplit) {
+              a0 = __uint_as_float(sv[2 * c]);
+              a1 = __uint_as_float(sv[2 * c + 1]);
+            } else {
+              a0 = fmaf(__uint_as_float(sv[2 * c]), sl2, nmu);
+              a1 = fmaf(__uint_as_float(sv[2 * c + 1]), sl2, nmu);
+            }
             float p0, p1;
             if (tc::kPolyEvery > 0 && !need_mask && (e % (tc::kPolyEvery > 0 ? tc::kPolyEvery : 1)) == tc::kPolyEvery - 1) {
               p0 = exp2_fma(a0);
@@ -602,7 +821,6 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
           }
           tmem_st16(sS + 16 * j, pk);
         }
-        l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
         if (tc::kPingPong && paired) {
           mbar_arrive(bar(Lay::B_ORD + (slot ^ 1)));
           ++oc;
@@ -623,6 +841,10 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(Lay::B_PFULL + slot));
+        tick(2);
+        l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+        tick(3);
+        if (tc::kTrace) ++tr[5];
       }
       if (!ok) break;
       // Epilogue: O / l -> global once the last P V MMA of this head is done.
@@ -632,46 +854,118 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
       tc_fence_after();
       const float inv = 1.f / l;
       const bool row_ok = i < p.g.Lq;
-      const int64_t orow =
-          (static_cast<int64_t>(x.b) * p.g.o_rows + static_cast<int64_t>(i) * p.g.o_ns + x.s) * p.Hq + h;
+      if constexpr (tc::kTmaStore) {
+        // O / l by 128-byte column chunks: this warp's 32 rows of a chunk go
+        // through its own 4 KB of staging (128-byte swizzle, the layout of
+        // the tensor map) and out with one TMA store; rows past Lq are
+        // clipped by it.  The tensor memory is released after the last
+        // chunk's load.
+        const int wq = warp & 3;
+        uint8_t* stg = smem + Lay::O_OFF + slot * Lay::BLK + wq * 32 * 128;
+        const uint32_t stg_s = smem_u32(stg);
+        const int row0 = q0 + 32 * wq;
+        const int rl = r & 31;
+        auto put = [&](int chunk, const uint4* w) {
+          if (lane == 0 && stored) bulk_wait_group_read<0>();
+          __syncwarp();
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t ov[32];
-        tmem_ld32(sO + c * 32, ov);
-        tmem_wait_ld();
-        if (row_ok) {
-          if (p.out_bf16) {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + orow * D + c * 32);
+          for (int uu = 0; uu < 8; ++uu)
+            *reinterpret_cast<uint4*>(stg + rl * 128 + ((uu ^ (rl & 7)) << 4)) = w[uu];
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && row0 < p.g.Lq) {
+            tma_store_5d(&tmO, stg_s, chunk * (p.out_bf16 ? 64 : 32), h, x.s, row0, x.b);
+            bulk_commit_group();
+            stored = true;
+          }
+        };
+        if (p.out_bf16) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              uint4 w;
-              w.x = pack_bf16x2(__uint_as_float(ov[8 * e + 0]) * inv, __uint_as_float(ov[8 * e + 1]) * inv);
-              w.y = pack_bf16x2(__uint_as_float(ov[8 * e + 2]) * inv, __uint_as_float(ov[8 * e + 3]) * inv);
-              w.z = pack_bf16x2(__uint_as_float(ov[8 * e + 4]) * inv, __uint_as_float(ov[8 * e + 5]) * inv);
-              w.w = pack_bf16x2(__uint_as_float(ov[8 * e + 6]) * inv, __uint_as_float(ov[8 * e + 7]) * inv);
-              dst[e] = w;
+          for (int ch = 0; ch < D / 64; ++ch) {
+            uint32_t ov[64];
+            tmem_ld32(sO + ch * 64, *reinterpret_cast<uint32_t(*)[32]>(&ov[0]));
+            tmem_ld32(sO + ch * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&ov[32]));
+            tmem_wait_ld();
+            if (ch == D / 64 - 1) {
+              tc_fence_before();
+              mbar_arrive(bar(Lay::B_OEMPTY + slot));
             }
-          } else {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow * D + c * 32);
+            uint4 w[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              dst[e] = make_float4(__uint_as_float(ov[4 * e + 0]) * inv, __uint_as_float(ov[4 * e + 1]) * inv,
-                                   __uint_as_float(ov[4 * e + 2]) * inv, __uint_as_float(ov[4 * e + 3]) * inv);
+            for (int uu = 0; uu < 8; ++uu) {
+              const int c0 = uu * 8;
+              w[uu].x = pack_bf16x2(__uint_as_float(ov[c0 + 0]) * inv, __uint_as_float(ov[c0 + 1]) * inv);
+              w[uu].y = pack_bf16x2(__uint_as_float(ov[c0 + 2]) * inv, __uint_as_float(ov[c0 + 3]) * inv);
+              w[uu].z = pack_bf16x2(__uint_as_float(ov[c0 + 4]) * inv, __uint_as_float(ov[c0 + 5]) * inv);
+              w[uu].w = pack_bf16x2(__uint_as_float(ov[c0 + 6]) * inv, __uint_as_float(ov[c0 + 7]) * inv);
+            }
+            put(ch, w);
+          }
+        } else {
+#pragma unroll
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t ov[32];
+            tmem_ld32(sO + ch * 32, ov);
+            tmem_wait_ld();
+            if (ch == D / 32 - 1) {
+              tc_fence_before();
+              mbar_arrive(bar(Lay::B_OEMPTY + slot));
+            }
+            uint4 w[8];
+#pragma unroll
+            for (int uu = 0; uu < 8; ++uu)
+              w[uu] = make_uint4(__float_as_uint(__uint_as_float(ov[4 * uu + 0]) * inv),
+                                 __float_as_uint(__uint_as_float(ov[4 * uu + 1]) * inv),
+                                 __float_as_uint(__uint_as_float(ov[4 * uu + 2]) * inv),
+                                 __float_as_uint(__uint_as_float(ov[4 * uu + 3]) * inv));
+            put(ch, w);
           }
         }
+      } else {
+        const int64_t orow =
+            (static_cast<int64_t>(x.b) * p.g.o_rows + static_cast<int64_t>(i) * p.g.o_ns + x.s) * p.Hq + h;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(sO + c * 32, ov);
+          tmem_wait_ld();
+          if (row_ok) {
+            if (p.out_bf16) {
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + orow * D + c * 32);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                uint4 w;
+                w.x = pack_bf16x2(__uint_as_float(ov[8 * e + 0]) * inv, __uint_as_float(ov[8 * e + 1]) * inv);
+                w.y = pack_bf16x2(__uint_as_float(ov[8 * e + 2]) * inv, __uint_as_float(ov[8 * e + 3]) * inv);
+                w.z = pack_bf16x2(__uint_as_float(ov[8 * e + 4]) * inv, __uint_as_float(ov[8 * e + 5]) * inv);
+                w.w = pack_bf16x2(__uint_as_float(ov[8 * e + 6]) * inv, __uint_as_float(ov[8 * e + 7]) * inv);
+                dst[e] = w;
+              }
+            } else {
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow * D + c * 32);
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                dst[e] = make_float4(__uint_as_float(ov[4 * e + 0]) * inv, __uint_as_float(ov[4 * e + 1]) * inv,
+                                     __uint_as_float(ov[4 * e + 2]) * inv, __uint_as_float(ov[4 * e + 3]) * inv);
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar(Lay::B_OEMPTY + slot));
       }
       if (row_ok && p.lse)
         p.lse[(static_cast<int64_t>(x.b) * p.Hq + h) * p.g.o_rows + static_cast<int64_t>(i) * p.g.o_ns + x.s] =
             (m + log2f(l)) * 0.69314718055994531f;
-      tc_fence_before();
-      mbar_arrive(bar(Lay::B_OEMPTY + slot));
+      tick(4);
     }
+    // Every TMA store has finished reading its staging before the CTA's
+    // shared memory can go away.
+    if (tc::kTmaStore && lane == 0 && stored) bulk_wait_group<0>();
     if (!ok) fail();
-  } else if (warp == tc::kWarpGather) {
-    // ------------------------------------------------------------- gather
-    if constexpr (kParts) {
-      if (kv.x.flags) gather_items<16>(kv.x, p.g.B, lane, abort_flag);
-    }
+#if HD_TC_TRACE
+    if (r == 0 && blockIdx.x < kTraceCtas)
+      for (int c = 0; c < 6; ++c) g_tc_trace[blockIdx.x * kTraceSlots + slot * 6 + c] = tr[c];
+#endif
   }
 
   __syncthreads();
@@ -700,6 +994,43 @@ static bool make_stream_view(const TmapKey& k, CUtensorMap* m) {
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// (D, H, ns, Ls, B) view of the output [B, ns*Ls, H, D], bf16 or f32 (element
+// bytes in the key's `pad`), with a box of one 128-byte column chunk x 32
+// rows: one warp's share of the epilogue's TMA stores.
+static bool make_out_view(const TmapKey& k, CUtensorMap* m) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) return false;
+  const cuuint64_t B = k.dims[0], Ls = k.dims[1], ns = k.dims[2], H = k.dims[3], D = k.dims[4];
+  const cuuint64_t e = static_cast<cuuint64_t>(k.pad);
+  const cuuint64_t dims[5] = {D, H, ns, Ls, B};
+  const cuuint64_t strides[4] = {D * e, H * D * e, ns * H * D * e, Ls * ns * H * D * e};
+  const cuuint32_t box[5] = {static_cast<cuuint32_t>(128 / e), 1, 1, 32, 1};
+  const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  return enc(m, e == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 5, const_cast<void*>(k.ptr),
+             dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The output view of a call's geometry (o [B, o_rows, Hq, D] with query (i, s)
+// at row i*o_ns + s, o_rows = o_ns*Lq); all zero when the epilogue stores
+// per thread.
+static bool encode_out_view(CUtensorMap* m, void* o, const AttnGeom& g, int Hq, int D, bool out_bf16) {
+  std::memset(m, 0, sizeof(*m));
+  if (!tc::kTmaStore) return true;
+  if (static_cast<int64_t>(g.o_ns) * g.Lq != g.o_rows) return false;
+  TmapKey k;
+  std::memset(&k, 0, sizeof(k));
+  k.ptr = o;
+  k.dims[0] = g.B;
+  k.dims[1] = g.Lq;
+  k.dims[2] = g.o_ns;
+  k.dims[3] = Hq;
+  k.dims[4] = D;
+  k.kind = 6;
+  k.pad = out_bf16 ? 2 : 4;
+  return tmap_cached(k, m, make_out_view);
 }
 
 bool encode_stream_view(CUtensorMap* m, const void* ptr, int B, int Ls, int ns, int H, int D) {
@@ -798,34 +1129,42 @@ static bool fill_params(TcParams& p, void* o, float* lse, const AttnGeom& g, int
     return (e && e[0] == '1') ? 1 : 0;
   }();
   p.stall_first_s = stall;
+  p.rope_tab = nullptr;
+  p.rope_half = 0;
+  p.rope_layout = 0;
   return true;
 }
 
 cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o, float* lse, const AttnGeom& g,
                            int Hq, int Hkv, int D, int W, float scale, bool out_bf16, int32_t* status, int sms,
-                           cudaStream_t st) {
-  CUtensorMap mq;
+                           cudaStream_t st, const float2* rope_tab, int rope_half, int rope_layout) {
+  CUtensorMap mq, mo;
   KvSrc<1> kv;
   if (!encode_stream_view(&mq, q, g.B, g.Lq, g.q_ns, Hq, D) ||
       !encode_stream_view(&kv.k[0], k, g.B, g.Lk, g.kv_ns, Hkv, D) ||
-      !encode_stream_view(&kv.v[0], v, g.B, g.Lk, g.kv_ns, Hkv, D))
+      !encode_stream_view(&kv.v[0], v, g.B, g.Lk, g.kv_ns, Hkv, D) || !encode_out_view(&mo, o, g, Hq, D, out_bf16))
     return cudaErrorInvalidValue;
   TcParams p;
   if (!fill_params(p, o, lse, g, Hq, Hkv, W, scale, out_bf16, status)) return cudaErrorInvalidValue;
   if (p.total_units == 0) return cudaSuccess;
+  if (rope_tab) {
+    if (rope_half < 4 || rope_half > 64 || rope_half % 4 || 2 * rope_half > D ||
+        (rope_layout == HD_ROPE_HALF && rope_half % 8))
+      return cudaErrorInvalidValue;
+    p.rope_tab = rope_tab;
+    p.rope_half = rope_half;
+    p.rope_layout = rope_layout;
+  }
   const int grid = p.total_units < sms ? p.total_units : sms;
   const int smem = attn_tc_smem_bytes(D);
-  cudaError_t err;
-  if (D == 64) {
-    err = cudaFuncSetAttribute(attn_tc_kernel<64, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  auto go = [&](auto kernel) {
+    cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
-    attn_tc_kernel<64, 1><<<grid, tc::kThreads, smem, st>>>(mq, kv, p);
-  } else {
-    err = cudaFuncSetAttribute(attn_tc_kernel<128, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (err != cudaSuccess) return err;
-    attn_tc_kernel<128, 1><<<grid, tc::kThreads, smem, st>>>(mq, kv, p);
-  }
-  return cudaGetLastError();
+    kernel<<<grid, tc::kThreads, smem, st>>>(mq, kv, mo, p);
+    return cudaGetLastError();
+  };
+  if (rope_tab) return D == 64 ? go(attn_tc_kernel<64, 1, true>) : go(attn_tc_kernel<128, 1, true>);
+  return D == 64 ? go(attn_tc_kernel<64, 1>) : go(attn_tc_kernel<128, 1>);
 }
 
 int64_t parts_flag_count(int B, int n, int L) {
@@ -833,8 +1172,8 @@ int64_t parts_flag_count(int B, int n, int L) {
 }
 
 template <int D>
-static cudaError_t launch_parts_kernel(const CUtensorMap& mq, const KvSrc<kPeerMaxRanks>& kv, const TcParams& p,
-                                       int grid, bool cooperative, cudaStream_t st) {
+static cudaError_t launch_parts_kernel(const CUtensorMap& mq, const KvSrc<kPeerMaxRanks>& kv, const CUtensorMap& mo,
+                                       const TcParams& p, int grid, bool cooperative, cudaStream_t st) {
   const int smem = attn_tc_smem_bytes(D);
   cudaError_t err =
       cudaFuncSetAttribute(attn_tc_kernel<D, kPeerMaxRanks>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -849,7 +1188,7 @@ static cudaError_t launch_parts_kernel(const CUtensorMap& mq, const KvSrc<kPeerM
   at[0].val.cooperative = 1;
   cfg.attrs = at;
   cfg.numAttrs = cooperative ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, attn_tc_kernel<D, kPeerMaxRanks>, mq, kv, p);
+  return cudaLaunchKernelEx(&cfg, attn_tc_kernel<D, kPeerMaxRanks>, mq, kv, mo, p);
 }
 
 cudaError_t launch_attn_tc_parts(const void* q, const PartsArgs& a, void* o, float* lse, const AttnGeom& g, int n,
@@ -863,8 +1202,9 @@ cudaError_t launch_attn_tc_parts(const void* q, const PartsArgs& a, void* o, flo
   const int64_t shard_rows = static_cast<int64_t>(nl) * L;
   const bool gather = R > 1 && a.k_dst[0 == a.self ? 1 : 0] != nullptr;
   const bool gself = gather && a.k_dst[a.self] != nullptr && a.v_dst[a.self] != nullptr;
-  CUtensorMap mq;
-  if (!encode_stream_view(&mq, q, g.B, g.Lq, g.q_ns, Hq, D)) return cudaErrorInvalidValue;
+  CUtensorMap mq, mo;
+  if (!encode_stream_view(&mq, q, g.B, g.Lq, g.q_ns, Hq, D) || !encode_out_view(&mo, o, g, Hq, D, out_bf16))
+    return cudaErrorInvalidValue;
   KvSrc<kPeerMaxRanks> kv;
   std::memset(&kv, 0, sizeof(kv));
   PartsInfo& x = kv.x;
@@ -927,8 +1267,20 @@ cudaError_t launch_attn_tc_parts(const void* q, const PartsArgs& a, void* o, flo
   }
   const int grid = p.total_units < sms ? p.total_units : sms;
   // A producer may wait for an item of any CTA: all CTAs must be resident.
-  return D == 64 ? launch_parts_kernel<64>(mq, kv, p, grid, gather, st)
-                 : launch_parts_kernel<128>(mq, kv, p, grid, gather, st);
+  return D == 64 ? launch_parts_kernel<64>(mq, kv, mo, p, grid, gather, st)
+                 : launch_parts_kernel<128>(mq, kv, mo, p, grid, gather, st);
 }
+
+#if HD_TC_TRACE
+// Diagnostic build only: copy (or clear) the per-CTA clock counters.
+extern "C" int hd_tc_trace_fetch(unsigned long long* dst, int count) {
+  if (count > kTraceCtas * kTraceSlots) count = kTraceCtas * kTraceSlots;
+  return static_cast<int>(cudaMemcpyFromSymbol(dst, g_tc_trace, sizeof(unsigned long long) * count));
+}
+extern "C" int hd_tc_trace_clear() {
+  static unsigned long long zeros[kTraceCtas * kTraceSlots];
+  return static_cast<int>(cudaMemcpyToSymbol(g_tc_trace, zeros, sizeof(zeros)));
+}
+#endif
 
 }  // namespace hd

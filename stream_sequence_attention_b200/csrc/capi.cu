@@ -188,6 +188,56 @@ size_t hd_attn_bwd_workspace(int B, int L, int n, int Hq, hd_mode mode) {
   return static_cast<size_t>(2 * bwd_plane(g, Hq)) * sizeof(float);
 }
 
+size_t hd_attn_rope_workspace(int L, int n, int rot_dim) {
+  if (L < 1 || n < 1 || rot_dim < 8 || rot_dim > 128 || rot_dim % 8) return 0;
+  const int64_t P = static_cast<int64_t>(n) * L;
+  if (P > (1ll << 30)) return 0;
+  return static_cast<size_t>(P) * (rot_dim / 2) * sizeof(float2);
+}
+
+hd_status hd_attn_fwd_rope(const void* q, void* k, const void* v, void* o, float* lse, int B, int L, int n, int Hq,
+                           int Hkv, int D, hd_mode mode, int window, float scale, int rot_dim, double base,
+                           hd_rope_layout layout, void* workspace, size_t ws_bytes, hd_dtype in_dt, hd_dtype out_dt,
+                           int32_t* dev_status, void* stream) {
+  hd_status stt = check_attn_args(q, k, v, o, lse, B, L, n, Hq, Hkv, D, mode, window, scale, in_dt, out_dt);
+  if (stt != HD_OK) return stt;
+  if (layout != HD_ROPE_HALF && layout != HD_ROPE_INTERLEAVED) return HD_ERR_INVALID_ARG;
+  if (rot_dim < 8 || rot_dim > D || rot_dim % (layout == HD_ROPE_HALF ? 16 : 8)) return HD_ERR_INVALID_ARG;
+  if (!std::isfinite(base) || !(base > 0.0)) return HD_ERR_INVALID_ARG;
+  if (in_dt != HD_BF16) return HD_ERR_UNSUPPORTED;
+  if (B == 0) return HD_OK;
+  const size_t need = hd_attn_rope_workspace(L, n, rot_dim);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || need == 0 || ws_bytes < need)
+    return HD_ERR_INVALID_ARG;
+  const int sms = sm_count();
+  if (sms <= 0) return HD_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t P = static_cast<int64_t>(n) * L;
+  RopeParams rp;
+  std::memset(&rp, 0, sizeof(rp));
+  rp.q = nullptr;
+  rp.k = k;
+  rp.pos0 = nullptr;
+  rp.B = B;
+  rp.P = static_cast<int>(P);
+  rp.Hq = 0;
+  rp.Hkv = Hkv;
+  rp.D = D;
+  rp.rot = rot_dim;
+  rp.layout = layout;
+  rp.pos_base = 0;
+  rp.pos_mult = 0;
+  rope_fill_turns(rp, rot_dim, base);
+  float2* tab = static_cast<float2*>(workspace);
+  // cos/sin of every position once; k rotated in place (what a cache of
+  // this layer keeps); the query rows rotated inside the attention kernel.
+  if (launch_rope_table(rp, P, tab, st) != cudaSuccess || launch_rope(rp, true, st) != cudaSuccess)
+    return HD_ERR_CUDA;
+  const AttnGeom g = regular_geom(B, L, n, mode);
+  return cuda_status(launch_attn_tc(q, k, v, o, lse, g, Hq, Hkv, D, window, scale, out_dt == HD_BF16, dev_status,
+                                    sms, st, tab, rot_dim / 2, layout));
+}
+
 static hd_status run_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
                               const float* lse, void* dq, void* dk, void* dv, const AttnGeom& g, int Hq, int Hkv,
                               int D, int window, float scale, hd_dtype dt, void* workspace, size_t ws_bytes,
@@ -517,13 +567,7 @@ hd_status hd_rope(void* q, void* k, const int32_t* pos0, int B, int P, int Hq, i
   p.layout = layout;
   p.pos_base = pos_base;
   p.pos_mult = pos_mult;
-  // theta_j / (2 pi) in turns, as a 64-bit binary fraction (long double:
-  // 64-bit mantissa); theta_j <= 1 so the fraction is below 1/(2 pi).
-  const long double two_pi = 6.283185307179586476925286766559005768L;
-  for (int j = 0; j < rot_dim / 2; ++j) {
-    const long double turns = powl(static_cast<long double>(base), -2.0L * j / rot_dim) / two_pi;
-    p.fturn[j] = static_cast<uint64_t>(ldexpl(turns, 64));
-  }
+  rope_fill_turns(p, rot_dim, base);
   return cuda_status(launch_rope(p, dt == HD_BF16, static_cast<cudaStream_t>(stream)));
 }
 

@@ -1,0 +1,72 @@
+"""Per-role clock counters of the tcgen05 attention kernel (diagnostic).
+
+    python -m stream_sequence_attention_b200.diag_trace [--mode intra|cross] [-D SWITCH=VALUE ...]
+
+Builds a diagnostic copy of the library with ``-DHD_TC_TRACE=1`` (plus any
+extra switches) next to libhd.so as ``libhd_trace.so``, runs one forward
+call of the bench's prefill workload (n=4, L=4096, B=2, 32q/8kv, D=128,
+bf16) after three warm-up calls, and prints, averaged over the CTAs, the
+cycles per tile each softmax warpgroup spends waiting for its scores, in the
+score load and row max, in the exponentials up to publishing P, in the row
+sum, and in the epilogue, and the MMA issuer's cycles waiting for P and for
+its Q/K/V/O stages.  The counters perturb the kernel (clock reads and a few
+more registers): compare them with each other, not with the timed build.
+"""
+
+from __future__ import annotations
+
+import argparse
+import ctypes
+import os
+
+import numpy as np
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--mode", default="intra", choices=["intra", "cross"])
+    ap.add_argument("-D", dest="defines", action="append", default=[])
+    a = ap.parse_args()
+    import torch
+
+    from stream_sequence_attention_b200 import build, hd, synth
+
+    out = os.path.join(os.path.dirname(build.LIB), "libhd_trace.so")
+    build.build(extra=["-DHD_TC_TRACE=1"] + [f"-D{d}" for d in a.defines], out=out)
+    hd.LIB_PATH = out
+    hd._lib = None
+    L = hd.lib()
+    L.hd_tc_trace_fetch.argtypes = [ctypes.c_void_p, ctypes.c_int]
+    B, n, Lt, Hq, Hkv, D = 2, 4, 4096, 32, 8, 128
+    P = n * Lt
+    q = synth.normal_device((B, P, Hq, D), 1)
+    k = synth.normal_device((B, P, Hkv, D), 2)
+    v = synth.normal_device((B, P, Hkv, D), 3)
+    o = torch.empty_like(q)
+    for _ in range(3):
+        hd.hd_attn_fwd(q, k, v, n, a.mode, out=o)
+    torch.cuda.synchronize()
+    L.hd_tc_trace_clear()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    hd.hd_attn_fwd(q, k, v, n, a.mode, out=o)
+    e1.record()
+    torch.cuda.synchronize()
+    slots = 20
+    buf = (ctypes.c_ulonglong * (1024 * slots))()
+    L.hd_tc_trace_fetch(buf, 1024 * slots)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    c = np.frombuffer(buf, dtype=np.uint64).reshape(1024, slots)[:sms].astype(np.float64)
+    print(f"{a.mode}: {e0.elapsed_time(e1):.3f} ms (trace build), {sms} CTAs")
+    print(f"  MMA issuer per CTA: waiting for P {c[:, 12].mean() / 1e6:.3f} M clk, for Q/K/V/O "
+          f"{c[:, 13].mean() / 1e6:.3f} M clk, total {c[:, 14].mean() / 1e6:.3f} M clk")
+    names = ["wait for S", "load + max", "exp -> P published", "row sum", "epilogue"]
+    for sl in (0, 1):
+        tiles = c[:, sl * 6 + 5].sum()
+        per = [c[:, sl * 6 + i].sum() / tiles for i in range(5)]
+        print(f"  softmax slot {sl}: {tiles / sms:.1f} tiles per CTA; clk per tile: " +
+              ", ".join(f"{nm} {x:.0f}" for nm, x in zip(names, per)))
+
+
+if __name__ == "__main__":
+    main()

@@ -143,6 +143,34 @@ def test_attn_fwd_matches_oracle(hd, dtype, B, n, L, Hq, Hkv, D, mode, W, out_f3
     assert int(st.item()) == 0
 
 
+@pytest.mark.parametrize("mode,W,n", [("intra", 0, 4), ("cross", 0, 4), ("intra", 150, 2), ("cross", 300, 2),
+                                      ("intra", 0, 1)])
+@pytest.mark.parametrize("out_f32", [False, True])
+def test_running_max_jumps(hd, mode, W, n, out_f32):
+    """Keys whose scores grow tile after tile, so a row's maximum rises by far
+    more than 2^8 (the kernel's rescale threshold, in log2 units) several
+    times within a unit: the rows that jump redo their exponentials against
+    the new maximum and rescale O.  Some rows see their first key tile fully
+    masked (windows), so their maximum starts at -inf."""
+    B, L, Hq, Hkv, D = 1, 700, 4, 2, 128
+    P = n * L
+    q, k, v = host_qkv(B, P, Hq, Hkv, D, 77, "bf16")
+    q = synth.bf16_round(np.abs(q).astype(np.float32) * np.float32(0.5))
+    # key j's features grow with its position: scores rise ~linearly along the
+    # sequence, a tile of 128 keys later by ~10 log2 units or more
+    grow = (1.0 + np.arange(P, dtype=np.float32) / 40.0)[None, :, None, None]
+    k = synth.bf16_round(np.abs(k).astype(np.float32) * grow * np.float32(0.25))
+    st = hd.new_status()
+    o, lse = hd.hd_attn_fwd(dev(q, "bf16"), dev(k, "bf16"), dev(v, "bf16"), n, mode, W,
+                            out_dtype=torch.float32 if out_f32 else None, lse=True, dev_status=st)
+    torch.cuda.synchronize()
+    ro, rl = oracle.attn(q, k, v, n, mode, W)
+    assert np.isfinite(to_f64(o)).all()
+    assert max_abs(to_f64(o), ro) <= TOL_BF16
+    assert max_abs(to_f64(lse), rl) <= 1e-3 * max(1.0, float(np.abs(rl).max()))
+    assert int(st.item()) == 0
+
+
 @pytest.mark.parametrize("dtype,mode,W", [("bf16", "intra", 0), ("bf16", "cross", 0), ("bf16", "intra", 60),
                                           ("bf16", "cross", 90), ("f32", "intra", 0), ("f32", "cross", 33)])
 def test_masked_keys_do_not_change_output_bits(hd, dtype, mode, W):
