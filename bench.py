@@ -737,15 +737,14 @@ def extras(torch, peaks, rank):
     rk = synth.normal_device((B, P, c["Hkv"], c["D"]), 7702 + rank)
     rv = synth.normal_device((B, P, c["Hkv"], c["D"]), 7703 + rank)
     ro = torch.empty_like(rq)
-    rws = torch.empty(hd.hd_attn_rope_workspace(c["L"], c["n"], c["D"]), dtype=torch.uint8, device="cuda")
     ms_sep = time_fn(lambda: (hd.hd_rope(rq, rk), hd.hd_attn_fwd(rq, rk, rv, c["n"], "intra", out=ro)))
-    ms_fused = time_fn(lambda: hd.hd_attn_fwd_rope(rq, rk, rv, c["n"], "intra", out=ro, workspace=rws))
+    ms_fused = time_fn(lambda: hd.hd_attn_fwd_rope(rq, rk, rv, c["n"], "intra", out=ro))
     fl = acc.attn_flops(B, c["L"], c["n"], c["Hq"], c["D"], "intra", 0)
     res["rope_fused_intra"] = {"separate_ms": round(ms_sep, 3), "fused_ms": round(ms_fused, 3),
                                "fused_attn_TFLOP/s": round(fl / (ms_fused * 1e-3) / 1e12, 1),
                                "note": "separate = hd_rope(q, k) + hd_attn_fwd; fused = hd_attn_fwd_rope "
-                                       "(table + rope(k) + attention with q rotated in the kernel)"}
-    del rq, rk, rv, ro, rws
+                                       "(rope(k) + attention with q rotated in the kernel)"}
+    del rq, rk, rv, ro
     torch.cuda.empty_cache()
     rp = Rope(WORKLOADS["rope"], 7401 + rank, torch, hd, synth)
     ms = time_fn(lambda: rp.step())

@@ -448,27 +448,24 @@ hd_status hd_rope(void* q, void* k, const int32_t* pos0, int B, int P, int Hq,
  * with rope as hd_rope at the contiguous positions of the expanded sequence
  * (row p of a sequence at position p = i*n + s; pos_base = 0, pos_mult = 0).
  *   q     [B, n*L, Hq, D]  bf16, read only: its rows are rotated inside the
- *                          attention kernel, as its tiles arrive, and never
- *                          written back
+ *                          attention kernel, in the tile, and never written
+ *                          back
  *   k     [B, n*L, Hkv, D] bf16, rotated IN PLACE (on return k holds rope(k),
  *                          the keys a cache of this layer keeps)
  *   v, o, lse, mode, window, scale: as hd_attn_fwd (out_dt bf16 or f32)
  *   rot_dim, base, layout: as hd_rope; rot_dim <= D, and a multiple of 16
  *                          (HD_ROPE_HALF) or of 8 (HD_ROPE_INTERLEAVED)
- *   workspace: device scratch of at least hd_attn_rope_workspace(L, n,
- *              rot_dim) bytes (the cos/sin table of the n*L positions),
- *              256-byte aligned, owned by the caller, no initialisation
- *              needed, dead after the call completes.
- * in_dt must be HD_BF16 (HD_ERR_UNSUPPORTED otherwise).  Three launches on
- * `stream`: the cos/sin table, the rotation of k, the attention.
+ * in_dt must be HD_BF16 (HD_ERR_UNSUPPORTED otherwise).  Two launches on
+ * `stream`: the rotation of k, then the attention.  The angles are reduced
+ * exactly as in hd_rope; the query rows' cos/sin are evaluated in float32 on
+ * the special-function unit (absolute error about 1e-6), so q's rotation can
+ * differ from hd_rope's in the last bit of a bf16 value.
  */
-size_t hd_attn_rope_workspace(int L, int n, int rot_dim);
 hd_status hd_attn_fwd_rope(const void* q, void* k, const void* v, void* o,
                            float* lse, int B, int L, int n, int Hq, int Hkv, int D,
                            hd_mode mode, int window, float scale, int rot_dim,
-                           double base, hd_rope_layout layout, void* workspace,
-                           size_t ws_bytes, hd_dtype in_dt, hd_dtype out_dt,
-                           int32_t* dev_status, void* stream);
+                           double base, hd_rope_layout layout, hd_dtype in_dt,
+                           hd_dtype out_dt, int32_t* dev_status, void* stream);
 
 /*
  * Final-stream gather ("Multi-Stream Expansion and Training Objective": only

@@ -65,6 +65,19 @@ constexpr int kThreads = 32 * (9 + kIssuers);
 constexpr int kWarpTMA = 8;
 constexpr int kWarpMMA = 9;
 constexpr int kWarpGather = 9 + kIssuers;  // rank-shard form with gather only
+// The MMA issuer's loop runs on all 32 lanes of its warp, one elected lane
+// issuing each MMA and commit (1), or on lane 0 alone (0).
+#ifndef HD_TC_MMA_WARP
+#define HD_TC_MMA_WARP 1
+#endif
+constexpr bool kMmaWarp = HD_TC_MMA_WARP != 0;
+// L2 policies on the TMA copies (1): K/V tiles, read again by every later
+// query block of their group, kept (evict_last); Q tiles and the O stores,
+// touched once, streamed (evict_first).  0: no policy.
+#ifndef HD_TC_L2HINT
+#define HD_TC_L2HINT 0
+#endif
+constexpr bool kL2Hint = HD_TC_L2HINT != 0;
 constexpr int VST = 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -140,11 +153,13 @@ struct TcParams {
   int out_bf16;
   int nqb, npairs;
   int total_units;
-  // Rotary embedding of the query rows inside the kernel (nullptr: q is
-  // used as given).  rope_tab[pos * rope_half + j] = (cos, sin) of
-  // pos * theta_j for positions pos = i * q_ns + s of the expanded sequence.
-  const float2* rope_tab;
+  // Rotary embedding of the query rows inside the kernel (the ROPE
+  // instantiation): rope_half pairs in layout rope_layout (hd_rope_layout),
+  // rope_fturn[j] = theta_j / (2 pi) as a 64-bit fixed-point fraction of a
+  // turn; query (i, s) sits at position i * q_ns + s of the expanded
+  // sequence.
   int rope_half, rope_layout;
+  uint64_t rope_fturn[kRopeMaxPairs / 2];
   // Test hook (environment HD_TEST_STALL_FIRST_S=1): the MMA warp of CTA 0
   // never signals its first S tile, so the softmax wait runs out and the
   // kernel must take its timeout path.  0 in normal use.
@@ -316,68 +331,68 @@ __device__ __forceinline__ void gather_items(const PartsInfo& x, int B, int lane
   }
 }
 
+// cos and sin of pos * theta_j: pos * fturn mod 2^64 is the angle's
+// fraction of a turn (exact); its top 32 bits as a signed fraction t in
+// [-1/2, 1/2) give the angle 2 pi t, whose sine and cosine come from the MUFU
+// unit (absolute error about 1e-6, far below the bf16 rounding of the row).
+__device__ __forceinline__ float2 rope_cos_sin(int64_t pos, uint64_t fturn) {
+  const uint64_t turns = static_cast<uint64_t>(pos) * fturn;
+  const float a = static_cast<float>(static_cast<int32_t>(turns >> 32)) * (6.28318530717958647692f * 0x1p-32f);
+  float sn, cn;
+  asm("sin.approx.f32 %0, %1;" : "=f"(sn) : "f"(a));
+  asm("cos.approx.f32 %0, %1;" : "=f"(cn) : "f"(a));
+  return make_float2(cn, sn);
+}
+
 // Rotary embedding of one query row in place in a 128-byte-swizzled Q tile
-// (row r at qrow; 64-feature blocks blk bytes apart): pairs (j, j + half) or
-// (2j, 2j + 1), j < half, (a, b) -> (a cos - b sin, a sin + b cos) with
-// (cos, sin) of pair j at t4[j / 2] (two pairs per float4).
-__device__ __forceinline__ void rope_rotate_row(uint8_t* qrow, int blk, int r, const float4* t4, int half,
-                                             int layout) {
-  // 16-byte unit holding features f .. f+7 (f a multiple of 8) of the
-  // row: 128-byte swizzle within each 64-feature block.
+// (row r at qrow; 64-feature blocks blk bytes apart), row position pos:
+// pairs (j, j + half) or (2j, 2j + 1), j < half, (a, b) -> (a cos - b sin,
+// a sin + b cos) at the angle pos * theta_j.
+template <int NP>
+__device__ __forceinline__ void rope_rotate_row(uint8_t* qrow, int blk, int r, int64_t pos, int half, int layout,
+                                                const uint64_t (&fturn)[NP]) {
+  // 16-byte unit holding features f .. f+7 (f a multiple of 8) of the row:
+  // 128-byte swizzle within each 64-feature block.
   auto unit = [&](int f) -> uint4* {
     return reinterpret_cast<uint4*>(qrow + (f >> 6) * blk + ((((f & 63) >> 3) ^ (r & 7)) << 4));
   };
-#pragma unroll 1
-  for (int qtr = 0; qtr < 4; ++qtr) {
-    float4 cs[8];
+  if (layout == HD_ROPE_HALF) {
+    // pairs (j, j + half): the units at features j = 8v and j + half
 #pragma unroll
-    for (int c = 0; c < 8; ++c)
-      if (16 * qtr + 2 * c < half) cs[c] = __ldg(t4 + 8 * qtr + c);
-    // pair 16*qtr + j of this quarter
-    auto cs_of = [&](int j) -> float2 {
-      const float4 c4 = cs[j >> 1];
-      return (j & 1) ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y);
-    };
-    if (16 * qtr >= half) {
-    } else if (layout == HD_ROPE_HALF) {
-      // pairs (j, j + half), (a, b) -> (a cos - b sin, a sin + b cos):
-      // the units at features j and j + half, j = 16*qtr + 8w
+    for (int v = 0; v < NP / 8; ++v) {
+      if (8 * v < half) {
+        uint4* pa = unit(8 * v);
+        uint4* pb = unit(8 * v + half);
+        const uint4 ua = *pa, ub = *pb;
+        uint32_t wa[4] = {ua.x, ua.y, ua.z, ua.w}, wb[4] = {ub.x, ub.y, ub.z, ub.w};
 #pragma unroll
-      for (int w = 0; w < 2; ++w) {
-        const int f = 16 * qtr + 8 * w;
-        if (f < half) {
-          uint4* pa = unit(f);
-          uint4* pb = unit(f + half);
-          const uint4 ua = *pa, ub = *pb;
-          uint32_t wa[4] = {ua.x, ua.y, ua.z, ua.w}, wb[4] = {ub.x, ub.y, ub.z, ub.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 fa = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wa[e]));
-            const float2 fb = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wb[e]));
-            const float2 t0 = cs_of(8 * w + 2 * e), t1 = cs_of(8 * w + 2 * e + 1);
-            wa[e] = pack_bf16x2(fmaf(fa.x, t0.x, -fb.x * t0.y), fmaf(fa.y, t1.x, -fb.y * t1.y));
-            wb[e] = pack_bf16x2(fmaf(fa.x, t0.y, fb.x * t0.x), fmaf(fa.y, t1.y, fb.y * t1.x));
-          }
-          *pa = make_uint4(wa[0], wa[1], wa[2], wa[3]);
-          *pb = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+        for (int e = 0; e < 4; ++e) {
+          const float2 fa = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wa[e]));
+          const float2 fb = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wb[e]));
+          const float2 t0 = rope_cos_sin(pos, fturn[8 * v + 2 * e]);
+          const float2 t1 = rope_cos_sin(pos, fturn[8 * v + 2 * e + 1]);
+          wa[e] = pack_bf16x2(fmaf(fa.x, t0.x, -fb.x * t0.y), fmaf(fa.y, t1.x, -fb.y * t1.y));
+          wb[e] = pack_bf16x2(fmaf(fa.x, t0.y, fb.x * t0.x), fmaf(fa.y, t1.y, fb.y * t1.x));
         }
+        *pa = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+        *pb = make_uint4(wb[0], wb[1], wb[2], wb[3]);
       }
-    } else {
-      // pairs (2j, 2j + 1): unit 4*qtr + w holds pairs 16*qtr + 4w .. + 3
+    }
+  } else {
+    // pairs (2j, 2j + 1): the unit at feature 8v holds pairs 4v .. 4v + 3
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        if (16 * qtr + 4 * w < half) {
-          uint4* pa = unit(32 * qtr + 8 * w);
-          const uint4 ua = *pa;
-          uint32_t wa[4] = {ua.x, ua.y, ua.z, ua.w};
+    for (int v = 0; v < NP / 4; ++v) {
+      if (4 * v < half) {
+        uint4* pa = unit(8 * v);
+        const uint4 ua = *pa;
+        uint32_t wa[4] = {ua.x, ua.y, ua.z, ua.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 fa = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wa[e]));
-            const float2 t = cs_of(4 * w + e);
-            wa[e] = pack_bf16x2(fmaf(fa.x, t.x, -fa.y * t.y), fmaf(fa.x, t.y, fa.y * t.x));
-          }
-          *pa = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+        for (int e = 0; e < 4; ++e) {
+          const float2 fa = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wa[e]));
+          const float2 t = rope_cos_sin(pos, fturn[4 * v + e]);
+          wa[e] = pack_bf16x2(fmaf(fa.x, t.x, -fa.y * t.y), fmaf(fa.x, t.y, fa.y * t.x));
         }
+        *pa = make_uint4(wa[0], wa[1], wa[2], wa[3]);
       }
     }
   }
@@ -456,7 +471,8 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
     report(p.status, HD_ERR_TIMEOUT);
   };
   // One 128-key tile of K or V into the stage at `dst`.
-  auto load_kv_tile = [&](const CUtensorMap* maps, uint32_t dst, uint32_t full, const TcUnit& x, int skv, int kt) {
+  auto load_kv_tile = [&](const CUtensorMap* maps, uint32_t dst, uint32_t full, const TcUnit& x, int skv, int kt,
+                          uint64_t pol) {
     if constexpr (kParts) {
       if (kv.x.stacked) {
         // One box covers the tile's rows of every rank, rank-major.
@@ -475,8 +491,12 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
       }
     } else {
 #pragma unroll
-      for (int kb = 0; kb < Lay::KB; ++kb)
-        tma_load_5d(dst + kb * Lay::BLK, &maps[0], full, kb * 64, x.kvh, skv, kt * tc::BN, x.b);
+      for (int kb = 0; kb < Lay::KB; ++kb) {
+        if constexpr (tc::kL2Hint)
+          tma_load_5d_hint(dst + kb * Lay::BLK, &maps[0], full, kb * 64, x.kvh, skv, kt * tc::BN, x.b, pol);
+        else
+          tma_load_5d(dst + kb * Lay::BLK, &maps[0], full, kb * 64, x.kvh, skv, kt * tc::BN, x.b);
+      }
     }
   };
 
@@ -485,6 +505,15 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
   if (warp == tc::kWarpTMA) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      const uint64_t pol_keep = tc::kL2Hint ? l2_policy_evict_last() : 0;
+      const uint64_t pol_once = tc::kL2Hint ? l2_policy_evict_first() : 0;
+      auto load = [&](uint32_t dst, const CUtensorMap* m, uint32_t b, int c0, int c1, int c2, int c3, int c4,
+                      uint64_t pol) {
+        if constexpr (tc::kL2Hint)
+          tma_load_5d_hint(dst, m, b, c0, c1, c2, c3, c4, pol);
+        else
+          tma_load_5d(dst, m, b, c0, c1, c2, c3, c4);
+      };
       int t = 0, ul = 0, q_issued = 0;
       int k_issued[Lay::KST] = {}, v_issued[tc::VST] = {};
       bool ok = true;
@@ -497,11 +526,11 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
         mbar_arrive_expect_tx(bar(Lay::B_QFULL), Lay::TILE * (x.h1 >= 0 ? 2 : 1));
 #pragma unroll
         for (int kb = 0; kb < Lay::KB; ++kb) {
-          tma_load_5d(sbase + Lay::Q_OFF + kb * Lay::BLK, &tmQ, bar(Lay::B_QFULL), kb * 64, x.h0, x.s,
-                      x.qblk * tc::BM, x.b);
+          load(sbase + Lay::Q_OFF + kb * Lay::BLK, &tmQ, bar(Lay::B_QFULL), kb * 64, x.h0, x.s, x.qblk * tc::BM,
+               x.b, pol_once);
           if (x.h1 >= 0)
-            tma_load_5d(sbase + Lay::Q_OFF + Lay::TILE + kb * Lay::BLK, &tmQ, bar(Lay::B_QFULL), kb * 64,
-                        x.h1, x.s, x.qblk * tc::BM, x.b);
+            load(sbase + Lay::Q_OFF + Lay::TILE + kb * Lay::BLK, &tmQ, bar(Lay::B_QFULL), kb * 64, x.h1, x.s,
+                 x.qblk * tc::BM, x.b, pol_once);
         }
         ++q_issued;
         const int skv = p.g.kv_stream >= 0 ? p.g.kv_stream : x.s;
@@ -517,12 +546,12 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
           const int ks = t % Lay::KST;
           if (!mbar_wait(bar(Lay::B_KEMPTY + ks), ((t / Lay::KST) & 1) ^ 1, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(bar(Lay::B_KFULL + ks), Lay::TILE);
-          load_kv_tile(kv.k, sbase + Lay::K_OFF + ks * Lay::TILE, bar(Lay::B_KFULL + ks), x, skv, kt);
+          load_kv_tile(kv.k, sbase + Lay::K_OFF + ks * Lay::TILE, bar(Lay::B_KFULL + ks), x, skv, kt, pol_keep);
           ++k_issued[ks];
           const int vs = t % tc::VST;
           if (!mbar_wait(bar(Lay::B_VEMPTY + vs), ((t / tc::VST) & 1) ^ 1, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(bar(Lay::B_VFULL + vs), Lay::TILE);
-          load_kv_tile(kv.v, sbase + Lay::V_OFF + vs * Lay::TILE, bar(Lay::B_VFULL + vs), x, skv, kt);
+          load_kv_tile(kv.v, sbase + Lay::V_OFF + vs * Lay::TILE, bar(Lay::B_VFULL + vs), x, skv, kt, pol_keep);
           ++v_issued[vs];
         }
         ++ul;
@@ -545,7 +574,27 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
     // from one thread executes in issue order, so PV_h(t) has read P_h(t) by
     // then.  Each issuer releases every Q/K/V stage once (its commit, or a
     // plain arrive when it has no head in the unit).
-    if (lane == 0) {
+    if (tc::kMmaWarp || lane == 0) {
+      // One lane issues (the loop on lane 0, or the whole warp's loop with an
+      // elected lane per MMA and commit).
+      auto mma_s = [&](uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+        if constexpr (tc::kMmaWarp)
+          mma_ss_elect(d, a, b, id, acc);
+        else
+          mma_ss(d, a, b, id, acc);
+      };
+      auto mma_t = [&](uint32_t d, uint32_t a, uint64_t b, uint32_t id, uint32_t acc) {
+        if constexpr (tc::kMmaWarp)
+          mma_ts_elect(d, a, b, id, acc);
+        else
+          mma_ts(d, a, b, id, acc);
+      };
+      auto commit = [&](uint32_t b) {
+        if constexpr (tc::kMmaWarp)
+          tc_commit_elect(b);
+        else
+          tc_commit(b);
+      };
       constexpr uint32_t idS = idesc_bf16_f32(tc::BM, tc::BN, false, false);
       constexpr uint32_t idO = idesc_bf16_f32(tc::BM, D, false, true);
       const int me = warp - tc::kWarpMMA;  // issuer index
@@ -556,16 +605,16 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off16 = ((kk >> 2) * Lay::BLK + (kk & 3) * 32) >> 4;
-          mma_ss(tmem + h * 128, qd + off16, kd + off16, idS, kk > 0 ? 1u : 0u);
+          mma_s(tmem + h * 128, qd + off16, kd + off16, idS, kk > 0 ? 1u : 0u);
         }
-        if (!(p.stall_first_s && blockIdx.x == 0)) tc_commit(bar(Lay::B_SFULL + h));
+        if (!(p.stall_first_s && blockIdx.x == 0)) commit(bar(Lay::B_SFULL + h));
       };
       auto issue_PV = [&](int h, int vst, bool acc) {
         // V tile is MN-major (D contiguous): 16 keys = 16 rows of 128 B.
         const uint64_t vd = smem_desc_sw128(sbase + Lay::V_OFF + vst * Lay::TILE, Lay::BLK, 1024);
 #pragma unroll
         for (int kk = 0; kk < tc::BN / 16; ++kk)
-          mma_ts(tmem + 256 + h * 128, tmem + h * 128 + kk * 8, vd + ((kk * 2048) >> 4), idO,
+          mma_t(tmem + 256 + h * 128, tmem + h * 128 + kk * 8, vd + ((kk * 2048) >> 4), idO,
                  (acc || kk > 0) ? 1u : 0u);
       };
       int t = 0, ul = 0;
@@ -596,8 +645,8 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
         const bool mine = h_hi > h_lo;
         auto release = [&](uint32_t b) {
           if (mine)
-            tc_commit(b);
-          else
+            commit(b);
+          else if (lane == 0)
             mbar_arrive(b);
         };
         const int nt = x.t_hi - x.t_lo + 1;
@@ -643,7 +692,7 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
               }
               issue_S(h, ksn);
             } else {
-              tc_commit(bar(Lay::B_ODONE + h));
+              commit(bar(Lay::B_ODONE + h));
             }
           }
           if (!ok) break;
@@ -658,11 +707,11 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
       }
       if (!ok) fail();
       // Drain: every MMA issued above has completed before TMEM is freed.
-      tc_commit(bar(Lay::B_DRAIN));
+      commit(bar(Lay::B_DRAIN));
       mbar_wait(bar(Lay::B_DRAIN), 0, no_abort);
 #if HD_TC_TRACE
       mw[2] = static_cast<unsigned long long>(clock64() - mt0);
-      if (blockIdx.x < kTraceCtas)
+      if (blockIdx.x < kTraceCtas && lane == 0)
         for (int c = 0; c < 3; ++c) g_tc_trace[blockIdx.x * kTraceSlots + 12 + 3 * me + c] = mw[c];
 #endif
     }
@@ -695,6 +744,23 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
       }
     };
     int uall = 0;  // units of this CTA so far (phases of B_QFULL)
+    int rot_done = -1;  // unit slot k whose query rows this warpgroup rotated ahead
+    // ROPE: rotate this thread's query row of unit xr (the uq-th unit of the
+    // CTA, B_QFULL phase uq & 1) in the Q tile, then publish the tile to the
+    // MMA issuer ("Multi-Stream Expansion and Training Objective": contiguous
+    // positions over the expanded sequence).
+    auto rotate_q = [&](const TcUnit& xr, int uq) -> bool {
+      const bool got = mbar_wait(bar(Lay::B_QFULL), uq & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) return false;
+      const int ir = xr.qblk * tc::BM + r;
+      if (ir < p.g.Lq)
+        rope_rotate_row(smem + Lay::Q_OFF + slot * Lay::TILE + r * 128, Lay::BLK, r,
+                        static_cast<int64_t>(ir) * p.g.q_ns + xr.s, p.rope_half, p.rope_layout, p.rope_fturn);
+      // The tensor core reads the tile through the async proxy.
+      fence_proxy_async_smem();
+      mbar_arrive(bar(Lay::B_QROT + slot));
+      return true;
+    };
     for (int k = 0; ok; ++k) {
       const int u = tc_unit_of(k, p.total_units);
       if (u == -1) break;
@@ -713,21 +779,11 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
       float m = -INFINITY, l = 0.f;
       const int nt = x.t_hi - x.t_lo + 1;
       if constexpr (ROPE) {
-        // Rotary embedding of this thread's query row, in the Q tile itself
-        // (position i*q_ns + s; "Multi-Stream Expansion and Training
-        // Objective": contiguous positions over the expanded sequence).  The
-        // cos/sin pairs are fetched before the tile lands.
-        const bool rok = i < p.g.Lq;
-        const int half = p.rope_half;
-        // (cos, sin) pairs of the row, 16 pairs (8 float4) at a time.
-        const float4* t4 =
-            reinterpret_cast<const float4*>(p.rope_tab + (static_cast<int64_t>(i) * p.g.q_ns + x.s) * half);
-        const bool got = mbar_wait(bar(Lay::B_QFULL), ucur & 1, abort_flag);
-        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-        if (rok) rope_rotate_row(smem + Lay::Q_OFF + slot * Lay::TILE + r * 128, Lay::BLK, r, t4, half, p.rope_layout);
-        // The tensor core reads the tile through the async proxy.
-        fence_proxy_async_smem();
-        mbar_arrive(bar(Lay::B_QROT + slot));
+        // Rotated ahead at the end of the previous unit, or now.
+        if (rot_done != k && !rotate_q(x, ucur)) {
+          ok = false;
+          break;
+        }
       }
       for (int jj = 0; jj < nt; ++jj, ++sc) {
         const int k0 = (x.t_lo + jj) * tc::BN;
@@ -843,6 +899,26 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
         mbar_arrive(bar(Lay::B_PFULL + slot));
         tick(2);
         l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+        if constexpr (ROPE) {
+          // After the unit's last P: rotate the next unit's query rows while
+          // the tensor core runs this unit's last P V, so that the next S can
+          // start right behind it.  Q(next) is on its way: the last S of this
+          // unit has released the tile.
+          if (jj == nt - 1) {
+            int k2 = k + 1, u2;
+            while ((u2 = tc_unit_of(k2, p.total_units)) == -2) ++k2;
+            if (u2 >= 0) {
+              const TcUnit x2 = tc_unit(u2, p);
+              if ((slot ? x2.h1 : x2.h0) >= 0) {
+                if (!rotate_q(x2, uall)) {
+                  ok = false;
+                  break;
+                }
+                rot_done = k2;
+              }
+            }
+          }
+        }
         tick(3);
         if (tc::kTrace) ++tr[5];
       }
@@ -874,7 +950,11 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0 && row0 < p.g.Lq) {
-            tma_store_5d(&tmO, stg_s, chunk * (p.out_bf16 ? 64 : 32), h, x.s, row0, x.b);
+            if constexpr (tc::kL2Hint)
+              tma_store_5d_hint(&tmO, stg_s, chunk * (p.out_bf16 ? 64 : 32), h, x.s, row0, x.b,
+                                l2_policy_evict_first());
+            else
+              tma_store_5d(&tmO, stg_s, chunk * (p.out_bf16 ? 64 : 32), h, x.s, row0, x.b);
             bulk_commit_group();
             stored = true;
           }
@@ -1129,7 +1209,6 @@ static bool fill_params(TcParams& p, void* o, float* lse, const AttnGeom& g, int
     return (e && e[0] == '1') ? 1 : 0;
   }();
   p.stall_first_s = stall;
-  p.rope_tab = nullptr;
   p.rope_half = 0;
   p.rope_layout = 0;
   return true;
@@ -1137,7 +1216,7 @@ static bool fill_params(TcParams& p, void* o, float* lse, const AttnGeom& g, int
 
 cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o, float* lse, const AttnGeom& g,
                            int Hq, int Hkv, int D, int W, float scale, bool out_bf16, int32_t* status, int sms,
-                           cudaStream_t st, const float2* rope_tab, int rope_half, int rope_layout) {
+                           cudaStream_t st, const RopeParams* rope) {
   CUtensorMap mq, mo;
   KvSrc<1> kv;
   if (!encode_stream_view(&mq, q, g.B, g.Lq, g.q_ns, Hq, D) ||
@@ -1147,13 +1226,14 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o,
   TcParams p;
   if (!fill_params(p, o, lse, g, Hq, Hkv, W, scale, out_bf16, status)) return cudaErrorInvalidValue;
   if (p.total_units == 0) return cudaSuccess;
-  if (rope_tab) {
-    if (rope_half < 4 || rope_half > 64 || rope_half % 4 || 2 * rope_half > D ||
-        (rope_layout == HD_ROPE_HALF && rope_half % 8))
+  if (rope) {
+    const int half = rope->rot / 2;
+    if (half < 4 || half > kRopeMaxPairs / 2 || half % 4 || 2 * half > D ||
+        (rope->layout == HD_ROPE_HALF && half % 8))
       return cudaErrorInvalidValue;
-    p.rope_tab = rope_tab;
-    p.rope_half = rope_half;
-    p.rope_layout = rope_layout;
+    p.rope_half = half;
+    p.rope_layout = rope->layout;
+    for (int j = 0; j < half; ++j) p.rope_fturn[j] = rope->fturn[j];
   }
   const int grid = p.total_units < sms ? p.total_units : sms;
   const int smem = attn_tc_smem_bytes(D);
@@ -1163,7 +1243,7 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o,
     kernel<<<grid, tc::kThreads, smem, st>>>(mq, kv, mo, p);
     return cudaGetLastError();
   };
-  if (rope_tab) return D == 64 ? go(attn_tc_kernel<64, 1, true>) : go(attn_tc_kernel<128, 1, true>);
+  if (rope) return D == 64 ? go(attn_tc_kernel<64, 1, true>) : go(attn_tc_kernel<128, 1, true>);
   return D == 64 ? go(attn_tc_kernel<64, 1>) : go(attn_tc_kernel<128, 1>);
 }
 

@@ -188,17 +188,10 @@ size_t hd_attn_bwd_workspace(int B, int L, int n, int Hq, hd_mode mode) {
   return static_cast<size_t>(2 * bwd_plane(g, Hq)) * sizeof(float);
 }
 
-size_t hd_attn_rope_workspace(int L, int n, int rot_dim) {
-  if (L < 1 || n < 1 || rot_dim < 8 || rot_dim > 128 || rot_dim % 8) return 0;
-  const int64_t P = static_cast<int64_t>(n) * L;
-  if (P > (1ll << 30)) return 0;
-  return static_cast<size_t>(P) * (rot_dim / 2) * sizeof(float2);
-}
-
 hd_status hd_attn_fwd_rope(const void* q, void* k, const void* v, void* o, float* lse, int B, int L, int n, int Hq,
                            int Hkv, int D, hd_mode mode, int window, float scale, int rot_dim, double base,
-                           hd_rope_layout layout, void* workspace, size_t ws_bytes, hd_dtype in_dt, hd_dtype out_dt,
-                           int32_t* dev_status, void* stream) {
+                           hd_rope_layout layout, hd_dtype in_dt, hd_dtype out_dt, int32_t* dev_status,
+                           void* stream) {
   hd_status stt = check_attn_args(q, k, v, o, lse, B, L, n, Hq, Hkv, D, mode, window, scale, in_dt, out_dt);
   if (stt != HD_OK) return stt;
   if (layout != HD_ROPE_HALF && layout != HD_ROPE_INTERLEAVED) return HD_ERR_INVALID_ARG;
@@ -206,20 +199,16 @@ hd_status hd_attn_fwd_rope(const void* q, void* k, const void* v, void* o, float
   if (!std::isfinite(base) || !(base > 0.0)) return HD_ERR_INVALID_ARG;
   if (in_dt != HD_BF16) return HD_ERR_UNSUPPORTED;
   if (B == 0) return HD_OK;
-  const size_t need = hd_attn_rope_workspace(L, n, rot_dim);
-  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || need == 0 || ws_bytes < need)
-    return HD_ERR_INVALID_ARG;
   const int sms = sm_count();
   if (sms <= 0) return HD_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int64_t P = static_cast<int64_t>(n) * L;
   RopeParams rp;
   std::memset(&rp, 0, sizeof(rp));
   rp.q = nullptr;
   rp.k = k;
   rp.pos0 = nullptr;
   rp.B = B;
-  rp.P = static_cast<int>(P);
+  rp.P = n * L;
   rp.Hq = 0;
   rp.Hkv = Hkv;
   rp.D = D;
@@ -228,14 +217,12 @@ hd_status hd_attn_fwd_rope(const void* q, void* k, const void* v, void* o, float
   rp.pos_base = 0;
   rp.pos_mult = 0;
   rope_fill_turns(rp, rot_dim, base);
-  float2* tab = static_cast<float2*>(workspace);
-  // cos/sin of every position once; k rotated in place (what a cache of
-  // this layer keeps); the query rows rotated inside the attention kernel.
-  if (launch_rope_table(rp, P, tab, st) != cudaSuccess || launch_rope(rp, true, st) != cudaSuccess)
-    return HD_ERR_CUDA;
+  // k rotated in place (what a cache of this layer keeps); the query rows
+  // rotated inside the attention kernel.
+  if (launch_rope(rp, true, st) != cudaSuccess) return HD_ERR_CUDA;
   const AttnGeom g = regular_geom(B, L, n, mode);
   return cuda_status(launch_attn_tc(q, k, v, o, lse, g, Hq, Hkv, D, window, scale, out_dt == HD_BF16, dev_status,
-                                    sms, st, tab, rot_dim / 2, layout));
+                                    sms, st, &rp));
 }
 
 static hd_status run_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,

@@ -58,13 +58,13 @@ bool encode_stream_view(CUtensorMap* m, const void* ptr, int B, int Ls, int ns, 
 cudaError_t launch_attn_f32(const float* q, const float* k, const float* v, void* o, float* lse,
                             const AttnGeom& g, int Hq, int Hkv, int D, int W, float scale, bool out_bf16,
                             cudaStream_t st);
-// rope_tab (nullable): the query rows are rotated inside the kernel, row (i,
-// s) at position i*q_ns + s with (cos, sin) pairs rope_tab[pos*rope_half + j]
-// (regular geometry only), pairs laid out per rope_layout (hd_rope_layout).
+struct RopeParams;
+// rope (nullable): the query rows are rotated inside the kernel, row (i, s)
+// at position i*q_ns + s (regular geometry only), with rope->rot, ->layout
+// and ->fturn as for launch_rope.
 cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o, float* lse, const AttnGeom& g,
                            int Hq, int Hkv, int D, int W, float scale, bool out_bf16, int32_t* status, int sms,
-                           cudaStream_t st, const float2* rope_tab = nullptr, int rope_half = 0,
-                           int rope_layout = 0);
+                           cudaStream_t st, const RopeParams* rope = nullptr);
 
 // Cross-stream prefill of one rank's queries (geometry as for the shard
 // call) with the keys/values held as R rank shards [B, (n/R)*L, Hkv, D]
@@ -129,9 +129,6 @@ struct RopeParams {
 cudaError_t launch_rope(const RopeParams& p, bool bf16, cudaStream_t st);
 // theta_j / (2 pi) as 64-bit fixed-point turns into p.fturn (j < rot/2).
 void rope_fill_turns(RopeParams& p, int rot_dim, double base);
-// (cos, sin) of pos * theta_j for pos in [0, P), j < p.rot/2, into
-// tab[pos * rot/2 + j], by rope_kernel's angle reduction.
-cudaError_t launch_rope_table(const RopeParams& p, int64_t P, float2* tab, cudaStream_t st);
 
 // Stream parallelism: re-interleave rank shards (copy rows of row_bytes),
 // and merge partial softmax results over disjoint key sets.

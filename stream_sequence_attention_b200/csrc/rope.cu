@@ -193,22 +193,6 @@ __global__ void __launch_bounds__(kRopeThreads) rope_kernel(const RopeParams p) 
   }
 }
 
-// cos/sin table of positions [0, P) (see launch_rope_table): the angle as
-// in rope_kernel, for kernels that rotate rows where they load them.
-__global__ void __launch_bounds__(256) rope_table_kernel(const RopeParams p, float2* __restrict__ tab, int64_t n) {
-  const int half = p.rot / 2;
-  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t pos = e / half;
-    const int j = static_cast<int>(e - pos * half);
-    const uint64_t turns = static_cast<uint64_t>(pos) * p.fturn[j];
-    const float tt = static_cast<float>(static_cast<int64_t>(turns)) * 0x1p-63f;
-    float sn, cn;
-    sincospif(tt, &sn, &cn);
-    tab[e] = make_float2(cn, sn);
-  }
-}
-
 // ------------------------------------------------------------------- host
 
 void rope_fill_turns(RopeParams& p, int rot_dim, double base) {
@@ -221,13 +205,6 @@ void rope_fill_turns(RopeParams& p, int rot_dim, double base) {
   }
 }
 
-cudaError_t launch_rope_table(const RopeParams& p, int64_t P, float2* tab, cudaStream_t st) {
-  const int64_t n = P * (p.rot / 2);
-  if (n <= 0) return cudaSuccess;
-  const int64_t blocks = (n + 255) / 256;
-  rope_table_kernel<<<static_cast<unsigned>(blocks < 4096 ? blocks : 4096), 256, 0, st>>>(p, tab, n);
-  return cudaGetLastError();
-}
 
 cudaError_t launch_rope(const RopeParams& p, bool bf16, cudaStream_t st) {
   const int64_t rows = static_cast<int64_t>(p.B) * p.P;

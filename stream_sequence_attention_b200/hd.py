@@ -47,7 +47,6 @@ EXPORTS = (
     "hd_attn_combine",
     "hd_final_stream_gather",
     "hd_rope",
-    "hd_attn_rope_workspace",
     "hd_attn_fwd_rope",
     "hd_status_string",
     "hd_version",
@@ -118,10 +117,8 @@ def lib() -> ctypes.CDLL:
         L.hd_ipc_open.restype = i32
         L.hd_ipc_close.argtypes = [vp]
         L.hd_ipc_close.restype = i32
-        L.hd_attn_rope_workspace.argtypes = [i32, i32, i32]
-        L.hd_attn_rope_workspace.restype = sz
         L.hd_attn_fwd_rope.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, f32, i32,
-                                       ctypes.c_double, i32, vp, sz, i32, i32, vp, vp]
+                                       ctypes.c_double, i32, i32, i32, vp, vp]
         L.hd_attn_fwd_rope.restype = i32
         L.hd_stream_interleave.argtypes = [vp, vp, i32, i32, i32, i32, i64, i32, vp]
         L.hd_stream_interleave.restype = i32
@@ -281,20 +278,13 @@ def hd_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n: int, mode=
     return (out, lse) if want_lse else out
 
 
-def hd_attn_rope_workspace(L: int, n: int, rot_dim: int) -> int:
-    return int(lib().hd_attn_rope_workspace(L, n, rot_dim))
-
-
 def hd_attn_fwd_rope(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n: int, mode="intra", window: int = 0,
                      scale: float | None = None, rot_dim: int | None = None, base: float = 10000.0,
                      layout: str = "half", out: torch.Tensor | None = None, out_dtype=None,
-                     lse: torch.Tensor | bool | None = None, workspace: torch.Tensor | None = None,
-                     dev_status: torch.Tensor | None = None, stream=None):
+                     lse: torch.Tensor | bool | None = None, dev_status: torch.Tensor | None = None, stream=None):
     """hd_attn_fwd on rope(q), rope(k) at the contiguous positions of the
     expanded sequence, the rotation fused in: k is rotated in place, q is
-    rotated inside the attention kernel and left as given.  bf16 only;
-    ``workspace`` (uint8, at least :func:`hd_attn_rope_workspace` bytes) is
-    allocated when not given."""
+    rotated inside the attention kernel and left as given.  bf16 only."""
     for t, nm in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, nm)
     B, P, Hq, D = q.shape
@@ -315,13 +305,10 @@ def hd_attn_fwd_rope(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n: int, 
         lse = torch.empty((B, Hq, P), dtype=torch.float32, device=q.device)
     elif lse is False:
         lse = None
-    nb = hd_attn_rope_workspace(L, n, rot)
-    if workspace is None:
-        workspace = torch.empty(max(nb, 1), dtype=torch.uint8, device=q.device)
     _check("hd_attn_fwd_rope", lib().hd_attn_fwd_rope(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, L, n, Hq, Hkv, D, _MODES[mode], int(window),
-        float(scale), rot, float(base), _ROPE_LAYOUTS[layout], _ptr(workspace),
-        workspace.numel() * workspace.element_size(), _dt(q), _dt(out), _ptr(dev_status), _stream(stream)))
+        float(scale), rot, float(base), _ROPE_LAYOUTS[layout], _dt(q), _dt(out), _ptr(dev_status),
+        _stream(stream)))
     return (out, lse) if want_lse else out
 
 

@@ -121,22 +121,15 @@ def test_attn_fwd_rope_bad_arguments(L):
     from stream_sequence_attention_b200 import hd
     vp = ctypes.c_void_p
     fake = vp(0x10000)  # never dereferenced: every call below fails validation first
-    ws = vp(0x20000)
-    assert hd.hd_attn_rope_workspace(300, 4, 128) == 4 * 300 * 64 * 8
-    assert hd.hd_attn_rope_workspace(300, 4, 12) == 0
-    args = lambda rot, layout, w, nb, dt: (fake, fake, fake, fake, None, 1, 300, 4, 4, 2, 128, 0, 0, 0.1,  # noqa
-                                           rot, 10000.0, layout, w, nb, dt, dt, None, None)
-    need = 4 * 300 * 64 * 8
+    args = lambda rot, layout, dt: (fake, fake, fake, fake, None, 1, 300, 4, 4, 2, 128, 0, 0, 0.1,  # noqa
+                                    rot, 10000.0, layout, dt, dt, None, None)
     # rot_dim not a multiple of 16 in the rotate-half form, or above D
-    assert L.hd_attn_fwd_rope(*args(40, hd.HD_ROPE_HALF, ws, need, hd.HD_BF16)) == hd.HD_ERR_INVALID_ARG
-    assert L.hd_attn_fwd_rope(*args(256, hd.HD_ROPE_HALF, ws, need, hd.HD_BF16)) == hd.HD_ERR_INVALID_ARG
-    # bad layout, missing / short / misaligned workspace
-    assert L.hd_attn_fwd_rope(*args(128, 7, ws, need, hd.HD_BF16)) == hd.HD_ERR_INVALID_ARG
-    assert L.hd_attn_fwd_rope(*args(128, hd.HD_ROPE_HALF, None, need, hd.HD_BF16)) == hd.HD_ERR_INVALID_ARG
-    assert L.hd_attn_fwd_rope(*args(128, hd.HD_ROPE_HALF, ws, need - 8, hd.HD_BF16)) == hd.HD_ERR_INVALID_ARG
-    assert L.hd_attn_fwd_rope(*args(128, hd.HD_ROPE_HALF, vp(0x20010), need, hd.HD_BF16)) == hd.HD_ERR_INVALID_ARG
-    # float32 inputs are not taken (the rotation runs in the tensor-core kernel)
-    assert L.hd_attn_fwd_rope(*args(128, hd.HD_ROPE_HALF, ws, need, hd.HD_F32)) == hd.HD_ERR_UNSUPPORTED
+    assert L.hd_attn_fwd_rope(*args(40, hd.HD_ROPE_HALF, hd.HD_BF16)) == hd.HD_ERR_INVALID_ARG
+    assert L.hd_attn_fwd_rope(*args(256, hd.HD_ROPE_HALF, hd.HD_BF16)) == hd.HD_ERR_INVALID_ARG
+    assert L.hd_attn_fwd_rope(*args(12, hd.HD_ROPE_INTERLEAVED, hd.HD_BF16)) == hd.HD_ERR_INVALID_ARG
+    # bad layout; float32 inputs are not taken (the rotation runs in the tensor-core kernel)
+    assert L.hd_attn_fwd_rope(*args(128, 7, hd.HD_BF16)) == hd.HD_ERR_INVALID_ARG
+    assert L.hd_attn_fwd_rope(*args(128, hd.HD_ROPE_HALF, hd.HD_F32)) == hd.HD_ERR_UNSUPPORTED
 
 
 def test_rope_bad_arguments(L):

@@ -1,8 +1,9 @@
 """hd_attn_fwd_rope: attention with the rotary embedding fused in (query rows
 rotated inside the attention kernel, k rotated in place), against the
-float64 oracle's attn(rope(q), rope(k), v), and bit-identical to the
-separate chain hd_rope + hd_attn_fwd (the rotation runs the same float32
-arithmetic on the same cos/sin values in both)."""
+float64 oracle's attn(rope(q), rope(k), v), and against the separate chain
+hd_rope + hd_attn_fwd (k bit-identical; the query rows' cos/sin come from the
+special-function unit inside the attention kernel, so O agrees with the
+chain to the bf16 bound rather than bit for bit)."""
 
 import numpy as np
 import pytest
@@ -48,11 +49,15 @@ def test_fused_rope_attention(hd, B, n, L, Hq, Hkv, D, mode, W, rot, layout, bas
     assert int(st.item()) == 0
     assert torch.equal(qd, q_before), "q must be left as given"
     kw = dict(layout=layout)
-    kr = oracle.rope(k, rot, base, **kw)
+    qr, kr = oracle.rope(q, rot, base, **kw), oracle.rope(k, rot, base, **kw)
     err_k = np.abs(to_f64(kd) - kr)
     assert np.all(err_k <= 2.0 ** -8 * np.abs(kr) + 1e-5), "k is not rope(k)"
-    ro, rl = oracle.attn(oracle.rope(q, rot, base, **kw), kr, v, n, mode, W)
+    ro, _ = oracle.attn(qr, kr, v, n, mode, W)
     assert max_abs(to_f64(o), ro) <= TOL_BF16
+    # The kernel attends over rope(q), rope(k) rounded to bf16 (the rotated
+    # rows are bf16 tiles); lse is checked against the oracle on those inputs,
+    # where the rounding moves scores by up to 2^-8 of their size.
+    _, rl = oracle.attn(synth.bf16_round(qr.astype(np.float32)), synth.bf16_round(kr.astype(np.float32)), v, n, mode, W)
     assert max_abs(to_f64(lse), rl) <= 1e-3
     # the separate chain: hd_rope on copies, then hd_attn_fwd
     q2, k2 = dev(q, "bf16"), dev(k, "bf16")
@@ -60,12 +65,14 @@ def test_fused_rope_attention(hd, B, n, L, Hq, Hkv, D, mode, W, rot, layout, bas
     o2, l2 = hd.hd_attn_fwd(q2, k2, vd, n, mode, W, out_dtype=odt, lse=True)
     torch.cuda.synchronize()
     assert torch.equal(k2, kd)
-    assert torch.equal(o2, o) and torch.equal(l2, lse)
+    assert float((o2.float() - o.float()).abs().max()) <= TOL_BF16
+    assert float((l2 - lse).abs().max()) <= 1e-3
 
 
 def test_fused_rope_full_size_sampled(hd):
-    """The intra prefill workload (n=4 L=4096 B=2 32q/8kv D=128): equal to
-    the separate chain bit for bit, and sampled rows against the oracle."""
+    """The intra prefill workload (n=4 L=4096 B=2 32q/8kv D=128): k equal to
+    the separate chain's bit for bit, O within the bf16 bound of it, and
+    sampled rows against the oracle."""
     B, n, L, Hq, Hkv, D = 2, 4, 4096, 32, 8, 128
     P = n * L
     q = synth.normal_device((B, P, Hq, D), 321)
@@ -77,7 +84,8 @@ def test_fused_rope_full_size_sampled(hd):
     hd.hd_rope(q2, k2)
     o2 = hd.hd_attn_fwd(q2, k2, v, n, "intra")
     torch.cuda.synchronize()
-    assert torch.equal(k, k2) and torch.equal(o, o2)
+    assert torch.equal(k, k2)
+    assert float((o.float() - o2.float()).abs().max()) <= TOL_BF16
     # sampled rows of stream 1, head 5, against the oracle on the de-interleaved stream
     s, h = 1, 5
     g = h // (Hq // Hkv)
