@@ -58,10 +58,24 @@ constexpr int BN = 128;
 #endif
 constexpr int kIssuers = HD_TC_ISSUERS;
 static_assert(kIssuers == 1 || kIssuers == 2, "one or two MMA issuers");
+// Register split (1): 12 warps, the third warpgroup (producer, MMA
+// issuer(s), gather, idle) gives registers to the two softmax warpgroups with
+// setmaxnreg: launched at 168 per thread (65536 / 384), it drops to kRegsAux
+// and the softmax warps rise to kRegsSoftmax.  (0): 10 or 11 warps, 168
+// registers for every thread.
+#ifndef HD_TC_REGSPLIT
+#define HD_TC_REGSPLIT 0
+#endif
+constexpr bool kRegSplit = HD_TC_REGSPLIT != 0;
+constexpr uint32_t kRegsAux = 104;
+constexpr uint32_t kRegsSoftmax = 200;
+static_assert(256 * kRegsSoftmax + 128 * kRegsAux <= 384 * 168, "register split exceeds the launch");
 // Warps: two softmax warpgroups (0-7), the TMA producer (8), the MMA
 // issuer(s) (9, and 10 with two), and in the rank-shard form with gather the
 // gather warp after them.
-constexpr int kThreads = 32 * (9 + kIssuers);
+constexpr int kThreads = kRegSplit ? 384 : 32 * (9 + kIssuers);
+// Threads of a launch of the form with NM key/value sources.
+__host__ __device__ constexpr int threads_of(int NM) { return kRegSplit ? 384 : (NM > 1 ? kThreads + 32 : kThreads); }
 constexpr int kWarpTMA = 8;
 constexpr int kWarpMMA = 9;
 constexpr int kWarpGather = 9 + kIssuers;  // rank-shard form with gather only
@@ -82,7 +96,7 @@ constexpr int VST = 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // On tiles without masking, one exp2 pair in kPolyEvery is evaluated on the
-// FMA pipe (0 = all on the MUFU unit).
+// FMA pipe in packed f32x2 arithmetic (exp2_fma2; 0 = all on the MUFU unit).
 #ifndef HD_TC_POLY_EVERY
 #define HD_TC_POLY_EVERY 0
 #endif
@@ -401,7 +415,7 @@ __device__ __forceinline__ void rope_rotate_row(uint8_t* qrow, int blk, int r, i
 // ROPE: the query rows are rotated in the Q tile at the start of each unit
 // (a separate instantiation, so the other forms carry none of its code).
 template <int D, int NM, bool ROPE = false>
-__global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
+__global__ void __launch_bounds__(tc::threads_of(NM), 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ KvSrc<NM> kv,
                    const __grid_constant__ CUtensorMap tmO, const TcParams p) {
   using Lay = tc::Layout<D>;
@@ -502,6 +516,7 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
 
   if (warp >= 8) {
   // Producer, MMA issuer, gather (each warp its own role).
+  if constexpr (tc::kRegSplit) regs_decrease<tc::kRegsAux>();
   if (warp == tc::kWarpTMA) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -723,6 +738,7 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
   }
   } else {
     // ------------------------------------------------- softmax + epilogue
+    if constexpr (tc::kRegSplit) regs_increase<tc::kRegsSoftmax>();
     const int slot = warp >> 2;
     const int r = threadIdx.x & 127;  // tensor-memory lane
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -866,8 +882,8 @@ __global__ void __launch_bounds__(NM > 1 ? tc::kThreads + 32 : tc::kThreads, 1)
             }
             float p0, p1;
             if (tc::kPolyEvery > 0 && !need_mask && (e % (tc::kPolyEvery > 0 ? tc::kPolyEvery : 1)) == tc::kPolyEvery - 1) {
-              p0 = exp2_fma(a0);
-              p1 = exp2_fma(a1);
+              // this pair on the FMA pipe (unmasked tiles: no -inf exponent)
+              unpack_f32x2(exp2_fma2(a0, a1), p0, p1);
             } else {
               p0 = ex2(a0);
               p1 = ex2(a1);
@@ -1240,7 +1256,7 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o,
   auto go = [&](auto kernel) {
     cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
-    kernel<<<grid, tc::kThreads, smem, st>>>(mq, kv, mo, p);
+    kernel<<<grid, tc::threads_of(1), smem, st>>>(mq, kv, mo, p);
     return cudaGetLastError();
   };
   if (rope) return D == 64 ? go(attn_tc_kernel<64, 1, true>) : go(attn_tc_kernel<128, 1, true>);
@@ -1260,7 +1276,7 @@ static cudaError_t launch_parts_kernel(const CUtensorMap& mq, const KvSrc<kPeerM
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(tc::kThreads + 32);
+  cfg.blockDim = dim3(tc::threads_of(kPeerMaxRanks));
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute at[1];

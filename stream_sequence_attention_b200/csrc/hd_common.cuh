@@ -441,6 +441,24 @@ __device__ __forceinline__ uint32_t pack_bf16x2_of(uint64_t v) {
   return pack_bf16x2(a, b);
 }
 
+// 2^x of a pair on the FMA pipe, as exp2_fma but in packed f32x2 arithmetic
+// (round to nearest, cubic, exponent add); inputs below -126 are clamped to
+// -126 (result ~2^-126, not 0): for exponents that are never -inf.
+__device__ __forceinline__ uint64_t exp2_fma2(float x0, float x1) {
+  const uint64_t m = pack_f32x2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+  const uint64_t x = pack_f32x2(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+  const uint64_t t = add_f32x2(x, m);
+  const uint64_t f = sub_f32x2(x, sub_f32x2(t, m));
+  uint64_t q = fma_f32x2(pack_f32x2(0.0551713444f, 0.0551713444f), f, pack_f32x2(0.242610335f, 0.242610335f));
+  q = fma_f32x2(q, f, pack_f32x2(0.693260968f, 0.693260968f));
+  q = fma_f32x2(q, f, pack_f32x2(0.999928117f, 0.999928117f));
+  float q0, q1, t0, t1;
+  unpack_f32x2(q, q0, q1);
+  unpack_f32x2(t, t0, t1);
+  return pack_f32x2(__int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23)),
+                    __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23)));
+}
+
 __device__ __forceinline__ int elect_one_lane() { return (threadIdx.x & 31) == 0; }
 
 }  // namespace hd

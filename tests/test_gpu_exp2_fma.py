@@ -1,8 +1,9 @@
 """The FMA-pipe exponential of the attention kernels (exp2_fma, an optional
-replacement for part of the MUFU exponentials) against the MUFU form and
-float64 2**x, over its whole input range: no NaN or negative result, exact
-zero below 2^-126 (as the flush-to-zero MUFU form gives, -inf included),
-relative error below 1e-4 elsewhere.  A small probe library is compiled
+replacement for part of the MUFU exponentials, and its packed f32x2 form
+exp2_fma2) against the MUFU form and float64 2**x, over its whole input
+range: no NaN or negative result, exact zero below 2^-126 (as the
+flush-to-zero MUFU form gives, -inf included; the packed form clamps there
+to ~2^-126), relative error below 1e-4 elsewhere.  A small probe library is compiled
 from tests/probes/exp2_fma_probe.cu against the kernels' shared header."""
 
 import ctypes
@@ -41,8 +42,9 @@ def test_exp2_fma_whole_range(probe):
     xt = torch.from_numpy(x).cuda()
     fo = torch.empty_like(xt)
     mo = torch.empty_like(xt)
+    po = torch.empty_like(xt)
     rc = probe.exp2_probe(ctypes.c_void_p(xt.data_ptr()), ctypes.c_void_p(fo.data_ptr()),
-                          ctypes.c_void_p(mo.data_ptr()), len(x))
+                          ctypes.c_void_p(mo.data_ptr()), ctypes.c_void_p(po.data_ptr()), len(x))
     assert rc == 0
     f = fo.cpu().numpy().astype(np.float64)
     m = mo.cpu().numpy().astype(np.float64)
@@ -58,3 +60,10 @@ def test_exp2_fma_whole_range(probe):
     assert (np.abs(f[normal] - m[normal]) / exact[normal]).max() < 1.2e-4
     edge = (x >= -126.0) & (x < -125.0)  # results near 2^-126: absolute bound
     assert (np.abs(f[edge] - exact[edge]) <= 2.0 ** -136).all()
+    # the packed form: the same values for x >= -126 (where the attention
+    # kernel uses it: exponents of unmasked tiles), clamped to ~2^-126 below
+    pr = po.cpu().numpy().astype(np.float64)
+    assert np.isfinite(pr).all() and (pr >= 0).all()
+    ok = x >= -126.0
+    assert np.array_equal(pr[ok], f[ok])
+    assert (pr[~ok] <= 2.0 ** -125).all()
