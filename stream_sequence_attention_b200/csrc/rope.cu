@@ -13,8 +13,6 @@
 // host passes theta_j/(2 pi) as a 64-bit fixed-point fraction of a turn F_j,
 // and pos*F_j mod 2^64 (an integer product) is the angle's fraction of a
 // turn; float32 sincospi of it is accurate to ~2e-7 rad.
-#include <cmath>
-
 #include "hd_common.cuh"
 #include "hd_launch.h"
 
@@ -204,7 +202,6 @@ void rope_fill_turns(RopeParams& p, int rot_dim, double base) {
     p.fturn[j] = static_cast<uint64_t>(ldexpl(turns, 64));
   }
 }
-
 
 cudaError_t launch_rope(const RopeParams& p, bool bf16, cudaStream_t st) {
   const int64_t rows = static_cast<int64_t>(p.B) * p.P;
