@@ -35,9 +35,17 @@
 // Softmax: running max m per row in log2 units; O is rescaled only when a
 // tile raises the max by more than 2^8 (the final 1/l makes the result
 // independent of which max was used).  The row max uses 3-input max.
-// Optionally (tc::kPolyEvery) part of the exponentials run on the FMA pipe
-// (round to nearest integer, cubic for 2^f on [-1/2, 1/2], exponent add;
-// relative error < 1e-4, below the bf16 rounding of P) to offload MUFU.
+// On tiles without masking one exponential pair in three (tc::kPolyEvery)
+// runs on the FMA pipe instead of the MUFU unit, whose 16 results per clock
+// per SM would otherwise bound the softmax at the tensor core's own rate:
+// the exponent is shifted and clamped by one saturating FMA per element
+// (masked -inf and anything below -126 land on -126; the top of the range
+// is the rescale threshold), then rounded to the nearest integer by the
+// 1.5 * 2^23 constant, a cubic gives 2^f on [-1/2, 1/2] and an integer
+// multiply-add puts n in the exponent field (relative error < 1e-4, below
+// the bf16 rounding of P).  Masked tiles stay on the MUFU unit, which
+// returns an exact 0 for -inf.
+#include <climits>
 #include <cstdlib>
 #include <cstring>
 #include <type_traits>
@@ -96,11 +104,38 @@ constexpr int VST = 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // On tiles without masking, one exp2 pair in kPolyEvery is evaluated on the
-// FMA pipe in packed f32x2 arithmetic (exp2_fma2; 0 = all on the MUFU unit).
+// FMA pipe in packed f32x2 arithmetic (0 = all on the MUFU unit): with
+// kPolySat its exponent is shifted and clamped by one saturating FMA per
+// element and exp2_sat2 takes it from there, else exp2_fma2 (ALU clamp and
+// exponent add; exponents above 0, up to the rescale threshold, included).
 #ifndef HD_TC_POLY_EVERY
-#define HD_TC_POLY_EVERY 0
+#define HD_TC_POLY_EVERY 3
 #endif
 constexpr int kPolyEvery = HD_TC_POLY_EVERY;
+#ifndef HD_TC_POLY_SAT
+#define HD_TC_POLY_SAT 1
+#endif
+constexpr bool kPolySat = HD_TC_POLY_SAT != 0;
+// Optional explicit choice of the FMA-pipe pairs: bit (c mod 16) of the mask
+// selects pair c of a tile row (kPolySat form; 0 = one in kPolyEvery).
+#ifndef HD_TC_POLY_PAT
+#define HD_TC_POLY_PAT 0
+#endif
+constexpr uint32_t kPolyPat = HD_TC_POLY_PAT;
+// The FMA-pipe pairs also in the fused-RoPE form (1), or MUFU only there (0).
+#ifndef HD_TC_ROPE_POLY
+#define HD_TC_ROPE_POLY 1
+#endif
+constexpr bool kRopePoly = HD_TC_ROPE_POLY != 0;
+// Row sums of P in packed f32x2 adds (1) or scalar adds (0).
+#ifndef HD_TC_PSUM
+#define HD_TC_PSUM 0
+#endif
+constexpr bool kPackedSum = HD_TC_PSUM != 0;
+__host__ __device__ constexpr bool poly_pair(int c) {
+  return kPolyPat != 0 ? ((kPolyPat >> (c & 15)) & 1u) != 0
+                       : (kPolyEvery > 0 && (c % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1);
+}
 // The two softmax warpgroups take turns (ping-pong) when nonzero.
 #ifndef HD_TC_PINGPONG
 #define HD_TC_PINGPONG 0
@@ -115,6 +150,18 @@ constexpr bool kTmaStore = HD_TC_TMA_STORE != 0;
 // Softmax arithmetic per tile: the exponents of the whole row first, as
 // packed f32x2 FMAs, then the exponentials (1); or exponent and exponential
 // column pair by column pair (0).
+#ifndef HD_TC_MASK2
+#define HD_TC_MASK2 1
+#endif
+// Masked tiles: the visible columns of a row are one interval [lo, hi] of
+// the tile, so each score takes two compares against constants.
+constexpr bool kMask2 = HD_TC_MASK2 != 0;
+#ifndef HD_TC_EPI_ALL
+#define HD_TC_EPI_ALL 1
+#endif
+// bf16 TMA-store epilogue: read all of O from tensor memory at once and
+// release it before the stores.
+constexpr bool kEpiAll = HD_TC_EPI_ALL != 0;
 #ifndef HD_TC_SPLIT
 #define HD_TC_SPLIT 1
 #endif
@@ -153,7 +200,7 @@ struct Layout {
 #if HD_TC_TRACE
 // Per-CTA clock counters of the diagnostic build: kTraceSlots per CTA.
 constexpr int kTraceCtas = 1024;
-constexpr int kTraceSlots = 20;
+constexpr int kTraceSlots = 32;
 __device__ unsigned long long g_tc_trace[kTraceCtas * kTraceSlots];
 #endif
 
@@ -345,17 +392,25 @@ __device__ __forceinline__ void gather_items(const PartsInfo& x, int B, int lane
   }
 }
 
-// cos and sin of pos * theta_j: pos * fturn mod 2^64 is the angle's
-// fraction of a turn (exact); its top 32 bits as a signed fraction t in
-// [-1/2, 1/2) give the angle 2 pi t, whose sine and cosine come from the MUFU
-// unit (absolute error about 1e-6, far below the bf16 rounding of the row).
-__device__ __forceinline__ float2 rope_cos_sin(int64_t pos, uint64_t fturn) {
-  const uint64_t turns = static_cast<uint64_t>(pos) * fturn;
-  const float a = static_cast<float>(static_cast<int32_t>(turns >> 32)) * (6.28318530717958647692f * 0x1p-32f);
+// cos and sin of the angle pos * theta_j, fturn = theta_j / (2 pi) as a
+// 64-bit fraction of a turn: bits 32..63 of pos * fturn (exact, mod 2^64)
+// are the fraction of a turn, from two 32-bit multiplies.  Its top bit
+// flipped and the next 22 bits under the exponent of 1.0f give 1.5 + the
+// signed fraction in [-1/2, 1/2); one FMA turns that into the angle in
+// [-pi, pi), where sin.approx / cos.approx are accurate to ~1e-6.
+__device__ __forceinline__ float2 rope_cos_sin(uint32_t pos, uint64_t fturn) {
+  const uint32_t t = pos * static_cast<uint32_t>(fturn >> 32) + __umulhi(pos, static_cast<uint32_t>(fturn));
+  const float f = __uint_as_float((t >> 9) ^ 0x3FC00000u);
+  const float a = fmaf(f, 6.28318530717958647692f, -9.42477796076937971538f);  // (f - 1.5) * 2 pi
   float sn, cn;
   asm("sin.approx.f32 %0, %1;" : "=f"(sn) : "f"(a));
   asm("cos.approx.f32 %0, %1;" : "=f"(cn) : "f"(a));
   return make_float2(cn, sn);
+}
+
+// bf16 pair (low, high half of w) as a packed f32 pair.
+__device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t w) {
+  return pack_f32x2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
 
 // Rotary embedding of one query row in place in a 128-byte-swizzled Q tile
@@ -363,7 +418,7 @@ __device__ __forceinline__ float2 rope_cos_sin(int64_t pos, uint64_t fturn) {
 // pairs (j, j + half) or (2j, 2j + 1), j < half, (a, b) -> (a cos - b sin,
 // a sin + b cos) at the angle pos * theta_j.
 template <int NP>
-__device__ __forceinline__ void rope_rotate_row(uint8_t* qrow, int blk, int r, int64_t pos, int half, int layout,
+__device__ __forceinline__ void rope_rotate_row(uint8_t* qrow, int blk, int r, uint32_t pos, int half, int layout,
                                                 const uint64_t (&fturn)[NP]) {
   // 16-byte unit holding features f .. f+7 (f a multiple of 8) of the row:
   // 128-byte swizzle within each 64-feature block.
@@ -381,12 +436,14 @@ __device__ __forceinline__ void rope_rotate_row(uint8_t* qrow, int blk, int r, i
         uint32_t wa[4] = {ua.x, ua.y, ua.z, ua.w}, wb[4] = {ub.x, ub.y, ub.z, ub.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float2 fa = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wa[e]));
-          const float2 fb = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wb[e]));
+          // features (j, j + 1) of both halves as packed pairs: a' = a c - b s,
+          // b' = a s + b c
+          const uint64_t a2 = bf16x2_to_f32x2(wa[e]), b2 = bf16x2_to_f32x2(wb[e]);
           const float2 t0 = rope_cos_sin(pos, fturn[8 * v + 2 * e]);
           const float2 t1 = rope_cos_sin(pos, fturn[8 * v + 2 * e + 1]);
-          wa[e] = pack_bf16x2(fmaf(fa.x, t0.x, -fb.x * t0.y), fmaf(fa.y, t1.x, -fb.y * t1.y));
-          wb[e] = pack_bf16x2(fmaf(fa.x, t0.y, fb.x * t0.x), fmaf(fa.y, t1.y, fb.y * t1.x));
+          const uint64_t c2 = pack_f32x2(t0.x, t1.x), s2 = pack_f32x2(t0.y, t1.y);
+          wa[e] = pack_bf16x2_of(sub_f32x2(mul_f32x2(a2, c2), mul_f32x2(b2, s2)));
+          wb[e] = pack_bf16x2_of(fma_f32x2(a2, s2, mul_f32x2(b2, c2)));
         }
         *pa = make_uint4(wa[0], wa[1], wa[2], wa[3]);
         *pb = make_uint4(wb[0], wb[1], wb[2], wb[3]);
@@ -727,7 +784,7 @@ __global__ void __launch_bounds__(tc::threads_of(NM), 1)
 #if HD_TC_TRACE
       mw[2] = static_cast<unsigned long long>(clock64() - mt0);
       if (blockIdx.x < kTraceCtas && lane == 0)
-        for (int c = 0; c < 3; ++c) g_tc_trace[blockIdx.x * kTraceSlots + 12 + 3 * me + c] = mw[c];
+        for (int c = 0; c < 3; ++c) g_tc_trace[blockIdx.x * kTraceSlots + 24 + 3 * me + c] = mw[c];
 #endif
     }
   } else if (warp == tc::kWarpGather) {
@@ -748,9 +805,12 @@ __global__ void __launch_bounds__(tc::threads_of(NM), 1)
     int sc = 0, uc = 0, oc = 0;
     bool ok = true;
     bool stored = false;  // this warp has TMA stores in flight (lane 0)
-    // Diagnostic counters (HD_TC_TRACE): wait for S, load + max, exponents
-    // to P published, row sum, epilogue, tiles.
-    unsigned long long tr[6] = {0, 0, 0, 0, 0, 0};
+    // Diagnostic counters (HD_TC_TRACE): wait for S, score load, max and
+    // mask, exponents to P published, row sum, epilogue wait for the last
+    // P V, rest of the epilogue, tiles; then the score load to P published
+    // on masked tiles and their count, and on a unit's first tile.
+    unsigned long long tr[12] = {0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0};
+    long long tfrom = 0;
     long long tmark = tc::kTrace ? clock64() : 0;
     auto tick = [&](int i) {
       if constexpr (tc::kTrace) {
@@ -771,7 +831,7 @@ __global__ void __launch_bounds__(tc::threads_of(NM), 1)
       const int ir = xr.qblk * tc::BM + r;
       if (ir < p.g.Lq)
         rope_rotate_row(smem + Lay::Q_OFF + slot * Lay::TILE + r * 128, Lay::BLK, r,
-                        static_cast<int64_t>(ir) * p.g.q_ns + xr.s, p.rope_half, p.rope_layout, p.rope_fturn);
+                        static_cast<uint32_t>(ir * p.g.q_ns + xr.s), p.rope_half, p.rope_layout, p.rope_fturn);
       // The tensor core reads the tile through the async proxy.
       fence_proxy_async_smem();
       mbar_arrive(bar(Lay::B_QROT + slot));
@@ -823,13 +883,25 @@ __global__ void __launch_bounds__(tc::threads_of(NM), 1)
         tmem_ld32(sS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
         tmem_ld32(sS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
         tmem_wait_ld();
+        tick(1);
+        if (tc::kTrace) tfrom = tmark;
         const bool need_mask = (k0 + tc::BN - 1 > pfirst) || (p.W > 0 && k0 < plast - p.W + 1);
         if (need_mask) {
+          if constexpr (tc::kMask2 && !kParts) {
+            // Column c holds key k0 + c: visible for k0 + c <= pi and, with
+            // a window, pi - (k0 + c) < W.
+            const int hi = pi - k0;
+            const int lo = p.W > 0 ? pi - p.W + 1 - k0 : INT_MIN;
 #pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            int j = k0 + c;
-            if constexpr (kParts) j = k0 + kv.x.perm[c];
-            if (j > pi || (p.W > 0 && pi - j >= p.W)) sv[c] = __float_as_uint(-INFINITY);
+            for (int c = 0; c < 128; ++c)
+              if (c > hi || c < lo) sv[c] = __float_as_uint(-INFINITY);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 128; ++c) {
+              int j = k0 + c;
+              if constexpr (kParts) j = k0 + kv.x.perm[c];
+              if (j > pi || (p.W > 0 && pi - j >= p.W)) sv[c] = __float_as_uint(-INFINITY);
+            }
           }
         }
         // Row max of the raw scores (scale > 0 commutes with max): 3-input
@@ -851,10 +923,62 @@ __global__ void __launch_bounds__(tc::threads_of(NM), 1)
           resc = true;
         }
         const float nmu = (m == -INFINITY) ? 0.f : -m;
-        tick(1);
+        tick(2);
         // P = 2^(s*scale - m) as bf16 pairs, written over the S columns 16 at
         // a time (column 16j of P holds S columns 32j.. already consumed).
         float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        uint64_t ls2[4] = {0, 0, 0, 0};  // packed pairs of 0.f
+        if ((tc::kPolyEvery > 0 || tc::kPolyPat != 0) && tc::kPolySat && tc::kSplit && (!ROPE || tc::kRopePoly) &&
+            !need_mask) {
+          // The exponent x = s * scale * log2 e - m lies in [-inf, T] (T =
+          // kRescaleThreshold: the max is raised only past it): the FMA-pipe
+          // pairs take y = sat((x + 126) / (126 + T)), the rest x itself.
+          constexpr int kHi = static_cast<int>(tc::kRescaleThreshold);
+          static_assert(kHi == tc::kRescaleThreshold, "integral threshold");
+          constexpr float kInvSpan = 1.f / (126.f + kHi);
+          const uint64_t s2 = pack_f32x2(sl2, sl2), n2 = pack_f32x2(nmu, nmu);
+          const float k1 = sl2 * kInvSpan, k2 = (nmu + 126.f) * kInvSpan;
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            if (tc::poly_pair(c)) {
+              sv[2 * c] = __float_as_uint(fma_sat(__uint_as_float(sv[2 * c]), k1, k2));
+              sv[2 * c + 1] = __float_as_uint(fma_sat(__uint_as_float(sv[2 * c + 1]), k1, k2));
+            } else {
+              float a0, a1;
+              unpack_f32x2(fma_f32x2(pack_f32x2(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1])), s2, n2),
+                           a0, a1);
+              sv[2 * c] = __float_as_uint(a0);
+              sv[2 * c + 1] = __float_as_uint(a1);
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int c = 16 * j + e;
+              float p0, p1;
+              if (tc::poly_pair(c)) {
+                unpack_f32x2(exp2_sat2<kHi>(pack_f32x2(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1]))), p0,
+                             p1);
+              } else {
+                p0 = ex2(__uint_as_float(sv[2 * c]));
+                p1 = ex2(__uint_as_float(sv[2 * c + 1]));
+              }
+              if constexpr (tc::kPackedSum) {
+                ls2[e & 3] = add_f32x2(ls2[e & 3], pack_f32x2(p0, p1));
+              } else {
+                ls[e & 7] += p0 + p1;
+              }
+              pk[e] = pack_bf16x2(p0, p1);
+            }
+            tmem_st16(sS + 16 * j, pk);
+          }
+          if constexpr (tc::kPackedSum) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) unpack_f32x2(ls2[e], ls[2 * e], ls[2 * e + 1]);
+          }
+        } else {
         if constexpr (tc::kSplit) {
           const uint64_t s2 = pack_f32x2(sl2, sl2), n2 = pack_f32x2(nmu, nmu);
 #pragma unroll
@@ -881,7 +1005,8 @@ __global__ void __launch_bounds__(tc::threads_of(NM), 1)
               a1 = fmaf(__uint_as_float(sv[2 * c + 1]), sl2, nmu);
             }
             float p0, p1;
-            if (tc::kPolyEvery > 0 && !need_mask && (e % (tc::kPolyEvery > 0 ? tc::kPolyEvery : 1)) == tc::kPolyEvery - 1) {
+            if (tc::kPolyEvery > 0 && !tc::kPolySat && !need_mask &&
+                (e % (tc::kPolyEvery > 0 ? tc::kPolyEvery : 1)) == tc::kPolyEvery - 1) {
               // this pair on the FMA pipe (unmasked tiles: no -inf exponent)
               unpack_f32x2(exp2_fma2(a0, a1), p0, p1);
             } else {
@@ -892,6 +1017,7 @@ __global__ void __launch_bounds__(tc::threads_of(NM), 1)
             pk[e] = pack_bf16x2(p0, p1);
           }
           tmem_st16(sS + 16 * j, pk);
+        }
         }
         if (tc::kPingPong && paired) {
           mbar_arrive(bar(Lay::B_ORD + (slot ^ 1)));
@@ -913,7 +1039,15 @@ __global__ void __launch_bounds__(tc::threads_of(NM), 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(Lay::B_PFULL + slot));
-        tick(2);
+        tick(3);
+        if constexpr (tc::kTrace) {
+          const unsigned long long d = static_cast<unsigned long long>(tmark - tfrom);
+          if (need_mask) {
+            tr[8] += d;
+            ++tr[9];
+          }
+          if (jj == 0) tr[10] += d;
+        }
         l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
         if constexpr (ROPE) {
           // After the unit's last P: rotate the next unit's query rows while
@@ -935,14 +1069,15 @@ __global__ void __launch_bounds__(tc::threads_of(NM), 1)
             }
           }
         }
-        tick(3);
-        if (tc::kTrace) ++tr[5];
+        tick(4);
+        if (tc::kTrace) ++tr[7];
       }
       if (!ok) break;
       // Epilogue: O / l -> global once the last P V MMA of this head is done.
       const bool got = mbar_wait(bar(Lay::B_ODONE + slot), uc & 1, abort_flag);
       ++uc;
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      tick(5);
       tc_fence_after();
       const float inv = 1.f / l;
       const bool row_ok = i < p.g.Lq;
@@ -975,7 +1110,27 @@ __global__ void __launch_bounds__(tc::threads_of(NM), 1)
             stored = true;
           }
         };
-        if (p.out_bf16) {
+        if (tc::kEpiAll && p.out_bf16) {
+          uint32_t ov[D];
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) tmem_ld32(sO + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&ov[c * 32]));
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(bar(Lay::B_OEMPTY + slot));
+#pragma unroll
+          for (int ch = 0; ch < D / 64; ++ch) {
+            uint4 w[8];
+#pragma unroll
+            for (int uu = 0; uu < 8; ++uu) {
+              const int c0 = ch * 64 + uu * 8;
+              w[uu].x = pack_bf16x2(__uint_as_float(ov[c0 + 0]) * inv, __uint_as_float(ov[c0 + 1]) * inv);
+              w[uu].y = pack_bf16x2(__uint_as_float(ov[c0 + 2]) * inv, __uint_as_float(ov[c0 + 3]) * inv);
+              w[uu].z = pack_bf16x2(__uint_as_float(ov[c0 + 4]) * inv, __uint_as_float(ov[c0 + 5]) * inv);
+              w[uu].w = pack_bf16x2(__uint_as_float(ov[c0 + 6]) * inv, __uint_as_float(ov[c0 + 7]) * inv);
+            }
+            put(ch, w);
+          }
+        } else if (p.out_bf16) {
 #pragma unroll
           for (int ch = 0; ch < D / 64; ++ch) {
             uint32_t ov[64];
@@ -1052,7 +1207,7 @@ __global__ void __launch_bounds__(tc::threads_of(NM), 1)
       if (row_ok && p.lse)
         p.lse[(static_cast<int64_t>(x.b) * p.Hq + h) * p.g.o_rows + static_cast<int64_t>(i) * p.g.o_ns + x.s] =
             (m + log2f(l)) * 0.69314718055994531f;
-      tick(4);
+      tick(6);
     }
     // Every TMA store has finished reading its staging before the CTA's
     // shared memory can go away.
@@ -1060,7 +1215,7 @@ __global__ void __launch_bounds__(tc::threads_of(NM), 1)
     if (!ok) fail();
 #if HD_TC_TRACE
     if (r == 0 && blockIdx.x < kTraceCtas)
-      for (int c = 0; c < 6; ++c) g_tc_trace[blockIdx.x * kTraceSlots + slot * 6 + c] = tr[c];
+      for (int c = 0; c < 12; ++c) g_tc_trace[blockIdx.x * kTraceSlots + slot * 12 + c] = tr[c];
 #endif
   }
 

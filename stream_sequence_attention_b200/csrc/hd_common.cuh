@@ -459,6 +459,40 @@ __device__ __forceinline__ uint64_t exp2_fma2(float x0, float x1) {
                     __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23)));
 }
 
+// Saturating scalar FMA: min(max(a * b + c, 0), 1) in one FMA-pipe
+// instruction (the clamp costs no ALU instruction).
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  float d;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^((126 + HI) y - 126) of a pair y in [0, 1] on the FMA pipe alone: the
+// caller maps an exponent x to y = sat((x + 126) / (126 + HI)), so x in
+// [-126, HI] keeps its value and x below (-inf included) lands on -126.
+// n = rint(x) through the 1.5 * 2^23 rounding constant, f = x - n in
+// [-1/2, 1/2] in one FMA, the cubic of exp2_fma2 for 2^f, and n added to the
+// exponent field with one integer multiply-add per element.
+template <int HI>
+__device__ __forceinline__ uint64_t exp2_sat2(uint64_t y) {
+  static_assert(HI >= 0 && HI <= 127, "exponent range");
+  constexpr float kSpan = 126.0f + HI;
+  const uint64_t k = pack_f32x2(kSpan, kSpan);
+  const uint64_t c = pack_f32x2(12582786.0f, 12582786.0f);  // 1.5 * 2^23 - 126
+  const uint64_t t = fma_f32x2(y, k, c);                     // 1.5 * 2^23 + n, exactly
+  const uint64_t f = fma_f32x2(y, k, sub_f32x2(c, t));       // x - n
+  uint64_t q = fma_f32x2(pack_f32x2(0.0551713444f, 0.0551713444f), f, pack_f32x2(0.242610335f, 0.242610335f));
+  q = fma_f32x2(q, f, pack_f32x2(0.693260968f, 0.693260968f));
+  q = fma_f32x2(q, f, pack_f32x2(0.999928117f, 0.999928117f));
+  float q0, q1, t0, t1;
+  unpack_f32x2(q, q0, q1);
+  unpack_f32x2(t, t0, t1);
+  // The low 9 bits of t's pattern hold n mod 2^9; times 2^23 they are n in
+  // the exponent field, mod 2^32.
+  return pack_f32x2(__uint_as_float(__float_as_uint(t0) * (1u << 23) + __float_as_uint(q0)),
+                    __uint_as_float(__float_as_uint(t1) * (1u << 23) + __float_as_uint(q1)));
+}
+
 __device__ __forceinline__ int elect_one_lane() { return (threadIdx.x & 31) == 0; }
 
 }  // namespace hd

@@ -7,8 +7,10 @@ extra switches) next to libhd.so as ``libhd_trace.so``, runs one forward
 call of the bench's prefill workload (n=4, L=4096, B=2, 32q/8kv, D=128,
 bf16) after three warm-up calls, and prints, averaged over the CTAs, the
 cycles per tile each softmax warpgroup spends waiting for its scores, in the
-score load and row max, in the exponentials up to publishing P, in the row
-sum, and in the epilogue, and the MMA issuer's cycles waiting for P and for
+score load, in the mask and row max, in the exponentials up to publishing P,
+in the row sum, and (per tile, amortised) in the epilogue's wait for the last
+P V and in writing O out; the score load to P published on masked tiles
+and on a unit's first tile; and the MMA issuer's cycles waiting for P and for
 its Q/K/V/O stages.  The counters perturb the kernel (clock reads and a few
 more registers): compare them with each other, not with the timed build.
 """
@@ -52,20 +54,25 @@ def main():
     hd.hd_attn_fwd(q, k, v, n, a.mode, out=o)
     e1.record()
     torch.cuda.synchronize()
-    slots = 20
+    slots = 32
     buf = (ctypes.c_ulonglong * (1024 * slots))()
     L.hd_tc_trace_fetch(buf, 1024 * slots)
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     c = np.frombuffer(buf, dtype=np.uint64).reshape(1024, slots)[:sms].astype(np.float64)
     print(f"{a.mode}: {e0.elapsed_time(e1):.3f} ms (trace build), {sms} CTAs")
-    print(f"  MMA issuer per CTA: waiting for P {c[:, 12].mean() / 1e6:.3f} M clk, for Q/K/V/O "
-          f"{c[:, 13].mean() / 1e6:.3f} M clk, total {c[:, 14].mean() / 1e6:.3f} M clk")
-    names = ["wait for S", "load + max", "exp -> P published", "row sum", "epilogue"]
+    print(f"  MMA issuer per CTA: waiting for P {c[:, 24].mean() / 1e6:.3f} M clk, for Q/K/V/O "
+          f"{c[:, 25].mean() / 1e6:.3f} M clk, total {c[:, 26].mean() / 1e6:.3f} M clk")
+    names = ["wait for S", "score load", "mask + max", "exp -> P published", "row sum",
+             "epilogue: wait for last P V", "epilogue: O out"]
     for sl in (0, 1):
-        tiles = c[:, sl * 6 + 5].sum()
-        per = [c[:, sl * 6 + i].sum() / tiles for i in range(5)]
+        b = sl * 12
+        tiles = c[:, b + 7].sum()
+        per = [c[:, b + i].sum() / tiles for i in range(7)]
         print(f"  softmax slot {sl}: {tiles / sms:.1f} tiles per CTA; clk per tile: " +
               ", ".join(f"{nm} {x:.0f}" for nm, x in zip(names, per)))
+        masked = c[:, b + 9].sum()
+        print(f"    score load to P published: masked tiles {c[:, b + 8].sum() / max(masked, 1):.0f} clk "
+              f"({masked / sms:.1f} per CTA), first tiles of units {c[:, b + 10].sum() / sms:.0f} clk per CTA")
 
 
 if __name__ == "__main__":

@@ -3,7 +3,8 @@ replacement for part of the MUFU exponentials, and its packed f32x2 form
 exp2_fma2) against the MUFU form and float64 2**x, over its whole input
 range: no NaN or negative result, exact zero below 2^-126 (as the
 flush-to-zero MUFU form gives, -inf included; the packed form clamps there
-to ~2^-126), relative error below 1e-4 elsewhere.  A small probe library is compiled
+to ~2^-126), relative error below 1e-4 elsewhere; and exp2_sat2 behind the
+saturating shift, on exponents up to 8.  A small probe library is compiled
 from tests/probes/exp2_fma_probe.cu against the kernels' shared header."""
 
 import ctypes
@@ -43,8 +44,10 @@ def test_exp2_fma_whole_range(probe):
     fo = torch.empty_like(xt)
     mo = torch.empty_like(xt)
     po = torch.empty_like(xt)
+    so = torch.empty_like(xt)
     rc = probe.exp2_probe(ctypes.c_void_p(xt.data_ptr()), ctypes.c_void_p(fo.data_ptr()),
-                          ctypes.c_void_p(mo.data_ptr()), ctypes.c_void_p(po.data_ptr()), len(x))
+                          ctypes.c_void_p(mo.data_ptr()), ctypes.c_void_p(po.data_ptr()),
+                          ctypes.c_void_p(so.data_ptr()), len(x))
     assert rc == 0
     f = fo.cpu().numpy().astype(np.float64)
     m = mo.cpu().numpy().astype(np.float64)
@@ -67,3 +70,13 @@ def test_exp2_fma_whole_range(probe):
     ok = x >= -126.0
     assert np.array_equal(pr[ok], f[ok])
     assert (pr[~ok] <= 2.0 ** -125).all()
+    # the saturating form, on exponents x <= 8 (the attention kernel's:
+    # up to its rescale threshold): the shift through y = sat((x + 126) / 134)
+    # costs about 134 * 2^-25 in x; x below -126 lands on ~2^-126
+    sr = so.cpu().numpy().astype(np.float64)
+    inr = x <= 8.0
+    assert np.isfinite(sr[inr]).all() and (sr[inr] >= 0).all()
+    sn = inr & (x >= -125.0)
+    rel = np.abs(sr[sn] - exact[sn]) / exact[sn]
+    assert rel.max() < 1e-4, (float(rel.max()), float(x[sn][np.argmax(rel)]))
+    assert (sr[inr & (x < -125.0)] <= 2.0 ** -124).all()
