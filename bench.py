@@ -727,6 +727,22 @@ def extras(torch, peaks, rank):
         "repeats": 10, "l2": "flushed before each timed launch"}
     del lc
     torch.cuda.empty_cache()
+    # A plain device-to-device copy of as many bytes as each gather moves
+    # (torch copy_, i.e. the driver's memcpy, not this library's kernel): the
+    # rate HBM gives a copy of that size, fixed launch and drain costs
+    # included, beside the gather's own.
+    res["copy_same_bytes_as_gather"] = {}
+    for wl in ("intra", "long"):
+        c = WORKLOADS[wl]
+        gb = acc.gather_bytes(c["B"], c["L"], c["dm"])
+        src = torch.empty(gb // 2, dtype=torch.uint8, device="cuda")
+        dst = torch.empty_like(src)
+        ms_c = time_fn(lambda: dst.copy_(src))
+        res["copy_same_bytes_as_gather"][wl] = {
+            "bytes": gb, "ms": round(ms_c, 4), "GB/s": round(gb / (ms_c * 1e-3) / 1e9, 1),
+            "frac_hbm": round(gb / (ms_c * 1e-3) / 1e9 / peaks["hbm"], 4)}
+        del src, dst
+    torch.cuda.empty_cache()
     # RoPE fused into the attention (intra workload): hd_rope on q and k then
     # hd_attn_fwd, against hd_attn_fwd_rope (k rotated in place, q rotated
     # inside the attention kernel).  Repeated rotation of the same buffers
