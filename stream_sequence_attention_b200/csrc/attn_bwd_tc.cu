@@ -50,13 +50,35 @@ constexpr int kWarpTMA = 8;
 constexpr int kWarpMMA = 9;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kLdBytes = BT * 8;  // -lse2[128] then delta[128] of one query tile
-// One exponential in four of the dK/dV kernel's P tile on the FMA pipe (the
-// cubic of exp2_fma, relative error < 1e-4, below the bf16 rounding of P)
-// when nonzero, to offload the MUFU unit.
-#ifndef HD_BW_POLY_EXP
-#define HD_BW_POLY_EXP 0
+// One exponential pair in kPolyEvery of the P tiles (both kernels) on the
+// FMA pipe, to offload the MUFU unit (0: all on MUFU): the exponent x
+// (<= 0 up to rounding for a visible pair; masked pairs are zeroed after)
+// is shifted and clamped to y = sat((x + 126) / (126 + kPolyHi)) by one
+// saturating FMA per element, then exp2_sat2 (relative error < 1e-4, below
+// the bf16 rounding of P).
+#ifndef HD_BW_POLY_EVERY
+#define HD_BW_POLY_EVERY 3
 #endif
-constexpr bool kPolyExp = HD_BW_POLY_EXP != 0;
+constexpr int kPolyEvery = HD_BW_POLY_EVERY;
+constexpr int kPolyHi = 1;
+constexpr float kPolyInv = 1.f / (126.f + kPolyHi);
+__host__ __device__ constexpr bool poly_pair(int c) {
+  return kPolyEvery > 0 && (c % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
+}
+// 2^x of the pairs of a 64-column row piece, x in pv (in place).
+__device__ __forceinline__ void exp2_row64(float (&pv)[64]) {
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    if (poly_pair(c)) {
+      const float y0 = fma_sat(pv[2 * c], kPolyInv, 126.f * kPolyInv);
+      const float y1 = fma_sat(pv[2 * c + 1], kPolyInv, 126.f * kPolyInv);
+      unpack_f32x2(exp2_sat2<kPolyHi>(pack_f32x2(y0, y1)), pv[2 * c], pv[2 * c + 1]);
+    } else {
+      pv[2 * c] = ex2(pv[2 * c]);
+      pv[2 * c + 1] = ex2(pv[2 * c + 1]);
+    }
+  }
+}
 // Elementwise arithmetic as packed f32x2 operations (exponents of P for a
 // whole tile first, then the exponentials; dS = P (dP - delta) in pairs)
 // when nonzero.
@@ -517,8 +539,7 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
                                    pack_f32x2(l.z, l.w)),
                          pv[4 * c4 + 2], pv[4 * c4 + 3]);
           }
-#pragma unroll
-          for (int c = 0; c < 64; ++c) pv[c] = (bw::kPolyExp && (c & 3) == 3) ? exp2_fma(pv[c]) : ex2(pv[c]);
+          bw::exp2_row64(pv);
         } else {
 #pragma unroll
           for (int c4 = 0; c4 < 16; ++c4) {
@@ -526,8 +547,7 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
             pv[4 * c4 + 0] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 0]), sl2, l.x));
             pv[4 * c4 + 1] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 1]), sl2, l.y));
             pv[4 * c4 + 2] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 2]), sl2, l.z));
-            const float a3 = fmaf(__uint_as_float(sv[4 * c4 + 3]), sl2, l.w);
-            pv[4 * c4 + 3] = bw::kPolyExp ? exp2_fma(a3) : ex2(a3);
+            pv[4 * c4 + 3] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 3]), sl2, l.w));
           }
         }
         if (need_mask) {
@@ -819,8 +839,7 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
           for (int c = 0; c < 32; ++c)
             unpack_f32x2(fma_f32x2(pack_f32x2(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1])), s2, l2),
                          pv[2 * c], pv[2 * c + 1]);
-#pragma unroll
-          for (int c = 0; c < 64; ++c) pv[c] = ex2(pv[c]);
+          bw::exp2_row64(pv);
         } else {
 #pragma unroll
           for (int c = 0; c < 64; ++c) pv[c] = ex2(fmaf(__uint_as_float(sv[c]), sl2, ld.x));
