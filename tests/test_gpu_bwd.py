@@ -70,6 +70,30 @@ def test_bwd_matches_oracle(hd, dtype, mode, W, B, L, n, Hq, Hkv, D):
         assert err <= _bound(ref, tol), (name, err, float(np.max(np.abs(ref))))
 
 
+@pytest.mark.parametrize("mode,W", [("intra", 0), ("cross", 70)])
+def test_bwd_scores_beyond_the_exponent_range(hd, mode, W):
+    """Queries scaled by 40: within a row many exponents s*scale - lse fall
+    below -126, where the FMA-pipe exponential clamps to ~2^-126 instead of
+    0; dQ, dK and dV still match the oracle and stay finite."""
+    B, L, n, Hq, Hkv, D = 1, 300, 2, 4, 2, 128
+    P = n * L
+    q, k, v = host_qkv(B, P, Hq, Hkv, D, 720, "bf16")
+    q = synth.bf16_round(q.astype(np.float32) * np.float32(40.0))
+    dO = synth.normal((B, P, Hq, D), 723, dtype="bf16")
+    ro, rl = oracle.attn(q, k, v, n, mode, W)
+    rdq, rdk, rdv = oracle.attn_bwd(q, k, v, dO, n, mode, W)
+    st = hd.new_status()
+    dq, dk, dv = hd.hd_attn_bwd(dev(q, "bf16"), dev(k, "bf16"), dev(v, "bf16"), dev(_round(ro, "bf16"), "bf16"),
+                                dev(dO, "bf16"), dev(rl, "f32"), n, mode, W, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    for name, got, ref in (("dq", dq, rdq), ("dk", dk, rdk), ("dv", dv, rdv)):
+        g = to_f64(got)
+        assert np.isfinite(g).all(), name
+        err = max_abs(g, ref)
+        assert err <= _bound(ref, TOL_BF16), (name, err, float(np.max(np.abs(ref))))
+
+
 @pytest.mark.parametrize("mode,W", [("intra", 0), ("cross", 0), ("cross", 300)])
 def test_forward_backward_chain(hd, mode, W):
     """O and lse from the library's forward feed its backward."""

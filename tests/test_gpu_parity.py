@@ -171,6 +171,28 @@ def test_running_max_jumps(hd, mode, W, n, out_f32):
     assert int(st.item()) == 0
 
 
+@pytest.mark.parametrize("mode,W", [("intra", 0), ("cross", 0), ("cross", 100)])
+def test_scores_beyond_the_exponent_range(hd, mode, W):
+    """Scores spread so widely within a row (queries scaled by 40: a score
+    spread of ~60 log2 units, hundreds between a row's extremes) that many
+    exponents fall below -126: there the FMA-pipe exponential of the
+    unmasked tiles clamps to ~2^-126 where MUFU gives 0, both negligible
+    next to the row sum (>= 1).  O and lse still match the oracle and stay
+    finite."""
+    B, n, L, Hq, Hkv, D = 1, 2, 400, 4, 2, 128
+    P = n * L
+    q, k, v = host_qkv(B, P, Hq, Hkv, D, 91, "bf16")
+    q = synth.bf16_round(q.astype(np.float32) * np.float32(40.0))
+    st = hd.new_status()
+    o, lse = hd.hd_attn_fwd(dev(q, "bf16"), dev(k, "bf16"), dev(v, "bf16"), n, mode, W, lse=True, dev_status=st)
+    torch.cuda.synchronize()
+    ro, rl = oracle.attn(q, k, v, n, mode, W)
+    assert int(st.item()) == 0
+    assert np.isfinite(to_f64(o)).all() and np.isfinite(to_f64(lse)).all()
+    assert max_abs(to_f64(o), ro) <= TOL_BF16
+    assert max_abs(to_f64(lse), rl) <= 1e-3 * max(1.0, float(np.abs(rl).max()))
+
+
 @pytest.mark.parametrize("dtype,mode,W", [("bf16", "intra", 0), ("bf16", "cross", 0), ("bf16", "intra", 60),
                                           ("bf16", "cross", 90), ("f32", "intra", 0), ("f32", "cross", 33)])
 def test_masked_keys_do_not_change_output_bits(hd, dtype, mode, W):
