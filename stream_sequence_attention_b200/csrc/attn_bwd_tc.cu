@@ -132,7 +132,19 @@ struct LayQ {
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int ALLOC = MISC_OFF + 16 + 1024;
 };
+// Diagnostic build only (HD_BW_TRACE): per-role clock counters of the dK/dV
+// kernel, kBwTraceSlots per CTA (see hd_bw_trace_fetch).
+#ifndef HD_BW_TRACE
+#define HD_BW_TRACE 0
+#endif
+constexpr bool kTrace = HD_BW_TRACE != 0;
 }  // namespace bw
+
+#if HD_BW_TRACE
+constexpr int kBwTraceCtas = 1024;
+constexpr int kBwTraceSlots = 16;
+__device__ unsigned long long g_bw_trace[kBwTraceCtas * kBwTraceSlots];
+#endif
 
 struct BwParams {
   BwdWs ws;  // -lse2 and delta planes, stream-major, padded
@@ -434,6 +446,20 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
       const uint32_t tS = tmem, tDP = tmem + 128, tDV = tmem + 256, tDK = tmem + 256 + D;
       int t = 0, ul = 0;
       bool ok = true;
+      // Diagnostic counters (HD_BW_TRACE): waiting for P, for dS, for the
+      // Q/dO/K/V stages and the accumulators; total.
+      unsigned long long mw[4] = {0, 0, 0, 0};
+      const long long mt0 = bw::kTrace ? clock64() : 0;
+      auto tw = [&](int which, uint32_t b, uint32_t par) {
+        if constexpr (bw::kTrace) {
+          const long long t0 = clock64();
+          const bool r = mbar_wait(b, par, abort_flag);
+          mw[which] += static_cast<unsigned long long>(clock64() - t0);
+          return r;
+        } else {
+          return mbar_wait(b, par, abort_flag);
+        }
+      };
       auto issue_S = [&](int tt) {
         const int st = tt % Lay::QST;
         mma_rows_rows<D>(tS, sbase + Lay::K_OFF, sbase + Lay::Q_OFF + st * T::TILE);
@@ -449,38 +475,38 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
         if (u < 0) continue;  // round k has no unit for this CTA
         const KvUnit x = kv_unit(u, p);
         const int nt = G * x.nqt;
-        if (!mbar_wait(bar(Lay::B_KVFULL), ul & 1, abort_flag)) { ok = false; break; }
+        if (!tw(2, bar(Lay::B_KVFULL), ul & 1)) { ok = false; break; }
         if (nt == 0) {  // no query sees this key block: nothing to accumulate
           tc_commit(bar(Lay::B_ACCFULL));
           tc_commit(bar(Lay::B_KVEMPTY));
           continue;
         }
-        if (!mbar_wait(bar(Lay::B_QFULL + t % Lay::QST), (t / Lay::QST) & 1, abort_flag)) { ok = false; break; }
+        if (!tw(2, bar(Lay::B_QFULL + t % Lay::QST), (t / Lay::QST) & 1)) { ok = false; break; }
         tc_fence_after();
         issue_S(t);
-        if (!mbar_wait(bar(Lay::B_OFULL + t % Lay::QST), (t / Lay::QST) & 1, abort_flag)) { ok = false; break; }
+        if (!tw(2, bar(Lay::B_OFULL + t % Lay::QST), (t / Lay::QST) & 1)) { ok = false; break; }
         tc_fence_after();
         issue_dP(t);
         for (int j = 0; j < nt; ++j, ++t) {
           const int st = t % Lay::QST;
           const int stn = (t + 1) % Lay::QST;
           const uint32_t phn = ((t + 1) / Lay::QST) & 1;
-          if (!mbar_wait(bar(Lay::B_PFULL), t & 1, abort_flag)) { ok = false; break; }
-          if (j == 0 && ul > 0 && !mbar_wait(bar(Lay::B_ACCEMPTY), (ul - 1) & 1, abort_flag)) { ok = false; break; }
+          if (!tw(0, bar(Lay::B_PFULL), t & 1)) { ok = false; break; }
+          if (j == 0 && ul > 0 && !tw(2, bar(Lay::B_ACCEMPTY), (ul - 1) & 1)) { ok = false; break; }
           tc_fence_after();
           mma_tmem_rows<D>(tDV, tS, sbase + Lay::O_OFF + st * T::TILE, j > 0);
           tc_commit(bar(Lay::B_OEMPTY + st));
           if (j + 1 < nt) {
-            if (!mbar_wait(bar(Lay::B_QFULL + stn), phn, abort_flag)) { ok = false; break; }
+            if (!tw(2, bar(Lay::B_QFULL + stn), phn)) { ok = false; break; }
             tc_fence_after();
             issue_S(t + 1);
           }
-          if (!mbar_wait(bar(Lay::B_DSFULL), t & 1, abort_flag)) { ok = false; break; }
+          if (!tw(1, bar(Lay::B_DSFULL), t & 1)) { ok = false; break; }
           tc_fence_after();
           mma_tmem_rows<D>(tDK, tDP, sbase + Lay::Q_OFF + st * T::TILE, j > 0);
           tc_commit(bar(Lay::B_QEMPTY + st));
           if (j + 1 < nt) {
-            if (!mbar_wait(bar(Lay::B_OFULL + stn), phn, abort_flag)) { ok = false; break; }
+            if (!tw(2, bar(Lay::B_OFULL + stn), phn)) { ok = false; break; }
             tc_fence_after();
             issue_dP(t + 1);
           }
@@ -492,6 +518,11 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
       if (!ok) fail();
       tc_commit(bar(Lay::B_DRAIN));
       mbar_wait(bar(Lay::B_DRAIN), 0, no_abort);
+#if HD_BW_TRACE
+      mw[3] = static_cast<unsigned long long>(clock64() - mt0);
+      if (blockIdx.x < kBwTraceCtas)
+        for (int c = 0; c < 4; ++c) g_bw_trace[blockIdx.x * kBwTraceSlots + 8 + c] = mw[c];
+#endif
     }
   } else {
     // ------------------------------------------- elementwise + epilogue
@@ -503,6 +534,17 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
     const float sl2 = p.scale_log2;
     int t = 0, ul = 0;
     bool ok = true;
+    // Diagnostic counters (HD_BW_TRACE): waiting for S, forming P, waiting
+    // for dP, forming dS, tiles, epilogue.
+    unsigned long long tr[6] = {0, 0, 0, 0, 0, 0};
+    long long tmark = bw::kTrace ? clock64() : 0;
+    auto tick = [&](int i) {
+      if constexpr (bw::kTrace) {
+        const long long tt = clock64();
+        tr[i] += static_cast<unsigned long long>(tt - tmark);
+        tmark = tt;
+      }
+    };
     for (int k = 0, u = bw_unit_of(0, p.total_units); ok && u != -1;
          ul += (u >= 0), u = bw_unit_of(++k, p.total_units)) {
       if (u < 0) continue;  // round k has no unit for this CTA
@@ -513,9 +555,11 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
       for (int j = 0; j < nt; ++j, ++t) {
         const int st = t % Lay::QST;
         const int q0 = kv_tile_qt(x, j, G) * bw::BT + 64 * ch;  // first query of this half
+        if (bw::kTrace) tmark = clock64();
         bool got = mbar_wait(bar(Lay::B_SFULL), t & 1, abort_flag);
         got = got && mbar_wait(bar(Lay::B_QFULL + st), (t / Lay::QST) & 1, abort_flag);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        tick(0);
         tc_fence_after();
         uint32_t sv[64];
         tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
@@ -569,8 +613,10 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(Lay::B_PFULL));
+        tick(1);
         got = mbar_wait(bar(Lay::B_DPFULL), t & 1, abort_flag);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        tick(2);
         tc_fence_after();
         tmem_ld32(tDP, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
         tmem_ld32(tDP + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
@@ -603,8 +649,11 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(Lay::B_DSFULL));
+        tick(3);
+        if (bw::kTrace) ++tr[4];
       }
       if (!ok) break;
+      if (bw::kTrace) tmark = clock64();
       // Epilogue: dV and scale*dK rows of this unit's keys.
       const bool got = mbar_wait(bar(Lay::B_ACCFULL), ul & 1, abort_flag);
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
@@ -628,8 +677,13 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(bar(Lay::B_ACCEMPTY));
+      tick(5);
     }
     if (!ok) fail();
+#if HD_BW_TRACE
+    if (threadIdx.x == 0 && blockIdx.x < kBwTraceCtas)
+      for (int c = 0; c < 6; ++c) g_bw_trace[blockIdx.x * kBwTraceSlots + c] = tr[c];
+#endif
   }
 
   __syncthreads();
@@ -968,5 +1022,18 @@ cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, cons
   if (D == 64) return launch_bwd_tc_d<64>(mq, mk, mv, mo, p, (int)kv_units, (int)q_units, sms, st);
   return launch_bwd_tc_d<128>(mq, mk, mv, mo, p, (int)kv_units, (int)q_units, sms, st);
 }
+
+#if HD_BW_TRACE
+// Diagnostic build only: copy out / reset the dK/dV kernel's per-role clock
+// counters (kBwTraceSlots per CTA).
+extern "C" int hd_bw_trace_fetch(unsigned long long* dst, int count) {
+  if (count > kBwTraceCtas * kBwTraceSlots) count = kBwTraceCtas * kBwTraceSlots;
+  return static_cast<int>(cudaMemcpyFromSymbol(dst, g_bw_trace, sizeof(unsigned long long) * count));
+}
+extern "C" int hd_bw_trace_clear() {
+  static unsigned long long zero[kBwTraceCtas * kBwTraceSlots];
+  return static_cast<int>(cudaMemcpyToSymbol(g_bw_trace, zero, sizeof(zero)));
+}
+#endif
 
 }  // namespace hd
