@@ -14,7 +14,7 @@ PKG = os.path.join(ROOT, "stream_sequence_attention_b200")
 PROBES = ["softmax_probe.cu", "mma_probe.cu"]
 
 
-@pytest.mark.parametrize("mod", ["diag_trace", "diag_softmax", "diag_mma"])
+@pytest.mark.parametrize("mod", ["diag_trace", "diag_softmax", "diag_mma", "diag_ab"])
 def test_diag_modules_import(mod):
     m = importlib.import_module(f"stream_sequence_attention_b200.{mod}")
     assert callable(m.main)
