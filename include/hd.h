@@ -457,9 +457,13 @@ hd_status hd_rope(void* q, void* k, const int32_t* pos0, int B, int P, int Hq,
  *                          (HD_ROPE_HALF) or of 8 (HD_ROPE_INTERLEAVED)
  * in_dt must be HD_BF16 (HD_ERR_UNSUPPORTED otherwise).  Two launches on
  * `stream`: the rotation of k, then the attention.  The angles are reduced
- * exactly as in hd_rope; the query rows' cos/sin are evaluated in float32 on
- * the special-function unit (absolute error about 1e-6), so q's rotation can
- * differ from hd_rope's in the last bit of a bf16 value.
+ * exactly as in hd_rope (position times the 64-bit fixed-point fraction of a
+ * turn, mod one turn); for the query rows the top 23 bits of that fraction
+ * give the angle in float32, whose cos/sin come from the special-function
+ * unit (absolute error about 1e-6), so q's rotation can differ from
+ * hd_rope's in the last bit of a bf16 value.  Measured at parity with
+ * hd_rope + hd_attn_fwd on the same inputs (the rotation of q costs the
+ * attention kernel about what hd_rope's pass over q costs).
  */
 hd_status hd_attn_fwd_rope(const void* q, void* k, const void* v, void* o,
                            float* lse, int B, int L, int n, int Hq, int Hkv, int D,
